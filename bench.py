@@ -1,0 +1,413 @@
+#!/usr/bin/env python
+"""Throughput of the MLA hot path on B200: one JSON line on stdout.
+
+A step is one pass of the whole hot path on seeded synthetic inputs that are
+resident in HBM: the Kimi-K2-shape causal prefill (B=1, T=2048, H=64,
+R=512, N=128, P=64, V=128, YaRN) followed by the absorbed decode over a
+latent cache (B=64, cache lengths uniform in [1000, 32768], Kimi-K2 heads).
+The headline ``value`` is the prefill's TFLOP/s (algorithmic FLOPs over the
+prefill's device time in each step); the decode's HBM GB/s is reported in
+the ``decode`` object of the same line. Between steps L2 is flushed by
+writing a 256 MiB buffer outside the per-step events.
+
+``--impl reference`` times the fp64 CPU oracle on a bounded sample of the
+same workload on the host cores instead (the reference arm).
+
+Multi-GPU: the path does not shard across GPUs here (one process per GPU runs
+an independent replica; no collective on the data path); ``value`` sums the
+replicas' work over the slowest rank's time ("scaling": "weak").
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from decode_latent_rmsnorm_b200 import mla  # noqa: E402
+from decode_latent_rmsnorm_b200 import workloads as W  # noqa: E402
+
+METRIC = "MLA causal prefill TFLOP/s (frac of BF16 peak); absorbed decode HBM GB/s"
+
+
+# ---------------------------------------------------------------- algorithmic work
+
+def prefill_flops(wl) -> dict:
+    """Algorithmic FLOPs: up-projection 2*T*R*H*(N+V); attention over the
+    unmasked causal pairs only, 2*H*(D+V) per pair."""
+    T = sum(wl.seqlens)
+    H, R, N, P, V = wl.num_heads, wl.kv_lora_rank, wl.qk_nope, wl.qk_rope, wl.v_head
+    up = 2.0 * T * R * H * (N + V)
+    pairs = sum(L * (L + 1) / 2 for L in wl.seqlens)
+    attn = 2.0 * H * (N + P + V) * pairs
+    return dict(up=up, attn=attn, total=up + attn)
+
+
+def decode_bytes(wl, lens) -> dict:
+    """Algorithmic HBM bytes: every cached row once, kv_b_proj once, q and out."""
+    H, R, N, P, V = wl.num_heads, wl.kv_lora_rank, wl.qk_nope, wl.qk_rope, wl.v_head
+    es = 2 if wl.dtype == "bf16" else 4
+    B = len(lens)
+    cache = float(sum(lens)) * (R + P) * es
+    weight = float(H) * (N + V) * R * es
+    io = float(B) * H * (N + P) * es + float(B) * H * V * es
+    flops = 2.0 * sum(lens) * H * ((R + P) + R)
+    return dict(cache=cache, weight=weight, io=io, total=cache + weight + io, flops=flops)
+
+
+# ---------------------------------------------------------------- environment
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm=p["hbm_gbs"], bf16=p["bf16_tflops"], bf16_sustained=p["bf16_tflops_sustained"],
+                    source="measured")
+    return dict(hbm=6650.0, bf16=1590.0, bf16_sustained=1400.0, source="fallback")
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while running."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) != 6:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                mx = float(parts[1])
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[2:]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- CPU oracle timing
+
+def oracle_prefill_sample(wl, inp, budget_s: float):
+    """Time the fp64 oracle on whole heads of the prefill workload until
+    ``budget_s`` is spent; returns (TFLOP/s, sample text, threads)."""
+    import numpy as np
+    import oracle as O
+    from threadpoolctl import threadpool_info
+    rope = O.RopeConfig(**wl.rope)
+    shape = O.MlaShape(wl.num_heads, wl.kv_lora_rank, wl.qk_nope, wl.qk_rope, wl.v_head,
+                       eps=wl.eps, interleaved=wl.interleaved)
+    scale = O.softmax_scale(rope, shape.qk_head_dim)
+    cos, sin = O.rope_tables(rope, W.max_position(wl))
+    a = {k: (v.double().numpy() if v.is_floating_point() else v.numpy()) for k, v in inp.items()}
+    heads_done, t_spent, h = 0, 0.0, 0
+    while t_spent < budget_s and h < wl.num_heads:
+        t0 = time.perf_counter()
+        O.prefill(a["latent"], a["q"], a["w_kvb"], a["w_norm"], a["positions"], a["cu_seqlens"], cos, sin,
+                  shape, scale, heads=[h])
+        t_spent += time.perf_counter() - t0
+        heads_done += 1
+        h += 1
+    fl = prefill_flops(wl)["total"] * heads_done / wl.num_heads
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] + [1])
+    return fl / t_spent / 1e12, "%s: %d of %d heads, all rows (%.1f s)" % (
+        wl.name, heads_done, wl.num_heads, t_spent), threads
+
+
+# ---------------------------------------------------------------- GPU bench
+
+def run_ours(args, rank, world, device):
+    torch.cuda.set_device(device)
+    peaks = measured_peaks()
+    pwl = W.KIMI
+    dwl = W.DECODE
+    # inputs, resident in HBM
+    pin = W.prefill_inputs(pwl)
+    din = W.decode_inputs(dwl)
+    lens = [int(x) for x in din["cache_lens"]]
+    rope_p = mla.rope_for(pwl)
+    dims_p = mla.dims_for(pwl, mla.mla_softmax_scale(rope_p, pwl.qk_head_dim))
+    dims_d = mla.dims_for(dwl, mla.mla_softmax_scale(mla.rope_for(dwl), dwl.qk_head_dim))
+    max_pos = max(W.max_position(pwl), W.max_position(dwl))
+    cos, sin = mla.mla_init_rope_tables(rope_p, max_pos)
+    P = {k: v.to(device) for k, v in pin.items()}
+    D = {k: v.to(device) for k, v in din.items()}
+    T = sum(pwl.seqlens)
+    p_out = torch.empty((T, pwl.num_heads, pwl.v_head), dtype=torch.bfloat16, device=device)
+    p_ws = torch.empty(mla.mla_prefill_workspace_size(dims_p, T, len(pwl.seqlens)), dtype=torch.uint8,
+                       device=device)
+    B = dwl.batch
+    max_len = max(lens)
+    d_out = torch.empty((B, dwl.num_heads, dwl.v_head), dtype=torch.bfloat16, device=device)
+    d_ws = torch.empty(mla.mla_decode_workspace_size(dims_d, B, max_len), dtype=torch.uint8, device=device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+
+    def prefill():
+        mla.mla_prefill(dims_p, P["latent"], P["q"], P["w_kvb"], P["w_norm"], P["positions"],
+                        P["cu_seqlens"], max(pwl.seqlens), cos, sin, out=p_out, workspace=p_ws)
+
+    def decode():
+        mla.mla_decode(dims_d, D["q"], D["cache"], D["cache_offsets"], D["cache_lens"], D["positions"],
+                       max_len, D["w_kvb"], cos, sin, out=d_out, workspace=d_ws)
+
+    for _ in range(args.warmup):
+        flush.fill_(1)
+        prefill()
+        decode()
+    torch.cuda.synchronize()
+    mla.mla_check_device_status()
+
+    # timed region: per-step events around prefill and decode, per-kernel events
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    kev_p, kev_d = [], []
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    launches0 = mla.mla_launch_count()
+    with ClockSampler(device.index if device.index is not None else 0) as clocks:
+        for i in range(args.steps):
+            flush.fill_(i & 0xff)
+            kp, kd = mla.KernelEvents(16), mla.KernelEvents(16)
+            ev[i][0].record()
+            with kp:
+                prefill()
+            ev[i][1].record()
+            with kd:
+                decode()
+            ev[i][2].record()
+            kev_p.append(kp)
+            kev_d.append(kd)
+        torch.cuda.synchronize()
+    launches = mla.mla_launch_count() - launches0
+    if world > 1:
+        torch.distributed.barrier()
+    mla.mla_check_device_status()
+    p_ms = [e[0].elapsed_time(e[1]) for e in ev]
+    d_ms = [e[1].elapsed_time(e[2]) for e in ev]
+    step_ms = [a + b for a, b in zip(p_ms, d_ms)]
+
+    def reduce_max(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        return float(t.item())
+
+    p_mean = reduce_max(statistics.mean(p_ms))
+    d_mean = reduce_max(statistics.mean(d_ms))
+    s_mean = reduce_max(statistics.mean(step_ms))
+    fl = prefill_flops(pwl)
+    by = decode_bytes(dwl, lens)
+    p_tflops = world * fl["total"] / (p_mean * 1e-3) / 1e12
+    d_gbs = world * by["total"] / (d_mean * 1e-3) / 1e9
+
+    # per-kernel mean durations (kernel names reported by the library)
+    def kernel_means(kev):
+        acc = {}
+        for k in kev:
+            for n, t in zip(k.names, k.durations_ms()):
+                acc.setdefault(n, []).append(t)
+        return {n: statistics.mean(v) for n, v in acc.items()}
+
+    kp_ms, kd_ms = kernel_means(kev_p), kernel_means(kev_d)
+    allk = {**{("prefill", n): t for n, t in kp_ms.items()}, **{("decode", n): t for n, t in kd_ms.items()}}
+    (phase, top), top_ms = max(allk.items(), key=lambda kv: kv[1])
+    if phase == "prefill":
+        algo = fl["attn"] if "attention" in top else fl["up"] if "proj" in top else fl["total"]
+        roof = dict(bound="tensor", achieved=algo / (top_ms * 1e-3) / 1e12, peak=peaks["bf16"],
+                    unit="TFLOP/s")
+    else:
+        algo = by["cache"] if "split" in top else by["total"]
+        roof = dict(bound="hbm", achieved=algo / (top_ms * 1e-3) / 1e9, peak=peaks["hbm"], unit="GB/s")
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["kernel"] = top
+    roof["peak_source"] = peaks["source"]
+
+    # end to end through the same C-ABI with pinned host buffers
+    e2e = run_e2e(args, pwl, dwl, pin, din, dims_p, dims_d, cos, sin, P, D, p_ws, d_ws, device, world,
+                  reduce_max, fl, by)
+
+    res = dict(
+        metric=METRIC, value=p_tflops, unit="TFLOP/s", n_gpus=world, steps=args.steps,
+        warmup=args.warmup, ms_per_step=s_mean, higher_is_better=True, scaling="weak",
+        vs_baseline=None, dtype="bf16", data="synthetic (seeded N(0,1) inputs, N(0,1/R) kv_b_proj)",
+        config=dict(workload="kimi_k2_prefill_bf16 + absorbed_decode_bf16",
+                    prefill="B=1 T=2048 H=64 R=512 N=128 P=64 V=128 YaRN(base 5e4, factor 32)",
+                    decode="B=64 H=64 R=512 N=128 P=64 V=128, cache lens U[1000,32768] sum=%d" % sum(lens),
+                    global_batch=world * (1 + B), parallelism="replicas x%d" % world,
+                    l2="flushed between steps (256 MiB write outside per-step events)"),
+        prefill=dict(ms=p_mean, tflops=p_tflops, frac_of_bf16_peak=p_tflops / (world * peaks["bf16"]),
+                     tokens_per_s=world * T / (p_mean * 1e-3), gflop=fl["total"] / 1e9),
+        decode=dict(metric="absorbed decode HBM GB/s", value=d_gbs, unit="GB/s", ms=d_mean,
+                    frac_of_hbm=d_gbs / (world * peaks["hbm"]), tokens_per_s=world * B / (d_mean * 1e-3),
+                    tflops=world * by["flops"] / (d_mean * 1e-3) / 1e12, bytes=by["total"]),
+        kernels_ms=dict(prefill=kp_ms, decode=kd_ms),
+        roofline=roof, e2e=e2e, gpu_launches=int(launches), clocks=clocks.summary(),
+        peaks=dict(hbm_gbs=peaks["hbm"], bf16_tflops=peaks["bf16"], source=peaks["source"]),
+    )
+    return res, (pwl, pin)
+
+
+def run_e2e(args, pwl, dwl, pin, din, dims_p, dims_d, cos, sin, P, D, p_ws, d_ws, device, world,
+            reduce_max, fl, by):
+    """Same calls with the step's inputs copied from pinned host memory and the
+    result read back inside the timed region. Weights, rotary tables and the
+    latent cache stay resident (model state); the step inputs are the
+    prefill's latent/q/positions/cu_seqlens and the decode's
+    q/positions/lengths/offsets."""
+    hp = {k: pin[k].pin_memory() for k in ("latent", "q", "positions", "cu_seqlens")}
+    hd = {k: din[k].pin_memory() for k in ("q", "positions", "cache_lens", "cache_offsets")}
+    T = sum(pwl.seqlens)
+    B = dwl.batch
+    max_len = int(din["cache_lens"].max())
+    p_out_h = torch.empty((T, pwl.num_heads, pwl.v_head), dtype=torch.bfloat16).pin_memory()
+    d_out_h = torch.empty((B, dwl.num_heads, dwl.v_head), dtype=torch.bfloat16).pin_memory()
+    dp = {k: torch.empty_like(v, device=device) for k, v in hp.items()}
+    dd = {k: torch.empty_like(v, device=device) for k, v in hd.items()}
+    p_out = torch.empty(p_out_h.shape, dtype=torch.bfloat16, device=device)
+    d_out = torch.empty(d_out_h.shape, dtype=torch.bfloat16, device=device)
+    h2d_p = sum(v.numel() * v.element_size() for v in hp.values())
+    h2d_d = sum(v.numel() * v.element_size() for v in hd.values())
+    d2h_p = p_out_h.numel() * 2
+    d2h_d = d_out_h.numel() * 2
+
+    def step(evs):
+        evs[0].record()
+        for k in hp:
+            dp[k].copy_(hp[k], non_blocking=True)
+        mla.mla_prefill(dims_p, dp["latent"], dp["q"], P["w_kvb"], P["w_norm"], dp["positions"],
+                        dp["cu_seqlens"], max(pwl.seqlens), cos, sin, out=p_out, workspace=p_ws)
+        p_out_h.copy_(p_out, non_blocking=True)
+        evs[1].record()
+        for k in hd:
+            dd[k].copy_(hd[k], non_blocking=True)
+        mla.mla_decode(dims_d, dd["q"], D["cache"], dd["cache_offsets"], dd["cache_lens"], dd["positions"],
+                       max_len, D["w_kvb"], cos, sin, out=d_out, workspace=d_ws)
+        d_out_h.copy_(d_out, non_blocking=True)
+        evs[2].record()
+
+    for _ in range(args.warmup):
+        step([torch.cuda.Event(enable_timing=True) for _ in range(3)])
+    torch.cuda.synchronize()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    for i in range(args.steps):
+        step(evs[i])
+    torch.cuda.synchronize()
+    p_ms = reduce_max(statistics.mean(e[0].elapsed_time(e[1]) for e in evs))
+    d_ms = reduce_max(statistics.mean(e[1].elapsed_time(e[2]) for e in evs))
+    return dict(value=world * fl["total"] / (p_ms * 1e-3) / 1e12, unit="TFLOP/s",
+                h2d_bytes_per_step=h2d_p + h2d_d, d2h_bytes_per_step=d2h_p + d2h_d,
+                prefill_ms=p_ms, decode_ms=d_ms,
+                decode_gbs=world * by["total"] / (d_ms * 1e-3) / 1e9)
+
+
+def cpu_baseline(budget_s=15.0):
+    pin = W.prefill_inputs(W.KIMI)
+    v, sample, threads = oracle_prefill_sample(W.KIMI, pin, budget_s)
+    return dict(value=v, unit="TFLOP/s", cores=threads, kind="oracle", sample=sample)
+
+
+def run_reference(args, rank, world):
+    """The reference arm: the fp64 oracle as it stands, on host cores."""
+    if rank != 0:
+        return None
+    pin = W.prefill_inputs(W.KIMI)
+    vals = []
+    sample = ""
+    threads = 1
+    for i in range(args.warmup + args.steps):
+        v, sample, threads = oracle_prefill_sample(W.KIMI, pin, budget_s=3.0)
+        if i >= args.warmup:
+            vals.append(v)
+    v = statistics.mean(vals)
+    fl = prefill_flops(W.KIMI)["total"]
+    return dict(metric=METRIC, value=v, unit="TFLOP/s", n_gpus=world, steps=args.steps, warmup=args.warmup,
+                ms_per_step=fl / (v * 1e12) * 1e3, higher_is_better=True, scaling="weak", vs_baseline=None,
+                dtype="f64", data="synthetic", impl="reference",
+                config=dict(workload="kimi_k2_prefill_bf16 (oracle on a sample of heads per step)"),
+                cpu_baseline=dict(kind="oracle", cores=threads, sample=sample, value=v, unit="TFLOP/s"),
+                e2e=dict(value=v, unit="TFLOP/s", h2d_bytes_per_step=0, d2h_bytes_per_step=0))
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        res = run_reference(args, rank, world)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(device)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    res, _ = run_ours(args, rank, world, device)
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline()
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

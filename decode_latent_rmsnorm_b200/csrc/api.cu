@@ -1,0 +1,416 @@
+// C-ABI of the MLA hot path (declared in include/mla.h). Host-side argument
+// checks, workspace carving and kernel launches; every step of the path runs
+// in the kernels included below.
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <atomic>
+
+#include "mla.h"
+#include "common.cuh"
+#include "rope.cuh"
+#include "simt_prefill.cuh"
+#include "simt_decode.cuh"
+
+namespace {
+
+thread_local char g_err[1024] = "no error";
+
+int fail(int code, const char* fmt, ...) {
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(g_err, sizeof(g_err), fmt, ap);
+  va_end(ap);
+  return code;
+}
+
+int cuda_status(cudaError_t e, const char* what) {
+  if (e == cudaSuccess) return MLA_OK;
+  return fail(MLA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ---- launch accounting and optional per-kernel events ---------------------
+std::atomic<uint64_t> g_launches{0};
+thread_local cudaEvent_t const* g_events = nullptr;
+thread_local int g_event_pairs = 0;
+thread_local int g_event_next = 0;
+constexpr int kMaxNamed = 256;
+thread_local const char* g_event_names[kMaxNamed];
+
+// Bracket one kernel launch: prof_begin before, prof_end after.
+void prof_begin(cudaStream_t st, const char* name) {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  if (g_events && g_event_next < g_event_pairs) {
+    if (g_event_next < kMaxNamed) g_event_names[g_event_next] = name;
+    cudaEventRecord(g_events[2 * g_event_next], st);
+  }
+}
+void prof_end(cudaStream_t st) {
+  if (g_events && g_event_next < g_event_pairs) {
+    cudaEventRecord(g_events[2 * g_event_next + 1], st);
+    ++g_event_next;
+  }
+}
+
+// ---- YaRN scalars (Kimi-K2 "RoPE coefficients" page, rope excerpt) -------
+double correction_dim(double rotations, int dim, double base, double max_pos) {
+  return (dim * log(max_pos / (rotations * 2.0 * M_PI))) / (2.0 * log(base));
+}
+double yarn_mscale(double scale, double m) {
+  return scale <= 1.0 ? 1.0 : 0.1 * m * log(scale) + 1.0;
+}
+
+int check_rope(const mla_rope_cfg* r) {
+  if (!r) return fail(MLA_ERR_INVALID_ARG, "rope config is NULL");
+  if (r->rope_dim < 2 || r->rope_dim > 256 || (r->rope_dim & 1))
+    return fail(MLA_ERR_INVALID_ARG, "rope_dim must be even and in [2, 256], got %d", r->rope_dim);
+  if (!(r->base > 1.0)) return fail(MLA_ERR_INVALID_ARG, "rope base must be > 1");
+  if (r->yarn != 0 && r->yarn != 1) return fail(MLA_ERR_INVALID_ARG, "yarn must be 0 or 1");
+  if (r->reserved != 0) return fail(MLA_ERR_INVALID_ARG, "reserved field must be 0");
+  if (r->yarn) {
+    if (!(r->factor > 0.0)) return fail(MLA_ERR_INVALID_ARG, "YaRN factor must be > 0");
+    if (r->original_max_pos < 1) return fail(MLA_ERR_INVALID_ARG, "original_max_pos must be >= 1");
+    if (!(r->beta_fast > 0.0) || !(r->beta_slow > 0.0))
+      return fail(MLA_ERR_INVALID_ARG, "beta_fast and beta_slow must be > 0");
+  }
+  return MLA_OK;
+}
+
+int check_dims(const mla_dims* d) {
+  if (!d) return fail(MLA_ERR_INVALID_ARG, "dims is NULL");
+  if (d->dtype != MLA_BF16 && d->dtype != MLA_FP32)
+    return fail(MLA_ERR_INVALID_ARG, "dtype must be MLA_BF16 (0) or MLA_FP32 (1), got %d", d->dtype);
+  if (d->num_heads < 1 || d->kv_lora_rank < 1 || d->qk_nope < 0 || d->qk_rope < 2 || d->v_head < 1)
+    return fail(MLA_ERR_INVALID_ARG, "non-positive head geometry");
+  if (d->qk_rope & 1) return fail(MLA_ERR_INVALID_ARG, "qk_rope must be even");
+  if (d->rope_interleaved != 0 && d->rope_interleaved != 1)
+    return fail(MLA_ERR_INVALID_ARG, "rope_interleaved must be 0 or 1");
+  if (!(d->eps >= 0.0f)) return fail(MLA_ERR_INVALID_ARG, "eps must be >= 0");
+  if (!(d->softmax_scale > 0.0f) || !isfinite(d->softmax_scale))
+    return fail(MLA_ERR_INVALID_ARG, "softmax_scale must be finite and > 0");
+  if (d->kv_lora_rank % 16 || d->kv_lora_rank > 512)
+    return fail(MLA_ERR_UNSUPPORTED_SHAPE, "kv_lora_rank must be a multiple of 16 and <= 512");
+  if (d->v_head % 8 || d->v_head > 256)
+    return fail(MLA_ERR_UNSUPPORTED_SHAPE, "v_head must be a multiple of 8 and <= 256");
+  if (d->qk_nope + d->qk_rope > 512 || d->qk_rope > 256)
+    return fail(MLA_ERR_UNSUPPORTED_SHAPE, "qk head dim must be <= 512 and qk_rope <= 256");
+  return MLA_OK;
+}
+
+size_t elem_size(const mla_dims* d) { return d->dtype == MLA_FP32 ? 4 : 2; }
+
+// Prefill workspace: k_nope [H, Ttot, N], values [H, Ttot, V], k_rot [Ttot, P].
+struct PrefillWs {
+  size_t k_nope, vals, k_rot, total;
+};
+PrefillWs prefill_ws_layout(const mla_dims* d, int64_t T) {
+  PrefillWs w;
+  const size_t es = elem_size(d);
+  size_t off = 0;
+  w.k_nope = off; off = align_up(off + es * (size_t)d->num_heads * T * d->qk_nope, 256);
+  w.vals = off;   off = align_up(off + es * (size_t)d->num_heads * T * d->v_head, 256);
+  w.k_rot = off;  off = align_up(off + es * (size_t)T * d->qk_rope, 256);
+  w.total = off;
+  return w;
+}
+
+// Decode workspace: q_lat [B, H, R], q_rot [B, H, P], per-split partials.
+struct DecodeWs {
+  int nsplit;
+  size_t q_lat, q_rot, o_part, m_part, l_part, total;
+};
+DecodeWs decode_ws_layout(const mla_dims* d, int B, int max_len) {
+  DecodeWs w;
+  const size_t H = d->num_heads, R = d->kv_lora_rank, P = d->qk_rope;
+  w.nsplit = (max_len + mla::simt::kDecChunk - 1) / mla::simt::kDecChunk;
+  if (w.nsplit < 1) w.nsplit = 1;
+  const size_t S = w.nsplit;
+  size_t off = 0;
+  w.q_lat = off;  off = align_up(off + 4 * (size_t)B * H * R, 256);
+  w.q_rot = off;  off = align_up(off + 4 * (size_t)B * H * P, 256);
+  w.o_part = off; off = align_up(off + 4 * (size_t)B * S * H * R, 256);
+  w.m_part = off; off = align_up(off + 4 * (size_t)B * S * H, 256);
+  w.l_part = off; off = align_up(off + 4 * (size_t)B * S * H, 256);
+  w.total = off;
+  return w;
+}
+
+template <typename T>
+int launch_prefill(const mla_dims* d, const void* latent, const void* q, const void* w_kvb,
+                   const void* w_norm, const int32_t* positions, const int32_t* cu_seqlens,
+                   int num_seqs, int max_seqlen, int64_t T_tot, const float* cos_t,
+                   const float* sin_t, int max_pos, void* out, void* workspace, cudaStream_t st) {
+  using namespace mla::simt;
+  const int H = d->num_heads, R = d->kv_lora_rank, N = d->qk_nope, P = d->qk_rope, V = d->v_head;
+  const PrefillWs L = prefill_ws_layout(d, T_tot);
+  char* ws = static_cast<char*>(workspace);
+  T* k_nope = reinterpret_cast<T*>(ws + L.k_nope);
+  T* vals = reinterpret_cast<T*>(ws + L.vals);
+  T* k_rot = reinterpret_cast<T*>(ws + L.k_rot);
+  const int NOUT = H * (N + V);
+  dim3 g1((unsigned)((T_tot + kGemmBM - 1) / kGemmBM), (unsigned)((NOUT + kGemmBN - 1) / kGemmBN));
+  prof_begin(st, "simt_norm_kv_b_proj");
+  norm_proj_kernel<T><<<g1, 256, 0, st>>>(static_cast<const T*>(latent), static_cast<const T*>(w_kvb),
+                                          static_cast<const T*>(w_norm), T_tot, R, P, H, N, V, d->eps,
+                                          k_nope, vals);
+  prof_end(st);
+  const int64_t npairs = T_tot * (P / 2);
+  prof_begin(st, "simt_rope_key");
+  rope_key_kernel<T><<<(unsigned)((npairs + 255) / 256), 256, 0, st>>>(
+      static_cast<const T*>(latent), positions, cos_t, sin_t, max_pos, T_tot, R, P, d->rope_interleaved,
+      k_rot);
+  prof_end(st);
+  const size_t smem = attention_smem_bytes(N + P, V);
+  cudaError_t e = cudaFuncSetAttribute(attention_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return cuda_status(e, "attention smem attribute");
+  dim3 g2((unsigned)((max_seqlen + kAttBQ - 1) / kAttBQ), (unsigned)num_seqs, (unsigned)H);
+  prof_begin(st, "simt_attention");
+  attention_kernel<T><<<g2, 256, smem, st>>>(static_cast<const T*>(q), k_nope, k_rot, vals, positions,
+                                             cu_seqlens, cos_t, sin_t, max_pos, max_seqlen, T_tot, H, N, P, V,
+                                             d->rope_interleaved, d->softmax_scale, static_cast<T*>(out));
+  prof_end(st);
+  return cuda_status(cudaGetLastError(), "prefill launch");
+}
+
+template <typename T>
+int launch_decode(const mla_dims* d, const void* q, const void* cache, int64_t cache_num_rows,
+                  const int64_t* offsets, const int32_t* lens, const int32_t* positions, int B,
+                  int max_len, const void* w_kvb, const float* cos_t, const float* sin_t, int max_pos,
+                  void* out, void* workspace, cudaStream_t st) {
+  using namespace mla::simt;
+  const int H = d->num_heads, R = d->kv_lora_rank, N = d->qk_nope, P = d->qk_rope, V = d->v_head;
+  const DecodeWs L = decode_ws_layout(d, B, max_len);
+  char* ws = static_cast<char*>(workspace);
+  float* q_lat = reinterpret_cast<float*>(ws + L.q_lat);
+  float* q_rot = reinterpret_cast<float*>(ws + L.q_rot);
+  float* o_part = reinterpret_cast<float*>(ws + L.o_part);
+  float* m_part = reinterpret_cast<float*>(ws + L.m_part);
+  float* l_part = reinterpret_cast<float*>(ws + L.l_part);
+  prof_begin(st, "simt_decode_qprep");
+  qprep_kernel<T><<<dim3(B, H), 256, 0, st>>>(static_cast<const T*>(q), static_cast<const T*>(w_kvb),
+                                              positions, cos_t, sin_t, max_pos, H, R, N, P, V,
+                                              d->rope_interleaved, q_lat, q_rot);
+  prof_end(st);
+  const size_t smem = split_smem_bytes(R, P);
+  cudaError_t e = cudaFuncSetAttribute(split_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return cuda_status(e, "decode smem attribute");
+  dim3 g2(L.nsplit, B, (H + kDecHeads - 1) / kDecHeads);
+  prof_begin(st, "simt_decode_split");
+  split_kernel<T><<<g2, 256, smem, st>>>(q_lat, q_rot, static_cast<const T*>(cache), cache_num_rows, offsets,
+                                         lens, max_len, H, R, P, d->softmax_scale, L.nsplit, o_part, m_part,
+                                         l_part);
+  prof_end(st);
+  prof_begin(st, "simt_decode_combine");
+  combine_kernel<T><<<dim3(B, H), 256, 0, st>>>(o_part, m_part, l_part, static_cast<const T*>(w_kvb), H,
+                                                R, N, V, L.nsplit, static_cast<T*>(out));
+  prof_end(st);
+  return cuda_status(cudaGetLastError(), "decode launch");
+}
+
+}  // namespace
+
+extern "C" {
+
+int mla_version(void) { return 100; }
+
+uint64_t mla_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+int mla_set_kernel_events(void* const* events, int32_t pairs) {
+  if (pairs < 0) return fail(MLA_ERR_INVALID_ARG, "pairs must be >= 0");
+  g_events = (pairs > 0 && events) ? reinterpret_cast<cudaEvent_t const*>(events) : nullptr;
+  g_event_pairs = g_events ? pairs : 0;
+  g_event_next = 0;
+  return MLA_OK;
+}
+
+const char* mla_recorded_kernel_name(int32_t i) {
+  if (i < 0 || i >= g_event_next || i >= kMaxNamed) return "";
+  return g_event_names[i];
+}
+
+int mla_recorded_kernel_events(int32_t* recorded) {
+  if (!recorded) return fail(MLA_ERR_INVALID_ARG, "recorded is NULL");
+  *recorded = g_event_next;
+  return MLA_OK;
+}
+
+const char* mla_last_error_string(void) { return g_err; }
+
+int mla_softmax_scale(const mla_rope_cfg* rope, int32_t qk_head_dim, float* scale_out) {
+  int rc = check_rope(rope);
+  if (rc) return rc;
+  if (qk_head_dim < 1) return fail(MLA_ERR_INVALID_ARG, "qk_head_dim must be >= 1");
+  if (!scale_out) return fail(MLA_ERR_INVALID_ARG, "scale_out is NULL");
+  double s = pow((double)qk_head_dim, -0.5);
+  if (rope->yarn && rope->mscale_all_dim != 0.0) {
+    const double m = yarn_mscale(rope->factor, rope->mscale_all_dim);
+    s *= m * m;
+  }
+  *scale_out = (float)s;
+  return MLA_OK;
+}
+
+int mla_init_rope_tables(const mla_rope_cfg* rope, int32_t max_pos, float* cos_table,
+                         float* sin_table, cudaStream_t stream) {
+  int rc = check_rope(rope);
+  if (rc) return rc;
+  if (max_pos < 1) return fail(MLA_ERR_INVALID_ARG, "max_pos must be >= 1");
+  if (!cos_table || !sin_table) return fail(MLA_ERR_INVALID_ARG, "table pointer is NULL");
+  mla::RopeTableParams p;
+  p.pairs = rope->rope_dim / 2;
+  p.rope_dim = rope->rope_dim;
+  p.yarn = rope->yarn;
+  p.base = rope->base;
+  p.factor = rope->factor;
+  p.ramp_lo = 0.0;
+  p.ramp_hi = 1.0;
+  p.table_mscale = 1.0;
+  if (rope->yarn) {
+    const int dim = rope->rope_dim;
+    double lo = floor(correction_dim(rope->beta_fast, dim, rope->base, rope->original_max_pos));
+    double hi = ceil(correction_dim(rope->beta_slow, dim, rope->base, rope->original_max_pos));
+    if (lo < 0.0) lo = 0.0;
+    if (hi > dim - 1) hi = dim - 1;
+    if (lo == hi) hi += 0.001;   // the ramp's singular case
+    p.ramp_lo = lo;
+    p.ramp_hi = hi;
+    p.table_mscale = yarn_mscale(rope->factor, rope->mscale) / yarn_mscale(rope->factor, rope->mscale_all_dim);
+  }
+  const int64_t n = (int64_t)max_pos * p.pairs;
+  prof_begin(stream, "rope_tables");
+  mla::rope_tables_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(p, max_pos, cos_table, sin_table);
+  prof_end(stream);
+  return cuda_status(cudaGetLastError(), "rope table launch");
+}
+
+int mla_prefill_workspace_size(const mla_dims* dims, int64_t total_tokens, int32_t num_seqs,
+                               size_t* bytes) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (total_tokens < 0 || num_seqs < 0) return fail(MLA_ERR_INVALID_ARG, "negative size");
+  if (!bytes) return fail(MLA_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = prefill_ws_layout(dims, total_tokens).total;
+  return MLA_OK;
+}
+
+int mla_prefill(const mla_dims* dims, const void* latent, const void* q, const void* w_kvb,
+                const void* w_norm, const int32_t* positions, const int32_t* cu_seqlens,
+                int32_t num_seqs, int32_t max_seqlen, int64_t total_tokens, const float* cos_table,
+                const float* sin_table, int32_t max_pos, void* out, void* workspace,
+                size_t workspace_bytes, cudaStream_t stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (num_seqs < 0 || total_tokens < 0 || max_seqlen < 0 || max_pos < 1)
+    return fail(MLA_ERR_INVALID_ARG, "negative size or max_pos < 1");
+  if (num_seqs > 65535) return fail(MLA_ERR_UNSUPPORTED_SHAPE, "num_seqs must be <= 65535");
+  if (total_tokens > (int64_t)1 << 31) return fail(MLA_ERR_UNSUPPORTED_SHAPE, "total_tokens too large");
+  if (max_seqlen > total_tokens) return fail(MLA_ERR_INVALID_ARG, "max_seqlen exceeds total_tokens");
+  if (!cu_seqlens) return fail(MLA_ERR_INVALID_ARG, "cu_seqlens is NULL");
+  if (total_tokens == 0 || num_seqs == 0 || max_seqlen == 0) return MLA_OK;   // nothing to attend
+  if (!latent || !q || !w_kvb || !w_norm || !positions || !cos_table || !sin_table || !out)
+    return fail(MLA_ERR_INVALID_ARG, "a tensor pointer is NULL");
+  const size_t need = prefill_ws_layout(dims, total_tokens).total;
+  if (!workspace || workspace_bytes < need)
+    return fail(MLA_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes, got %zu", need, workspace_bytes);
+  if (dims->dtype == MLA_FP32)
+    return launch_prefill<float>(dims, latent, q, w_kvb, w_norm, positions, cu_seqlens, num_seqs,
+                                 max_seqlen, total_tokens, cos_table, sin_table, max_pos, out, workspace,
+                                 stream);
+  return launch_prefill<__nv_bfloat16>(dims, latent, q, w_kvb, w_norm, positions, cu_seqlens, num_seqs,
+                                       max_seqlen, total_tokens, cos_table, sin_table, max_pos, out,
+                                       workspace, stream);
+}
+
+int mla_decode_workspace_size(const mla_dims* dims, int32_t batch, int32_t max_cache_len, size_t* bytes) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (batch < 0 || max_cache_len < 0) return fail(MLA_ERR_INVALID_ARG, "negative size");
+  if (!bytes) return fail(MLA_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = decode_ws_layout(dims, batch, max_cache_len).total;
+  return MLA_OK;
+}
+
+int mla_decode(const mla_dims* dims, const void* q, const void* cache, int64_t cache_num_rows,
+               const int64_t* cache_offsets,
+               const int32_t* cache_lens, const int32_t* positions, int32_t batch,
+               int32_t max_cache_len, const void* w_kvb, const float* cos_table,
+               const float* sin_table, int32_t max_pos, void* out, void* workspace,
+               size_t workspace_bytes, cudaStream_t stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (batch < 0) return fail(MLA_ERR_INVALID_ARG, "batch must be >= 0");
+  if (batch == 0) return MLA_OK;
+  if (max_cache_len < 1) return fail(MLA_ERR_INVALID_ARG, "max_cache_len must be >= 1");
+  if (max_pos < 1) return fail(MLA_ERR_INVALID_ARG, "max_pos must be >= 1");
+  if (batch > 65535) return fail(MLA_ERR_UNSUPPORTED_SHAPE, "batch must be <= 65535");
+  if ((max_cache_len + mla::simt::kDecChunk - 1) / mla::simt::kDecChunk > 256)
+    return fail(MLA_ERR_UNSUPPORTED_SHAPE, "max_cache_len must be <= %d", 256 * mla::simt::kDecChunk);
+  if (!q || !cache || !cache_offsets || !cache_lens || !positions || !w_kvb || !cos_table || !sin_table ||
+      !out)
+    return fail(MLA_ERR_INVALID_ARG, "a tensor pointer is NULL");
+  if (dims->qk_nope > 512) return fail(MLA_ERR_UNSUPPORTED_SHAPE, "qk_nope must be <= 512");
+  if (cache_num_rows < 1) return fail(MLA_ERR_INVALID_ARG, "cache_num_rows must be >= 1");
+  const size_t need = decode_ws_layout(dims, batch, max_cache_len).total;
+  if (!workspace || workspace_bytes < need)
+    return fail(MLA_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes, got %zu", need, workspace_bytes);
+  if (dims->dtype == MLA_FP32)
+    return launch_decode<float>(dims, q, cache, cache_num_rows, cache_offsets, cache_lens, positions, batch,
+                                max_cache_len, w_kvb, cos_table, sin_table, max_pos, out, workspace, stream);
+  return launch_decode<__nv_bfloat16>(dims, q, cache, cache_num_rows, cache_offsets, cache_lens, positions,
+                                      batch, max_cache_len, w_kvb, cos_table, sin_table, max_pos, out,
+                                      workspace, stream);
+}
+
+int mla_cache_append(const mla_dims* dims, const void* latent, const void* w_norm,
+                     const int32_t* positions, int64_t n, const float* cos_table, const float* sin_table,
+                     int32_t max_pos, void* cache, int64_t cache_num_rows, const int64_t* cache_rows,
+                     cudaStream_t stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (n < 0) return fail(MLA_ERR_INVALID_ARG, "n must be >= 0");
+  if (n == 0) return MLA_OK;
+  if (n > 0x7fffffff) return fail(MLA_ERR_UNSUPPORTED_SHAPE, "too many rows");
+  if (max_pos < 1) return fail(MLA_ERR_INVALID_ARG, "max_pos must be >= 1");
+  if (!latent || !w_norm || !positions || !cos_table || !sin_table || !cache || !cache_rows)
+    return fail(MLA_ERR_INVALID_ARG, "a tensor pointer is NULL");
+  if (cache_num_rows < 1) return fail(MLA_ERR_INVALID_ARG, "cache_num_rows must be >= 1");
+  using namespace mla::simt;
+  const int R = dims->kv_lora_rank, P = dims->qk_rope;
+  prof_begin(stream, "simt_cache_append");
+  if (dims->dtype == MLA_FP32)
+    cache_append_kernel<float><<<(unsigned)n, 256, 0, stream>>>(
+        static_cast<const float*>(latent), static_cast<const float*>(w_norm), positions, cos_table, sin_table,
+        max_pos, R, P, dims->rope_interleaved, dims->eps, static_cast<float*>(cache), cache_num_rows,
+        cache_rows);
+  else
+    cache_append_kernel<__nv_bfloat16><<<(unsigned)n, 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(latent), static_cast<const __nv_bfloat16*>(w_norm), positions,
+        cos_table, sin_table, max_pos, R, P, dims->rope_interleaved, dims->eps,
+        static_cast<__nv_bfloat16*>(cache), cache_num_rows, cache_rows);
+  prof_end(stream);
+  return cuda_status(cudaGetLastError(), "cache append launch");
+}
+
+int mla_check_device_status(cudaStream_t stream) {
+  cudaError_t e = cudaStreamSynchronize(stream);
+  if (e != cudaSuccess) return cuda_status(e, "stream synchronize");
+  uint32_t v = 0;
+  e = cudaMemcpyFromSymbol(&v, mla::g_device_error, sizeof(v));
+  if (e != cudaSuccess) return cuda_status(e, "read device error word");
+  if (v) {
+    const uint32_t zero = 0;
+    e = cudaMemcpyToSymbol(mla::g_device_error, &zero, sizeof(zero));
+    if (e != cudaSuccess) return cuda_status(e, "clear device error word");
+    if (v & mla::kDevErrTimeout) return fail(MLA_ERR_DEVICE_TIMEOUT, "a device-side wait timed out (0x%x)", v);
+    return fail(MLA_ERR_INVALID_ARG, "device-side input check failed (0x%x)", v);
+  }
+  return MLA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,203 @@
+/*
+ * mla.h -- C-ABI of the B200 (sm_100a) multi-head latent attention hot path.
+ *
+ * The operations follow the eager MLA definition printed on these pages:
+ *   [EQ]  "Eager latent expansion" equation page ("Read the equation", and the
+ *         code under "Original context");
+ *   [KQ]  Kimi-K2 "Query content heads" page ("Split content heads",
+ *         "Join query parts");
+ *   [GLM] GLM-5 "Normalized key-value latent" page ("Key-value compression",
+ *         "KV cache");
+ *   [ROT] Kimi-K2 "RoPE coefficients" page ("Generate RoPE coefficients",
+ *         "Query heads", "Key heads").
+ *
+ * Conventions for every entry point:
+ *   - Tensor pointers are DEVICE pointers owned by the caller; the library
+ *     keeps no pointer after a call returns and allocates no device memory.
+ *     Scratch space is the caller's `workspace` buffer, sized by the matching
+ *     *_workspace_size query.
+ *   - Tensors are dense and row-major (last index contiguous) unless stated.
+ *   - Calls are asynchronous on `stream`; none synchronises the device except
+ *     mla_check_device_status. Host-side argument errors are reported before
+ *     anything is launched.
+ *   - The return value is an mla_status. mla_last_error_string() gives a
+ *     text for the last non-zero status of the calling thread.
+ *   - MLA_BF16 runs read and write bfloat16 tensors and accumulate in fp32;
+ *     MLA_FP32 runs are fp32 throughout (exact-fp32 SIMT kernels).
+ */
+#ifndef MLA_H_
+#define MLA_H_
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum mla_status {
+  MLA_OK = 0,
+  MLA_ERR_INVALID_ARG = 1,        /* null pointer, negative size, bad value     */
+  MLA_ERR_UNSUPPORTED_SHAPE = 2,  /* head geometry / alignment not supported    */
+  MLA_ERR_WORKSPACE_TOO_SMALL = 3,
+  MLA_ERR_CUDA = 4,               /* a CUDA runtime call failed                 */
+  MLA_ERR_DEVICE_TIMEOUT = 5      /* a bounded device-side wait gave up         */
+} mla_status;
+
+typedef enum mla_dtype { MLA_BF16 = 0, MLA_FP32 = 1 } mla_dtype;
+
+/* Rotary configuration; field names follow config.rope_scaling ([ROT]
+ * "Generate RoPE coefficients", model-args and rope excerpts).
+ *   yarn = 0: default rotary embedding, inv_freq[i] = base^(-2i/rope_dim).
+ *   yarn = 1: YaRN blend of base and factor-interpolated frequencies over the
+ *             correction range of (beta_fast, beta_slow) turns measured over
+ *             original_max_pos positions; tables multiplied by
+ *             get_mscale(factor, mscale) / get_mscale(factor, mscale_all_dim). */
+typedef struct mla_rope_cfg {
+  int32_t rope_dim;          /* qk_rope_head_dim, even, 2..256              */
+  int32_t yarn;              /* 0 or 1                                       */
+  int32_t original_max_pos;  /* YaRN original_max_position_embeddings        */
+  int32_t reserved;          /* must be 0                                    */
+  double base;               /* rope_theta (> 1)                             */
+  double factor;             /* YaRN scaling factor                          */
+  double beta_fast;
+  double beta_slow;
+  double mscale;
+  double mscale_all_dim;
+} mla_rope_cfg;
+
+/* Head geometry ([ROT] "Query heads" mla-init; [GLM] mla-init). */
+typedef struct mla_dims {
+  int32_t num_heads;         /* H                                            */
+  int32_t kv_lora_rank;      /* R                                            */
+  int32_t qk_nope;           /* N: non-rotary part of each query/key head    */
+  int32_t qk_rope;           /* P: rotary part, shared key across heads      */
+  int32_t v_head;            /* V                                            */
+  int32_t dtype;             /* mla_dtype                                    */
+  int32_t rope_interleaved;  /* 0: pair (i, i+P/2); 1: pair (2i, 2i+1)       */
+  float eps;                 /* latent RMSNorm epsilon ([GLM]: 1e-6)         */
+  float softmax_scale;       /* from mla_softmax_scale()                     */
+} mla_dims;
+
+/* Softmax scale ([ROT] model-args; [GLM] mla-init yarn_apply_mscale):
+ * qk_head_dim^-0.5, times get_mscale(factor, mscale_all_dim)^2 when yarn = 1
+ * and mscale_all_dim != 0. Host only; *scale_out is a host pointer. */
+int mla_softmax_scale(const mla_rope_cfg* rope, int32_t qk_head_dim, float* scale_out);
+
+/* Rotary cos/sin tables ([ROT] rope excerpt, _set_cos_sin_cache): for
+ * pos < max_pos and pair i < rope_dim/2,
+ *   cos_table[pos * rope_dim/2 + i] = cos(pos * inv_freq[i]) * table_mscale
+ * (sin likewise). The angle is formed in fp64; values are stored as fp32.
+ * cos_table/sin_table: device, fp32 [max_pos, rope_dim/2] each. */
+int mla_init_rope_tables(const mla_rope_cfg* rope, int32_t max_pos,
+                         float* cos_table, float* sin_table, cudaStream_t stream);
+
+/* Workspace bytes mla_prefill needs for `total_tokens` packed tokens. */
+int mla_prefill_workspace_size(const mla_dims* dims, int64_t total_tokens,
+                               int32_t num_seqs, size_t* bytes);
+
+/* Causal MLA prefill over packed sequences ([ROT] "Key heads" mla-kv and
+ * mla-prefill; [KQ] "Join query parts"; [EQ]).
+ *   latent     [Ttot, R + P]  compressed_kv before the split: latent then k_pe
+ *   q          [Ttot, H, N + P]  per-head query, non-rotary part first
+ *   w_kvb      [H * (N + V), R]  kv_b_proj weight (nn.Linear layout, no bias)
+ *   w_norm     [R]            latent RMSNorm weight
+ *   positions  int32 [Ttot]   rotary position of each token (< max_pos)
+ *   cu_seqlens int32 [num_seqs + 1]  sequence boundaries, cu[0] = 0,
+ *              non-decreasing, cu[num_seqs] = total_tokens; empty sequences
+ *              are allowed. max_seqlen (host) >= every sequence length.
+ *   cos_table, sin_table  fp32 [max_pos, P/2] from mla_init_rope_tables
+ *   out        [Ttot, H, V]   attention output, token-major
+ * Computes, per sequence and head: c_hat = RMSNorm(latent[:, :R]);
+ * [k_nope | v] = c_hat W^T split per head; q_pe and the one shared k_pe
+ * rotated at `positions`; softmax(scale * [q_nope|q_pe'][k_nope|k_pe']^T
+ * with a causal mask) @ v. All tensors use dims->dtype; positions and
+ * cu_seqlens are read on the device and range-checked there: a sequence with
+ * bad bounds (outside 0..total_tokens, or longer than max_seqlen) is skipped
+ * and a position outside the table is not used; either sets the device error
+ * word (see mla_check_device_status). */
+int mla_prefill(const mla_dims* dims,
+                const void* latent, const void* q, const void* w_kvb, const void* w_norm,
+                const int32_t* positions, const int32_t* cu_seqlens,
+                int32_t num_seqs, int32_t max_seqlen, int64_t total_tokens,
+                const float* cos_table, const float* sin_table, int32_t max_pos,
+                void* out, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* Workspace bytes mla_decode needs for `batch` sequences whose longest
+ * cache has max_cache_len rows. */
+int mla_decode_workspace_size(const mla_dims* dims, int32_t batch, int32_t max_cache_len,
+                              size_t* bytes);
+
+/* Absorbed decode: one new query per sequence over a latent cache
+ * ([GLM] "KV cache": the cache holds the normalized latent and the rotated
+ * shared key; [EQ] "Read the equation": the absorbed path contracts the
+ * projection weights with the query and with the latent aggregate).
+ *   q             [B, H, N + P]
+ *   cache         [cache_num_rows, R + P]  each row = c_hat (R) || rotated k_pe (P)
+ *   cache_offsets int64 [B]       first cache row of sequence b
+ *   cache_lens    int32 [B]       cached rows of sequence b, 1..max_cache_len
+ *   positions     int32 [B]       rotary position of the new query (< max_pos)
+ *   w_kvb         [H * (N + V), R]
+ *   out           [B, H, V]
+ * Per (b, h): q_lat = W_UK_h^T q_nope, q_pe' = rope(q_pe, positions[b]),
+ * s_t = scale (q_lat . c_hat_t + q_pe' . k_pe_t) over the sequence's rows,
+ * o_lat = softmax(s) . c_hat, out = W_UV_h o_lat, where W_UK_h / W_UV_h are
+ * the k_nope / value rows of head h in w_kvb. Attention is split over rows
+ * and the pieces are merged by their log-sum-exp.
+ * Device-resident arguments are range-checked on the device: a sequence whose
+ * rows fall outside the cache, whose length is outside 1..max_cache_len or
+ * whose position is outside the table is skipped (its output is zero) and the
+ * device error word is set (see mla_check_device_status). */
+int mla_decode(const mla_dims* dims, const void* q, const void* cache, int64_t cache_num_rows,
+               const int64_t* cache_offsets, const int32_t* cache_lens,
+               const int32_t* positions, int32_t batch, int32_t max_cache_len,
+               const void* w_kvb, const float* cos_table, const float* sin_table,
+               int32_t max_pos, void* out, void* workspace, size_t workspace_bytes,
+               cudaStream_t stream);
+
+/* New cache rows ([GLM] "KV cache" and "Key-value compression": the cache is
+ * written while the latent is still compressed, with the normalized latent
+ * and the rotated key).
+ *   latent     [n, R + P]  rows of compressed_kv
+ *   w_norm     [R]
+ *   positions  int32 [n]
+ *   cache      [cache_num_rows, R + P]  destination; row i goes to cache_rows[i]
+ *   cache_rows int64 [n]   destination row of each new token
+ * Row = RMSNorm(latent[:R]) || rope(latent[R:], position). A destination
+ * row or position out of range is skipped and sets the device error word. */
+int mla_cache_append(const mla_dims* dims, const void* latent, const void* w_norm,
+                     const int32_t* positions, int64_t n, const float* cos_table,
+                     const float* sin_table, int32_t max_pos, void* cache,
+                     int64_t cache_num_rows, const int64_t* cache_rows, cudaStream_t stream);
+
+/* Synchronises `stream`, then reads and clears the device error word that
+ * the kernels' bounded waits set. Returns MLA_ERR_DEVICE_TIMEOUT if one gave
+ * up since the last check, MLA_ERR_CUDA on a CUDA error, else MLA_OK. */
+int mla_check_device_status(cudaStream_t stream);
+
+/* Text of the calling thread's last error (static storage, never NULL). */
+const char* mla_last_error_string(void);
+
+/* Profiling support. Registers `pairs` pairs of host cudaEvent_t handles
+ * (`events` points to 2 * pairs handles created by the caller). Every kernel
+ * the calling thread's later calls launch records events[2i] on its stream
+ * right before the i-th launch and events[2i+1] right after it, for
+ * i < pairs; later launches are not recorded. pairs = 0 (or events = NULL)
+ * stops recording. Returns the number of launches recorded so far under the
+ * current registration in *recorded when `recorded` is not NULL. */
+int mla_set_kernel_events(void* const* events, int32_t pairs);
+int mla_recorded_kernel_events(int32_t* recorded);
+/* Kernel name of the i-th recorded launch ("" when i is out of range). */
+const char* mla_recorded_kernel_name(int32_t i);
+
+/* Number of kernels this library has launched in this process. */
+uint64_t mla_launch_count(void);
+
+/* Library version, major * 10000 + minor * 100 + patch. */
+int mla_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* MLA_H_ */

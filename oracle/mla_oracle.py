@@ -391,21 +391,22 @@ def decode_absorbed(q, cache, cache_offsets, cache_lens, positions, W, cos, sin,
     B = q.shape[0]
     batches = list(range(B)) if batches is None else batches
     heads = list(range(H)) if heads is None else heads
-    Wh = W.reshape(H, N + V, R)
+    Wh = W.reshape(H, N + V, R)[heads]
+    W_UK, W_UV = Wh[:, :N, :], Wh[:, N:, :]                  # [h, N, R], [h, V, R]
     out = np.full((B, H, V), np.nan)
     for b in batches:
         rows = _cache_rows(cache, cache_offsets, cache_lens, b)
         c_hat, k_rot = rows[:, :R], rows[:, R:]
         p = int(positions[b])
-        for h in heads:
-            W_UK, W_UV = Wh[h, :N], Wh[h, N:]
-            q_lat = W_UK.T @ q[b, h, :N]
-            q_pe_rot = apply_rope(q[b, h, N:], cos[p], sin[p], shape.interleaved)
-            s = (c_hat @ q_lat + k_rot @ q_pe_rot) * scale
-            s = s - s.max()
-            e = np.exp(s)
-            o_lat = (e / e.sum()) @ c_hat
-            out[b, h] = W_UV @ o_lat
+        q_lat = np.einsum("hnr,hn->hr", W_UK, q[b, heads, :N])          # [h, R]
+        q_pe_rot = apply_rope(q[b, heads, N:], cos[p][None, :], sin[p][None, :],
+                              shape.interleaved)                         # [h, P]
+        s = (c_hat @ q_lat.T + k_rot @ q_pe_rot.T) * scale               # [L, h]
+        s = s - s.max(axis=0, keepdims=True)
+        e = np.exp(s)
+        probs = e / e.sum(axis=0, keepdims=True)                         # softmax over rows
+        o_lat = probs.T @ c_hat                                          # [h, R]
+        out[b, heads] = np.einsum("hvr,hr->hv", W_UV, o_lat)
     return out
 
 

@@ -1,0 +1,125 @@
+"""C-ABI checks that need no GPU: the library loads, exports every symbol the
+header declares, and rejects bad arguments on the host before any launch."""
+
+import ctypes
+import math
+import os
+import re
+
+import pytest
+
+from decode_latent_rmsnorm_b200 import mla
+import oracle as O
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+FAKE = ctypes.c_void_p(0x1000)   # never dereferenced: every call below fails on the host
+
+
+def declared_functions():
+    text = open(os.path.join(ROOT, "include", "mla.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mla_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_exports_every_declared_symbol():
+    lib = mla.load()
+    names = declared_functions()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(lib, n), n
+        assert n in mla.SIGNATURES, n
+    assert mla.mla_version() >= 100
+
+
+def kimi_dims(**kw):
+    d = dict(num_heads=64, kv_lora_rank=512, qk_nope=128, qk_rope=64, v_head=128, dtype=0,
+             rope_interleaved=0, eps=1e-6, softmax_scale=0.13)
+    d.update(kw)
+    return mla.Dims(**d)
+
+
+def test_softmax_scale_matches_oracle():
+    kimi = mla.RopeCfg.make(64, 50000.0, yarn=True, factor=32.0, original_max_pos=4096,
+                            beta_fast=32.0, beta_slow=1.0, mscale=1.0, mscale_all_dim=1.0)
+    glm = mla.RopeCfg.make(64, 10000.0)
+    s = mla.mla_softmax_scale(kimi, 192)
+    ref = O.softmax_scale(O.RopeConfig(64, 50000.0, True, 32.0, 4096, 32.0, 1.0, 1.0, 1.0), 192)
+    assert s == pytest.approx(ref, rel=1e-7)
+    assert mla.mla_softmax_scale(glm, 256) == 0.0625
+    assert mla.mla_softmax_scale(mla.RopeCfg.make(8, 10000.0), 24) == pytest.approx(24 ** -0.5, rel=1e-7)
+
+
+def test_rope_config_rejections():
+    with pytest.raises(mla.MlaError) as e:
+        mla.mla_softmax_scale(mla.RopeCfg.make(63, 10000.0), 128)
+    assert e.value.status == 1
+    with pytest.raises(mla.MlaError):
+        mla.mla_softmax_scale(mla.RopeCfg.make(64, 1.0), 128)
+    with pytest.raises(mla.MlaError):
+        mla.mla_softmax_scale(mla.RopeCfg.make(64, 10000.0, yarn=True, factor=-1.0), 128)
+    lib = mla.load()
+    assert lib.mla_init_rope_tables(ctypes.byref(mla.RopeCfg.make(64, 1e4)), 0, FAKE, FAKE, None) == 1
+    assert lib.mla_init_rope_tables(ctypes.byref(mla.RopeCfg.make(64, 1e4)), 8, None, FAKE, None) == 1
+
+
+def _prefill(lib, dims, **over):
+    a = dict(latent=FAKE, q=FAKE, w=FAKE, wn=FAKE, pos=FAKE, cu=FAKE, nseq=1, maxlen=16, T=16,
+             cos=FAKE, sin=FAKE, maxpos=16, out=FAKE, ws=FAKE, wsb=1 << 40)
+    a.update(over)
+    return lib.mla_prefill(ctypes.byref(dims) if dims is not None else None, a["latent"], a["q"], a["w"],
+                           a["wn"], a["pos"], a["cu"], a["nseq"], a["maxlen"], a["T"], a["cos"],
+                           a["sin"], a["maxpos"], a["out"], a["ws"], a["wsb"], None)
+
+
+def test_prefill_host_validation():
+    lib = mla.load()
+    assert _prefill(lib, None) == 1
+    assert _prefill(lib, kimi_dims(dtype=7)) == 1
+    assert _prefill(lib, kimi_dims(qk_rope=63)) == 1
+    assert _prefill(lib, kimi_dims(kv_lora_rank=100)) == 2
+    assert _prefill(lib, kimi_dims(v_head=260)) == 2
+    assert _prefill(lib, kimi_dims(softmax_scale=float("nan"))) == 1
+    assert _prefill(lib, kimi_dims(), latent=None) == 1
+    assert _prefill(lib, kimi_dims(), cu=None) == 1
+    assert _prefill(lib, kimi_dims(), maxlen=17) == 1          # longer than all tokens
+    assert _prefill(lib, kimi_dims(), maxpos=0) == 1
+    assert _prefill(lib, kimi_dims(), wsb=10) == 3
+    assert "workspace" in mla.mla_last_error_string()
+    assert _prefill(lib, kimi_dims(), ws=None) == 3
+    # empty work is a successful no-op (nothing is launched)
+    assert _prefill(lib, kimi_dims(), T=0, maxlen=0) == 0
+    assert _prefill(lib, kimi_dims(), nseq=0) == 0
+
+
+def test_decode_host_validation():
+    lib = mla.load()
+    d = kimi_dims()
+
+    def call(**over):
+        a = dict(q=FAKE, cache=FAKE, offs=FAKE, lens=FAKE, pos=FAKE, B=4, maxlen=100, w=FAKE, cos=FAKE,
+                 sin=FAKE, maxpos=200, out=FAKE, ws=FAKE, wsb=1 << 40)
+        a.update(over)
+        return lib.mla_decode(ctypes.byref(d), a["q"], a["cache"], a.get("rows", 10 ** 6), a["offs"], a["lens"], a["pos"], a["B"],
+                              a["maxlen"], a["w"], a["cos"], a["sin"], a["maxpos"], a["out"], a["ws"],
+                              a["wsb"], None)
+
+    assert call(B=-1) == 1
+    assert call(B=0) == 0
+    assert call(maxlen=0) == 1
+    assert call(cache=None) == 1
+    assert call(lens=None) == 1
+    assert call(wsb=16) == 3
+    assert call(rows=0) == 1
+
+
+def test_workspace_sizes_are_monotone():
+    d = kimi_dims()
+    a = mla.mla_prefill_workspace_size(d, 1000, 1)
+    b = mla.mla_prefill_workspace_size(d, 2000, 1)
+    assert 0 < a < b
+    # at least the bf16 k_nope, values and rotated key of every token
+    assert b >= 2 * 2000 * (64 * (128 + 128) + 64)
+    assert mla.mla_decode_workspace_size(d, 64, 32768) > mla.mla_decode_workspace_size(d, 8, 32768)
+    with pytest.raises(mla.MlaError):
+        mla.mla_prefill_workspace_size(d, -1, 1)

@@ -1,0 +1,193 @@
+"""GPU parity: the CUDA library against the fp64 oracle on seeded inputs.
+
+Small cases compare every element; the full-size workloads compare every
+element the oracle evaluates (all of the Kimi-K2 prefill; sampled heads and
+rows elsewhere). All calls go through the C-ABI via the ctypes binding.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from decode_latent_rmsnorm_b200 import mla
+from decode_latent_rmsnorm_b200 import workloads as W
+from _parity import (compare, f64, oracle_cfg, oracle_decode, oracle_prefill, run_decode,
+                     run_prefill)
+
+pytestmark = pytest.mark.gpu
+
+
+# ---------------------------------------------------------------- rotary tables
+
+@pytest.mark.parametrize("wl", [W.TINY, W.KIMI, W.GLM], ids=lambda w: w.name)
+def test_rope_tables_match_oracle(gpu_lib, wl):
+    rope, shape, _ = oracle_cfg(wl)
+    max_pos = 40000
+    cos, sin = mla.mla_init_rope_tables(mla.rope_for(wl), max_pos)
+    rc, rs = O.rope_tables(rope, max_pos)
+    m = O.rope_table_mscale(rope)
+    assert np.abs(f64(cos) - rc).max() <= 1e-7 * m
+    assert np.abs(f64(sin) - rs).max() <= 1e-7 * m
+
+
+def test_rope_tables_yarn_mscale_ratio(gpu_lib):
+    # mscale != mscale_all_dim: tables carry get_mscale(f, m) / get_mscale(f, m_all)
+    rope = O.RopeConfig(rope_dim=64, base=50000.0, yarn=True, factor=32.0, mscale=0.707,
+                        mscale_all_dim=0.0)
+    cfg = mla.RopeCfg.make(64, 50000.0, yarn=True, factor=32.0, mscale=0.707, mscale_all_dim=0.0)
+    cos, sin = mla.mla_init_rope_tables(cfg, 5000)
+    rc, rs = O.rope_tables(rope, 5000)
+    assert np.abs(f64(cos) - rc).max() <= 2e-7 and np.abs(f64(sin) - rs).max() <= 2e-7
+
+
+# ---------------------------------------------------------------- prefill
+
+def test_prefill_tiny_fp32(gpu_lib):
+    inp = W.prefill_inputs(W.TINY)
+    got = run_prefill(W.TINY, inp)
+    compare(f64(got), oracle_prefill(W.TINY, inp), "fp32", "tiny")
+
+
+@pytest.mark.parametrize("seqlens", [(1,), (127,), (129, 1, 300), (0, 200, 0, 77, 0)],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_prefill_kimi_heads_ragged(gpu_lib, seqlens):
+    wl = W.scaled(W.KIMI, seqlens=seqlens, seed=11)
+    inp = W.prefill_inputs(wl)
+    got = run_prefill(wl, inp)
+    compare(f64(got), oracle_prefill(wl, inp), "bf16", "kimi ragged")
+
+
+def test_prefill_glm_heads_small(gpu_lib):
+    wl = W.scaled(W.GLM, seqlens=(300, 129), seed=12)
+    inp = W.prefill_inputs(wl)
+    got = run_prefill(wl, inp)
+    compare(f64(got), oracle_prefill(wl, inp), "bf16", "glm small")
+
+
+def test_prefill_fp32_other_geometry(gpu_lib):
+    # fp32, half-split pairs, a geometry unlike the configs (H=3, N=32, P=16, V=24)
+    wl = W.Workload("odd_fp32", "prefill", 3, 128, 32, 16, 24, "fp32", dict(W.KIMI_ROPE, rope_dim=16),
+                    21, seqlens=(70, 33))
+    inp = W.prefill_inputs(wl)
+    got = run_prefill(wl, inp)
+    compare(f64(got), oracle_prefill(wl, inp), "fp32", "odd fp32")
+
+
+def test_prefill_kimi_full(gpu_lib):
+    inp = W.prefill_inputs(W.KIMI)
+    got = run_prefill(W.KIMI, inp)
+    compare(f64(got), oracle_prefill(W.KIMI, inp), "bf16", "kimi full")
+
+
+def test_prefill_glm_full_sampled_heads(gpu_lib):
+    inp = W.prefill_inputs(W.GLM)
+    got = run_prefill(W.GLM, inp)
+    compare(f64(got), oracle_prefill(W.GLM, inp, heads=[0, 1, 31, 63]), "bf16", "glm full")
+
+
+def _varlen_rows(seqlens, seed=0):
+    """Sampled query rows of long sequences: first/last 32, rows around every
+    128-row tile boundary, and seeded random rows (256 in all)."""
+    rng = np.random.default_rng(seed)
+    rows = {}
+    for s, L in enumerate(seqlens):
+        if L <= 4096:
+            continue
+        pick = set(range(32)) | set(range(L - 32, L))
+        for t in range(128, L, 128 * 16):
+            pick |= {t - 1, t}
+        while len(pick) < 256:
+            pick.add(int(rng.integers(0, L)))
+        rows[s] = np.array(sorted(pick))
+    return rows
+
+
+def test_prefill_varlen_sampled(gpu_lib):
+    wl = W.VARLEN
+    inp = W.prefill_inputs(wl)
+    got = run_prefill(wl, inp)
+    ref = oracle_prefill(wl, inp, heads=[0, 1, 31, 63], rows=_varlen_rows(wl.seqlens))
+    compare(f64(got), ref, "bf16", "varlen")
+
+
+def test_prefill_output_guard_bytes(gpu_lib):
+    # Writes stay inside `out`: guard regions around it keep their bytes.
+    wl = W.scaled(W.KIMI, seqlens=(200, 57), seed=13)
+    inp = W.prefill_inputs(wl)
+    T = 257
+    n = T * 64 * 128
+    buf = torch.full((n + 2 * 4096,), 7.0, dtype=torch.bfloat16, device="cuda")
+    out = buf[4096:4096 + n].view(T, 64, 128)
+    rope, shape, _ = oracle_cfg(wl)
+    dims = mla.dims_for(wl, mla.mla_softmax_scale(mla.rope_for(wl), 192))
+    cos, sin = mla.mla_init_rope_tables(mla.rope_for(wl), 256)
+    d = {k: v.cuda() for k, v in inp.items()}
+    mla.mla_prefill(dims, d["latent"], d["q"], d["w_kvb"], d["w_norm"], d["positions"], d["cu_seqlens"],
+                    200, cos, sin, out=out)
+    torch.cuda.synchronize()
+    assert torch.all(buf[:4096] == 7.0) and torch.all(buf[4096 + n:] == 7.0)
+
+
+# ---------------------------------------------------------------- decode
+
+def test_decode_small_all_heads(gpu_lib):
+    wl = W.scaled(W.DECODE, batch=5, cache_lens=(1, 2, 63, 700, 2049), seed=14)
+    inp = W.decode_inputs(wl)
+    got = run_decode(wl, inp)
+    ref = oracle_decode(wl, inp, batches=range(5))
+    compare(f64(got), ref, "bf16", "decode small")
+
+
+def test_decode_fp32_tiny_geometry(gpu_lib):
+    wl = W.Workload("tiny_decode_fp32", "decode", 2, 64, 16, 8, 16, "fp32", W.TINY_ROPE, 15,
+                    batch=3, cache_lens=(1, 40, 333))
+    inp = W.decode_inputs(wl)
+    got = run_decode(wl, inp)
+    compare(f64(got), oracle_decode(wl, inp, batches=range(3)), "fp32", "decode fp32")
+
+
+def test_decode_full_sampled(gpu_lib):
+    wl = W.DECODE
+    inp = W.decode_inputs(wl)
+    got = f64(run_decode(wl, inp))
+    eager = oracle_decode(wl, inp, batches=[0, 9, 17, 25, 33, 41, 50, 63], heads=[0, 1, 31, 63])
+    compare(got, eager, "bf16", "decode vs eager")
+    absorbed = oracle_decode(wl, inp, batches=range(0, 64, 4), absorbed=True)
+    compare(got, absorbed, "bf16", "decode vs absorbed")
+
+
+def test_cache_append_then_decode_matches_prefill_row(gpu_lib):
+    # Append every token of two sequences to a latent cache on the GPU, then a
+    # decode step for each sequence's last token must reproduce the oracle's
+    # prefill output for that token.
+    wl = W.scaled(W.KIMI, seqlens=(333, 1000), seed=16)
+    inp = W.prefill_inputs(wl)
+    rope, shape, scale = oracle_cfg(wl)
+    dims = mla.dims_for(wl, mla.mla_softmax_scale(mla.rope_for(wl), 192))
+    cos, sin = mla.mla_init_rope_tables(mla.rope_for(wl), 1000)
+    d = {k: v.cuda() for k, v in inp.items()}
+    T = 1333
+    cache = torch.zeros((T, 576), dtype=torch.bfloat16, device="cuda")
+    rows = torch.arange(T, dtype=torch.int64, device="cuda")
+    mla.mla_cache_append(dims, d["latent"], d["w_norm"], d["positions"], cos, sin, cache, rows)
+    torch.cuda.synchronize()
+    # the appended rows themselves
+    ocos, osin = O.rope_tables(rope, 1000)
+    ref_rows = O.cache_append(f64(inp["latent"]), f64(inp["w_norm"]), inp["positions"].numpy(),
+                              ocos, osin, shape)
+    compare(f64(cache), ref_rows, "bf16", "cache rows")
+    last = torch.tensor([332, 1332])
+    qd = d["q"][last.cuda()].contiguous()
+    offs = torch.tensor([0, 333], dtype=torch.int64, device="cuda")
+    lens = torch.tensor([333, 1000], dtype=torch.int32, device="cuda")
+    pos = torch.tensor([332, 999], dtype=torch.int32, device="cuda")
+    got = mla.mla_decode(dims, qd, cache, offs, lens, pos, 1000, d["w_kvb"], cos, sin)
+    torch.cuda.synchronize()
+    rows_sel = {0: np.array([332]), 1: np.array([999])}
+    ref = oracle_prefill(wl, inp, rows=rows_sel)
+    compare(f64(got), ref[[332, 1332]], "bf16", "decode vs prefill row")
+
+
+def test_device_status_clean(gpu_lib):
+    mla.mla_check_device_status()
