@@ -13,6 +13,10 @@
 #include "rope.cuh"
 #include "simt_prefill.cuh"
 #include "simt_decode.cuh"
+#include "tc_gemm.cuh"
+#include "tc_attention.cuh"
+
+#include <cudaTypedefs.h>
 
 namespace {
 
@@ -32,6 +36,39 @@ int cuda_status(cudaError_t e, const char* what) {
 }
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// ---- TMA tensor maps (driver entry point fetched through the runtime) --------
+PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
+
+int get_encode() {
+  if (g_encode) return MLA_OK;
+  void* fn = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q);
+  if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !fn)
+    return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled is not available");
+  g_encode = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(fn);
+  return MLA_OK;
+}
+
+// 16-bit tensor map with the 128-byte swizzle; dims/strides innermost first
+// (strides in bytes, for dims 1..rank-1).
+int make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, const uint64_t* strides,
+             const uint32_t* box, CUtensorMapDataType dtype = CU_TENSOR_MAP_DATA_TYPE_BFLOAT16) {
+  int rc = get_encode();
+  if (rc) return rc;
+  cuuint64_t d[5], st[4];
+  cuuint32_t b[5], es[5];
+  for (int i = 0; i < rank; ++i) { d[i] = dims[i]; b[i] = box[i]; es[i] = 1; }
+  for (int i = 0; i < rank - 1; ++i) st[i] = strides[i];
+  CUresult r = g_encode(m, dtype, rank, const_cast<void*>(base), d, st, b, es,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(MLA_ERR_CUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return MLA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // ---- launch accounting and optional per-kernel events ---------------------
 std::atomic<uint64_t> g_launches{0};
@@ -103,19 +140,60 @@ int check_dims(const mla_dims* d) {
 
 size_t elem_size(const mla_dims* d) { return d->dtype == MLA_FP32 ? 4 : 2; }
 
-// Prefill workspace: k_nope [H, Ttot, N], values [H, Ttot, V], k_rot [Ttot, P].
+// Shapes the tensor-core prefill takes (bf16; otherwise the SIMT kernels run).
+bool prefill_tc_shape(const mla_dims* d) {
+  return d->dtype == MLA_BF16 && d->kv_lora_rank % 64 == 0 && d->kv_lora_rank <= 512 && d->qk_nope % 64 == 0 &&
+         d->qk_nope >= 64 && d->qk_rope == 64 && d->v_head % 64 == 0 && d->v_head <= 256 &&
+         d->qk_nope + d->qk_rope <= 256;
+}
+
+// SIMT prefill workspace: k_nope [H, Ttot, N], values [H, Ttot, V], k_rot [Ttot, P].
+// Tensor-core workspace: tile schedule, then the padded k_nope [H, Tpad, N],
+// transposed values [H, V, Tpad] and k_rot [Tpad, P], with Tpad = 128 * cap
+// and cap = ceil(Ttot / 128) + num_seqs bounding the number of 128-row tiles.
 struct PrefillWs {
+  int64_t cap, Tpad;
+  int gemm_tiles_per_cta, gemm_gy;
+  size_t seq_tile0, tile_seq, tile_q0, order, lo;
   size_t k_nope, vals, k_rot, total;
 };
-PrefillWs prefill_ws_layout(const mla_dims* d, int64_t T) {
-  PrefillWs w;
+PrefillWs prefill_ws_layout(const mla_dims* d, int64_t T, int nseq, bool tc) {
+  PrefillWs w = {};
   const size_t es = elem_size(d);
   size_t off = 0;
-  w.k_nope = off; off = align_up(off + es * (size_t)d->num_heads * T * d->qk_nope, 256);
-  w.vals = off;   off = align_up(off + es * (size_t)d->num_heads * T * d->v_head, 256);
-  w.k_rot = off;  off = align_up(off + es * (size_t)T * d->qk_rope, 256);
+  if (tc) {
+    w.cap = (T + 127) / 128 + nseq;
+    w.Tpad = w.cap * 128;
+    // GEMM grid: (cap, gy) CTAs, each with tiles_per_cta output tiles of 256 columns
+    const int NOUT = d->num_heads * (d->qk_nope + d->v_head);
+    const int n_total = (NOUT + mla::tc::kGemmBN - 1) / mla::tc::kGemmBN;
+    int splits = (int)(148 / (w.cap > 0 ? w.cap : 1));
+    if (splits < 1) splits = 1;
+    if (splits > n_total) splits = n_total;
+    w.gemm_tiles_per_cta = (n_total + splits - 1) / splits;
+    w.gemm_gy = (n_total + w.gemm_tiles_per_cta - 1) / w.gemm_tiles_per_cta;
+    w.seq_tile0 = off; off = align_up(off + 4 * (size_t)(nseq + 1), 256);
+    w.tile_seq = off;  off = align_up(off + 4 * (size_t)w.cap, 256);
+    w.tile_q0 = off;   off = align_up(off + 4 * (size_t)w.cap, 256);
+    w.order = off;     off = align_up(off + 4 * (size_t)w.cap, 256);
+    w.lo = off;        off = align_up(off + 2 * (size_t)w.cap * w.gemm_gy * 128 * d->kv_lora_rank, 256);
+  } else {
+    w.Tpad = T;
+  }
+  const size_t Tp = (size_t)w.Tpad;
+  w.k_nope = off; off = align_up(off + es * (size_t)d->num_heads * Tp * d->qk_nope, 256);
+  w.vals = off;   off = align_up(off + es * (size_t)d->num_heads * Tp * d->v_head, 256);
+  w.k_rot = off;  off = align_up(off + es * Tp * d->qk_rope, 256);
   w.total = off;
   return w;
+}
+size_t prefill_ws_bytes(const mla_dims* d, int64_t T, int nseq) {
+  size_t a = prefill_ws_layout(d, T, nseq, false).total;
+  if (prefill_tc_shape(d)) {
+    const size_t b = prefill_ws_layout(d, T, nseq, true).total;
+    if (b > a) a = b;
+  }
+  return a;
 }
 
 // Decode workspace: q_lat [B, H, R], q_rot [B, H, P], per-split partials.
@@ -146,7 +224,7 @@ int launch_prefill(const mla_dims* d, const void* latent, const void* q, const v
                    const float* sin_t, int max_pos, void* out, void* workspace, cudaStream_t st) {
   using namespace mla::simt;
   const int H = d->num_heads, R = d->kv_lora_rank, N = d->qk_nope, P = d->qk_rope, V = d->v_head;
-  const PrefillWs L = prefill_ws_layout(d, T_tot);
+  const PrefillWs L = prefill_ws_layout(d, T_tot, num_seqs, false);
   char* ws = static_cast<char*>(workspace);
   T* k_nope = reinterpret_cast<T*>(ws + L.k_nope);
   T* vals = reinterpret_cast<T*>(ws + L.vals);
@@ -165,16 +243,180 @@ int launch_prefill(const mla_dims* d, const void* latent, const void* q, const v
       k_rot);
   prof_end(st);
   const size_t smem = attention_smem_bytes(N + P, V);
-  cudaError_t e = cudaFuncSetAttribute(attention_kernel<T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(attention_kernel<T, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return cuda_status(e, "attention smem attribute");
   dim3 g2((unsigned)((max_seqlen + kAttBQ - 1) / kAttBQ), (unsigned)num_seqs, (unsigned)H);
   prof_begin(st, "simt_attention");
-  attention_kernel<T><<<g2, 256, smem, st>>>(static_cast<const T*>(q), k_nope, k_rot, vals, positions,
-                                             cu_seqlens, cos_t, sin_t, max_pos, max_seqlen, T_tot, H, N, P, V,
-                                             d->rope_interleaved, d->softmax_scale, static_cast<T*>(out));
+  attention_kernel<T, false><<<g2, 256, smem, st>>>(static_cast<const T*>(q), k_nope, k_rot, vals, positions,
+                                                    cu_seqlens, cos_t, sin_t, max_pos, max_seqlen, T_tot, H, N, P,
+                                                    V, d->rope_interleaved, d->softmax_scale, static_cast<T*>(out),
+                                                    nullptr, T_tot);
   prof_end(st);
   return cuda_status(cudaGetLastError(), "prefill launch");
+}
+
+template <int kN, int kV>
+int launch_attention_tc_t(unsigned grid, const CUtensorMap& mq, const CUtensorMap& mkn, const CUtensorMap& mkr,
+                          const CUtensorMap& mvt, const mla::tc::AttParams& ap, cudaStream_t st) {
+  // deepest K/V pipeline that fits next to Q and P in 227 KB of shared memory
+  constexpr size_t kBase = mla::tc::AttCfg<kN, kV, 1>::kSmem - mla::tc::AttCfg<kN, kV, 1>::kStageBytes;
+  constexpr size_t kStage = mla::tc::AttCfg<kN, kV, 1>::kStageBytes;
+  constexpr int kFit = (int)((232448 - 1024 - kBase) / kStage);
+  constexpr int kStages = kFit >= 3 ? 3 : 2;
+  static_assert(kFit >= 2, "attention tile does not fit in shared memory");
+  using C = mla::tc::AttCfg<kN, kV, kStages>;
+  auto kern = mla::tc::attention_kernel<kN, kV, kStages>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
+  if (e != cudaSuccess) return cuda_status(e, "attention smem attribute");
+  prof_begin(st, "tc_attention");
+  kern<<<grid, mla::tc::kAttThreads, C::kSmem, st>>>(mq, mkn, mkr, mvt, ap);
+  prof_end(st);
+  return cuda_status(cudaGetLastError(), "attention launch");
+}
+
+int launch_attention_tc(int N, int V, unsigned grid, const CUtensorMap& mq, const CUtensorMap& mkn,
+                        const CUtensorMap& mkr, const CUtensorMap& mvt, const mla::tc::AttParams& ap,
+                        cudaStream_t st) {
+#define MLA_ATT_CASE(n, v) \
+  if (N == n && V == v) return launch_attention_tc_t<n, v>(grid, mq, mkn, mkr, mvt, ap, st);
+  MLA_ATT_CASE(64, 64) MLA_ATT_CASE(64, 128) MLA_ATT_CASE(64, 192) MLA_ATT_CASE(64, 256)
+  MLA_ATT_CASE(128, 64) MLA_ATT_CASE(128, 128) MLA_ATT_CASE(128, 192) MLA_ATT_CASE(128, 256)
+  MLA_ATT_CASE(192, 64) MLA_ATT_CASE(192, 128) MLA_ATT_CASE(192, 192) MLA_ATT_CASE(192, 256)
+#undef MLA_ATT_CASE
+  return fail(MLA_ERR_UNSUPPORTED_SHAPE, "no tensor-core attention for qk_nope=%d v_head=%d", N, V);
+}
+
+// Tensor-core prefill: tile schedule -> fused RMSNorm + kv_b_proj (tcgen05)
+// -> causal attention over the padded layout.
+int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, const void* w_kvb,
+                      const void* w_norm, const int32_t* positions, const int32_t* cu_seqlens, int num_seqs,
+                      int max_seqlen, int64_t T_tot, const float* cos_t, const float* sin_t, int max_pos,
+                      void* out, void* workspace, cudaStream_t st) {
+  using bf16 = __nv_bfloat16;
+  const int H = d->num_heads, R = d->kv_lora_rank, N = d->qk_nope, P = d->qk_rope, V = d->v_head;
+  const PrefillWs L = prefill_ws_layout(d, T_tot, num_seqs, true);
+  char* ws = static_cast<char*>(workspace);
+  int32_t* seq_tile0 = reinterpret_cast<int32_t*>(ws + L.seq_tile0);
+  int32_t* tile_seq = reinterpret_cast<int32_t*>(ws + L.tile_seq);
+  int32_t* tile_q0 = reinterpret_cast<int32_t*>(ws + L.tile_q0);
+  int32_t* order = reinterpret_cast<int32_t*>(ws + L.order);
+  __half* k_nope = reinterpret_cast<__half*>(ws + L.k_nope);
+  __half* vt = reinterpret_cast<__half*>(ws + L.vals);
+  __half* k_rot = reinterpret_cast<__half*>(ws + L.k_rot);
+  const int cap = (int)L.cap;
+  const int NOUT = H * (N + V);
+
+  CUtensorMap map_lat, map_w;
+  {
+    const uint64_t dims[2] = {(uint64_t)(R + P), (uint64_t)T_tot};
+    const uint64_t strides[1] = {(uint64_t)(R + P) * 2};
+    const uint32_t box[2] = {64, 128};
+    int rc = make_map(&map_lat, latent, 2, dims, strides, box);
+    if (rc) return rc;
+  }
+  {
+    const uint64_t dims[2] = {(uint64_t)R, (uint64_t)NOUT};
+    const uint64_t strides[1] = {(uint64_t)R * 2};
+    const uint32_t box[2] = {64, 256};
+    int rc = make_map(&map_w, w_kvb, 2, dims, strides, box);
+    if (rc) return rc;
+  }
+
+  bf16* lo = reinterpret_cast<bf16*>(ws + L.lo);
+  const int gy = L.gemm_gy;
+  CUtensorMap map_lo;
+  {
+    const uint64_t dims[2] = {(uint64_t)R, (uint64_t)cap * gy * 128};
+    const uint64_t strides[1] = {(uint64_t)R * 2};
+    const uint32_t box[2] = {64, 128};
+    int rc = make_map(&map_lo, lo, 2, dims, strides, box);
+    if (rc) return rc;
+  }
+
+  prof_begin(st, "tc_schedule");
+  mla::tc::schedule_kernel<<<1, 1024, 0, st>>>(cu_seqlens, num_seqs, T_tot, max_seqlen, cap, seq_tile0, tile_seq,
+                                                tile_q0, order);
+  prof_end(st);
+
+  mla::tc::GemmParams gp;
+  gp.latent = static_cast<const bf16*>(latent);
+  gp.w_norm = static_cast<const bf16*>(w_norm);
+  gp.positions = positions;
+  gp.cu = cu_seqlens;
+  gp.tile_seq = tile_seq;
+  gp.tile_q0 = tile_q0;
+  gp.cos_t = cos_t;
+  gp.sin_t = sin_t;
+  gp.k_nope = k_nope;
+  gp.vt = vt;
+  gp.k_rot = k_rot;
+  gp.lo_scratch = lo;
+  gp.Ttot = T_tot;
+  gp.Tpad = (int)L.Tpad;
+  gp.R = R; gp.P = P; gp.H = H; gp.N = N; gp.V = V; gp.NOUT = NOUT;
+  gp.max_pos = max_pos;
+  gp.interleaved = d->rope_interleaved;
+  gp.eps = d->eps;
+  gp.tiles_per_cta = L.gemm_tiles_per_cta;
+  cudaError_t e = cudaFuncSetAttribute(mla::tc::norm_kvb_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)mla::tc::kGemmSmemBytes);
+  if (e != cudaSuccess) return cuda_status(e, "gemm smem attribute");
+  prof_begin(st, "tc_norm_kv_b_proj");
+  mla::tc::norm_kvb_gemm_kernel<<<dim3(cap, gy), mla::tc::kGemmThreads, mla::tc::kGemmSmemBytes, st>>>(
+      map_lat, map_w, map_lo, gp);
+  prof_end(st);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_status(e, "gemm launch");
+
+  // attention tensor maps over the padded workspace and q [Ttot, H, D]
+  const int D = N + P;
+  CUtensorMap map_q, map_kn, map_kr, map_vt;
+  {
+    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)H, (uint64_t)T_tot};
+    const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)H * D * 2};
+    const uint32_t box[3] = {64, 1, 128};
+    int rc = make_map(&map_q, q, 3, dims, strides, box);
+    if (rc) return rc;
+  }
+  {
+    const uint64_t dims[2] = {(uint64_t)N, (uint64_t)H * L.Tpad};
+    const uint64_t strides[1] = {(uint64_t)N * 2};
+    const uint32_t box[2] = {64, (uint32_t)mla::tc::kAttBKV};
+    int rc = make_map(&map_kn, k_nope, 2, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+    if (rc) return rc;
+  }
+  {
+    const uint64_t dims[2] = {(uint64_t)P, (uint64_t)L.Tpad};
+    const uint64_t strides[1] = {(uint64_t)P * 2};
+    const uint32_t box[2] = {64, (uint32_t)mla::tc::kAttBKV};
+    int rc = make_map(&map_kr, k_rot, 2, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+    if (rc) return rc;
+  }
+  {
+    const uint64_t dims[2] = {(uint64_t)L.Tpad, (uint64_t)H * V};
+    const uint64_t strides[1] = {(uint64_t)L.Tpad * 2};
+    const uint32_t box[2] = {64, (uint32_t)V};
+    int rc = make_map(&map_vt, vt, 2, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+    if (rc) return rc;
+  }
+  mla::tc::AttParams ap;
+  ap.cu = cu_seqlens;
+  ap.positions = positions;
+  ap.seq_tile0 = seq_tile0;
+  ap.tile_seq = tile_seq;
+  ap.tile_q0 = tile_q0;
+  ap.order = order;
+  ap.cos_t = cos_t;
+  ap.sin_t = sin_t;
+  ap.out = static_cast<bf16*>(out);
+  ap.H = H;
+  ap.Tpad = (int)L.Tpad;
+  ap.max_pos = max_pos;
+  ap.interleaved = d->rope_interleaved;
+  ap.scale_log2 = d->softmax_scale * 1.4426950408889634f;
+  const unsigned grid = (unsigned)(cap * H);
+  return launch_attention_tc(N, V, grid, map_q, map_kn, map_kr, map_vt, ap, st);
 }
 
 template <typename T>
@@ -295,7 +537,7 @@ int mla_prefill_workspace_size(const mla_dims* dims, int64_t total_tokens, int32
   if (rc) return rc;
   if (total_tokens < 0 || num_seqs < 0) return fail(MLA_ERR_INVALID_ARG, "negative size");
   if (!bytes) return fail(MLA_ERR_INVALID_ARG, "bytes is NULL");
-  *bytes = prefill_ws_layout(dims, total_tokens).total;
+  *bytes = prefill_ws_bytes(dims, total_tokens, num_seqs);
   return MLA_OK;
 }
 
@@ -315,9 +557,13 @@ int mla_prefill(const mla_dims* dims, const void* latent, const void* q, const v
   if (total_tokens == 0 || num_seqs == 0 || max_seqlen == 0) return MLA_OK;   // nothing to attend
   if (!latent || !q || !w_kvb || !w_norm || !positions || !cos_table || !sin_table || !out)
     return fail(MLA_ERR_INVALID_ARG, "a tensor pointer is NULL");
-  const size_t need = prefill_ws_layout(dims, total_tokens).total;
+  const size_t need = prefill_ws_bytes(dims, total_tokens, num_seqs);
   if (!workspace || workspace_bytes < need)
     return fail(MLA_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes, got %zu", need, workspace_bytes);
+  if (prefill_tc_shape(dims) && aligned16(latent) && aligned16(w_kvb) && aligned16(q) && aligned16(workspace) &&
+      aligned16(w_norm))
+    return launch_prefill_tc(dims, latent, q, w_kvb, w_norm, positions, cu_seqlens, num_seqs, max_seqlen,
+                             total_tokens, cos_table, sin_table, max_pos, out, workspace, stream);
   if (dims->dtype == MLA_FP32)
     return launch_prefill<float>(dims, latent, q, w_kvb, w_norm, positions, cu_seqlens, num_seqs,
                                  max_seqlen, total_tokens, cos_table, sin_table, max_pos, out, workspace,
@@ -408,6 +654,8 @@ int mla_check_device_status(cudaStream_t stream) {
     e = cudaMemcpyToSymbol(mla::g_device_error, &zero, sizeof(zero));
     if (e != cudaSuccess) return cuda_status(e, "clear device error word");
     if (v & mla::kDevErrTimeout) return fail(MLA_ERR_DEVICE_TIMEOUT, "a device-side wait timed out (0x%x)", v);
+    if (v & mla::kDevErrRange)
+      return fail(MLA_ERR_INVALID_ARG, "a q, key or value exceeded the fp16 range of the internal buffers (0x%x)", v);
     return fail(MLA_ERR_INVALID_ARG, "device-side input check failed (0x%x)", v);
   }
   return MLA_OK;

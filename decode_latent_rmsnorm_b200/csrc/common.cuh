@@ -4,6 +4,7 @@
 
 #include <cuda_runtime.h>
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <stdint.h>
 
 namespace mla {
@@ -13,6 +14,7 @@ namespace mla {
 enum : uint32_t {
   kDevErrTimeout = 1u,      // an mbarrier / flag wait exceeded its limit
   kDevErrBadInput = 2u,     // a device-resident argument was out of range
+  kDevErrRange = 4u,        // a value exceeded the fp16 range of an internal buffer
 };
 
 __device__ uint32_t g_device_error;

@@ -119,13 +119,18 @@ constexpr int kAttBQ = 32, kAttBKV = 32, kAttMaxVPerThread = 32;
 // Causal attention for one (query block, sequence, head). 256 threads: each
 // query row is owned by 8 consecutive lanes; scores are kept online (running
 // max and sum), so the [L, L] matrix is never formed.
-template <typename T>
+// kPadded = false: k_nope [H, Ttot, N], vals [H, Ttot, V], k_rot [Ttot, P];
+// kPadded = true: the tensor-core GEMM's padded layout, k_nope [H, Tpad, N],
+// vals transposed [H, V, Tpad], k_rot [Tpad, P], sequence s starting at
+// padded row 128 * seq_tile0[s].
+template <typename T, bool kPadded>
 __global__ void __launch_bounds__(256)
 attention_kernel(const T* __restrict__ q, const T* __restrict__ k_nope, const T* __restrict__ k_rot,
                  const T* __restrict__ vals, const int32_t* __restrict__ positions,
                  const int32_t* __restrict__ cu_seqlens, const float* __restrict__ cos_t,
                  const float* __restrict__ sin_t, int max_pos, int max_seqlen, int64_t Ttot, int H,
-                 int N, int P, int V, int interleaved, float scale, T* __restrict__ out) {
+                 int N, int P, int V, int interleaved, float scale, T* __restrict__ out,
+                 const int32_t* __restrict__ seq_tile0, int64_t Tpad) {
   extern __shared__ float smem[];
   const int D = N + P;
   float* Qs = smem;                       // [BQ][D]
@@ -143,6 +148,8 @@ attention_kernel(const T* __restrict__ q, const T* __restrict__ k_nope, const T*
   const int q0 = blockIdx.x * kAttBQ;
   if (q0 >= L) return;
   const int half = P / 2;
+  const int64_t kv0 = kPadded ? (int64_t)seq_tile0[s] * 128 : seq0;   // row of key 0 in the K/V buffers
+  const int64_t kv_rows = kPadded ? Tpad : Ttot;
 
   for (int e = tid; e < kAttBQ * D; e += 256) {
     const int r = e / D, d = e % D;
@@ -182,15 +189,18 @@ attention_kernel(const T* __restrict__ q, const T* __restrict__ k_nope, const T*
       const int r = e / D, d = e % D;
       float v = 0.f;
       if (k0 + r < L) {
-        const int64_t t = seq0 + k0 + r;
-        v = d < N ? to_f32(k_nope[((int64_t)h * Ttot + t) * N + d]) : to_f32(k_rot[t * P + (d - N)]);
+        const int64_t t = kv0 + k0 + r;
+        v = d < N ? to_f32(k_nope[((int64_t)h * kv_rows + t) * N + d]) : to_f32(k_rot[t * P + (d - N)]);
       }
       Ks[e] = v;
     }
     for (int e = tid; e < kAttBKV * V; e += 256) {
       const int r = e / V, d = e % V;
-      const int64_t t = seq0 + k0 + r;
-      Vs[e] = (k0 + r < L) ? to_f32(vals[((int64_t)h * Ttot + t) * V + d]) : 0.f;
+      const int64_t t = kv0 + k0 + r;
+      float v = 0.f;
+      if (k0 + r < L)
+        v = kPadded ? to_f32(vals[((int64_t)h * V + d) * kv_rows + t]) : to_f32(vals[((int64_t)h * kv_rows + t) * V + d]);
+      Vs[e] = v;
     }
     __syncthreads();
     float sc[kAttBKV / 8];

@@ -1,0 +1,356 @@
+// Tensor-core (tcgen05) causal attention over the padded k_nope / transposed
+// value / rotated k_rot workspace written by norm_kvb_gemm_kernel.
+//
+// Sources: Kimi-K2 "Query content heads" page, "Join query parts" and the
+// Kimi-K2 "RoPE coefficients" page, "Key heads" (mla-prefill excerpt): the
+// rotary parts are rotated; each head's query and key join their non-rotary
+// and rotary parts, the key's rotary part being the one shared rotary key;
+// scores are scaled, causally masked, normalized with a softmax in fp32 and
+// used to mix the values.
+//
+// Operands of both tensor-core products are fp16 (q is converted in shared
+// memory after its TMA load; k_nope, k_rot and the values come in fp16 from
+// the GEMM; P is packed to fp16), accumulators fp32, output bf16.
+//
+// One CTA = one (128-query tile, head). Warp 0 issues TMA loads, warp 1 issues
+// the MMAs, warps 2-5 own one query row per thread (TMEM lane = row):
+//   S_j   = Q K_j^T           (tcgen05, fp32 in TMEM, double buffered)
+//   P_j   = exp2(S_j * scale * log2 e - m)   (online softmax, registers)
+//   O    += P_j V_j           (tcgen05, fp32 accumulator in TMEM)
+// The shared rotary key tile is loaded once per key tile and serves every
+// query row of the head; q's rotary part is rotated in shared memory right
+// after its TMA load. O is rescaled (in TMEM, by the softmax warps) whenever
+// a row's running max grows.
+#pragma once
+#include "tc_gemm.cuh"
+
+namespace mla {
+namespace tc {
+
+constexpr int kAttBKV = 64;                       // keys per tile (MMA N of S, K of PV)
+constexpr int kAttThreads = 192;
+
+template <int kN, int kV, int kStages>
+struct AttCfg {
+  static constexpr int D = kN + 64;
+  static constexpr int kQAtoms = D / 64;
+  static constexpr int kQBytes = kQAtoms * kTile * 128;
+  static constexpr int kKAtomBytes = kAttBKV * 128;
+  static constexpr int kKBytes = kQAtoms * kKAtomBytes;
+  static constexpr int kVBytes = kV * 128;         // [kV rows x 64 keys]
+  static constexpr int kStageBytes = kKBytes + kVBytes;
+  static constexpr int kPBytes = kTile * 128;      // [128 rows x 64 keys]
+  static constexpr size_t kSmem = (size_t)kQBytes + (size_t)kStages * kStageBytes + kPBytes + 1024;
+  static constexpr int kSCol = 0;                  // S buffers: columns [0, 128)
+  static constexpr int kOCol = 2 * kAttBKV;        // O: columns [128, 128 + kV)
+  static constexpr uint32_t kTmemCols = (kOCol + kV) <= 256 ? 256 : 512;
+};
+
+struct AttParams {
+  const int32_t* cu;
+  const int32_t* positions;
+  const int32_t* seq_tile0;
+  const int32_t* tile_seq;
+  const int32_t* tile_q0;
+  const int32_t* order;
+  const float* cos_t;
+  const float* sin_t;
+  __nv_bfloat16* out;
+  int H, Tpad, max_pos, interleaved;
+  float scale_log2;             // softmax scale * log2(e)
+};
+
+template <int kStages>
+struct AttBarriers {
+  uint64_t q_full, q_ready;
+  uint64_t kv_full[kStages], kv_empty[kStages];
+  uint64_t s_full[2], s_free[2];
+  uint64_t p_full, pv_done, mma_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+template <int kN, int kV, int kStages>
+__global__ void __launch_bounds__(kAttThreads, 1)
+attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_kn,
+                 const __grid_constant__ CUtensorMap map_kr, const __grid_constant__ CUtensorMap map_vt,
+                 AttParams p) {
+  using C = AttCfg<kN, kV, kStages>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ AttBarriers<kStages> bars;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int rank = blockIdx.x / p.H, h = blockIdx.x % p.H;
+  const int tile = p.order[rank];
+  if (tile < 0) return;   // uniform over the CTA
+  const int seq = p.tile_seq[tile];
+  const int q0 = p.tile_q0[tile];
+  const int64_t seq0 = p.cu[seq];
+  const int L = (int)(p.cu[seq + 1] - seq0);
+  const int kv_pad0 = p.seq_tile0[seq] * kTile;           // padded row of key 0
+  const int kv_len = min(L, q0 + kTile);
+  const int n_kv = (kv_len + kAttBKV - 1) / kAttBKV;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sKV = smem + C::kQBytes;
+  uint8_t* sP = sKV + kStages * C::kStageBytes;
+  volatile int* abort_flag = &bars.abort_flag;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars.q_full, 1);
+    mbar_init(&bars.q_ready, 128);
+    for (int s = 0; s < kStages; ++s) { mbar_init(&bars.kv_full[s], 1); mbar_init(&bars.kv_empty[s], 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&bars.s_full[b], 1); mbar_init(&bars.s_free[b], 128); }
+    mbar_init(&bars.p_full, 128);
+    mbar_init(&bars.pv_done, 1);
+    mbar_init(&bars.mma_done, 1);
+    bars.abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 1) tmem_alloc(&bars.tmem_base, C::kTmemCols);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars.tmem_base;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0) {
+      tma_prefetch_desc(&map_q);
+      tma_prefetch_desc(&map_kn);
+      tma_prefetch_desc(&map_kr);
+      tma_prefetch_desc(&map_vt);
+      mbar_arrive_expect_tx(&bars.q_full, C::kQBytes);
+      for (int a = 0; a < C::kQAtoms; ++a)
+        tma_load_3d(sQ + a * kTile * 128, &map_q, &bars.q_full, a * 64, h, (int)(seq0 + q0));
+      bool ok = true;
+      int j = 0;
+      for (; j < n_kv; ++j) {
+        const int s = j % kStages;
+        if (!mbar_wait(&bars.kv_empty[s], ((uint32_t)(j / kStages) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+        uint8_t* sK = sKV + s * C::kStageBytes;
+        uint8_t* sV = sK + C::kKBytes;
+        const int kv_row = kv_pad0 + j * kAttBKV;
+        mbar_arrive_expect_tx(&bars.kv_full[s], C::kStageBytes);
+        for (int a = 0; a < kN / 64; ++a)
+          tma_load_2d(sK + a * C::kKAtomBytes, &map_kn, &bars.kv_full[s], a * 64, h * p.Tpad + kv_row);
+        tma_load_2d(sK + (kN / 64) * C::kKAtomBytes, &map_kr, &bars.kv_full[s], 0, kv_row);
+        tma_load_2d(sV, &map_vt, &bars.kv_full[s], kv_row, h * kV);
+      }
+      if (!ok) {   // let every copy already issued land before the CTA exits
+        mbar_wait_drain(&bars.q_full, 0);
+        for (int i = (j > kStages ? j - kStages : 0); i < j; ++i)
+          mbar_wait_drain(&bars.kv_full[i % kStages], (uint32_t)(i / kStages) & 1u);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0) {
+      const uint32_t idesc_s = idesc_f16_f32(kTile, kAttBKV);
+      const uint32_t idesc_o = idesc_f16_f32(kTile, kV);
+      const uint32_t o_tmem = tmem + C::kOCol;
+      bool ok = mbar_wait(&bars.q_ready, 0, abort_flag);
+      tc_fence_after();
+      auto issue_pv = [&](int jj) -> bool {
+        if (!mbar_wait(&bars.p_full, (uint32_t)jj & 1u, abort_flag)) return false;
+        tc_fence_after();
+        const int s = jj % kStages;
+        const uint64_t pd = desc_kmajor_sw128(smem_u32(sP));
+        const uint64_t vd = desc_kmajor_sw128(smem_u32(sKV + s * C::kStageBytes + C::kKBytes));
+#pragma unroll
+        for (int k = 0; k < kAttBKV / 16; ++k)
+          mma_bf16_ss(o_tmem, desc_advance(pd, k * 32), desc_advance(vd, k * 32), idesc_o, (jj | k) != 0);
+        mma_commit(&bars.kv_empty[s]);
+        mma_commit(&bars.pv_done);
+        return true;
+      };
+      for (int j = 0; j < n_kv && ok; ++j) {
+        const int s = j % kStages, b = j & 1;
+        if (!mbar_wait(&bars.kv_full[s], (uint32_t)(j / kStages) & 1u, abort_flag)) { ok = false; break; }
+        if (!mbar_wait(&bars.s_free[b], ((uint32_t)(j >> 1) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint8_t* sK = sKV + s * C::kStageBytes;
+        const uint32_t s_tmem = tmem + C::kSCol + b * kAttBKV;
+#pragma unroll
+        for (int a = 0; a < C::kQAtoms; ++a) {
+          const uint64_t qd = desc_kmajor_sw128(smem_u32(sQ + a * kTile * 128));
+          const uint64_t kd = desc_kmajor_sw128(smem_u32(sK + a * C::kKAtomBytes));
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_bf16_ss(s_tmem, desc_advance(qd, k * 32), desc_advance(kd, k * 32), idesc_s, (a | k) != 0);
+        }
+        mma_commit(&bars.s_full[b]);
+        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+      }
+      if (ok && n_kv > 0) issue_pv(n_kv - 1);
+      mma_commit(&bars.mma_done);     // every MMA done before TMEM is freed
+      mbar_wait_drain(&bars.mma_done, 0);
+    }
+  } else {
+    // ---------------- softmax / correction / epilogue (warps 2-5) ----------------
+    const int grp = warp & 3;
+    const int row = grp * 32 + lane;
+    const uint32_t lane_base = (uint32_t)(grp * 32) << 16;
+    const bool valid = (q0 + row) < L;
+    const int qi = min(q0 + row, L - 1);          // in-sequence query index used by the mask
+    const int64_t t = seq0 + q0 + row;
+    bool ok = mbar_wait_warp(&bars.q_full, 0, abort_flag);
+    if (ok) {
+      // this row of q: bf16 -> fp16 in place; the rotary part (last atom) is
+      // rotated at the token's position on the way
+      float qmax = 0.f;
+#pragma unroll 1
+      for (int a = 0; a < C::kQAtoms - 1; ++a) {
+        uint8_t* qa = sQ + a * kTile * 128;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint4* ptr = reinterpret_cast<uint4*>(qa + sw128_offset(row, c));
+          const uint4 v = *ptr;
+          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+          uint32_t o4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = unpack_bf16x2(w4[e]);
+            qmax = fmaxf(qmax, fmaxf(fabsf(f.x), fabsf(f.y)));
+            o4[e] = pack_f16x2(f.x, f.y);
+          }
+          *ptr = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+        }
+      }
+      uint8_t* qr = sQ + (C::kQAtoms - 1) * kTile * 128;
+      float x[64];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint4 v = *reinterpret_cast<const uint4*>(qr + sw128_offset(row, c));
+        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const float2 f = unpack_bf16x2(w4[e]);
+          x[c * 8 + 2 * e] = f.x;
+          x[c * 8 + 2 * e + 1] = f.y;
+        }
+      }
+      const int64_t pos = valid ? checked_pos(p.positions[t], p.max_pos) : 0;
+      const float* ct = p.cos_t + pos * 32;
+      const float* st = p.sin_t + pos * 32;
+      float y[64];
+      if (p.interleaved) {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) rope_turn(x[2 * i], x[2 * i + 1], ct[i], st[i], y[2 * i], y[2 * i + 1]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) rope_turn(x[i], x[i + 32], ct[i], st[i], y[i], y[i + 32]);
+      }
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        uint4 v;
+        v.x = pack_f16x2(y[c * 8 + 0], y[c * 8 + 1]);
+        v.y = pack_f16x2(y[c * 8 + 2], y[c * 8 + 3]);
+        v.z = pack_f16x2(y[c * 8 + 4], y[c * 8 + 5]);
+        v.w = pack_f16x2(y[c * 8 + 6], y[c * 8 + 7]);
+        *reinterpret_cast<uint4*>(qr + sw128_offset(row, c)) = v;
+#pragma unroll
+        for (int e = 0; e < 8; ++e) qmax = fmaxf(qmax, fabsf(y[c * 8 + e]));
+      }
+      if (valid && !(qmax <= kF16Max)) raise_device_error(kDevErrRange);
+    }
+    fence_proxy_async_smem();
+    mbar_arrive(&bars.q_ready);
+
+    float m = -INFINITY;      // running max (log2 units) used as the exponent's reference
+    float l = 0.f;            // running sum of P at that reference
+    for (int j = 0; j < n_kv && ok; ++j) {
+      const int b = j & 1;
+      if (!mbar_wait_warp(&bars.s_full[b], (uint32_t)(j >> 1) & 1u, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      float sc[kAttBKV];
+#pragma unroll
+      for (int c = 0; c < kAttBKV / 16; ++c) {
+        uint32_t v[16];
+        tmem_ld16(tmem + lane_base + (uint32_t)(C::kSCol + b * kAttBKV + c * 16), v);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) sc[c * 16 + e] = __uint_as_float(v[e]);
+      }
+      tc_fence_before();
+      mbar_arrive(&bars.s_free[b]);
+      const int kv0 = j * kAttBKV;
+      float mx = -INFINITY;
+#pragma unroll
+      for (int e = 0; e < kAttBKV; ++e) {
+        const float v = (kv0 + e <= qi) ? sc[e] * p.scale_log2 : -INFINITY;   // causal mask
+        sc[e] = v;
+        mx = fmaxf(mx, v);
+      }
+      // the reference is the exact running max, so the dominant key of a row
+      // gets the weight 1.0 exactly (a lazier reference would round it)
+      float alpha = 1.f;
+      bool rescale = false;
+      if (mx > m) {
+        if (m != -INFINITY) { alpha = ex2_approx(m - mx); rescale = true; }
+        m = mx;
+      }
+      float rs = 0.f;
+      uint32_t pk[kAttBKV / 2];
+#pragma unroll
+      for (int e = 0; e < kAttBKV; e += 2) {
+        const float p0 = ex2_approx(sc[e] - m), p1 = ex2_approx(sc[e + 1] - m);
+        pk[e / 2] = pack_f16x2(p0, p1);
+        // the row sum uses the same rounded weights the P V product sees, so
+        // the output is an exact convex combination of those weights
+        const float2 pr = unpack_f16x2(pk[e / 2]);
+        rs += pr.x + pr.y;
+      }
+      l = l * alpha + rs;
+      if (j >= 1) {
+        // P buffer free and O stable once the previous P V product is done
+        if (!mbar_wait_warp(&bars.pv_done, (uint32_t)(j - 1) & 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        if (__any_sync(0xffffffffu, rescale)) {   // warp-collective TMEM access: whole warp, alpha = 1 elsewhere
+          for (int c = 0; c < kV / 16; ++c) {
+            uint32_t v[16];
+            const uint32_t ta = tmem + lane_base + (uint32_t)(C::kOCol + c * 16);
+            tmem_ld16(ta, v);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+            tmem_st16(ta, v);
+          }
+          tmem_st_wait();
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < 8; ++c)
+        *reinterpret_cast<uint4*>(sP + sw128_offset(row, c)) =
+            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bars.p_full);
+    }
+    if (ok && n_kv > 0) ok = mbar_wait_warp(&bars.pv_done, (uint32_t)(n_kv - 1) & 1u, abort_flag);
+    if (ok) {
+      tc_fence_after();
+      const float inv = 1.f / l;
+      __nv_bfloat16* dst = p.out + (t * p.H + h) * kV;
+      for (int c = 0; c < kV / 16; ++c) {
+        uint32_t v[16];
+        tmem_ld16(tmem + lane_base + (uint32_t)(C::kOCol + c * 16), v);
+        if (valid) {
+          uint32_t o[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            o[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * inv, __uint_as_float(v[2 * e + 1]) * inv);
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 16);
+          d4[0] = make_uint4(o[0], o[1], o[2], o[3]);
+          d4[1] = make_uint4(o[4], o[5], o[6], o[7]);
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+}  // namespace tc
+}  // namespace mla

@@ -1,0 +1,377 @@
+// Tensor-core (tcgen05) prefill front half: tile schedule of the packed
+// sequences, and the fused latent RMSNorm + kv_b_proj up-projection.
+//
+// Sources: "Eager latent expansion" equation page (normalize the compressed
+// latent, apply the learned up-projection, reshape into heads, split into
+// non-rotary key and value); Kimi-K2 "RoPE coefficients" page, "Key heads"
+// (mla-kv: split the joint latent into the 512-wide latent and k_pe, view
+// k_pe as one head shared by all heads).
+//
+// Precision: the normalized latent c_hat = w * x / rms(x) is formed in fp32
+// and handed to the tensor cores exactly, as c_hat = hi + lo with hi =
+// bf16(c_hat) and lo = bf16(c_hat - hi) (|lo| <= 2^-9 |c_hat|; the pair keeps
+// about 17 significant bits). Both halves multiply the same weight tile and
+// accumulate in fp32, so k_nope and the values carry one rounding only: their
+// own storage, in fp16 (11 significant bits; attention runs its tensor-core
+// products on fp16 operands). A value beyond the fp16 range sets the device
+// error word.
+//
+// Workspace layout ("padded token space"): every sequence starts on a
+// 128-row boundary, so a 128-token tile never straddles two sequences and
+// every TMA coordinate along tokens is a multiple of 64 elements. Rows past a
+// sequence's end are written as zeros.
+//   k_nope [H, Tpad, N]  fp16   (row tp, N contiguous)
+//   vt     [H, V, Tpad]  fp16   (values transposed: tokens contiguous)
+//   k_rot  [Tpad, P]     fp16   (the shared rotary key, rotated)
+#pragma once
+#include "tc_ptx.cuh"
+
+namespace mla {
+namespace tc {
+
+constexpr int kTile = 128;            // token rows per tile (M of the MMAs)
+
+// ---- tile schedule --------------------------------------------------------
+// tile_seq[i] / tile_q0[i]: sequence and first in-sequence row of tile i in
+// natural order (padded rows tp = 128 i ...); order[j]: tiles sorted by
+// decreasing causal work (largest q0 first), for the attention grid.
+// Entries past the real tile count are -1. Bad cu_seqlens set the device error
+// word and leave every entry at -1.
+__global__ void __launch_bounds__(1024)
+schedule_kernel(const int32_t* __restrict__ cu, int nseq, int64_t Ttot, int max_seqlen, int cap,
+                int32_t* __restrict__ seq_tile0, int32_t* __restrict__ tile_seq, int32_t* __restrict__ tile_q0,
+                int32_t* __restrict__ order) {
+  constexpr int kBuckets = 2048;
+  __shared__ int s_bad;
+  __shared__ int s_carry;
+  __shared__ int s_scan[1024];
+  __shared__ int s_cnt[kBuckets];
+  __shared__ int s_off[kBuckets];
+  const int tid = threadIdx.x;
+  if (tid == 0) { s_bad = 0; s_carry = 0; }
+  for (int i = tid; i < cap; i += blockDim.x) { tile_seq[i] = -1; tile_q0[i] = -1; order[i] = -1; }
+  for (int k = tid; k < kBuckets; k += blockDim.x) { s_cnt[k] = 0; s_off[k] = 0; }
+  __syncthreads();
+  // 1) per-sequence tile counts -> exclusive scan into seq_tile0
+  for (int base = 0; base <= nseq; base += blockDim.x) {
+    const int s = base + tid;
+    int nt = 0;
+    if (s < nseq) {
+      const int64_t a = cu[s], b = cu[s + 1];
+      if (a < 0 || b < a || b > Ttot || b - a > max_seqlen) s_bad = 1;
+      else nt = (int)((b - a + kTile - 1) / kTile);
+    }
+    s_scan[tid] = nt;
+    __syncthreads();
+    for (int off = 1; off < (int)blockDim.x; off <<= 1) {
+      const int v = tid >= off ? s_scan[tid - off] : 0;
+      __syncthreads();
+      s_scan[tid] += v;
+      __syncthreads();
+    }
+    if (s <= nseq) seq_tile0[s] = s_carry + s_scan[tid] - nt;
+    __syncthreads();
+    if (tid == (int)blockDim.x - 1) s_carry += s_scan[tid];
+    __syncthreads();
+  }
+  if (s_bad) {
+    if (tid == 0) raise_device_error(kDevErrBadInput);
+    return;
+  }
+  if (s_carry > cap) {   // cannot happen for valid input; guards the arrays
+    if (tid == 0) raise_device_error(kDevErrBadInput);
+    return;
+  }
+  __syncthreads();
+  // 2) tiles in natural order; 3) bucket counts of causal work (tile index)
+  for (int s = tid; s < nseq; s += blockDim.x) {
+    const int t0 = seq_tile0[s], nt = seq_tile0[s + 1] - t0;
+    for (int k = 0; k < nt; ++k) {
+      tile_seq[t0 + k] = s;
+      tile_q0[t0 + k] = k * kTile;
+      atomicAdd(&s_cnt[min(k, kBuckets - 1)], 1);
+    }
+  }
+  __syncthreads();
+  if (tid == 0) {   // descending exclusive offsets (kBuckets steps, once per call)
+    int run = 0;
+    for (int k = kBuckets - 1; k >= 0; --k) { s_off[k] = run; run += s_cnt[k]; }
+  }
+  __syncthreads();
+  for (int s = tid; s < nseq; s += blockDim.x) {
+    const int t0 = seq_tile0[s], nt = seq_tile0[s + 1] - t0;
+    for (int k = 0; k < nt; ++k) {
+      const int pos = atomicAdd(&s_off[min(k, kBuckets - 1)], 1);
+      order[pos] = t0 + k;
+    }
+  }
+}
+
+// ---- fused RMSNorm + kv_b_proj GEMM ------------------------------------------
+constexpr int kGemmBN = 256;                    // output columns per tile (MMA N)
+constexpr int kGemmStages = 2;                  // (weight tile, lo tile) pipeline depth
+constexpr int kAtomBytes = kTile * 128;         // 128 rows x 64 bf16
+constexpr int kBStageBytes = kGemmBN * 128;     // 256 rows x 64 bf16
+constexpr int kStageBytes = kBStageBytes + kAtomBytes;   // weight chunk + lo chunk
+constexpr int kGemmThreads = 192;               // warp 0 TMA, warp 1 MMA, warps 2-5 norm + epilogue
+constexpr int kGemmMaxAtoms = 8;                // R <= 512
+constexpr size_t kGemmSmemBytes = (size_t)kGemmMaxAtoms * kAtomBytes + (size_t)kGemmStages * kStageBytes + 1024;
+
+struct GemmParams {
+  const __nv_bfloat16* latent;   // [Ttot, R + P]
+  const __nv_bfloat16* w_norm;   // [R]
+  const int32_t* positions;
+  const int32_t* cu;
+  const int32_t* tile_seq;
+  const int32_t* tile_q0;
+  const float* cos_t;
+  const float* sin_t;
+  __half* k_nope;
+  __half* vt;
+  __half* k_rot;
+  __nv_bfloat16* lo_scratch;     // [CTAs * 128, R]: each CTA's lo half of c_hat
+  int64_t Ttot;
+  int Tpad, R, P, H, N, V, NOUT;
+  int tiles_per_cta;             // n tiles (256 columns) per CTA
+  int max_pos, interleaved;
+  float eps;
+};
+
+struct GemmBarriers {
+  uint64_t a_full, a_ready;
+  uint64_t b_full[kGemmStages], b_empty[kGemmStages];
+  uint64_t acc_full[2], acc_empty[2];
+  uint64_t mma_done;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+// grid: (tile capacity, ceil(NOUT / (256 * tiles_per_cta))). The TMA-fed
+// prologue normalizes the CTA's 128 x R latent tile: hi stays resident in
+// shared memory, lo goes to the CTA's private scratch rows (L2-resident) and
+// streams back with the weight tiles through a 2-stage TMA pipeline. The fp32
+// accumulator is double buffered in TMEM (2 x 256 columns) so the epilogue of
+// one output tile overlaps the MMAs of the next.
+__global__ void __launch_bounds__(kGemmThreads, 1)
+norm_kvb_gemm_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant__ CUtensorMap map_w,
+                     const __grid_constant__ CUtensorMap map_lo, GemmParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ GemmBarriers bars;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x;
+  const int seq = p.tile_seq[tile];
+  if (seq < 0) return;   // past the real tiles (uniform over the CTA)
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;                                        // R/64 atoms of [128 x 64] (hi)
+  uint8_t* sB = smem + kGemmMaxAtoms * kAtomBytes;           // stages: [256 x 64] weight + [128 x 64] lo
+  const int cta_id = blockIdx.y * gridDim.x + blockIdx.x;
+  __nv_bfloat16* lo_rows = p.lo_scratch + (int64_t)cta_id * kTile * p.R;
+  const int q0 = p.tile_q0[tile];
+  const int64_t seq0 = p.cu[seq];
+  const int L = (int)(p.cu[seq + 1] - seq0);
+  const int tp0 = tile * kTile;                              // padded row of the tile
+  const int natoms = p.R / 64;
+  const int n_begin = blockIdx.y * p.tiles_per_cta;
+  const int n_tiles_total = (p.NOUT + kGemmBN - 1) / kGemmBN;
+  const int n_end = min(n_tiles_total, n_begin + p.tiles_per_cta);
+  const int my_tiles = n_end - n_begin;
+  volatile int* abort_flag = &bars.abort_flag;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars.a_full, 1);
+    mbar_init(&bars.a_ready, 128);
+    for (int s = 0; s < kGemmStages; ++s) { mbar_init(&bars.b_full[s], 1); mbar_init(&bars.b_empty[s], 1); }
+    for (int s = 0; s < 2; ++s) { mbar_init(&bars.acc_full[s], 1); mbar_init(&bars.acc_empty[s], 128); }
+    mbar_init(&bars.mma_done, 1);
+    bars.abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 1) tmem_alloc(&bars.tmem_base, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars.tmem_base;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0 && my_tiles > 0) {
+      tma_prefetch_desc(&map_lat);
+      tma_prefetch_desc(&map_w);
+      tma_prefetch_desc(&map_lo);
+      mbar_arrive_expect_tx(&bars.a_full, natoms * kAtomBytes);
+      for (int a = 0; a < natoms; ++a)
+        tma_load_2d(sA + a * kAtomBytes, &map_lat, &bars.a_full, a * 64, (int)(seq0 + q0));
+      int it = 0;
+      // the lo rows exist once the prologue has written them
+      bool ok = mbar_wait(&bars.a_ready, 0, abort_flag);
+      for (int nt = n_begin; nt < n_end && ok; ++nt) {
+        for (int kc = 0; kc < natoms; ++kc, ++it) {
+          const int s = it % kGemmStages;
+          const uint32_t ph = (uint32_t)(it / kGemmStages) & 1u;
+          if (!mbar_wait(&bars.b_empty[s], ph ^ 1u, abort_flag)) { ok = false; break; }
+          uint8_t* st = sB + s * kStageBytes;
+          mbar_arrive_expect_tx(&bars.b_full[s], kStageBytes);
+          tma_load_2d(st, &map_w, &bars.b_full[s], kc * 64, nt * kGemmBN);
+          tma_load_2d(st + kBStageBytes, &map_lo, &bars.b_full[s], kc * 64, cta_id * kTile);
+        }
+      }
+      if (!ok) {   // drain the loads that may still be in flight before the CTA exits
+        mbar_wait_drain(&bars.a_full, 0);
+        for (int j = (it > kGemmStages ? it - kGemmStages : 0); j < it; ++j)
+          mbar_wait_drain(&bars.b_full[j % kGemmStages], (uint32_t)(j / kGemmStages) & 1u);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer ----------------
+    if (lane == 0 && my_tiles > 0) {
+      const uint32_t idesc = idesc_bf16_f32(kTile, kGemmBN);
+      bool ok = mbar_wait(&bars.a_ready, 0, abort_flag);
+      tc_fence_after();
+      int it = 0;
+      for (int i = 0; i < my_tiles && ok; ++i) {
+        const int acc = i & 1;
+        if (!mbar_wait(&bars.acc_empty[acc], ((uint32_t)(i >> 1) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(acc * kGemmBN);
+        for (int kc = 0; kc < natoms; ++kc, ++it) {
+          const int s = it % kGemmStages;
+          if (!mbar_wait(&bars.b_full[s], (uint32_t)(it / kGemmStages) & 1u, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t ad = desc_kmajor_sw128(smem_u32(sA + kc * kAtomBytes));
+          const uint64_t ld = desc_kmajor_sw128(smem_u32(sB + s * kStageBytes + kBStageBytes));
+          const uint64_t bd = desc_kmajor_sw128(smem_u32(sB + s * kStageBytes));
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_bf16_ss(d, desc_advance(ad, k * 32), desc_advance(bd, k * 32), idesc, (kc | k) != 0);
+#pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_bf16_ss(d, desc_advance(ld, k * 32), desc_advance(bd, k * 32), idesc, 1u);
+          mma_commit(&bars.b_empty[s]);
+        }
+        if (!ok) break;
+        mma_commit(&bars.acc_full[acc]);
+      }
+      mma_commit(&bars.mma_done);          // every MMA done before TMEM is freed
+      mbar_wait_drain(&bars.mma_done, 0);
+    }
+  } else {
+    // ---------------- RMSNorm prologue, then epilogue (warps 2-5) ----------------
+    const int grp = warp & 3;                 // TMEM lane group this warp may access
+    const int row = grp * 32 + lane;          // tile row == TMEM lane
+    const bool valid = (q0 + row) < L;
+    const int64_t t = seq0 + q0 + row;        // token of this row (when valid)
+    const int tp = tp0 + row;                 // padded row
+    bool ok = my_tiles > 0 ? mbar_wait_warp(&bars.a_full, 0, abort_flag) : false;
+    if (ok) {
+      // sum of squares of the R latent columns of this row
+      float ss = 0.f;
+      for (int a = 0; a < natoms; ++a) {
+        const uint8_t* base = sA + a * kAtomBytes;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint4 v = *reinterpret_cast<const uint4*>(base + sw128_offset(row, c));
+          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = unpack_bf16x2(w4[e]);
+            ss = fmaf(f.x, f.x, fmaf(f.y, f.y, ss));
+          }
+        }
+      }
+      const float r = valid ? 1.0f / sqrtf(ss / (float)p.R + p.eps) : 0.f;
+      // c_hat = w * x * r: hi in place, lo to this CTA's scratch row (rows past
+      // the sequence become zeros)
+      uint4* lo_dst = reinterpret_cast<uint4*>(lo_rows + (int64_t)row * p.R);
+      for (int a = 0; a < natoms; ++a) {
+        uint8_t* base = sA + a * kAtomBytes;
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint4* ptr = reinterpret_cast<uint4*>(base + sw128_offset(row, c));
+          const uint4 v = *ptr;
+          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
+          const int k0 = a * 64 + c * 8;
+          const uint4 wv = *reinterpret_cast<const uint4*>(p.w_norm + k0);
+          const uint32_t g4[4] = {wv.x, wv.y, wv.z, wv.w};
+          uint32_t hi4[4], lo4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = unpack_bf16x2(w4[e]);
+            const float2 g = unpack_bf16x2(g4[e]);
+            const float c0 = g.x * (f.x * r), c1 = g.y * (f.y * r);
+            hi4[e] = pack_bf16x2(c0, c1);
+            const float2 hb = unpack_bf16x2(hi4[e]);
+            lo4[e] = pack_bf16x2(c0 - hb.x, c1 - hb.y);
+          }
+          *ptr = make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
+          lo_dst[k0 / 8] = make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
+        }
+      }
+      fence_proxy_async_smem();
+      fence_proxy_async_global();
+    }
+    mbar_arrive(&bars.a_ready);
+    // rotated shared key of this row (one CTA column per tile writes it)
+    if (blockIdx.y == 0) {
+      const int half = p.P / 2;
+      __half* dst = p.k_rot + (int64_t)tp * p.P;
+      if (valid) {
+        const __nv_bfloat16* src = p.latent + t * (p.R + p.P) + p.R;
+        const int64_t pos = checked_pos(p.positions[t], p.max_pos);
+        for (int i = 0; i < half; ++i) {
+          int ia, ib;
+          rope_pair_slots(i, p.P, p.interleaved, ia, ib);
+          float ox, oy;
+          rope_turn(__bfloat162float(src[ia]), __bfloat162float(src[ib]), p.cos_t[pos * half + i],
+                    p.sin_t[pos * half + i], ox, oy);
+          dst[ia] = __float2half_rn(ox);
+          dst[ib] = __float2half_rn(oy);
+        }
+      } else {
+        for (int i = 0; i < p.P; ++i) dst[i] = __float2half_rn(0.f);
+      }
+    }
+    // epilogue: TMEM -> bf16 k_nope / transposed values
+    const int NV = p.N + p.V;
+    float vmax = 0.f;
+    for (int i = 0; i < my_tiles && ok; ++i) {
+      const int acc = i & 1;
+      if (!mbar_wait_warp(&bars.acc_full[acc], (uint32_t)(i >> 1) & 1u, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      const int o_base = (n_begin + i) * kGemmBN;
+      for (int ch = 0; ch < kGemmBN / 16; ++ch) {
+        uint32_t v[16];
+        tmem_ld16(tmem + ((uint32_t)(grp * 32) << 16) + (uint32_t)(acc * kGemmBN + ch * 16), v);
+        const int o0 = o_base + ch * 16;
+        if (o0 >= p.NOUT) continue;
+        const int h = o0 / NV, c0 = o0 % NV;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) vmax = fmaxf(vmax, fabsf(__uint_as_float(v[e])));
+        if (c0 < p.N) {
+          uint32_t pk[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e)
+            pk[e] = pack_f16x2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+          uint4* dst = reinterpret_cast<uint4*>(p.k_nope + ((int64_t)h * p.Tpad + tp) * p.N + c0);
+          dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        } else {
+          __half* dst = p.vt + ((int64_t)h * p.V + (c0 - p.N)) * p.Tpad + tp;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) dst[(int64_t)e * p.Tpad] = __float2half_rn(__uint_as_float(v[e]));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&bars.acc_empty[acc]);
+    }
+    if (!(vmax <= kF16Max)) raise_device_error(kDevErrRange);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace tc
+}  // namespace mla

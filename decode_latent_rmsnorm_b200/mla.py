@@ -232,6 +232,8 @@ class KernelEvents:
 
     def __init__(self, pairs: int):
         self.events = [torch.cuda.Event(enable_timing=True) for _ in range(2 * pairs)]
+        for e in self.events:   # torch creates the CUDA event on its first record
+            e.record()
         self._handles = (c_vp * (2 * pairs))(*[e.cuda_event for e in self.events])
         self.pairs = pairs
         self.recorded = 0

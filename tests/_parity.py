@@ -5,6 +5,9 @@ Tolerances: fp32 runs max-abs <= 1e-4; bf16 runs rel-L2 <= 5e-3 and
 max-abs <= 2e-2 (on the evaluated elements).
 """
 
+import json
+import os
+
 import numpy as np
 import torch
 
@@ -40,6 +43,10 @@ def compare(got, ref, dtype, what=""):
     max_abs = float(np.abs(err).max())
     rel_l2 = float(np.linalg.norm(err) / max(np.linalg.norm(r), 1e-300))
     m = dict(max_abs=max_abs, rel_l2=rel_l2, n=int(sel.sum()))
+    log = os.environ.get("MLA_PARITY_LOG")
+    if log:
+        with open(log, "a") as f:
+            f.write(json.dumps(dict(what=what, dtype=dtype, **m)) + "\n")
     if dtype == "fp32":
         assert max_abs <= FP32_MAX_ABS, "%s fp32 %s" % (what, m)
     else:
