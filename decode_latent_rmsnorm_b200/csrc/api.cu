@@ -7,6 +7,7 @@
 #include <string.h>
 
 #include <atomic>
+#include <mutex>
 
 #include "mla.h"
 #include "common.cuh"
@@ -17,6 +18,10 @@
 #include "tc_attention.cuh"
 
 #include <cudaTypedefs.h>
+
+// Scratch of mla_prefill_noalloc: the workspace for callers that cannot
+// allocate. It lives on every device that loads this library.
+static __device__ __align__(256) uint8_t g_noalloc_scratch[MLA_NOALLOC_SCRATCH_BYTES];
 
 namespace {
 
@@ -641,6 +646,49 @@ int mla_cache_append(const mla_dims* dims, const void* latent, const void* w_nor
         static_cast<__nv_bfloat16*>(cache), cache_num_rows, cache_rows);
   prof_end(stream);
   return cuda_status(cudaGetLastError(), "cache append launch");
+}
+
+// Device address of g_noalloc_scratch, looked up once per device (host code
+// cannot use the array's name as a device address).
+namespace {
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_ptr[kMaxDevices] = {};
+
+int noalloc_scratch(void** ptr) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_status(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxDevices) return fail(MLA_ERR_UNSUPPORTED_SHAPE, "device index %d too large", dev);
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (!g_noalloc_ptr[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return cuda_status(e, "cudaGetSymbolAddress of the static scratch");
+    g_noalloc_ptr[dev] = p;
+  }
+  *ptr = g_noalloc_ptr[dev];
+  return MLA_OK;
+}
+}  // namespace
+
+int mla_prefill_noalloc(const mla_dims* dims, const void* latent, const void* q, const void* w_kvb,
+                        const void* w_norm, const int32_t* positions, const int32_t* cu_seqlens, int32_t num_seqs,
+                        int32_t max_seqlen, int64_t total_tokens, const float* cos_table, const float* sin_table,
+                        int32_t max_pos, void* out, cudaStream_t stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (total_tokens < 0 || num_seqs < 0) return fail(MLA_ERR_INVALID_ARG, "negative size");
+  const size_t need = prefill_ws_bytes(dims, total_tokens, num_seqs);
+  if (need > (size_t)MLA_NOALLOC_SCRATCH_BYTES)
+    return fail(MLA_ERR_WORKSPACE_TOO_SMALL,
+                "this prefill needs %zu bytes of scratch; the static scratch of mla_prefill_noalloc holds %zu",
+                need, (size_t)MLA_NOALLOC_SCRATCH_BYTES);
+  void* scratch = nullptr;
+  rc = noalloc_scratch(&scratch);
+  if (rc) return rc;
+  return mla_prefill(dims, latent, q, w_kvb, w_norm, positions, cu_seqlens, num_seqs, max_seqlen, total_tokens,
+                     cos_table, sin_table, max_pos, out, scratch, (size_t)MLA_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 int mla_check_device_status(cudaStream_t stream) {

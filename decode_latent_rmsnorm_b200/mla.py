@@ -42,7 +42,12 @@ SIGNATURES = {
     "mla_recorded_kernel_events": (c_i32, [ctypes.POINTER(c_i32)]),
     "mla_launch_count": (ctypes.c_uint64, []),
     "mla_recorded_kernel_name": (ctypes.c_char_p, [c_i32]),
+    "mla_prefill_noalloc": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_i32, c_i32, c_i64,
+                                    c_vp, c_vp, c_i32, c_vp, c_vp]),
 }
+
+# Bytes of the static scratch behind mla_prefill_noalloc (MLA_NOALLOC_SCRATCH_BYTES).
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024
 
 
 class RopeCfg(ctypes.Structure):
@@ -160,6 +165,24 @@ def mla_prefill(dims: Dims, latent, q, w_kvb, w_norm, positions, cu_seqlens, max
         int(nseq), int(max_seqlen), int(T), _dev(cos, "cos", torch.float32),
         _dev(sin, "sin", torch.float32), int(cos.shape[0]), _dev(out, "out", dt, (T, H, V)),
         _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream()))
+    return out
+
+
+def mla_prefill_noalloc(dims: Dims, latent, q, w_kvb, w_norm, positions, cu_seqlens, max_seqlen: int,
+                        cos, sin, out):
+    """mla_prefill without a workspace, for callers that cannot allocate
+    device memory: the library's static scratch array serves as workspace.
+    ``out`` must be given (this call allocates nothing)."""
+    dt = dims.torch_dtype
+    H, R, N, P, V = dims.num_heads, dims.kv_lora_rank, dims.qk_nope, dims.qk_rope, dims.v_head
+    T = latent.shape[0]
+    nseq = cu_seqlens.numel() - 1
+    _check(load().mla_prefill_noalloc(
+        ctypes.byref(dims), _dev(latent, "latent", dt, (T, R + P)), _dev(q, "q", dt, (T, H, N + P)),
+        _dev(w_kvb, "w_kvb", dt, (H * (N + V), R)), _dev(w_norm, "w_norm", dt, (R,)),
+        _dev(positions, "positions", torch.int32, (T,)), _dev(cu_seqlens, "cu_seqlens", torch.int32),
+        int(nseq), int(max_seqlen), int(T), _dev(cos, "cos", torch.float32),
+        _dev(sin, "sin", torch.float32), int(cos.shape[0]), _dev(out, "out", dt, (T, H, V)), _stream()))
     return out
 
 

@@ -171,6 +171,41 @@ int mla_cache_append(const mla_dims* dims, const void* latent, const void* w_nor
                      const float* sin_table, int32_t max_pos, void* cache,
                      int64_t cache_num_rows, const int64_t* cache_rows, cudaStream_t stream);
 
+/* Size of the scratch array behind mla_prefill_noalloc (32 MiB). */
+#define MLA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+/* Prefill for callers that cannot allocate device memory. Some code that
+ * calls this library owns no device allocator of its own: a plugin inside a
+ * host application whose framework has already reserved the GPU's memory in
+ * its caching allocator, or a latency-bound loop that may not call
+ * cudaMalloc because that call can block until the whole device is idle.
+ * This entry point takes the same arguments as mla_prefill except the
+ * workspace, and allocates nothing: its scratch is a file-scope static
+ * __device__ array of MLA_NOALLOC_SCRATCH_BYTES bytes that exists on every
+ * GPU that loads this library, until the process exits. The pages have no
+ * counterpart to this entry point; it changes how scratch is provided, not
+ * what is computed (the results equal mla_prefill's).
+ *   - The first call on a device, with that device current, looks up the
+ *     array's device address (cudaGetSymbolAddress) and keeps it; make that
+ *     first call before any stream capture.
+ *   - A call whose workspace need (mla_prefill_workspace_size) exceeds
+ *     MLA_NOALLOC_SCRATCH_BYTES returns MLA_ERR_WORKSPACE_TOO_SMALL and
+ *     launches nothing. About 20 MiB of the array go to per-block scratch
+ *     whatever the size; for the Kimi-K2 head geometry the rest holds one
+ *     sequence of up to 256 tokens (each sequence is padded to 128-token
+ *     tiles, plus one tile per sequence of headroom).
+ *   - All calls on a device share the one array, and it keeps what the last
+ *     call left there (no part of it needs to start at zero: every call
+ *     writes what it reads). Calls that can overlap on the GPU (different
+ *     streams without ordering between them) race on it and must not be
+ *     issued. */
+int mla_prefill_noalloc(const mla_dims* dims,
+                        const void* latent, const void* q, const void* w_kvb, const void* w_norm,
+                        const int32_t* positions, const int32_t* cu_seqlens,
+                        int32_t num_seqs, int32_t max_seqlen, int64_t total_tokens,
+                        const float* cos_table, const float* sin_table, int32_t max_pos,
+                        void* out, cudaStream_t stream);
+
 /* Synchronises `stream`, then reads and clears the device error word that
  * the kernels' bounded waits set. Returns MLA_ERR_DEVICE_TIMEOUT if one gave
  * up since the last check, MLA_ERR_CUDA on a CUDA error, else MLA_OK. */
