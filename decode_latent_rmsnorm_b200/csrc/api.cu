@@ -16,6 +16,7 @@
 #include "simt_decode.cuh"
 #include "tc_gemm.cuh"
 #include "tc_attention.cuh"
+#include "tc_decode.cuh"
 
 #include <cudaTypedefs.h>
 
@@ -201,18 +202,53 @@ size_t prefill_ws_bytes(const mla_dims* d, int64_t T, int nseq) {
   return a;
 }
 
-// Decode workspace: q_lat [B, H, R], q_rot [B, H, P], per-split partials.
+// Shapes the tensor-core decode takes (bf16, 64 heads, 512 + 64 latent row).
+bool decode_tc_shape(const mla_dims* d) {
+  return d->dtype == MLA_BF16 && d->num_heads == mla::tc::kDecHeads && d->kv_lora_rank == 512 &&
+         d->qk_rope == 64 && d->qk_nope <= 384;
+}
+
+int g_num_sms[64] = {};
+int num_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!g_num_sms[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    g_num_sms[dev] = n;
+  }
+  return g_num_sms[dev];
+}
+
+// SIMT decode workspace: q_lat [B, H, R], q_rot [B, H, P], per-split partials.
+// Tensor-core decode workspace: prefix [B + 1] and meta [2] (int64), q [B, H,
+// R + P] bf16, partials of B + G slots, o_lat [B, H, R] fp32.
 struct DecodeWs {
   int nsplit;
   size_t q_lat, q_rot, o_part, m_part, l_part, total;
+  size_t prefix, meta, qf, o_lat;
+  int G;
 };
-DecodeWs decode_ws_layout(const mla_dims* d, int B, int max_len) {
-  DecodeWs w;
+DecodeWs decode_ws_layout(const mla_dims* d, int B, int max_len, bool tc) {
+  DecodeWs w = {};
   const size_t H = d->num_heads, R = d->kv_lora_rank, P = d->qk_rope;
+  size_t off = 0;
+  if (tc) {
+    w.G = num_sms();
+    const size_t slots = (size_t)B + w.G;
+    w.prefix = off; off = align_up(off + 8 * (size_t)(B + 1), 256);
+    w.meta = off;   off = align_up(off + 16, 256);
+    w.qf = off;     off = align_up(off + 2 * (size_t)B * H * (R + P), 256);
+    w.o_part = off; off = align_up(off + 4 * slots * H * R, 256);
+    w.m_part = off; off = align_up(off + 4 * slots * H, 256);
+    w.l_part = off; off = align_up(off + 4 * slots * H, 256);
+    w.o_lat = off;  off = align_up(off + 4 * (size_t)B * H * R, 256);
+    w.total = off;
+    return w;
+  }
   w.nsplit = (max_len + mla::simt::kDecChunk - 1) / mla::simt::kDecChunk;
   if (w.nsplit < 1) w.nsplit = 1;
   const size_t S = w.nsplit;
-  size_t off = 0;
   w.q_lat = off;  off = align_up(off + 4 * (size_t)B * H * R, 256);
   w.q_rot = off;  off = align_up(off + 4 * (size_t)B * H * P, 256);
   w.o_part = off; off = align_up(off + 4 * (size_t)B * S * H * R, 256);
@@ -220,6 +256,14 @@ DecodeWs decode_ws_layout(const mla_dims* d, int B, int max_len) {
   w.l_part = off; off = align_up(off + 4 * (size_t)B * S * H, 256);
   w.total = off;
   return w;
+}
+size_t decode_ws_bytes(const mla_dims* d, int B, int max_len) {
+  size_t a = decode_ws_layout(d, B, max_len, false).total;
+  if (decode_tc_shape(d)) {
+    const size_t b = decode_ws_layout(d, B, max_len, true).total;
+    if (b > a) a = b;
+  }
+  return a;
 }
 
 template <typename T>
@@ -431,7 +475,7 @@ int launch_decode(const mla_dims* d, const void* q, const void* cache, int64_t c
                   void* out, void* workspace, cudaStream_t st) {
   using namespace mla::simt;
   const int H = d->num_heads, R = d->kv_lora_rank, N = d->qk_nope, P = d->qk_rope, V = d->v_head;
-  const DecodeWs L = decode_ws_layout(d, B, max_len);
+  const DecodeWs L = decode_ws_layout(d, B, max_len, false);
   char* ws = static_cast<char*>(workspace);
   float* q_lat = reinterpret_cast<float*>(ws + L.q_lat);
   float* q_rot = reinterpret_cast<float*>(ws + L.q_rot);
@@ -456,6 +500,84 @@ int launch_decode(const mla_dims* d, const void* q, const void* cache, int64_t c
   prof_begin(st, "simt_decode_combine");
   combine_kernel<T><<<dim3(B, H), 256, 0, st>>>(o_part, m_part, l_part, static_cast<const T*>(w_kvb), H,
                                                 R, N, V, L.nsplit, static_cast<T*>(out));
+  prof_end(st);
+  return cuda_status(cudaGetLastError(), "decode launch");
+}
+
+// Tensor-core decode: split schedule -> q absorb + rope -> split-KV attention
+// (tcgen05) -> log-sum-exp combine -> W_UV un-absorb.
+int launch_decode_tc(const mla_dims* d, const void* q, const void* cache, int64_t cache_rows,
+                     const int64_t* offsets, const int32_t* lens, const int32_t* positions, int B, int max_len,
+                     const void* w_kvb, const float* cos_t, const float* sin_t, int max_pos, void* out,
+                     void* workspace, cudaStream_t st) {
+  using bf16 = __nv_bfloat16;
+  namespace T = mla::tc;
+  const int H = d->num_heads, R = d->kv_lora_rank, N = d->qk_nope, P = d->qk_rope, V = d->v_head;
+  const DecodeWs L = decode_ws_layout(d, B, max_len, true);
+  char* ws = static_cast<char*>(workspace);
+  int64_t* prefix = reinterpret_cast<int64_t*>(ws + L.prefix);
+  int64_t* meta = reinterpret_cast<int64_t*>(ws + L.meta);
+  bf16* qf = reinterpret_cast<bf16*>(ws + L.qf);
+  float* o_part = reinterpret_cast<float*>(ws + L.o_part);
+  float* m_part = reinterpret_cast<float*>(ws + L.m_part);
+  float* l_part = reinterpret_cast<float*>(ws + L.l_part);
+  float* o_lat = reinterpret_cast<float*>(ws + L.o_lat);
+
+  CUtensorMap map_cache, map_q;
+  {
+    const uint64_t dims[2] = {(uint64_t)(R + P), (uint64_t)cache_rows};
+    const uint64_t strides[1] = {(uint64_t)(R + P) * 2};
+    const uint32_t box[2] = {64, (uint32_t)T::kDecRows};
+    int rc = make_map(&map_cache, cache, 2, dims, strides, box);
+    if (rc) return rc;
+  }
+  {
+    const uint64_t dims[2] = {(uint64_t)(R + P), (uint64_t)B * H};
+    const uint64_t strides[1] = {(uint64_t)(R + P) * 2};
+    const uint32_t box[2] = {64, (uint32_t)T::kDecHeads};
+    int rc = make_map(&map_q, qf, 2, dims, strides, box);
+    if (rc) return rc;
+  }
+  prof_begin(st, "tc_decode_schedule");
+  T::decode_schedule_kernel<<<1, 1024, 0, st>>>(lens, offsets, B, max_len, cache_rows, L.G, prefix, meta);
+  prof_end(st);
+
+  const size_t qsm = (size_t)N * 128 * sizeof(float);
+  cudaError_t e = cudaFuncSetAttribute(T::decode_qprep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qsm);
+  if (e != cudaSuccess) return cuda_status(e, "qprep smem attribute");
+  prof_begin(st, "tc_decode_qprep");
+  T::decode_qprep_kernel<<<dim3(H, R / 128 + 1), 256, qsm, st>>>(
+      static_cast<const bf16*>(q), static_cast<const bf16*>(w_kvb), positions, cos_t, sin_t, max_pos, B, H, R, N, P, V,
+      d->rope_interleaved, qf);
+  prof_end(st);
+
+  T::DecParams dp;
+  dp.prefix = prefix;
+  dp.meta = meta;
+  dp.offsets = offsets;
+  dp.o_part = o_part;
+  dp.m_part = m_part;
+  dp.l_part = l_part;
+  dp.B = B;
+  dp.H = H;
+  dp.R = R;
+  dp.scale_log2 = d->softmax_scale * 1.4426950408889634f;
+  e = cudaFuncSetAttribute(T::decode_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)T::kDecSmem);
+  if (e != cudaSuccess) return cuda_status(e, "decode smem attribute");
+  prof_begin(st, "tc_decode_attention");
+  T::decode_attn_kernel<<<L.G, T::kDecThreads, T::kDecSmem, st>>>(map_cache, map_q, dp);
+  prof_end(st);
+
+  prof_begin(st, "tc_decode_combine");
+  T::decode_combine_kernel<<<dim3(B, H), 128, 0, st>>>(o_part, m_part, l_part, prefix, meta, H, R, o_lat);
+  prof_end(st);
+
+  const size_t usm = (size_t)32 * R * sizeof(float);
+  e = cudaFuncSetAttribute(T::decode_unabsorb_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)usm);
+  if (e != cudaSuccess) return cuda_status(e, "unabsorb smem attribute");
+  prof_begin(st, "tc_decode_unabsorb");
+  T::decode_unabsorb_kernel<<<dim3(H, (V + 31) / 32), 256, usm, st>>>(o_lat, static_cast<const bf16*>(w_kvb), B, H, R,
+                                                                      N, V, static_cast<bf16*>(out));
   prof_end(st);
   return cuda_status(cudaGetLastError(), "decode launch");
 }
@@ -583,7 +705,7 @@ int mla_decode_workspace_size(const mla_dims* dims, int32_t batch, int32_t max_c
   if (rc) return rc;
   if (batch < 0 || max_cache_len < 0) return fail(MLA_ERR_INVALID_ARG, "negative size");
   if (!bytes) return fail(MLA_ERR_INVALID_ARG, "bytes is NULL");
-  *bytes = decode_ws_layout(dims, batch, max_cache_len).total;
+  *bytes = decode_ws_bytes(dims, batch, max_cache_len);
   return MLA_OK;
 }
 
@@ -607,9 +729,12 @@ int mla_decode(const mla_dims* dims, const void* q, const void* cache, int64_t c
     return fail(MLA_ERR_INVALID_ARG, "a tensor pointer is NULL");
   if (dims->qk_nope > 512) return fail(MLA_ERR_UNSUPPORTED_SHAPE, "qk_nope must be <= 512");
   if (cache_num_rows < 1) return fail(MLA_ERR_INVALID_ARG, "cache_num_rows must be >= 1");
-  const size_t need = decode_ws_layout(dims, batch, max_cache_len).total;
+  const size_t need = decode_ws_bytes(dims, batch, max_cache_len);
   if (!workspace || workspace_bytes < need)
     return fail(MLA_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes, got %zu", need, workspace_bytes);
+  if (decode_tc_shape(dims) && cache_num_rows < ((int64_t)1 << 31) && aligned16(cache) && aligned16(workspace))
+    return launch_decode_tc(dims, q, cache, cache_num_rows, cache_offsets, cache_lens, positions, batch, max_cache_len,
+                            w_kvb, cos_table, sin_table, max_pos, out, workspace, stream);
   if (dims->dtype == MLA_FP32)
     return launch_decode<float>(dims, q, cache, cache_num_rows, cache_offsets, cache_lens, positions, batch,
                                 max_cache_len, w_kvb, cos_table, sin_table, max_pos, out, workspace, stream);

@@ -41,7 +41,7 @@ __global__ void __launch_bounds__(1024)
 schedule_kernel(const int32_t* __restrict__ cu, int nseq, int64_t Ttot, int max_seqlen, int cap,
                 int32_t* __restrict__ seq_tile0, int32_t* __restrict__ tile_seq, int32_t* __restrict__ tile_q0,
                 int32_t* __restrict__ order) {
-  constexpr int kBuckets = 2048;
+  constexpr int kBuckets = 2048;   // = 2 * blockDim.x (launched with 1024 threads)
   __shared__ int s_bad;
   __shared__ int s_carry;
   __shared__ int s_scan[1024];
@@ -93,9 +93,22 @@ schedule_kernel(const int32_t* __restrict__ cu, int nseq, int64_t Ttot, int max_
     }
   }
   __syncthreads();
-  if (tid == 0) {   // descending exclusive offsets (kBuckets steps, once per call)
-    int run = 0;
-    for (int k = kBuckets - 1; k >= 0; --k) { s_off[k] = run; run += s_cnt[k]; }
+  {
+    // descending exclusive offsets: s_off[k] = sum of s_cnt[k'] for k' > k.
+    // Thread i owns reversed buckets 2i and 2i + 1 (bucket kBuckets-1-2i, ...).
+    const int k0 = kBuckets - 1 - 2 * tid, k1 = k0 - 1;
+    const int c0 = s_cnt[k0], c1 = s_cnt[k1];
+    s_scan[tid] = c0 + c1;
+    __syncthreads();
+    for (int off = 1; off < (int)blockDim.x; off <<= 1) {
+      const int v = tid >= off ? s_scan[tid - off] : 0;
+      __syncthreads();
+      s_scan[tid] += v;
+      __syncthreads();
+    }
+    const int before = s_scan[tid] - (c0 + c1);
+    s_off[k0] = before;
+    s_off[k1] = before + c0;
   }
   __syncthreads();
   for (int s = tid; s < nseq; s += blockDim.x) {
