@@ -160,7 +160,7 @@ bool prefill_tc_shape(const mla_dims* d) {
 struct PrefillWs {
   int64_t cap, Tpad;
   int gemm_tiles_per_cta, gemm_gy;
-  size_t seq_tile0, tile_seq, tile_q0, order, lo;
+  size_t seq_tile0, tile_seq, tile_q0, order, w16;
   size_t k_nope, vals, k_rot, total;
 };
 PrefillWs prefill_ws_layout(const mla_dims* d, int64_t T, int nseq, bool tc) {
@@ -182,7 +182,7 @@ PrefillWs prefill_ws_layout(const mla_dims* d, int64_t T, int nseq, bool tc) {
     w.tile_seq = off;  off = align_up(off + 4 * (size_t)w.cap, 256);
     w.tile_q0 = off;   off = align_up(off + 4 * (size_t)w.cap, 256);
     w.order = off;     off = align_up(off + 4 * (size_t)w.cap, 256);
-    w.lo = off;        off = align_up(off + 2 * (size_t)w.cap * w.gemm_gy * 128 * d->kv_lora_rank, 256);
+    w.w16 = off;       off = align_up(off + 2 * (size_t)NOUT * d->kv_lora_rank, 256);
   } else {
     w.Tpad = T;
   }
@@ -205,7 +205,7 @@ size_t prefill_ws_bytes(const mla_dims* d, int64_t T, int nseq) {
 // Shapes the tensor-core decode takes (bf16, 64 heads, 512 + 64 latent row).
 bool decode_tc_shape(const mla_dims* d) {
   return d->dtype == MLA_BF16 && d->num_heads == mla::tc::kDecHeads && d->kv_lora_rank == 512 &&
-         d->qk_rope == 64 && d->qk_nope <= 384;
+         d->qk_rope == 64;
 }
 
 int g_num_sms[64] = {};
@@ -368,20 +368,17 @@ int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, cons
     const uint64_t dims[2] = {(uint64_t)R, (uint64_t)NOUT};
     const uint64_t strides[1] = {(uint64_t)R * 2};
     const uint32_t box[2] = {64, 256};
-    int rc = make_map(&map_w, w_kvb, 2, dims, strides, box);
+    int rc = make_map(&map_w, ws + L.w16, 2, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
     if (rc) return rc;
   }
 
-  bf16* lo = reinterpret_cast<bf16*>(ws + L.lo);
+  __half* w16 = reinterpret_cast<__half*>(ws + L.w16);
   const int gy = L.gemm_gy;
-  CUtensorMap map_lo;
-  {
-    const uint64_t dims[2] = {(uint64_t)R, (uint64_t)cap * gy * 128};
-    const uint64_t strides[1] = {(uint64_t)R * 2};
-    const uint32_t box[2] = {64, 128};
-    int rc = make_map(&map_lo, lo, 2, dims, strides, box);
-    if (rc) return rc;
-  }
+
+  const int64_t n8 = (int64_t)NOUT * R / 8;
+  prof_begin(st, "tc_weight_f16");
+  mla::tc::weight_to_f16_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(static_cast<const bf16*>(w_kvb), w16, n8);
+  prof_end(st);
 
   prof_begin(st, "tc_schedule");
   mla::tc::schedule_kernel<<<1, 1024, 0, st>>>(cu_seqlens, num_seqs, T_tot, max_seqlen, cap, seq_tile0, tile_seq,
@@ -400,7 +397,6 @@ int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, cons
   gp.k_nope = k_nope;
   gp.vt = vt;
   gp.k_rot = k_rot;
-  gp.lo_scratch = lo;
   gp.Ttot = T_tot;
   gp.Tpad = (int)L.Tpad;
   gp.R = R; gp.P = P; gp.H = H; gp.N = N; gp.V = V; gp.NOUT = NOUT;
@@ -413,7 +409,7 @@ int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, cons
   if (e != cudaSuccess) return cuda_status(e, "gemm smem attribute");
   prof_begin(st, "tc_norm_kv_b_proj");
   mla::tc::norm_kvb_gemm_kernel<<<dim3(cap, gy), mla::tc::kGemmThreads, mla::tc::kGemmSmemBytes, st>>>(
-      map_lat, map_w, map_lo, gp);
+      map_lat, map_w, gp);
   prof_end(st);
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_status(e, "gemm launch");
@@ -542,13 +538,17 @@ int launch_decode_tc(const mla_dims* d, const void* q, const void* cache, int64_
   T::decode_schedule_kernel<<<1, 1024, 0, st>>>(lens, offsets, B, max_len, cache_rows, L.G, prefix, meta);
   prof_end(st);
 
-  const size_t qsm = (size_t)N * 128 * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(T::decode_qprep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)qsm);
-  if (e != cudaSuccess) return cuda_status(e, "qprep smem attribute");
-  prof_begin(st, "tc_decode_qprep");
-  T::decode_qprep_kernel<<<dim3(H, R / 128 + 1), 256, qsm, st>>>(
-      static_cast<const bf16*>(q), static_cast<const bf16*>(w_kvb), positions, cos_t, sin_t, max_pos, B, H, R, N, P, V,
-      d->rope_interleaved, qf);
+  // q_lat[b, h, :] = q_nope[b, h, :] W_UK_h  (W_UK_h rows j < N of head h: [N, R], R contiguous)
+  prof_begin(st, "tc_decode_qabsorb");
+  T::small_gemm_kernel<bf16, true><<<dim3(H, R / T::kSgBN, (B + T::kSgBM - 1) / T::kSgBM), 256, 0, st>>>(
+      static_cast<const bf16*>(q), (int64_t)H * (N + P), (int64_t)(N + P), static_cast<const bf16*>(w_kvb),
+      (int64_t)(N + V) * R, (int64_t)R, qf, (int64_t)H * (R + P), (int64_t)(R + P), B, R, N);
+  prof_end(st);
+  const int64_t nrope = (int64_t)B * H * (P / 2);
+  prof_begin(st, "tc_decode_qrope");
+  T::decode_qrope_kernel<<<(unsigned)((nrope + 255) / 256), 256, 0, st>>>(static_cast<const bf16*>(q), positions,
+                                                                           cos_t, sin_t, max_pos, B, H, R, N, P,
+                                                                           d->rope_interleaved, qf);
   prof_end(st);
 
   T::DecParams dp;
@@ -562,7 +562,7 @@ int launch_decode_tc(const mla_dims* d, const void* q, const void* cache, int64_
   dp.H = H;
   dp.R = R;
   dp.scale_log2 = d->softmax_scale * 1.4426950408889634f;
-  e = cudaFuncSetAttribute(T::decode_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)T::kDecSmem);
+  cudaError_t e = cudaFuncSetAttribute(T::decode_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)T::kDecSmem);
   if (e != cudaSuccess) return cuda_status(e, "decode smem attribute");
   prof_begin(st, "tc_decode_attention");
   T::decode_attn_kernel<<<L.G, T::kDecThreads, T::kDecSmem, st>>>(map_cache, map_q, dp);
@@ -572,12 +572,12 @@ int launch_decode_tc(const mla_dims* d, const void* q, const void* cache, int64_
   T::decode_combine_kernel<<<dim3(B, H), 128, 0, st>>>(o_part, m_part, l_part, prefix, meta, H, R, o_lat);
   prof_end(st);
 
-  const size_t usm = (size_t)32 * R * sizeof(float);
-  e = cudaFuncSetAttribute(T::decode_unabsorb_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)usm);
-  if (e != cudaSuccess) return cuda_status(e, "unabsorb smem attribute");
+  // out[b, h, :] = W_UV_h o_lat[b, h, :]  (W_UV_h rows N.. N+V-1 of head h: [V, R], R contiguous)
   prof_begin(st, "tc_decode_unabsorb");
-  T::decode_unabsorb_kernel<<<dim3(H, (V + 31) / 32), 256, usm, st>>>(o_lat, static_cast<const bf16*>(w_kvb), B, H, R,
-                                                                      N, V, static_cast<bf16*>(out));
+  T::small_gemm_kernel<float, false><<<dim3(H, (V + T::kSgBN - 1) / T::kSgBN, (B + T::kSgBM - 1) / T::kSgBM), 256, 0,
+                                       st>>>(o_lat, (int64_t)H * R, (int64_t)R,
+                                             static_cast<const bf16*>(w_kvb) + (int64_t)N * R, (int64_t)(N + V) * R,
+                                             (int64_t)R, static_cast<bf16*>(out), (int64_t)H * V, (int64_t)V, B, V, R);
   prof_end(st);
   return cuda_status(cudaGetLastError(), "decode launch");
 }

@@ -8,13 +8,11 @@
 // k_pe as one head shared by all heads).
 //
 // Precision: the normalized latent c_hat = w * x / rms(x) is formed in fp32
-// and handed to the tensor cores exactly, as c_hat = hi + lo with hi =
-// bf16(c_hat) and lo = bf16(c_hat - hi) (|lo| <= 2^-9 |c_hat|; the pair keeps
-// about 17 significant bits). Both halves multiply the same weight tile and
-// accumulate in fp32, so k_nope and the values carry one rounding only: their
-// own storage, in fp16 (11 significant bits; attention runs its tensor-core
-// products on fp16 operands). A value beyond the fp16 range sets the device
-// error word.
+// and handed to the tensor cores in fp16 (11 significant bits), against an
+// fp16 copy of the weight (exact for weights in fp16's normal range), with
+// fp32 accumulation; k_nope and the values are stored in fp16 (attention runs
+// its tensor-core products on fp16 operands). A value beyond the fp16 range
+// sets the device error word.
 //
 // Workspace layout ("padded token space"): every sequence starts on a
 // 128-row boundary, so a 128-token tile never straddles two sequences and
@@ -120,12 +118,32 @@ schedule_kernel(const int32_t* __restrict__ cu, int nseq, int64_t Ttot, int max_
   }
 }
 
+// ---- fp16 copy of the kv_b_proj weight ------------------------------------------
+// 8 values per thread; a weight beyond the fp16 range sets the device error word.
+__global__ void __launch_bounds__(256)
+weight_to_f16_kernel(const __nv_bfloat16* __restrict__ w, __half* __restrict__ w16, int64_t n8) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const uint4 v = reinterpret_cast<const uint4*>(w)[i];
+  const uint32_t in[4] = {v.x, v.y, v.z, v.w};
+  uint32_t o[4];
+  float mx = 0.f;
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 f = unpack_bf16x2(in[e]);
+    mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
+    o[e] = pack_f16x2(f.x, f.y);
+  }
+  if (!(mx <= kF16Max)) raise_device_error(kDevErrRange);
+  reinterpret_cast<uint4*>(w16)[i] = make_uint4(o[0], o[1], o[2], o[3]);
+}
+
 // ---- fused RMSNorm + kv_b_proj GEMM ------------------------------------------
 constexpr int kGemmBN = 256;                    // output columns per tile (MMA N)
-constexpr int kGemmStages = 2;                  // (weight tile, lo tile) pipeline depth
-constexpr int kAtomBytes = kTile * 128;         // 128 rows x 64 bf16
-constexpr int kBStageBytes = kGemmBN * 128;     // 256 rows x 64 bf16
-constexpr int kStageBytes = kBStageBytes + kAtomBytes;   // weight chunk + lo chunk
+constexpr int kGemmStages = 3;                  // weight pipeline depth
+constexpr int kAtomBytes = kTile * 128;         // 128 rows x 64 16-bit values
+constexpr int kBStageBytes = kGemmBN * 128;     // 256 rows x 64 fp16
+constexpr int kStageBytes = kBStageBytes;
 constexpr int kGemmThreads = 192;               // warp 0 TMA, warp 1 MMA, warps 2-5 norm + epilogue
 constexpr int kGemmMaxAtoms = 8;                // R <= 512
 constexpr size_t kGemmSmemBytes = (size_t)kGemmMaxAtoms * kAtomBytes + (size_t)kGemmStages * kStageBytes + 1024;
@@ -142,7 +160,6 @@ struct GemmParams {
   __half* k_nope;
   __half* vt;
   __half* k_rot;
-  __nv_bfloat16* lo_scratch;     // [CTAs * 128, R]: each CTA's lo half of c_hat
   int64_t Ttot;
   int Tpad, R, P, H, N, V, NOUT;
   int tiles_per_cta;             // n tiles (256 columns) per CTA
@@ -160,14 +177,14 @@ struct GemmBarriers {
 };
 
 // grid: (tile capacity, ceil(NOUT / (256 * tiles_per_cta))). The TMA-fed
-// prologue normalizes the CTA's 128 x R latent tile: hi stays resident in
-// shared memory, lo goes to the CTA's private scratch rows (L2-resident) and
-// streams back with the weight tiles through a 2-stage TMA pipeline. The fp32
-// accumulator is double buffered in TMEM (2 x 256 columns) so the epilogue of
-// one output tile overlaps the MMAs of the next.
+// prologue normalizes the CTA's 128 x R latent tile in shared memory (fp16,
+// resident for all its output tiles); the fp16 weight streams through a
+// 3-stage TMA pipeline. The fp32 accumulator is double buffered in TMEM
+// (2 x 256 columns) so the epilogue of one output tile overlaps the MMAs of
+// the next.
 __global__ void __launch_bounds__(kGemmThreads, 1)
 norm_kvb_gemm_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant__ CUtensorMap map_w,
-                     const __grid_constant__ CUtensorMap map_lo, GemmParams p) {
+                     GemmParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ GemmBarriers bars;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -175,10 +192,8 @@ norm_kvb_gemm_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_c
   const int seq = p.tile_seq[tile];
   if (seq < 0) return;   // past the real tiles (uniform over the CTA)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* sA = smem;                                        // R/64 atoms of [128 x 64] (hi)
-  uint8_t* sB = smem + kGemmMaxAtoms * kAtomBytes;           // stages: [256 x 64] weight + [128 x 64] lo
-  const int cta_id = blockIdx.y * gridDim.x + blockIdx.x;
-  __nv_bfloat16* lo_rows = p.lo_scratch + (int64_t)cta_id * kTile * p.R;
+  uint8_t* sA = smem;                                        // R/64 atoms of [128 x 64]
+  uint8_t* sB = smem + kGemmMaxAtoms * kAtomBytes;           // stages of [256 x 64] weight
   const int q0 = p.tile_q0[tile];
   const int64_t seq0 = p.cu[seq];
   const int L = (int)(p.cu[seq + 1] - seq0);
@@ -210,13 +225,11 @@ norm_kvb_gemm_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_c
     if (lane == 0 && my_tiles > 0) {
       tma_prefetch_desc(&map_lat);
       tma_prefetch_desc(&map_w);
-      tma_prefetch_desc(&map_lo);
       mbar_arrive_expect_tx(&bars.a_full, natoms * kAtomBytes);
       for (int a = 0; a < natoms; ++a)
         tma_load_2d(sA + a * kAtomBytes, &map_lat, &bars.a_full, a * 64, (int)(seq0 + q0));
       int it = 0;
-      // the lo rows exist once the prologue has written them
-      bool ok = mbar_wait(&bars.a_ready, 0, abort_flag);
+      bool ok = true;
       for (int nt = n_begin; nt < n_end && ok; ++nt) {
         for (int kc = 0; kc < natoms; ++kc, ++it) {
           const int s = it % kGemmStages;
@@ -225,7 +238,6 @@ norm_kvb_gemm_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_c
           uint8_t* st = sB + s * kStageBytes;
           mbar_arrive_expect_tx(&bars.b_full[s], kStageBytes);
           tma_load_2d(st, &map_w, &bars.b_full[s], kc * 64, nt * kGemmBN);
-          tma_load_2d(st + kBStageBytes, &map_lo, &bars.b_full[s], kc * 64, cta_id * kTile);
         }
       }
       if (!ok) {   // drain the loads that may still be in flight before the CTA exits
@@ -237,7 +249,7 @@ norm_kvb_gemm_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_c
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0 && my_tiles > 0) {
-      const uint32_t idesc = idesc_bf16_f32(kTile, kGemmBN);
+      const uint32_t idesc = idesc_f16_f32(kTile, kGemmBN);
       bool ok = mbar_wait(&bars.a_ready, 0, abort_flag);
       tc_fence_after();
       int it = 0;
@@ -251,14 +263,10 @@ norm_kvb_gemm_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_c
           if (!mbar_wait(&bars.b_full[s], (uint32_t)(it / kGemmStages) & 1u, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint64_t ad = desc_kmajor_sw128(smem_u32(sA + kc * kAtomBytes));
-          const uint64_t ld = desc_kmajor_sw128(smem_u32(sB + s * kStageBytes + kBStageBytes));
           const uint64_t bd = desc_kmajor_sw128(smem_u32(sB + s * kStageBytes));
 #pragma unroll
           for (int k = 0; k < 4; ++k)
             mma_bf16_ss(d, desc_advance(ad, k * 32), desc_advance(bd, k * 32), idesc, (kc | k) != 0);
-#pragma unroll
-          for (int k = 0; k < 4; ++k)
-            mma_bf16_ss(d, desc_advance(ld, k * 32), desc_advance(bd, k * 32), idesc, 1u);
           mma_commit(&bars.b_empty[s]);
         }
         if (!ok) break;
@@ -292,9 +300,7 @@ norm_kvb_gemm_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_c
         }
       }
       const float r = valid ? 1.0f / sqrtf(ss / (float)p.R + p.eps) : 0.f;
-      // c_hat = w * x * r: hi in place, lo to this CTA's scratch row (rows past
-      // the sequence become zeros)
-      uint4* lo_dst = reinterpret_cast<uint4*>(lo_rows + (int64_t)row * p.R);
+      // c_hat = w * x * r in place, as fp16 (rows past the sequence become zeros)
       for (int a = 0; a < natoms; ++a) {
         uint8_t* base = sA + a * kAtomBytes;
 #pragma unroll
@@ -305,22 +311,17 @@ norm_kvb_gemm_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_c
           const int k0 = a * 64 + c * 8;
           const uint4 wv = *reinterpret_cast<const uint4*>(p.w_norm + k0);
           const uint32_t g4[4] = {wv.x, wv.y, wv.z, wv.w};
-          uint32_t hi4[4], lo4[4];
+          uint32_t o4[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const float2 f = unpack_bf16x2(w4[e]);
             const float2 g = unpack_bf16x2(g4[e]);
-            const float c0 = g.x * (f.x * r), c1 = g.y * (f.y * r);
-            hi4[e] = pack_bf16x2(c0, c1);
-            const float2 hb = unpack_bf16x2(hi4[e]);
-            lo4[e] = pack_bf16x2(c0 - hb.x, c1 - hb.y);
+            o4[e] = pack_f16x2(g.x * (f.x * r), g.y * (f.y * r));
           }
-          *ptr = make_uint4(hi4[0], hi4[1], hi4[2], hi4[3]);
-          lo_dst[k0 / 8] = make_uint4(lo4[0], lo4[1], lo4[2], lo4[3]);
+          *ptr = make_uint4(o4[0], o4[1], o4[2], o4[3]);
         }
       }
       fence_proxy_async_smem();
-      fence_proxy_async_global();
     }
     mbar_arrive(&bars.a_ready);
     // rotated shared key of this row (one CTA column per tile writes it)

@@ -203,6 +203,18 @@ __device__ __forceinline__ uint64_t desc_mnmajor_sw128(uint32_t smem_addr, uint3
   return d;
 }
 
+// Shared-memory matrix descriptor of a K-major operand tile without swizzle:
+// 8 x 8 core matrices of 16-byte rows (128 bytes each); the two core matrices
+// of one 16-wide K step are `lbo_bytes` apart and 8-row groups `sbo_bytes`.
+__device__ __forceinline__ uint64_t desc_kmajor_noswz(uint32_t smem_addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr & 0x3FFFFu) >> 4);
+  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
+  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
+  d |= static_cast<uint64_t>(1) << 46;
+  return d;   // swizzle mode 0
+}
+
 // Next 16-element (32-byte) K step inside a 128-byte swizzle row.
 __device__ __forceinline__ uint64_t desc_advance(uint64_t d, uint32_t bytes) { return d + (bytes >> 4); }
 
@@ -213,8 +225,9 @@ __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(N >> 3) << 17) |
          (static_cast<uint32_t>(M >> 4) << 24);
 }
-// Bit 15 of the instruction descriptor: A is MN-major (transposed).
+// Bits 15 / 16 of the instruction descriptor: A / B is MN-major (transposed).
 constexpr uint32_t kIdescAMajorMN = 1u << 15;
+constexpr uint32_t kIdescBMajorMN = 1u << 16;
 __host__ __device__ constexpr uint32_t idesc_f16_f32(int M, int N) {
   return (1u << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (static_cast<uint32_t>(M >> 4) << 24);
 }

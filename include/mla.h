@@ -190,8 +190,8 @@ int mla_cache_append(const mla_dims* dims, const void* latent, const void* w_nor
  *     first call before any stream capture.
  *   - A call whose workspace need (mla_prefill_workspace_size) exceeds
  *     MLA_NOALLOC_SCRATCH_BYTES returns MLA_ERR_WORKSPACE_TOO_SMALL and
- *     launches nothing. About 20 MiB of the array go to per-block scratch
- *     whatever the size; for the Kimi-K2 head geometry the rest holds one
+ *     launches nothing. For the Kimi-K2 head geometry half of the array
+ *     holds the call's fp16 copy of kv_b_proj and the rest holds one
  *     sequence of up to 256 tokens (each sequence is padded to 128-token
  *     tiles, plus one tile per sequence of headroom).
  *   - All calls on a device share the one array, and it keeps what the last
