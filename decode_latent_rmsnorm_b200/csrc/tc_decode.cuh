@@ -18,31 +18,28 @@
 // sum) goes to its own slot, b + cta, and `combine` merges the slots of a
 // sequence by their log-sum-exp.
 //
-// Tensor-core mapping, 32-row cache tiles (32 x 576 bf16 = 36 KB) in a
-// 4-stage TMA ring, so three tiles are in flight while one is computed:
-//   S[h, t] : M = 64 heads, N = 32 rows, K = 576; A = q (resident), B = tile
-//             (K-major); fp32 in TMEM lanes (h % 16) + 32 (h / 16).
-//   O[h, d] : M = 64 heads, N = 256 latent dims (two accumulators, lower and
-//             upper 16 lanes of each quadrant), K = 32 rows; A = P (smem),
-//             B = the same cache tile read MN-major.
+// Tensor-core mapping (M = 128 for both products, the shape tcgen05 runs at
+// full rate; see decode_attn_kernel for the data flow):
+//   S^T[t, h] : M = 128 cache rows, N = 64 heads, K = 576.
+//   O^T[d, h] : M = 128 latent dims (4 blocks), N = 64 heads, K = 128 rows.
 #pragma once
 #include "tc_gemm.cuh"
 
 namespace mla {
 namespace tc {
 
-constexpr int kDecRows = 32;                    // cache rows per tile
-constexpr int kDecStages = 4;                   // TMA ring depth
-constexpr int kDecHeads = 64;                   // heads per CTA (M of S)
+constexpr int kDecRows = 128;                   // cache rows per tile (M of the score MMAs)
+constexpr int kDecHeads = 64;                   // heads per CTA (N of both MMAs)
 constexpr int kDecBoxes = 9;                    // 576 columns = 9 x 64
-constexpr int kDecBoxBytes = kDecRows * 128;    // [32 rows x 64 cols] bf16
-constexpr int kDecTileBytes = kDecBoxes * kDecBoxBytes;
+constexpr int kDecLatBoxes = 8;                 // the 512 latent columns
+constexpr int kDecBoxBytes = kDecRows * 128;    // [128 rows x 64 cols] bf16 = 16 KB
+constexpr int kDecRing = 8;                     // TMA ring slots
 constexpr int kDecQBytes = kDecBoxes * kDecHeads * 128;
-constexpr int kDecPBytes = 2 * kDecHeads * kDecRows * 2;   // two [64 heads x 32 rows] bf16
+constexpr int kDecPBytes = kDecRows * 128;      // P^T [128 rows x 64 heads] bf16
 constexpr int kDecThreads = 192;
-constexpr size_t kDecSmem = (size_t)kDecQBytes + kDecStages * (size_t)kDecTileBytes + kDecPBytes + 1024;
-constexpr int kDecOCol = 0;                     // O: 256 columns (both lane halves)
-constexpr int kDecSCol = 256;                   // S: 2 x 32 columns (M = 64 layout)
+constexpr size_t kDecSmem = (size_t)kDecQBytes + kDecRing * (size_t)kDecBoxBytes + kDecPBytes + 1024;
+constexpr int kDecOCol = 0;                     // O^T: 4 blocks x 64 columns
+constexpr int kDecSCol = 256;                   // S^T: 2 buffers x 64 columns
 
 // ---- split schedule -----------------------------------------------------------
 // prefix[b] = rows of sequences before b (invalid sequences count 0 rows);
@@ -218,24 +215,121 @@ struct DecParams {
   float scale_log2;
 };
 
-struct DecBarriers {
-  uint64_t q_full, q_empty;
-  uint64_t c_full[kDecStages], c_empty[kDecStages];
-  uint64_t s_full[2], s_free[2];     // S double buffer (TMEM)
-  uint64_t p_full[2], pv_done[2];    // P double buffer (smem)
-  uint64_t o_free, mma_done;
-  uint32_t tmem_base;
-  int abort_flag;
+// The (segment, tile) stream every role of a CTA walks in the same order.
+struct DecTile {
+  int seg, b;
+  int64_t row0;      // first cache row of the tile
+  int nvalid;        // rows of the tile inside the segment
+  bool first, last;  // first / last tile of its segment
+};
+struct DecTileIter {
+  DecSegIter segs;
+  const int64_t* offsets;
+  DecSeg cur;
+  bool have;
+  int segi, k, nt;
+  __device__ void init(const DecParams& p, int64_t lo, int64_t hi) {
+    segs.init(p.prefix, p.B, lo, hi);
+    offsets = p.offsets;
+    have = segs.next(cur);
+    segi = 0;
+    k = 0;
+    nt = have ? (int)((cur.hi - cur.lo + kDecRows - 1) / kDecRows) : 0;
+  }
+  __device__ bool next(DecTile& t) {
+    if (!have) return false;
+    t.seg = segi;
+    t.b = cur.b;
+    const int64_t r = cur.lo + (int64_t)k * kDecRows;
+    t.row0 = offsets[cur.b] + r;
+    t.nvalid = (int)min((int64_t)kDecRows, cur.hi - r);
+    t.first = (k == 0);
+    t.last = (k == nt - 1);
+    if (++k == nt) {
+      ++segi;
+      k = 0;
+      have = segs.next(cur);
+      nt = have ? (int)((cur.hi - cur.lo + kDecRows - 1) / kDecRows) : 0;
+    }
+    return true;
+  }
 };
 
+struct DecBarriers {
+  uint64_t q_full, q_empty;
+  uint64_t full[kDecRing], empty[kDecRing];
+  uint64_t s_full[2], s_free[2];     // S^T double buffer (TMEM)
+  uint64_t p_full, pv_done;          // P^T buffer (smem)
+  uint64_t o_free, mma_done;
+  uint64_t sm_sync;                  // bounded barrier of the 128 softmax threads
+  uint32_t tmem_base;
+  int abort_flag;
+  int vote[2][4];                    // per tile parity: a vote is read after one sync, rewritten after two
+  float m_ref[kDecHeads];            // per-head reference max (log2 units)
+  float alpha[kDecHeads];
+  float red[4][kDecHeads];           // per-warp column maxima / sums
+};
+
+// Column reduction of a warp: lane l holds v[0..63] (one value per head) and
+// ends with the reduction over the warp's 32 lanes of heads 2l and 2l + 1
+// (a halving exchange: 32 + 16 + 8 + 4 + 2 shuffles).
+template <bool kMax>
+__device__ __forceinline__ float2 warp_column_reduce(float (&v)[kDecHeads], int lane) {
+#pragma unroll
+  for (int c = 0; c < 32; ++c) {
+    const bool up = lane & 16;
+    const float send = up ? v[c] : v[c + 32];
+    const float keep = up ? v[c + 32] : v[c];
+    const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
+    v[c] = kMax ? fmaxf(keep, recv) : keep + recv;
+  }
+#pragma unroll
+  for (int c = 0; c < 16; ++c) {
+    const bool up = lane & 8;
+    const float send = up ? v[c] : v[c + 16];
+    const float keep = up ? v[c + 16] : v[c];
+    const float recv = __shfl_xor_sync(0xffffffffu, send, 8);
+    v[c] = kMax ? fmaxf(keep, recv) : keep + recv;
+  }
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const bool up = lane & 4;
+    const float send = up ? v[c] : v[c + 8];
+    const float keep = up ? v[c + 8] : v[c];
+    const float recv = __shfl_xor_sync(0xffffffffu, send, 4);
+    v[c] = kMax ? fmaxf(keep, recv) : keep + recv;
+  }
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const bool up = lane & 2;
+    const float send = up ? v[c] : v[c + 4];
+    const float keep = up ? v[c + 4] : v[c];
+    const float recv = __shfl_xor_sync(0xffffffffu, send, 2);
+    v[c] = kMax ? fmaxf(keep, recv) : keep + recv;
+  }
+#pragma unroll
+  for (int c = 0; c < 2; ++c) {
+    const bool up = lane & 1;
+    const float send = up ? v[c] : v[c + 2];
+    const float keep = up ? v[c + 2] : v[c];
+    const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
+    v[c] = kMax ? fmaxf(keep, recv) : keep + recv;
+  }
+  return make_float2(v[0], v[1]);
+}
+
 // One persistent CTA per SM; warp 0 issues TMA loads, warp 1 the MMAs, warps
-// 2-5 run the softmax. TMEM (512 columns):
-//   O[h, d]  (M = 64 accumulators): d < 256 in the lower 16 lanes of each
-//            32-lane quadrant, d >= 256 in the upper 16 lanes, columns 0-255;
-//   S[h, t]  two 32-column buffers at columns 256 and 288, lower lanes.
-// Head h = 16 q + i (quadrant q, lane i < 16) is owned by lanes i and i + 16
-// of warp q: the lower lane runs h's online softmax, both rescale their half
-// of h's O row, so the softmax needs no exchange across warps.
+// 2-5 run the softmax (one cache row per thread: S^T lane = row).
+//   S^T[t, h] = C[t, :] . q[h, :]      M = 128 rows, N = 64 heads, K = 576
+//   O^T[d, h] += C[:, d]^T . P^T[:, h]  M = 128 latent dims (4 blocks), N = 64, K = 128
+// The 128 x 576 tile does not fit next to the resident q (72 KB), so the
+// tile's 16 KB boxes stream through an 8-slot ring twice: all 9 for S^T, the
+// 8 latent ones again (from L2) for O^T. Per tile the stream holds 9 boxes,
+// one empty slot (so latent box pairs start on even slots and an MN-major
+// A operand never wraps around the ring), then the previous tile's 8 latent
+// boxes. The softmax keeps a per-head reference max that it raises only when
+// a score exceeds it by more than 8 (2^8 bounds P), so the common path needs
+// one CTA-wide vote per tile and no column reduction.
 __global__ void __launch_bounds__(kDecThreads, 1)
 decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_constant__ CUtensorMap map_q,
                    DecParams p) {
@@ -249,26 +343,24 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_c
   if (r_lo >= r_hi) return;   // uniform over the CTA
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
-  uint8_t* sC = smem + kDecQBytes;
-  uint8_t* sP = sC + kDecStages * kDecTileBytes;            // 2 x [64 heads x 32 rows], no swizzle
-  constexpr int kPBuf = kDecHeads * kDecRows * 2;           // 4 KB
+  uint8_t* sRing = smem + kDecQBytes;
+  uint8_t* sP = sRing + kDecRing * kDecBoxBytes;
   volatile int* abort_flag = &bars.abort_flag;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars.q_full, 1);
     mbar_init(&bars.q_empty, 1);
-    for (int s = 0; s < kDecStages; ++s) { mbar_init(&bars.c_full[s], 1); mbar_init(&bars.c_empty[s], 1); }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&bars.s_full[b], 1);
-      mbar_init(&bars.s_free[b], 128);
-      mbar_init(&bars.p_full[b], 128);
-      mbar_init(&bars.pv_done[b], 1);
-    }
+    for (int s = 0; s < kDecRing; ++s) { mbar_init(&bars.full[s], 1); mbar_init(&bars.empty[s], 1); }
+    for (int b = 0; b < 2; ++b) { mbar_init(&bars.s_full[b], 1); mbar_init(&bars.s_free[b], 128); }
+    mbar_init(&bars.p_full, 128);
+    mbar_init(&bars.pv_done, 1);
     mbar_init(&bars.o_free, 128);
     mbar_init(&bars.mma_done, 1);
+    mbar_init(&bars.sm_sync, 128);
     bars.abort_flag = 0;
     mbar_fence_init();
   }
+  if (threadIdx.x < kDecHeads) bars.m_ref[threadIdx.x] = -INFINITY;
   if (warp == 1) tmem_alloc(&bars.tmem_base, 512);
   tc_fence_before();
   __syncthreads();
@@ -280,245 +372,277 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_c
     if (lane == 0) {
       tma_prefetch_desc(&map_cache);
       tma_prefetch_desc(&map_q);
-      DecSegIter itr;
-      itr.init(p.prefix, p.B, r_lo, r_hi);
-      DecSeg sg;
-      int it = 0, segi = 0;
+      int it = 0;
       bool ok = true;
-      while (ok && itr.next(sg)) {
-        if (!mbar_wait(&bars.q_empty, ((uint32_t)segi & 1u) ^ 1u, abort_flag)) { ok = false; break; }
-        mbar_arrive_expect_tx(&bars.q_full, kDecQBytes);
-        for (int a = 0; a < kDecBoxes; ++a)
-          tma_load_2d(sQ + a * kDecHeads * 128, &map_q, &bars.q_full, a * 64, sg.b * kDecHeads);
-        const int64_t row0 = p.offsets[sg.b] + sg.lo;
-        const int ntiles = (int)((sg.hi - sg.lo + kDecRows - 1) / kDecRows);
-        for (int k = 0; k < ntiles; ++k, ++it) {
-          const int s = it % kDecStages;
-          if (!mbar_wait(&bars.c_empty[s], ((uint32_t)(it / kDecStages) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
-          mbar_arrive_expect_tx(&bars.c_full[s], kDecTileBytes);
-          uint8_t* st = sC + s * kDecTileBytes;
+      auto push_box = [&](int64_t row0, int a) -> bool {
+        const int s = it % kDecRing;
+        if (!mbar_wait(&bars.empty[s], ((uint32_t)(it / kDecRing) & 1u) ^ 1u, abort_flag)) return false;
+        mbar_arrive_expect_tx(&bars.full[s], kDecBoxBytes);
+        tma_load_2d(sRing + s * kDecBoxBytes, &map_cache, &bars.full[s], a * 64, (int)row0);
+        ++it;
+        return true;
+      };
+      auto push_bubble = [&]() -> bool {
+        const int s = it % kDecRing;
+        if (!mbar_wait(&bars.empty[s], ((uint32_t)(it / kDecRing) & 1u) ^ 1u, abort_flag)) return false;
+        mbar_arrive(&bars.full[s]);
+        ++it;
+        return true;
+      };
+      DecTileIter tiles;
+      tiles.init(p, r_lo, r_hi);
+      DecTile t, prev;
+      bool have_prev = false;
+      while (ok && tiles.next(t)) {
+        if (t.first) {
+          if (!mbar_wait(&bars.q_empty, ((uint32_t)t.seg & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&bars.q_full, kDecQBytes);
           for (int a = 0; a < kDecBoxes; ++a)
-            tma_load_2d(st + a * kDecBoxBytes, &map_cache, &bars.c_full[s], a * 64,
-                        (int)(row0 + (int64_t)k * kDecRows));
+            tma_load_2d(sQ + a * kDecHeads * 128, &map_q, &bars.q_full, a * 64, t.b * kDecHeads);
         }
-        ++segi;
+        for (int a = 0; a < kDecBoxes && ok; ++a) ok = push_box(t.row0, a);
+        if (ok) ok = push_bubble();
+        if (ok && have_prev)
+          for (int a = 0; a < kDecLatBoxes && ok; ++a) ok = push_box(prev.row0, a);
+        prev = t;
+        have_prev = true;
       }
+      if (ok && have_prev)
+        for (int a = 0; a < kDecLatBoxes && ok; ++a) ok = push_box(prev.row0, a);
       if (!ok) {   // let the copies in flight land before the CTA exits
-        if (segi > 0) mbar_wait_drain(&bars.q_full, (uint32_t)(segi - 1) & 1u);
-        for (int i = (it > kDecStages ? it - kDecStages : 0); i < it; ++i)
-          mbar_wait_drain(&bars.c_full[i % kDecStages], (uint32_t)(i / kDecStages) & 1u);
+        mbar_wait_drain(&bars.q_full, 0);
+        for (int i = (it > kDecRing ? it - kDecRing : 0); i < it; ++i)
+          mbar_wait_drain(&bars.full[i % kDecRing], (uint32_t)(i / kDecRing) & 1u);
       }
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer ----------------
     if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16_f32(kDecHeads, kDecRows);
-      const uint32_t idesc_o = idesc_bf16_f32(kDecHeads, 256) | kIdescBMajorMN;
-      // The (segment, tile) items form one stream. S runs two items ahead of
-      // P V: S(j + 2) is issued right after P V(j).
-      struct Item { int seg; bool first, last; };
-      DecSegIter itr;
-      itr.init(p.prefix, p.B, r_lo, r_hi);
-      DecSeg cur;
-      bool have = itr.next(cur);
-      int segi = 0, k_in_seg = 0;
-      int nt = have ? (int)((cur.hi - cur.lo + kDecRows - 1) / kDecRows) : 0;
-      auto next_item = [&](Item& out) -> bool {
-        if (!have) return false;
-        out.seg = segi;
-        out.first = (k_in_seg == 0);
-        out.last = (k_in_seg == nt - 1);
-        if (++k_in_seg == nt) {
-          ++segi;
-          k_in_seg = 0;
-          have = itr.next(cur);
-          nt = have ? (int)((cur.hi - cur.lo + kDecRows - 1) / kDecRows) : 0;
-        }
+      const uint32_t idesc_s = idesc_bf16_f32(kDecRows, kDecHeads);
+      const uint32_t idesc_o = idesc_bf16_f32(128, kDecHeads) | kIdescAMajorMN | kIdescBMajorMN;
+      int it = 0;
+      bool ok = true;
+      auto take = [&](int& slot) -> bool {   // wait for the next ring item
+        slot = it % kDecRing;
+        if (!mbar_wait(&bars.full[slot], (uint32_t)(it / kDecRing) & 1u, abort_flag)) return false;
+        ++it;
         return true;
       };
-      auto issue_s = [&](int j, const Item& itm) -> bool {
-        const int s = j % kDecStages, b = j & 1;
-        if (itm.first && !mbar_wait(&bars.q_full, (uint32_t)itm.seg & 1u, abort_flag)) return false;
-        if (!mbar_wait(&bars.c_full[s], (uint32_t)(j / kDecStages) & 1u, abort_flag)) return false;
+      auto issue_s = [&](int j, const DecTile& t) -> bool {
+        const int b = j & 1;
+        if (t.first && !mbar_wait(&bars.q_full, (uint32_t)t.seg & 1u, abort_flag)) return false;
         if (!mbar_wait(&bars.s_free[b], ((uint32_t)(j >> 1) & 1u) ^ 1u, abort_flag)) return false;
         tc_fence_after();
-        const uint8_t* st = sC + s * kDecTileBytes;
-        const uint32_t s_tmem = tmem + kDecSCol + b * kDecRows;
-#pragma unroll 1
+        const uint32_t d = tmem + kDecSCol + b * kDecHeads;
         for (int a = 0; a < kDecBoxes; ++a) {
+          int slot;
+          if (!take(slot)) return false;
+          tc_fence_after();
+          const uint64_t cd = desc_kmajor_sw128(smem_u32(sRing + slot * kDecBoxBytes));
           const uint64_t qd = desc_kmajor_sw128(smem_u32(sQ + a * kDecHeads * 128));
-          const uint64_t cd = desc_kmajor_sw128(smem_u32(st + a * kDecBoxBytes));
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            mma_bf16_ss(s_tmem, desc_advance(qd, k * 32), desc_advance(cd, k * 32), idesc_s, (a | k) != 0);
+            mma_bf16_ss(d, desc_advance(cd, k * 32), desc_advance(qd, k * 32), idesc_s, (a | k) != 0);
+          mma_commit(&bars.empty[slot]);
         }
         mma_commit(&bars.s_full[b]);
-        if (itm.last) mma_commit(&bars.q_empty);   // q may be replaced once these are done
+        if (t.last) mma_commit(&bars.q_empty);     // q may be replaced once these are done
+        int bslot;                                 // the empty slot of the stream
+        if (!take(bslot)) return false;
+        mbar_arrive(&bars.empty[bslot]);
         return true;
       };
-      auto issue_pv = [&](int j, const Item& itm) -> bool {
-        const int s = j % kDecStages, b = j & 1;
-        if (itm.first && itm.seg > 0 && !mbar_wait(&bars.o_free, (uint32_t)(itm.seg - 1) & 1u, abort_flag))
+      auto issue_pv = [&](int j, const DecTile& t) -> bool {
+        if (t.first && t.seg > 0 && !mbar_wait(&bars.o_free, (uint32_t)(t.seg - 1) & 1u, abort_flag))
           return false;
-        if (!mbar_wait(&bars.p_full[b], (uint32_t)(j >> 1) & 1u, abort_flag)) return false;
+        if (!mbar_wait(&bars.p_full, (uint32_t)j & 1u, abort_flag)) return false;
         tc_fence_after();
-        const uint8_t* st = sC + s * kDecTileBytes;
-        const uint64_t pd = desc_kmajor_noswz(smem_u32(sP + b * kPBuf), 128, 512);
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          // latent columns [256 half, 256 half + 256) = boxes 4 half .. 4 half + 3, read MN-major
-          const uint64_t cd = desc_mnmajor_sw128(smem_u32(st + 4 * half * kDecBoxBytes), kDecBoxBytes, 1024);
-          const uint32_t o_tmem = tmem + kDecOCol + ((uint32_t)(16 * half) << 16);
+        const uint64_t pd = desc_mnmajor_sw128(smem_u32(sP), kDecPBytes, 1024);
+        for (int blk = 0; blk < 4; ++blk) {
+          int s0, s1;
+          if (!take(s0) || !take(s1)) return false;   // s1 == s0 + 1 (even start, never wraps)
+          tc_fence_after();
+          // latent columns [128 blk, 128 blk + 128): the pair of boxes, read MN-major
+          const uint64_t ad = desc_mnmajor_sw128(smem_u32(sRing + s0 * kDecBoxBytes), kDecBoxBytes, 1024);
 #pragma unroll
           for (int k = 0; k < kDecRows / 16; ++k)
-            mma_bf16_ss(o_tmem, desc_advance(pd, k * 256), desc_advance(cd, k * 2048), idesc_o,
-                        (itm.first && k == 0) ? 0u : 1u);
+            mma_bf16_ss(tmem + kDecOCol + blk * kDecHeads, desc_advance(ad, k * 2048), desc_advance(pd, k * 2048),
+                        idesc_o, (t.first && k == 0) ? 0u : 1u);
+          mma_commit(&bars.empty[s0]);
+          mma_commit(&bars.empty[s1]);
         }
-        mma_commit(&bars.c_empty[s]);
-        mma_commit(&bars.pv_done[b]);
+        mma_commit(&bars.pv_done);
         return true;
       };
-      Item win[3];   // items j, j+1, j+2
-      int nwin = 0;
-      for (; nwin < 2 && next_item(win[nwin]); ++nwin) {}
-      bool ok = true;
-      for (int i = 0; i < nwin && ok; ++i) ok = issue_s(i, win[i]);
+      DecTileIter tiles;
+      tiles.init(p, r_lo, r_hi);
+      DecTile t, prev;
       int j = 0;
-      while (ok && nwin > 0) {
-        if (!issue_pv(j, win[0])) break;
-        Item nx;
-        const bool more = next_item(nx);
-        win[0] = win[1];
-        if (more) {
-          win[1] = nx;
-          if (!issue_s(j + 2, nx)) break;
-        } else {
-          --nwin;
-        }
+      bool have_prev = false;
+      while (ok && tiles.next(t)) {
+        if (!(ok = issue_s(j, t))) break;
+        if (have_prev && !(ok = issue_pv(j - 1, prev))) break;
+        prev = t;
+        have_prev = true;
         ++j;
-        if (nwin == 1 && !more) {
-          // one item left (j): its S is issued; finish with its P V
-          if (!issue_pv(j, win[0])) break;
-          break;
-        }
       }
+      if (ok && have_prev) issue_pv(j - 1, prev);
       mma_commit(&bars.mma_done);          // every MMA done before TMEM is freed
       mbar_wait_drain(&bars.mma_done, 0);
     }
   } else {
     // ---------------- softmax / correction / partial epilogue (warps 2-5) ----------------
     const int grp = warp & 3;                       // TMEM quadrant
-    const bool lower = lane < 16;                   // S row owner (M = 64 layout)
-    const int h = grp * 16 + (lane & 15);           // head of this lane pair
+    const int tix = grp * 32 + lane;                // cache row of the tile == O^T latent row
     const uint32_t lane_base = (uint32_t)(grp * 32) << 16;
-    DecSegIter itr;
-    itr.init(p.prefix, p.B, r_lo, r_hi);
-    DecSeg sg;
-    int j = 0, segi = 0;
+    int sync_ph = 0;
+    auto cta_sync = [&]() -> bool {                 // bounded barrier of the 128 softmax threads
+      mbar_arrive(&bars.sm_sync);
+      const bool r = mbar_wait_warp(&bars.sm_sync, (uint32_t)sync_ph & 1u, abort_flag);
+      ++sync_ph;
+      return r;
+    };
+    float lpart[kDecHeads];
+#pragma unroll
+    for (int h = 0; h < kDecHeads; ++h) lpart[h] = 0.f;
+    DecTileIter tiles;
+    tiles.init(p, r_lo, r_hi);
+    DecTile t;
+    int j = 0;
     bool ok = true;
-    while (ok && itr.next(sg)) {
-      const int slot = sg.b + c;
-      const int ntiles = (int)((sg.hi - sg.lo + kDecRows - 1) / kDecRows);
-      float m = -INFINITY, l = 0.f;
-      for (int k = 0; k < ntiles; ++k, ++j) {
-        const int b = j & 1;
-        if (!mbar_wait_warp(&bars.s_full[b], (uint32_t)(j >> 1) & 1u, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        float sc[kDecRows];
-#pragma unroll
-        for (int cc = 0; cc < kDecRows / 16; ++cc) {
-          uint32_t v[16];
-          tmem_ld16(tmem + lane_base + (uint32_t)(kDecSCol + b * kDecRows + cc * 16), v);
-#pragma unroll
-          for (int e = 0; e < 16; ++e) sc[cc * 16 + e] = __uint_as_float(v[e]);
-        }
-        tc_fence_before();
-        mbar_arrive(&bars.s_free[b]);
-        const int64_t t0 = sg.lo + (int64_t)k * kDecRows;
-        const int nvalid = (int)min((int64_t)kDecRows, sg.hi - t0);
-        float mx = -INFINITY;
-#pragma unroll
-        for (int e = 0; e < kDecRows; ++e) {
-          const float x = (e < nvalid) ? sc[e] * p.scale_log2 : -INFINITY;
-          sc[e] = x;
-          mx = fmaxf(mx, x);
-        }
-        // reference max: raised only when the row max grows by more than 8
-        // (P then stays below 2^8), so O is rarely rescaled
-        float alpha = 1.f;
-        bool need = false;
-        if (lower && mx > m + 8.f) {
-          alpha = (m == -INFINITY) ? 0.f : ex2_approx(m - mx);
-          need = (k > 0);
-          m = mx;
-        }
-        uint32_t pk[kDecRows / 2];
-        float rs = 0.f;
-#pragma unroll
-        for (int e = 0; e < kDecRows; e += 2) {
-          pk[e / 2] = pack_bf16x2(ex2_approx(sc[e] - m), ex2_approx(sc[e + 1] - m));
-          const float2 pr = unpack_bf16x2(pk[e / 2]);
-          rs += pr.x + pr.y;
-        }
-        l = l * alpha + rs;
-        // both lanes of a head take the lower lane's alpha
-        const float alpha_h = __shfl_sync(0xffffffffu, alpha, lane & 15);
-        if (__any_sync(0xffffffffu, need)) {
-          // O must be stable: the previous tile's P V is done
-          if (k > 0 && !mbar_wait_warp(&bars.pv_done[(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1u, abort_flag)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-#pragma unroll 1
-          for (int cc = 0; cc < 256 / 16; ++cc) {
-            uint32_t v[16];
-            const uint32_t ta = tmem + lane_base + (uint32_t)(kDecOCol + cc * 16);
-            tmem_ld16(ta, v);
-#pragma unroll
-            for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha_h);
-            tmem_st16(ta, v);
-          }
-          tmem_st_wait();
-        }
-        // P buffer b is free once P V of tile j - 2 is done
-        if (j >= 2 && !mbar_wait_warp(&bars.pv_done[b], (uint32_t)((j - 2) >> 1) & 1u, abort_flag)) {
-          ok = false;
-          break;
-        }
-        if (lower) {
-          // no-swizzle K-major layout: core matrix (h / 8, chunk) at (h / 8) * 512 + chunk * 128
-          uint8_t* prow = sP + b * kPBuf + (h >> 3) * 512 + (h & 7) * 16;
-#pragma unroll
-          for (int cc = 0; cc < kDecRows / 8; ++cc)
-            *reinterpret_cast<uint4*>(prow + cc * 128) = make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
-        }
-        fence_proxy_async_smem();
-        tc_fence_before();
-        mbar_arrive(&bars.p_full[b]);
-      }
-      if (!ok) break;
-      // segment epilogue: unnormalized partial to slot (b + cta)
-      if (!mbar_wait_warp(&bars.pv_done[(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1u, abort_flag)) { ok = false; break; }
+    while (ok && tiles.next(t)) {
+      const int b2 = j & 1;
+      if (!mbar_wait_warp(&bars.s_full[b2], (uint32_t)(j >> 1) & 1u, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      float* op = p.o_part + ((int64_t)slot * p.H + h) * p.R + (lower ? 0 : 256);
-#pragma unroll 1
-      for (int cc = 0; cc < 256 / 16; ++cc) {
+      float x[kDecHeads];
+#pragma unroll
+      for (int cc = 0; cc < kDecHeads / 16; ++cc) {
         uint32_t v[16];
-        tmem_ld16(tmem + lane_base + (uint32_t)(kDecOCol + cc * 16), v);
-        float4* o4 = reinterpret_cast<float4*>(op + cc * 16);
-        o4[0] = make_float4(__uint_as_float(v[0]), __uint_as_float(v[1]), __uint_as_float(v[2]), __uint_as_float(v[3]));
-        o4[1] = make_float4(__uint_as_float(v[4]), __uint_as_float(v[5]), __uint_as_float(v[6]), __uint_as_float(v[7]));
-        o4[2] = make_float4(__uint_as_float(v[8]), __uint_as_float(v[9]), __uint_as_float(v[10]), __uint_as_float(v[11]));
-        o4[3] = make_float4(__uint_as_float(v[12]), __uint_as_float(v[13]), __uint_as_float(v[14]), __uint_as_float(v[15]));
-      }
-      if (lower) {
-        p.m_part[(int64_t)slot * p.H + h] = m;
-        p.l_part[(int64_t)slot * p.H + h] = l;
+        tmem_ld16(tmem + lane_base + (uint32_t)(kDecSCol + b2 * kDecHeads + cc * 16), v);
+#pragma unroll
+        for (int e = 0; e < 16; ++e) x[cc * 16 + e] = __uint_as_float(v[e]);
       }
       tc_fence_before();
-      mbar_arrive(&bars.o_free);
-      ++segi;
+      mbar_arrive(&bars.s_free[b2]);
+      const bool valid = tix < t.nvalid;
+      bool exceed = false;
+#pragma unroll
+      for (int q4 = 0; q4 < kDecHeads / 4; ++q4) {
+        const float4 mr = *reinterpret_cast<const float4*>(&bars.m_ref[q4 * 4]);
+        const float mrv[4] = {mr.x, mr.y, mr.z, mr.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int h = q4 * 4 + e;
+          const float xv = valid ? x[h] * p.scale_log2 : -INFINITY;
+          x[h] = xv;
+          exceed |= xv > mrv[e] + 8.f;
+        }
+      }
+      const unsigned wv = __ballot_sync(0xffffffffu, exceed);
+      if (lane == 0) bars.vote[b2][grp] = wv != 0u;
+      if (!cta_sync()) { ok = false; break; }
+      const bool any = (bars.vote[b2][0] | bars.vote[b2][1] | bars.vote[b2][2] | bars.vote[b2][3]) != 0;
+      bool o_stable = false;
+      if (any) {
+        // rare path: raise the reference max of heads whose scores outgrew it
+        float tmp[kDecHeads];
+#pragma unroll
+        for (int h = 0; h < kDecHeads; ++h) tmp[h] = x[h];
+        const float2 cm = warp_column_reduce<true>(tmp, lane);
+        bars.red[grp][2 * lane] = cm.x;
+        bars.red[grp][2 * lane + 1] = cm.y;
+        if (!cta_sync()) { ok = false; break; }
+        if (tix < kDecHeads) {
+          const float mo = bars.m_ref[tix];
+          const float mt = fmaxf(fmaxf(bars.red[0][tix], bars.red[1][tix]), fmaxf(bars.red[2][tix], bars.red[3][tix]));
+          float a = 1.f;
+          if (mt > mo) {
+            a = (mo == -INFINITY) ? 0.f : ex2_approx(mo - mt);
+            bars.m_ref[tix] = mt;
+          }
+          bars.alpha[tix] = a;
+        }
+        if (!cta_sync()) { ok = false; break; }
+#pragma unroll
+        for (int h = 0; h < kDecHeads; ++h) lpart[h] *= bars.alpha[h];
+        if (!t.first) {
+          // O^T must be stable: the previous tile's P V is done
+          if (!mbar_wait_warp(&bars.pv_done, (uint32_t)(j - 1) & 1u, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          o_stable = true;
+#pragma unroll 1
+          for (int blk = 0; blk < 4; ++blk)
+#pragma unroll 1
+            for (int cc = 0; cc < kDecHeads / 16; ++cc) {
+              uint32_t v[16];
+              const uint32_t ta = tmem + lane_base + (uint32_t)(kDecOCol + blk * kDecHeads + cc * 16);
+              tmem_ld16(ta, v);
+#pragma unroll
+              for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * bars.alpha[cc * 16 + e]);
+              tmem_st16(ta, v);
+            }
+          tmem_st_wait();
+        }
+      }
+      // P^T row of this thread (relative to the reference max), bf16
+      uint32_t pk[kDecHeads / 2];
+#pragma unroll
+      for (int q4 = 0; q4 < kDecHeads / 4; ++q4) {
+        const float4 mr = *reinterpret_cast<const float4*>(&bars.m_ref[q4 * 4]);
+        const uint32_t a0 = pack_bf16x2(ex2_approx(x[q4 * 4] - mr.x), ex2_approx(x[q4 * 4 + 1] - mr.y));
+        const uint32_t a1 = pack_bf16x2(ex2_approx(x[q4 * 4 + 2] - mr.z), ex2_approx(x[q4 * 4 + 3] - mr.w));
+        pk[q4 * 2] = a0;
+        pk[q4 * 2 + 1] = a1;
+        const float2 f0 = unpack_bf16x2(a0), f1 = unpack_bf16x2(a1);
+        lpart[q4 * 4] += f0.x;
+        lpart[q4 * 4 + 1] += f0.y;
+        lpart[q4 * 4 + 2] += f1.x;
+        lpart[q4 * 4 + 3] += f1.y;
+      }
+      // P^T buffer free once the previous tile's P V is done
+      if (j > 0 && !o_stable && !mbar_wait_warp(&bars.pv_done, (uint32_t)(j - 1) & 1u, abort_flag)) {
+        ok = false;
+        break;
+      }
+#pragma unroll
+      for (int cc = 0; cc < 8; ++cc)
+        *reinterpret_cast<uint4*>(sP + sw128_offset(tix, cc)) =
+            make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(&bars.p_full);
+      if (t.last) {
+        // segment epilogue: unnormalized partial to slot (b + cta)
+        const int slot = t.b + c;
+        if (!mbar_wait_warp(&bars.pv_done, (uint32_t)j & 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+#pragma unroll 1
+        for (int blk = 0; blk < 4; ++blk)
+#pragma unroll 1
+          for (int cc = 0; cc < kDecHeads / 16; ++cc) {
+            uint32_t v[16];
+            tmem_ld16(tmem + lane_base + (uint32_t)(kDecOCol + blk * kDecHeads + cc * 16), v);
+#pragma unroll
+            for (int e = 0; e < 16; ++e)
+              p.o_part[((int64_t)slot * p.H + cc * 16 + e) * p.R + blk * 128 + tix] = __uint_as_float(v[e]);
+          }
+        const float2 ls = warp_column_reduce<false>(lpart, lane);
+        bars.red[grp][2 * lane] = ls.x;
+        bars.red[grp][2 * lane + 1] = ls.y;
+        if (!cta_sync()) { ok = false; break; }
+        if (tix < kDecHeads) {
+          p.m_part[(int64_t)slot * p.H + tix] = bars.m_ref[tix];
+          p.l_part[(int64_t)slot * p.H + tix] =
+              bars.red[0][tix] + bars.red[1][tix] + bars.red[2][tix] + bars.red[3][tix];
+          bars.m_ref[tix] = -INFINITY;   // the next segment starts afresh
+        }
+#pragma unroll
+        for (int h = 0; h < kDecHeads; ++h) lpart[h] = 0.f;
+        if (!cta_sync()) { ok = false; break; }
+        tc_fence_before();
+        mbar_arrive(&bars.o_free);
+      }
+      ++j;
     }
   }
   tc_fence_before();
