@@ -33,13 +33,13 @@ constexpr int kDecHeads = 64;                   // heads per CTA (N of both MMAs
 constexpr int kDecBoxes = 9;                    // 576 columns = 9 x 64
 constexpr int kDecLatBoxes = 8;                 // the 512 latent columns
 constexpr int kDecBoxBytes = kDecRows * 128;    // [128 rows x 64 cols] bf16 = 16 KB
-constexpr int kDecRing = 8;                     // TMA ring slots
+constexpr int kDecSlots = kDecBoxes;            // one smem slot per box of a tile
 constexpr int kDecQBytes = kDecBoxes * kDecHeads * 128;
 constexpr int kDecPBytes = kDecRows * 128;      // P^T [128 rows x 64 heads] bf16
 constexpr int kDecThreads = 192;
-constexpr size_t kDecSmem = (size_t)kDecQBytes + kDecRing * (size_t)kDecBoxBytes + kDecPBytes + 1024;
+constexpr size_t kDecSmem = (size_t)kDecQBytes + kDecSlots * (size_t)kDecBoxBytes + 1024;   // P^T reuses the rope slot
 constexpr int kDecOCol = 0;                     // O^T: 4 blocks x 64 columns
-constexpr int kDecSCol = 256;                   // S^T: 2 buffers x 64 columns
+constexpr int kDecSCol = 256;                   // S^T: 64 columns
 
 // ---- split schedule -----------------------------------------------------------
 // prefix[b] = rows of sequences before b (invalid sequences count 0 rows);
@@ -257,9 +257,9 @@ struct DecTileIter {
 
 struct DecBarriers {
   uint64_t q_full, q_empty;
-  uint64_t full[kDecRing], empty[kDecRing];
-  uint64_t s_full[2], s_free[2];     // S^T double buffer (TMEM)
-  uint64_t p_full, pv_done;          // P^T buffer (smem)
+  uint64_t full[kDecSlots], empty[kDecSlots];
+  uint64_t s_full, s_free;           // S^T (TMEM)
+  uint64_t p_full, pv_done;          // P^T (smem, in the rope slot)
   uint64_t o_free, mma_done;
   uint64_t sm_sync;                  // bounded barrier of the 128 softmax threads
   uint32_t tmem_base;
@@ -322,14 +322,14 @@ __device__ __forceinline__ float2 warp_column_reduce(float (&v)[kDecHeads], int 
 // 2-5 run the softmax (one cache row per thread: S^T lane = row).
 //   S^T[t, h] = C[t, :] . q[h, :]      M = 128 rows, N = 64 heads, K = 576
 //   O^T[d, h] += C[:, d]^T . P^T[:, h]  M = 128 latent dims (4 blocks), N = 64, K = 128
-// The 128 x 576 tile does not fit next to the resident q (72 KB), so the
-// tile's 16 KB boxes stream through an 8-slot ring twice: all 9 for S^T, the
-// 8 latent ones again (from L2) for O^T. Per tile the stream holds 9 boxes,
-// one empty slot (so latent box pairs start on even slots and an MN-major
-// A operand never wraps around the ring), then the previous tile's 8 latent
-// boxes. The softmax keeps a per-head reference max that it raises only when
-// a score exceeds it by more than 8 (2^8 bounds P), so the common path needs
-// one CTA-wide vote per tile and no column reduction.
+// Shared memory holds the resident q (72 KB) and one 128 x 576 tile as nine
+// 16 KB boxes, one slot per box. The 8 latent boxes stay from the scores to
+// the latent product; P^T is written into the rope box's slot once the
+// scores have read it. Slots free up block by block as the latent product
+// retires, and the next tile's boxes stream into them right away. The
+// softmax keeps a per-head reference max that it raises only when a score
+// exceeds it by more than 8 (2^8 bounds P), so the common path needs one
+// CTA-wide vote per tile and no column reduction.
 __global__ void __launch_bounds__(kDecThreads, 1)
 decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_constant__ CUtensorMap map_q,
                    DecParams p) {
@@ -343,15 +343,16 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_c
   if (r_lo >= r_hi) return;   // uniform over the CTA
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
-  uint8_t* sRing = smem + kDecQBytes;
-  uint8_t* sP = sRing + kDecRing * kDecBoxBytes;
+  uint8_t* sSlot = smem + kDecQBytes;                       // slot a holds box a of the current tile
+  uint8_t* sP = sSlot + (kDecSlots - 1) * kDecBoxBytes;     // P^T [128 rows x 64 heads] in the rope slot
   volatile int* abort_flag = &bars.abort_flag;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars.q_full, 1);
     mbar_init(&bars.q_empty, 1);
-    for (int s = 0; s < kDecRing; ++s) { mbar_init(&bars.full[s], 1); mbar_init(&bars.empty[s], 1); }
-    for (int b = 0; b < 2; ++b) { mbar_init(&bars.s_full[b], 1); mbar_init(&bars.s_free[b], 128); }
+    for (int a = 0; a < kDecSlots; ++a) { mbar_init(&bars.full[a], 1); mbar_init(&bars.empty[a], 1); }
+    mbar_init(&bars.s_full, 1);
+    mbar_init(&bars.s_free, 128);
     mbar_init(&bars.p_full, 128);
     mbar_init(&bars.pv_done, 1);
     mbar_init(&bars.o_free, 128);
@@ -372,27 +373,11 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_c
     if (lane == 0) {
       tma_prefetch_desc(&map_cache);
       tma_prefetch_desc(&map_q);
-      int it = 0;
       bool ok = true;
-      auto push_box = [&](int64_t row0, int a) -> bool {
-        const int s = it % kDecRing;
-        if (!mbar_wait(&bars.empty[s], ((uint32_t)(it / kDecRing) & 1u) ^ 1u, abort_flag)) return false;
-        mbar_arrive_expect_tx(&bars.full[s], kDecBoxBytes);
-        tma_load_2d(sRing + s * kDecBoxBytes, &map_cache, &bars.full[s], a * 64, (int)row0);
-        ++it;
-        return true;
-      };
-      auto push_bubble = [&]() -> bool {
-        const int s = it % kDecRing;
-        if (!mbar_wait(&bars.empty[s], ((uint32_t)(it / kDecRing) & 1u) ^ 1u, abort_flag)) return false;
-        mbar_arrive(&bars.full[s]);
-        ++it;
-        return true;
-      };
+      int j = 0;
       DecTileIter tiles;
       tiles.init(p, r_lo, r_hi);
-      DecTile t, prev;
-      bool have_prev = false;
+      DecTile t;
       while (ok && tiles.next(t)) {
         if (t.first) {
           if (!mbar_wait(&bars.q_empty, ((uint32_t)t.seg & 1u) ^ 1u, abort_flag)) { ok = false; break; }
@@ -400,19 +385,16 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_c
           for (int a = 0; a < kDecBoxes; ++a)
             tma_load_2d(sQ + a * kDecHeads * 128, &map_q, &bars.q_full, a * 64, t.b * kDecHeads);
         }
-        for (int a = 0; a < kDecBoxes && ok; ++a) ok = push_box(t.row0, a);
-        if (ok) ok = push_bubble();
-        if (ok && have_prev)
-          for (int a = 0; a < kDecLatBoxes && ok; ++a) ok = push_box(prev.row0, a);
-        prev = t;
-        have_prev = true;
+        for (int a = 0; a < kDecBoxes; ++a) {   // latent boxes first: they free up first
+          if (!mbar_wait(&bars.empty[a], ((uint32_t)j & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&bars.full[a], kDecBoxBytes);
+          tma_load_2d(sSlot + a * kDecBoxBytes, &map_cache, &bars.full[a], a * 64, (int)t.row0);
+        }
+        ++j;
       }
-      if (ok && have_prev)
-        for (int a = 0; a < kDecLatBoxes && ok; ++a) ok = push_box(prev.row0, a);
       if (!ok) {   // let the copies in flight land before the CTA exits
         mbar_wait_drain(&bars.q_full, 0);
-        for (int i = (it > kDecRing ? it - kDecRing : 0); i < it; ++i)
-          mbar_wait_drain(&bars.full[i % kDecRing], (uint32_t)(i / kDecRing) & 1u);
+        for (int a = 0; a < kDecSlots; ++a) mbar_wait_drain(&bars.full[a], (uint32_t)(j > 0 ? j - 1 : 0) & 1u);
       }
     }
   } else if (warp == 1) {
@@ -420,73 +402,48 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_c
     if (lane == 0) {
       const uint32_t idesc_s = idesc_bf16_f32(kDecRows, kDecHeads);
       const uint32_t idesc_o = idesc_bf16_f32(128, kDecHeads) | kIdescAMajorMN | kIdescBMajorMN;
-      int it = 0;
       bool ok = true;
-      auto take = [&](int& slot) -> bool {   // wait for the next ring item
-        slot = it % kDecRing;
-        if (!mbar_wait(&bars.full[slot], (uint32_t)(it / kDecRing) & 1u, abort_flag)) return false;
-        ++it;
-        return true;
-      };
-      auto issue_s = [&](int j, const DecTile& t) -> bool {
-        const int b = j & 1;
-        if (t.first && !mbar_wait(&bars.q_full, (uint32_t)t.seg & 1u, abort_flag)) return false;
-        if (!mbar_wait(&bars.s_free[b], ((uint32_t)(j >> 1) & 1u) ^ 1u, abort_flag)) return false;
+      int j = 0;
+      DecTileIter tiles;
+      tiles.init(p, r_lo, r_hi);
+      DecTile t;
+      while (ok && tiles.next(t)) {
+        const uint32_t ph = (uint32_t)j & 1u;
+        // ---- S^T(j) ----
+        if (t.first && !(ok = mbar_wait(&bars.q_full, (uint32_t)t.seg & 1u, abort_flag))) break;
+        if (!(ok = mbar_wait(&bars.s_free, ph ^ 1u, abort_flag))) break;
         tc_fence_after();
-        const uint32_t d = tmem + kDecSCol + b * kDecHeads;
-        for (int a = 0; a < kDecBoxes; ++a) {
-          int slot;
-          if (!take(slot)) return false;
+        for (int a = 0; a < kDecBoxes && ok; ++a) {
+          if (!(ok = mbar_wait(&bars.full[a], ph, abort_flag))) break;
           tc_fence_after();
-          const uint64_t cd = desc_kmajor_sw128(smem_u32(sRing + slot * kDecBoxBytes));
+          const uint64_t cd = desc_kmajor_sw128(smem_u32(sSlot + a * kDecBoxBytes));
           const uint64_t qd = desc_kmajor_sw128(smem_u32(sQ + a * kDecHeads * 128));
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            mma_bf16_ss(d, desc_advance(cd, k * 32), desc_advance(qd, k * 32), idesc_s, (a | k) != 0);
-          mma_commit(&bars.empty[slot]);
+            mma_bf16_ss(tmem + kDecSCol, desc_advance(cd, k * 32), desc_advance(qd, k * 32), idesc_s, (a | k) != 0);
         }
-        mma_commit(&bars.s_full[b]);
+        if (!ok) break;
+        mma_commit(&bars.s_full);
         if (t.last) mma_commit(&bars.q_empty);     // q may be replaced once these are done
-        int bslot;                                 // the empty slot of the stream
-        if (!take(bslot)) return false;
-        mbar_arrive(&bars.empty[bslot]);
-        return true;
-      };
-      auto issue_pv = [&](int j, const DecTile& t) -> bool {
-        if (t.first && t.seg > 0 && !mbar_wait(&bars.o_free, (uint32_t)(t.seg - 1) & 1u, abort_flag))
-          return false;
-        if (!mbar_wait(&bars.p_full, (uint32_t)j & 1u, abort_flag)) return false;
+        // ---- O^T(j) += C^T P^T ----
+        if (t.first && t.seg > 0 && !(ok = mbar_wait(&bars.o_free, (uint32_t)(t.seg - 1) & 1u, abort_flag))) break;
+        if (!(ok = mbar_wait(&bars.p_full, ph, abort_flag))) break;
         tc_fence_after();
-        const uint64_t pd = desc_mnmajor_sw128(smem_u32(sP), kDecPBytes, 1024);
+        const uint64_t pd = desc_mnmajor_sw128(smem_u32(sP), kDecBoxBytes, 1024);
         for (int blk = 0; blk < 4; ++blk) {
-          int s0, s1;
-          if (!take(s0) || !take(s1)) return false;   // s1 == s0 + 1 (even start, never wraps)
-          tc_fence_after();
-          // latent columns [128 blk, 128 blk + 128): the pair of boxes, read MN-major
-          const uint64_t ad = desc_mnmajor_sw128(smem_u32(sRing + s0 * kDecBoxBytes), kDecBoxBytes, 1024);
+          // latent columns [128 blk, 128 blk + 128): slots 2 blk, 2 blk + 1, read MN-major
+          const uint64_t ad = desc_mnmajor_sw128(smem_u32(sSlot + 2 * blk * kDecBoxBytes), kDecBoxBytes, 1024);
 #pragma unroll
           for (int k = 0; k < kDecRows / 16; ++k)
             mma_bf16_ss(tmem + kDecOCol + blk * kDecHeads, desc_advance(ad, k * 2048), desc_advance(pd, k * 2048),
                         idesc_o, (t.first && k == 0) ? 0u : 1u);
-          mma_commit(&bars.empty[s0]);
-          mma_commit(&bars.empty[s1]);
+          mma_commit(&bars.empty[2 * blk]);
+          mma_commit(&bars.empty[2 * blk + 1]);
         }
+        mma_commit(&bars.empty[kDecSlots - 1]);    // P^T read: the rope slot is free
         mma_commit(&bars.pv_done);
-        return true;
-      };
-      DecTileIter tiles;
-      tiles.init(p, r_lo, r_hi);
-      DecTile t, prev;
-      int j = 0;
-      bool have_prev = false;
-      while (ok && tiles.next(t)) {
-        if (!(ok = issue_s(j, t))) break;
-        if (have_prev && !(ok = issue_pv(j - 1, prev))) break;
-        prev = t;
-        have_prev = true;
         ++j;
       }
-      if (ok && have_prev) issue_pv(j - 1, prev);
       mma_commit(&bars.mma_done);          // every MMA done before TMEM is freed
       mbar_wait_drain(&bars.mma_done, 0);
     }
@@ -512,18 +469,18 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_c
     bool ok = true;
     while (ok && tiles.next(t)) {
       const int b2 = j & 1;
-      if (!mbar_wait_warp(&bars.s_full[b2], (uint32_t)(j >> 1) & 1u, abort_flag)) { ok = false; break; }
+      if (!mbar_wait_warp(&bars.s_full, (uint32_t)j & 1u, abort_flag)) { ok = false; break; }
       tc_fence_after();
       float x[kDecHeads];
 #pragma unroll
       for (int cc = 0; cc < kDecHeads / 16; ++cc) {
         uint32_t v[16];
-        tmem_ld16(tmem + lane_base + (uint32_t)(kDecSCol + b2 * kDecHeads + cc * 16), v);
+        tmem_ld16(tmem + lane_base + (uint32_t)(kDecSCol + cc * 16), v);
 #pragma unroll
         for (int e = 0; e < 16; ++e) x[cc * 16 + e] = __uint_as_float(v[e]);
       }
       tc_fence_before();
-      mbar_arrive(&bars.s_free[b2]);
+      mbar_arrive(&bars.s_free);
       const bool valid = tix < t.nvalid;
       bool exceed = false;
 #pragma unroll
@@ -542,7 +499,6 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_c
       if (lane == 0) bars.vote[b2][grp] = wv != 0u;
       if (!cta_sync()) { ok = false; break; }
       const bool any = (bars.vote[b2][0] | bars.vote[b2][1] | bars.vote[b2][2] | bars.vote[b2][3]) != 0;
-      bool o_stable = false;
       if (any) {
         // rare path: raise the reference max of heads whose scores outgrew it
         float tmp[kDecHeads];
@@ -566,10 +522,7 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_c
 #pragma unroll
         for (int h = 0; h < kDecHeads; ++h) lpart[h] *= bars.alpha[h];
         if (!t.first) {
-          // O^T must be stable: the previous tile's P V is done
-          if (!mbar_wait_warp(&bars.pv_done, (uint32_t)(j - 1) & 1u, abort_flag)) { ok = false; break; }
-          tc_fence_after();
-          o_stable = true;
+          // O^T holds the segment's earlier tiles (their P V finished before S^T(j) began)
 #pragma unroll 1
           for (int blk = 0; blk < 4; ++blk)
 #pragma unroll 1
@@ -584,7 +537,7 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_c
           tmem_st_wait();
         }
       }
-      // P^T row of this thread (relative to the reference max), bf16
+      // P^T row of this thread (relative to the reference max), bf16, into the rope slot
       uint32_t pk[kDecHeads / 2];
 #pragma unroll
       for (int q4 = 0; q4 < kDecHeads / 4; ++q4) {
@@ -598,11 +551,6 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_c
         lpart[q4 * 4 + 1] += f0.y;
         lpart[q4 * 4 + 2] += f1.x;
         lpart[q4 * 4 + 3] += f1.y;
-      }
-      // P^T buffer free once the previous tile's P V is done
-      if (j > 0 && !o_stable && !mbar_wait_warp(&bars.pv_done, (uint32_t)(j - 1) & 1u, abort_flag)) {
-        ok = false;
-        break;
       }
 #pragma unroll
       for (int cc = 0; cc < 8; ++cc)
