@@ -205,7 +205,7 @@ size_t prefill_ws_bytes(const mla_dims* d, int64_t T, int nseq) {
 // Shapes the tensor-core decode takes (bf16, 64 heads, 512 + 64 latent row).
 bool decode_tc_shape(const mla_dims* d) {
   return d->dtype == MLA_BF16 && d->num_heads == mla::tc::kDecHeads && d->kv_lora_rank == 512 &&
-         d->qk_rope == 64;
+         d->qk_rope == 64 && d->qk_nope % 64 == 0 && d->qk_nope >= 64;
 }
 
 int g_num_sms[64] = {};
@@ -242,7 +242,7 @@ DecodeWs decode_ws_layout(const mla_dims* d, int B, int max_len, bool tc) {
     w.o_part = off; off = align_up(off + 4 * slots * H * R, 256);
     w.m_part = off; off = align_up(off + 4 * slots * H, 256);
     w.l_part = off; off = align_up(off + 4 * slots * H, 256);
-    w.o_lat = off;  off = align_up(off + 4 * (size_t)B * H * R, 256);
+    w.o_lat = off;  off = align_up(off + 2 * (size_t)B * H * R, 256);
     w.total = off;
     return w;
   }
@@ -517,7 +517,7 @@ int launch_decode_tc(const mla_dims* d, const void* q, const void* cache, int64_
   float* o_part = reinterpret_cast<float*>(ws + L.o_part);
   float* m_part = reinterpret_cast<float*>(ws + L.m_part);
   float* l_part = reinterpret_cast<float*>(ws + L.l_part);
-  float* o_lat = reinterpret_cast<float*>(ws + L.o_lat);
+  bf16* o_lat = reinterpret_cast<bf16*>(ws + L.o_lat);
 
   CUtensorMap map_cache, map_q;
   {
@@ -538,12 +538,51 @@ int launch_decode_tc(const mla_dims* d, const void* q, const void* cache, int64_
   T::decode_schedule_kernel<<<1, 1024, 0, st>>>(lens, offsets, B, max_len, cache_rows, L.G, prefix, meta);
   prof_end(st);
 
-  // q_lat[b, h, :] = q_nope[b, h, :] W_UK_h  (W_UK_h rows j < N of head h: [N, R], R contiguous)
-  prof_begin(st, "tc_decode_qabsorb");
-  T::small_gemm_kernel<bf16, true><<<dim3(H, R / T::kSgBN, (B + T::kSgBM - 1) / T::kSgBM), 256, 0, st>>>(
-      static_cast<const bf16*>(q), (int64_t)H * (N + P), (int64_t)(N + P), static_cast<const bf16*>(w_kvb),
-      (int64_t)(N + V) * R, (int64_t)R, qf, (int64_t)H * (R + P), (int64_t)(R + P), B, R, N);
-  prof_end(st);
+  // q_lat[b, h, :] = q_nope[b, h, :] W_UK_h   (W_UK_h = rows j < N of head h: [N, R], R contiguous)
+  CUtensorMap map_wk, map_qn, map_wv, map_ol;
+  {
+    const uint64_t dims[2] = {(uint64_t)R, (uint64_t)H * (N + V)};
+    const uint64_t strides[1] = {(uint64_t)R * 2};
+    const uint32_t box[2] = {64, 64};
+    int rc = make_map(&map_wk, w_kvb, 2, dims, strides, box);
+    if (rc) return rc;
+    const uint32_t box2[2] = {64, 128};
+    rc = make_map(&map_wv, w_kvb, 2, dims, strides, box2);
+    if (rc) return rc;
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)(N + P), (uint64_t)H, (uint64_t)B};
+    const uint64_t strides[2] = {(uint64_t)(N + P) * 2, (uint64_t)H * (N + P) * 2};
+    const uint32_t box[3] = {64, 1, 64};
+    int rc = make_map(&map_qn, q, 3, dims, strides, box);
+    if (rc) return rc;
+  }
+  {
+    const uint64_t dims[3] = {(uint64_t)R, (uint64_t)H, (uint64_t)B};
+    const uint64_t strides[2] = {(uint64_t)R * 2, (uint64_t)H * R * 2};
+    const uint32_t box[3] = {64, 1, 64};
+    int rc = make_map(&map_ol, o_lat, 3, dims, strides, box);
+    if (rc) return rc;
+  }
+  cudaError_t e = cudaFuncSetAttribute(T::head_gemm_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)T::kHgSmem);
+  if (e != cudaSuccess) return cuda_status(e, "head gemm smem attribute");
+  e = cudaFuncSetAttribute(T::head_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)T::kHgSmem);
+  if (e != cudaSuccess) return cuda_status(e, "head gemm smem attribute");
+  {
+    T::HgParams hp;
+    hp.out = qf;
+    hp.out_bs = (int64_t)H * (R + P);
+    hp.out_hs = R + P;
+    hp.B = B;
+    hp.Nout = R;
+    hp.K = N;
+    hp.a_row0 = 0;
+    hp.a_hstride = N + V;
+    prof_begin(st, "tc_decode_qabsorb");
+    T::head_gemm_kernel<true><<<dim3(H, R / 128, (B + 63) / 64), 192, T::kHgSmem, st>>>(map_wk, map_qn, hp);
+    prof_end(st);
+  }
   const int64_t nrope = (int64_t)B * H * (P / 2);
   prof_begin(st, "tc_decode_qrope");
   T::decode_qrope_kernel<<<(unsigned)((nrope + 255) / 256), 256, 0, st>>>(static_cast<const bf16*>(q), positions,
@@ -562,23 +601,31 @@ int launch_decode_tc(const mla_dims* d, const void* q, const void* cache, int64_
   dp.H = H;
   dp.R = R;
   dp.scale_log2 = d->softmax_scale * 1.4426950408889634f;
-  cudaError_t e = cudaFuncSetAttribute(T::decode_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)T::kDecSmem);
+  e = cudaFuncSetAttribute(T::decode_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)T::kDecSmem);
   if (e != cudaSuccess) return cuda_status(e, "decode smem attribute");
   prof_begin(st, "tc_decode_attention");
   T::decode_attn_kernel<<<L.G, T::kDecThreads, T::kDecSmem, st>>>(map_cache, map_q, dp);
   prof_end(st);
 
   prof_begin(st, "tc_decode_combine");
-  T::decode_combine_kernel<<<dim3(B, H), 128, 0, st>>>(o_part, m_part, l_part, prefix, meta, H, R, o_lat);
+  T::decode_combine_kernel<<<dim3(B, (H + 3) / 4), 256, 0, st>>>(o_part, m_part, l_part, prefix, meta, H, R, o_lat);
   prof_end(st);
 
-  // out[b, h, :] = W_UV_h o_lat[b, h, :]  (W_UV_h rows N.. N+V-1 of head h: [V, R], R contiguous)
-  prof_begin(st, "tc_decode_unabsorb");
-  T::small_gemm_kernel<float, false><<<dim3(H, (V + T::kSgBN - 1) / T::kSgBN, (B + T::kSgBM - 1) / T::kSgBM), 256, 0,
-                                       st>>>(o_lat, (int64_t)H * R, (int64_t)R,
-                                             static_cast<const bf16*>(w_kvb) + (int64_t)N * R, (int64_t)(N + V) * R,
-                                             (int64_t)R, static_cast<bf16*>(out), (int64_t)H * V, (int64_t)V, B, V, R);
-  prof_end(st);
+  // out[b, h, :] = W_UV_h o_lat[b, h, :]   (W_UV_h = rows N .. N+V-1 of head h: [V, R], R contiguous)
+  {
+    T::HgParams hp;
+    hp.out = static_cast<bf16*>(out);
+    hp.out_bs = (int64_t)H * V;
+    hp.out_hs = V;
+    hp.B = B;
+    hp.Nout = V;
+    hp.K = R;
+    hp.a_row0 = N;
+    hp.a_hstride = N + V;
+    prof_begin(st, "tc_decode_unabsorb");
+    T::head_gemm_kernel<false><<<dim3(H, (V + 127) / 128, (B + 63) / 64), 192, T::kHgSmem, st>>>(map_wv, map_ol, hp);
+    prof_end(st);
+  }
   return cuda_status(cudaGetLastError(), "decode launch");
 }
 

@@ -80,73 +80,6 @@ decode_schedule_kernel(const int32_t* __restrict__ lens, const int64_t* __restri
   }
 }
 
-// ---- per-head batched GEMM on CUDA cores (q absorption, un-absorption) ----------
-// For head h (grid x) and a 64-column block (grid y) and 64-row block (grid z):
-//   C[m, n] = sum_k A[m, k] * Bm[k, n]   (fp32 accumulate, bf16 output)
-// with A[m, k] = a[m * a_ms + h * a_hs + k] and
-//   b_kn = true : Bm[k, n] = w[h * w_hs + k * w_ks + n]   (rows k, n contiguous)
-//   b_kn = false: Bm[k, n] = w[h * w_hs + n * w_ks + k]   (rows n, k contiguous)
-// C[m, n] goes to c[m * c_ms + h * c_hs + n]. 256 threads, 4 x 4 outputs per
-// thread, K in chunks of 32 staged in smem ([k][m], [k][n], fp32).
-constexpr int kSgBM = 64, kSgBN = 64, kSgBK = 32, kSgPad = 68;
-template <typename TA, bool kBKN>
-__global__ void __launch_bounds__(256)
-small_gemm_kernel(const TA* __restrict__ a, int64_t a_ms, int64_t a_hs, const __nv_bfloat16* __restrict__ w,
-                  int64_t w_hs, int64_t w_ks, __nv_bfloat16* __restrict__ cout, int64_t c_ms, int64_t c_hs,
-                  int M, int N, int K) {
-  __shared__ __align__(16) float sA[kSgBK][kSgPad];
-  __shared__ __align__(16) float sB[kSgBK][kSgPad];
-  const int h = blockIdx.x, n0 = blockIdx.y * kSgBN, m0 = blockIdx.z * kSgBM;
-  const int tid = threadIdx.x;
-  const int tm = (tid >> 4) * 4, tn = (tid & 15) * 4;
-  float acc[4][4] = {};
-  const TA* ah = a + (int64_t)h * a_hs;
-  const __nv_bfloat16* wh = w + (int64_t)h * w_hs;
-  for (int k0 = 0; k0 < K; k0 += kSgBK) {
-    __syncthreads();
-    for (int e = tid; e < kSgBM * kSgBK; e += 256) {          // A chunk, k fastest (coalesced)
-      const int mm = e / kSgBK, kk = e % kSgBK;
-      const int m = m0 + mm, k = k0 + kk;
-      float v = 0.f;
-      if (m < M && k < K) v = to_f32(ah[(int64_t)m * a_ms + k]);
-      sA[kk][mm] = v;
-    }
-    for (int e = tid; e < kSgBN * kSgBK; e += 256) {
-      int nn, kk;
-      if (kBKN) { kk = e / kSgBN; nn = e % kSgBN; } else { nn = e / kSgBK; kk = e % kSgBK; }
-      const int n = n0 + nn, k = k0 + kk;
-      float v = 0.f;
-      if (n < N && k < K) v = __bfloat162float(kBKN ? wh[(int64_t)k * w_ks + n] : wh[(int64_t)n * w_ks + k]);
-      sB[kk][nn] = v;
-    }
-    __syncthreads();
-#pragma unroll 8
-    for (int kk = 0; kk < kSgBK; ++kk) {
-      const float4 av = *reinterpret_cast<const float4*>(&sA[kk][tm]);
-      const float4 bv = *reinterpret_cast<const float4*>(&sB[kk][tn]);
-      const float ar[4] = {av.x, av.y, av.z, av.w}, br[4] = {bv.x, bv.y, bv.z, bv.w};
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int jx = 0; jx < 4; ++jx) acc[i][jx] = fmaf(ar[i], br[jx], acc[i][jx]);
-    }
-  }
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int m = m0 + tm + i;
-    if (m >= M) continue;
-    __nv_bfloat16* dst = cout + (int64_t)m * c_ms + (int64_t)h * c_hs + n0 + tn;
-    if (n0 + tn + 3 < N) {
-      uint2 v2 = make_uint2(pack_bf16x2(acc[i][0], acc[i][1]), pack_bf16x2(acc[i][2], acc[i][3]));
-      *reinterpret_cast<uint2*>(dst) = v2;
-    } else {
-#pragma unroll
-      for (int jx = 0; jx < 4; ++jx)
-        if (n0 + tn + jx < N) dst[jx] = __float2bfloat16_rn(acc[i][jx]);
-    }
-  }
-}
-
 // q_pe rotated at the query position, into the last P columns of qf rows.
 __global__ void decode_qrope_kernel(const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ positions,
                                     const float* __restrict__ cos_t, const float* __restrict__ sin_t, int max_pos,
@@ -603,36 +536,159 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_c
 
 // ---- merge the partials of each (b, h) ----------------------------------------
 // o_lat[b, h, :] = sum_s 2^(m_s - M) o_s / sum_s 2^(m_s - M) l_s over the slots
-// b + c of the CTAs c whose ranges touch sequence b.
-__global__ void __launch_bounds__(128)
+// b + c of the CTAs c whose ranges touch sequence b. One block per (b, 4
+// heads), 8 latent values per thread; output bf16 (the MMA operand of the
+// un-absorption).
+__global__ void __launch_bounds__(256)
 decode_combine_kernel(const float* __restrict__ o_part, const float* __restrict__ m_part,
                       const float* __restrict__ l_part, const int64_t* __restrict__ prefix,
-                      const int64_t* __restrict__ meta, int H, int R, float* __restrict__ o_lat) {
-  const int b = blockIdx.x, h = blockIdx.y;
+                      const int64_t* __restrict__ meta, int H, int R, __nv_bfloat16* __restrict__ o_lat) {
+  const int b = blockIdx.x;
+  const int h = blockIdx.y * 4 + (threadIdx.x >> 6);
+  const int d0 = (threadIdx.x & 63) * 8;
+  if (h >= H || d0 >= R) return;
   const int64_t per = meta[0];
   const int64_t p0 = prefix[b], p1 = prefix[b + 1];
-  float* dst = o_lat + ((int64_t)b * H + h) * R;
+  uint4* dst = reinterpret_cast<uint4*>(o_lat + ((int64_t)b * H + h) * R + d0);
   if (p1 <= p0 || per <= 0) {   // a skipped sequence: no row to attend
-    for (int d = threadIdx.x; d < R; d += blockDim.x) dst[d] = 0.f;
+    *dst = make_uint4(0, 0, 0, 0);
     return;
   }
   const int c0 = (int)(p0 / per), c1 = (int)((p1 - 1) / per);
   float M = -INFINITY;
   for (int cc = c0; cc <= c1; ++cc) M = fmaxf(M, m_part[(int64_t)(b + cc) * H + h]);
-  float Lsum = 0.f;
+  float Lsum = 0.f, acc[8] = {};
   for (int cc = c0; cc <= c1; ++cc) {
-    const float ms = m_part[(int64_t)(b + cc) * H + h];
-    Lsum += (ms == -INFINITY ? 0.f : exp2f(ms - M)) * l_part[(int64_t)(b + cc) * H + h];
+    const int64_t slot = b + cc;
+    const float ms = m_part[slot * H + h];
+    if (ms == -INFINITY) continue;
+    const float w = ex2_approx(ms - M);
+    Lsum = fmaf(w, l_part[slot * H + h], Lsum);
+    const float4* src = reinterpret_cast<const float4*>(o_part + (slot * H + h) * R + d0);
+    const float4 a = src[0], bq = src[1];
+    acc[0] = fmaf(w, a.x, acc[0]); acc[1] = fmaf(w, a.y, acc[1]);
+    acc[2] = fmaf(w, a.z, acc[2]); acc[3] = fmaf(w, a.w, acc[3]);
+    acc[4] = fmaf(w, bq.x, acc[4]); acc[5] = fmaf(w, bq.y, acc[5]);
+    acc[6] = fmaf(w, bq.z, acc[6]); acc[7] = fmaf(w, bq.w, acc[7]);
   }
   const float inv = 1.f / Lsum;
-  for (int d = threadIdx.x; d < R; d += blockDim.x) {
-    float a = 0.f;
-    for (int cc = c0; cc <= c1; ++cc) {
-      const int64_t slot = b + cc;
-      const float ms = m_part[slot * H + h];
-      if (ms != -INFINITY) a = fmaf(exp2f(ms - M), o_part[(slot * H + h) * R + d], a);
+  *dst = make_uint4(pack_bf16x2(acc[0] * inv, acc[1] * inv), pack_bf16x2(acc[2] * inv, acc[3] * inv),
+                    pack_bf16x2(acc[4] * inv, acc[5] * inv), pack_bf16x2(acc[6] * inv, acc[7] * inv));
+}
+
+// ---- per-head GEMM on tensor cores (q absorption, un-absorption) -----------------
+// For head h (grid x), a block of 128 output features n (grid y) and a block of
+// 64 batch rows b (grid z):   out[b, n] = sum_k A_h[n, k] Bm[b, k]
+// A_h is a weight slice of kv_b_proj, Bm the per-head activations. On the
+// tensor core it is D^T[n, b] = A[n, :] . Bm[b, :] with M = 128 (n), N = 64 (b):
+//   kAMN = true : A is read MN-major (the weight stored [k][n]: W_UK_h), its
+//                 TMA box [64 k x 64 n] twice per 64-wide K chunk;
+//   kAMN = false: A is read K-major (the weight stored [n][k]: W_UV_h), its box
+//                 [128 n x 64 k] per K chunk.
+// Bm comes through a 3D map {K, H, B} as [64 b x 64 k] boxes. The output row
+// of b is out[b * out_bs + h * out_hs + n] (bf16).
+constexpr int kHgStages = 4;
+constexpr int kHgABytes = 128 * 128;            // 128 n x 64 k bf16
+constexpr int kHgBBytes = 64 * 128;             // 64 b x 64 k bf16
+constexpr size_t kHgSmem = (size_t)kHgStages * (kHgABytes + kHgBBytes) + 1024;
+
+struct HgParams {
+  __nv_bfloat16* out;
+  int64_t out_bs, out_hs;
+  int B, Nout, K;
+  int a_row0;            // first weight row of head h: a_row0 + h * a_hstride
+  int a_hstride;
+};
+
+template <bool kAMN>
+__global__ void __launch_bounds__(192, 1)
+head_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b, HgParams p) {
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ uint64_t full[kHgStages], empty[kHgStages], done;
+  __shared__ uint32_t tmem_base;
+  __shared__ int abort_flag;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int h = blockIdx.x, n0 = blockIdx.y * 128, b0 = blockIdx.z * 64;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kHgStages * kHgABytes;
+  const int nk = p.K / 64;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kHgStages; ++s) { mbar_init(&full[s], 1); mbar_init(&empty[s], 1); }
+    mbar_init(&done, 1);
+    abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 1) tmem_alloc(&tmem_base, 64);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = tmem_base;
+  const int arow = p.a_row0 + h * p.a_hstride;
+  if (warp == 0) {
+    if (lane == 0) {
+      int kc = 0;
+      bool ok = true;
+      for (; kc < nk; ++kc) {
+        const int s = kc % kHgStages;
+        if (!mbar_wait(&empty[s], ((uint32_t)(kc / kHgStages) & 1u) ^ 1u, &abort_flag)) { ok = false; break; }
+        mbar_arrive_expect_tx(&full[s], kHgABytes + kHgBBytes);
+        uint8_t* a = sA + s * kHgABytes;
+        if (kAMN) {   // rows k, columns n: two [64 k x 64 n] boxes
+          tma_load_2d(a, &map_a, &full[s], n0, arow + kc * 64);
+          tma_load_2d(a + kHgABytes / 2, &map_a, &full[s], n0 + 64, arow + kc * 64);
+        } else {      // rows n, columns k: one [128 n x 64 k] box
+          tma_load_2d(a, &map_a, &full[s], kc * 64, arow + n0);
+        }
+        tma_load_3d(sB + s * kHgBBytes, &map_b, &full[s], kc * 64, h, b0);
+      }
+      if (!ok)
+        for (int i = (kc > kHgStages ? kc - kHgStages : 0); i < kc; ++i)
+          mbar_wait_drain(&full[i % kHgStages], (uint32_t)(i / kHgStages) & 1u);
     }
-    dst[d] = a * inv;
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16_f32(128, 64) | (kAMN ? kIdescAMajorMN : 0u);
+      for (int kc = 0; kc < nk; ++kc) {
+        const int s = kc % kHgStages;
+        if (!mbar_wait(&full[s], (uint32_t)(kc / kHgStages) & 1u, &abort_flag)) break;
+        tc_fence_after();
+        const uint32_t aaddr = smem_u32(sA + s * kHgABytes);
+        const uint64_t ad = kAMN ? desc_mnmajor_sw128(aaddr, kHgABytes / 2, 1024) : desc_kmajor_sw128(aaddr);
+        const uint64_t bd = desc_kmajor_sw128(smem_u32(sB + s * kHgBBytes));
+#pragma unroll
+        for (int k = 0; k < 4; ++k)
+          mma_bf16_ss(tmem, desc_advance(ad, kAMN ? k * 2048 : k * 32), desc_advance(bd, k * 32), idesc,
+                      (kc | k) != 0);
+        mma_commit(&empty[s]);
+      }
+      mma_commit(&done);
+      mbar_wait_drain(&done, 0);
+    }
+  } else {
+    const int grp = warp & 3;
+    const int n = n0 + grp * 32 + lane;
+    if (mbar_wait_warp(&done, 0, &abort_flag)) {
+      tc_fence_after();
+#pragma unroll 1
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t v[16];
+        tmem_ld16(tmem + ((uint32_t)(grp * 32) << 16) + (uint32_t)(cc * 16), v);
+        if (n < p.Nout) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int b = b0 + cc * 16 + e;
+            if (b < p.B) p.out[(int64_t)b * p.out_bs + (int64_t)h * p.out_hs + n] = __float2bfloat16_rn(__uint_as_float(v[e]));
+          }
+        }
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 64);
   }
 }
 
