@@ -78,59 +78,119 @@ def measured_peaks():
 
 
 class ClockSampler:
-    """nvidia-smi samples of SM clock and throttle reasons while running."""
+    """SM clock and clock-event reasons sampled while the timed region runs.
 
-    FIELDS = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
-              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
-              "clocks_event_reasons.sw_power_cap")
+    NVML is polled from a thread every ``period_s`` (the timed region of a
+    default run lasts only tens of milliseconds, too short for
+    ``nvidia-smi -lms``); if NVML cannot be loaded, ``nvidia-smi`` is used."""
 
-    def __init__(self, index: int):
-        self.index = index
-        self.proc = None
-        self.lines = []
+    REASONS = (("hw_slowdown", 0x8), ("sw_thermal_slowdown", 0x20),
+               ("hw_thermal_slowdown", 0x40), ("sw_power_cap", 0x4),
+               ("hw_power_brake_slowdown", 0x80))
+
+    def __init__(self, device: torch.device, period_s: float = 0.0005):
+        self.device = device
+        self.period_s = period_s
+        self.samples = []          # (sm_mhz, reason mask)
+        self.max_mhz = None
+        self._nvml = None
+        self._handle = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._proc = None
+        self._lines = []
+
+    def _open_nvml(self):
+        import pynvml
+        pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.device)
+        uuid = str(props.uuid)
+        if not uuid.startswith("GPU-"):
+            uuid = "GPU-" + uuid
+        self._handle = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+        self._nvml = pynvml
+        self.max_mhz = float(pynvml.nvmlDeviceGetMaxClockInfo(self._handle, pynvml.NVML_CLOCK_SM))
+
+    def _sample_nvml(self):
+        nv = self._nvml
+        mhz = nv.nvmlDeviceGetClockInfo(self._handle, nv.NVML_CLOCK_SM)
+        mask = nv.nvmlDeviceGetCurrentClocksEventReasons(self._handle)
+        self.samples.append((float(mhz), int(mask)))
+
+    def _poll(self):
+        while not self._stop.is_set():
+            try:
+                self._sample_nvml()
+            except Exception:  # a failed read drops one sample
+                pass
+            time.sleep(self.period_s)
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), "--query-gpu=" + self.FIELDS,
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
-            self.thread.start()
-        except (OSError, FileNotFoundError):
-            self.proc = None
+            self._open_nvml()
+            self._sample_nvml()
+            self._thread = threading.Thread(target=self._poll, daemon=True)
+            self._thread.start()
+        except Exception:
+            self._nvml = None
+            self._start_smi()
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def _start_smi(self):
+        fields = ("clocks.sm,clocks.max.sm,clocks_event_reasons.hw_slowdown,"
+                  "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+                  "clocks_event_reasons.sw_power_cap")
+        idx = self.device.index if self.device.index is not None else 0
+        try:
+            self._proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(idx), "--query-gpu=" + fields,
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self._thread = threading.Thread(target=self._read_smi, daemon=True)
+            self._thread.start()
+        except OSError:
+            self._proc = None
 
-    def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except subprocess.TimeoutExpired:
-                self.proc.kill()
-        return False
-
-    def summary(self):
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
+    def _read_smi(self):
+        names = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
+        bits = dict(self.REASONS)
+        for line in self._proc.stdout:
+            parts = [p.strip() for p in line.split(",")]
             if len(parts) != 6:
                 continue
             try:
-                sm.append(float(parts[0]))
-                mx = float(parts[1])
+                mhz, self.max_mhz = float(parts[0]), float(parts[1])
             except ValueError:
                 continue
+            mask = 0
             for n, v in zip(names, parts[2:]):
                 if v.lower() == "active":
-                    reasons.add(n)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                    mask |= bits[n]
+            self.samples.append((mhz, mask))
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._nvml is not None:
+            try:
+                self._sample_nvml()
+            except Exception:
+                pass
+        if self._proc is not None:
+            self._proc.terminate()
+            try:
+                self._proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self._proc.kill()
+        if self._thread is not None:
+            self._thread.join(timeout=5)
+        return False
+
+    def summary(self):
+        sm = [s[0] for s in self.samples]
+        reasons = sorted({n for _, m in self.samples for n, b in self.REASONS if m & b})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(sm),
+                "source": "nvml" if self._nvml is not None else "nvidia-smi"}
 
 
 # ---------------------------------------------------------------- CPU oracle timing
@@ -211,7 +271,7 @@ def run_ours(args, rank, world, device):
         torch.distributed.barrier()
     torch.cuda.synchronize()
     launches0 = mla.mla_launch_count()
-    with ClockSampler(device.index if device.index is not None else 0) as clocks:
+    with ClockSampler(device) as clocks:
         for i in range(args.steps):
             flush.fill_(i & 0xff)
             kp, kd = mla.KernelEvents(16), mla.KernelEvents(16)
@@ -264,7 +324,7 @@ def run_ours(args, rank, world, device):
         roof = dict(bound="tensor", achieved=algo / (top_ms * 1e-3) / 1e12, peak=peaks["bf16"],
                     unit="TFLOP/s")
     else:
-        algo = by["cache"] if "split" in top else by["total"]
+        algo = by["cache"] if "attention" in top else by["total"]
         roof = dict(bound="hbm", achieved=algo / (top_ms * 1e-3) / 1e9, peak=peaks["hbm"], unit="GB/s")
     roof["frac"] = roof["achieved"] / roof["peak"]
     roof["traffic"] = None

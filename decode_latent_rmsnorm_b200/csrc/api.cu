@@ -16,6 +16,7 @@
 #include "simt_decode.cuh"
 #include "tc_gemm.cuh"
 #include "tc_attention.cuh"
+#include "tc_attention_pair.cuh"
 #include "tc_decode.cuh"
 
 #include <cudaTypedefs.h>
@@ -160,7 +161,7 @@ bool prefill_tc_shape(const mla_dims* d) {
 struct PrefillWs {
   int64_t cap, Tpad;
   int gemm_tiles_per_cta, gemm_gy;
-  size_t seq_tile0, tile_seq, tile_q0, order, w16;
+  size_t seq_tile0, tile_seq, tile_q0, order, pair_order, w16;
   size_t k_nope, vals, k_rot, total;
 };
 PrefillWs prefill_ws_layout(const mla_dims* d, int64_t T, int nseq, bool tc) {
@@ -182,6 +183,7 @@ PrefillWs prefill_ws_layout(const mla_dims* d, int64_t T, int nseq, bool tc) {
     w.tile_seq = off;  off = align_up(off + 4 * (size_t)w.cap, 256);
     w.tile_q0 = off;   off = align_up(off + 4 * (size_t)w.cap, 256);
     w.order = off;     off = align_up(off + 4 * (size_t)w.cap, 256);
+    w.pair_order = off; off = align_up(off + 4 * (size_t)w.cap, 256);
     w.w16 = off;       off = align_up(off + 2 * (size_t)NOUT * d->kv_lora_rank, 256);
   } else {
     w.Tpad = T;
@@ -336,6 +338,33 @@ int launch_attention_tc(int N, int V, unsigned grid, const CUtensorMap& mq, cons
   return fail(MLA_ERR_UNSUPPORTED_SHAPE, "no tensor-core attention for qk_nope=%d v_head=%d", N, V);
 }
 
+// Head geometries of the two-tile attention kernel (two fp32 O accumulators
+// of V columns next to two 128-column S buffers in 512 TMEM columns).
+bool attention_pair_shape(int N, int V) { return (N == 64 || N == 128) && (V == 64 || V == 128); }
+
+template <int kN, int kV>
+int launch_attention_pair_t(unsigned grid, const CUtensorMap& mq, const CUtensorMap& mkn, const CUtensorMap& mkr,
+                            const CUtensorMap& mvt, const mla::tc::AttParams& ap, cudaStream_t st) {
+  using C = mla::tc::PairCfg<kN, kV>;
+  auto kern = mla::tc::attention_pair_kernel<kN, kV>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
+  if (e != cudaSuccess) return cuda_status(e, "attention smem attribute");
+  prof_begin(st, "tc_attention");
+  kern<<<grid, mla::tc::kPrThreads, C::kSmem, st>>>(mq, mkn, mkr, mvt, ap);
+  prof_end(st);
+  return cuda_status(cudaGetLastError(), "attention launch");
+}
+
+int launch_attention_pair(int N, int V, unsigned grid, const CUtensorMap& mq, const CUtensorMap& mkn,
+                          const CUtensorMap& mkr, const CUtensorMap& mvt, const mla::tc::AttParams& ap,
+                          cudaStream_t st) {
+#define MLA_PAIR_CASE(n, v) \
+  if (N == n && V == v) return launch_attention_pair_t<n, v>(grid, mq, mkn, mkr, mvt, ap, st);
+  MLA_PAIR_CASE(64, 64) MLA_PAIR_CASE(64, 128) MLA_PAIR_CASE(128, 64) MLA_PAIR_CASE(128, 128)
+#undef MLA_PAIR_CASE
+  return fail(MLA_ERR_UNSUPPORTED_SHAPE, "no two-tile attention for qk_nope=%d v_head=%d", N, V);
+}
+
 // Tensor-core prefill: tile schedule -> fused RMSNorm + kv_b_proj (tcgen05)
 // -> causal attention over the padded layout.
 int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, const void* w_kvb,
@@ -350,6 +379,7 @@ int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, cons
   int32_t* tile_seq = reinterpret_cast<int32_t*>(ws + L.tile_seq);
   int32_t* tile_q0 = reinterpret_cast<int32_t*>(ws + L.tile_q0);
   int32_t* order = reinterpret_cast<int32_t*>(ws + L.order);
+  int32_t* pair_order = reinterpret_cast<int32_t*>(ws + L.pair_order);
   __half* k_nope = reinterpret_cast<__half*>(ws + L.k_nope);
   __half* vt = reinterpret_cast<__half*>(ws + L.vals);
   __half* k_rot = reinterpret_cast<__half*>(ws + L.k_rot);
@@ -364,10 +394,13 @@ int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, cons
     int rc = make_map(&map_lat, latent, 2, dims, strides, box);
     if (rc) return rc;
   }
+  // heads with V = 128 and qk_nope 64 or 128 take the GEMM that writes the
+  // value half transposed straight from TMEM (one head's weight rows per stage)
+  const bool vt_gemm = (N == 64 || N == 128) && V == 128;
   {
     const uint64_t dims[2] = {(uint64_t)R, (uint64_t)NOUT};
     const uint64_t strides[1] = {(uint64_t)R * 2};
-    const uint32_t box[2] = {64, 256};
+    const uint32_t box[2] = {64, vt_gemm ? (uint32_t)(N + V) : 256u};
     int rc = make_map(&map_w, ws + L.w16, 2, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
     if (rc) return rc;
   }
@@ -376,13 +409,12 @@ int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, cons
   const int gy = L.gemm_gy;
 
   const int64_t n8 = (int64_t)NOUT * R / 8;
-  prof_begin(st, "tc_weight_f16");
-  mla::tc::weight_to_f16_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, st>>>(static_cast<const bf16*>(w_kvb), w16, n8);
-  prof_end(st);
-
-  prof_begin(st, "tc_schedule");
-  mla::tc::schedule_kernel<<<1, 1024, 0, st>>>(cu_seqlens, num_seqs, T_tot, max_seqlen, cap, seq_tile0, tile_seq,
-                                                tile_q0, order);
+  const int64_t per_block = (int64_t)mla::tc::kPrepThreads * mla::tc::kPrepUnroll;
+  const unsigned prep_blocks = (unsigned)(1 + (n8 + per_block - 1) / per_block);
+  prof_begin(st, "tc_prep");
+  mla::tc::prefill_prep_kernel<<<prep_blocks, mla::tc::kPrepThreads, 0, st>>>(
+      cu_seqlens, num_seqs, T_tot, max_seqlen, cap, seq_tile0, tile_seq, tile_q0, order, pair_order,
+      static_cast<const bf16*>(w_kvb), w16, n8);
   prof_end(st);
 
   mla::tc::GemmParams gp;
@@ -404,17 +436,37 @@ int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, cons
   gp.interleaved = d->rope_interleaved;
   gp.eps = d->eps;
   gp.tiles_per_cta = L.gemm_tiles_per_cta;
-  cudaError_t e = cudaFuncSetAttribute(mla::tc::norm_kvb_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)mla::tc::kGemmSmemBytes);
-  if (e != cudaSuccess) return cuda_status(e, "gemm smem attribute");
-  prof_begin(st, "tc_norm_kv_b_proj");
-  mla::tc::norm_kvb_gemm_kernel<<<dim3(cap, gy), mla::tc::kGemmThreads, mla::tc::kGemmSmemBytes, st>>>(
-      map_lat, map_w, gp);
-  prof_end(st);
+  cudaError_t e;
+  if (vt_gemm) {
+    // grid: (tiles, head groups); about one CTA per SM over the real tiles
+    const int real_tiles = (int)((T_tot + 127) / 128) + (num_seqs > 1 ? num_seqs - 1 : 0);
+    int groups = num_sms() / (real_tiles > 0 ? real_tiles : 1);
+    if (groups < 1) groups = 1;
+    if (groups > H) groups = H;
+    gp.tiles_per_cta = (H + groups - 1) / groups;
+    const int gy2 = (H + gp.tiles_per_cta - 1) / gp.tiles_per_cta;
+    auto kern = N == 64 ? mla::tc::norm_kvb_gemm_vt_kernel<64> : mla::tc::norm_kvb_gemm_vt_kernel<128>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mla::tc::kG2SmemBytes);
+    if (e != cudaSuccess) return cuda_status(e, "gemm smem attribute");
+    prof_begin(st, "tc_norm_kv_b_proj");
+    kern<<<dim3(cap, gy2), mla::tc::kG2Threads, mla::tc::kG2SmemBytes, st>>>(map_lat, map_w, gp);
+    prof_end(st);
+  } else {
+    e = cudaFuncSetAttribute(mla::tc::norm_kvb_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)mla::tc::kGemmSmemBytes);
+    if (e != cudaSuccess) return cuda_status(e, "gemm smem attribute");
+    prof_begin(st, "tc_norm_kv_b_proj");
+    mla::tc::norm_kvb_gemm_kernel<<<dim3(cap, gy), mla::tc::kGemmThreads, mla::tc::kGemmSmemBytes, st>>>(
+        map_lat, map_w, gp);
+    prof_end(st);
+  }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_status(e, "gemm launch");
 
-  // attention tensor maps over the padded workspace and q [Ttot, H, D]
+  // attention tensor maps over the padded workspace and q [Ttot, H, D]; the
+  // two-tile kernel reads 128 keys per step, the one-tile kernel 64
+  const bool pair = attention_pair_shape(N, V) && d->softmax_scale > 0.f;
+  const uint32_t kv_box = pair ? (uint32_t)mla::tc::kPrBKV : (uint32_t)mla::tc::kAttBKV;
   const int D = N + P;
   CUtensorMap map_q, map_kn, map_kr, map_vt;
   {
@@ -427,14 +479,14 @@ int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, cons
   {
     const uint64_t dims[2] = {(uint64_t)N, (uint64_t)H * L.Tpad};
     const uint64_t strides[1] = {(uint64_t)N * 2};
-    const uint32_t box[2] = {64, (uint32_t)mla::tc::kAttBKV};
+    const uint32_t box[2] = {64, kv_box};
     int rc = make_map(&map_kn, k_nope, 2, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
     if (rc) return rc;
   }
   {
     const uint64_t dims[2] = {(uint64_t)P, (uint64_t)L.Tpad};
     const uint64_t strides[1] = {(uint64_t)P * 2};
-    const uint32_t box[2] = {64, (uint32_t)mla::tc::kAttBKV};
+    const uint32_t box[2] = {64, kv_box};
     int rc = make_map(&map_kr, k_rot, 2, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
     if (rc) return rc;
   }
@@ -451,7 +503,7 @@ int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, cons
   ap.seq_tile0 = seq_tile0;
   ap.tile_seq = tile_seq;
   ap.tile_q0 = tile_q0;
-  ap.order = order;
+  ap.order = pair ? pair_order : order;
   ap.cos_t = cos_t;
   ap.sin_t = sin_t;
   ap.out = static_cast<bf16*>(out);
@@ -460,6 +512,13 @@ int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, cons
   ap.max_pos = max_pos;
   ap.interleaved = d->rope_interleaved;
   ap.scale_log2 = d->softmax_scale * 1.4426950408889634f;
+  if (pair) {
+    // blocks of two tiles: sum over sequences of ceil(tiles / 2) <= (tiles + nseq) / 2
+    const int64_t tiles_ub = (T_tot + 127) / 128 + num_seqs;
+    int64_t blocks = (tiles_ub + num_seqs) / 2;
+    if (blocks > L.cap) blocks = L.cap;
+    return launch_attention_pair(N, V, (unsigned)(blocks * H), map_q, map_kn, map_kr, map_vt, ap, st);
+  }
   const unsigned grid = (unsigned)(cap * H);
   return launch_attention_tc(N, V, grid, map_q, map_kn, map_kr, map_vt, ap, st);
 }

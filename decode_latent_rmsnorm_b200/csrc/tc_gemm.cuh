@@ -33,12 +33,15 @@ constexpr int kTile = 128;            // token rows per tile (M of the MMAs)
 // tile_seq[i] / tile_q0[i]: sequence and first in-sequence row of tile i in
 // natural order (padded rows tp = 128 i ...); order[j]: tiles sorted by
 // decreasing causal work (largest q0 first), for the attention grid.
-// Entries past the real tile count are -1. Bad cu_seqlens set the device error
-// word and leave every entry at -1.
-__global__ void __launch_bounds__(1024)
-schedule_kernel(const int32_t* __restrict__ cu, int nseq, int64_t Ttot, int max_seqlen, int cap,
-                int32_t* __restrict__ seq_tile0, int32_t* __restrict__ tile_seq, int32_t* __restrict__ tile_q0,
-                int32_t* __restrict__ order) {
+// pair_order[j]: the first tile of each 256-row block (tiles 2k and 2k + 1 of
+// one sequence; the second may not exist), blocks sorted by decreasing k.
+// Entries past the real tile / block count are -1. Bad cu_seqlens set the
+// device error word and leave every entry at -1.
+// Run by one block of 1024 threads.
+__device__ __forceinline__ void schedule_block(const int32_t* __restrict__ cu, int nseq, int64_t Ttot,
+                                               int max_seqlen, int cap, int32_t* __restrict__ seq_tile0,
+                                               int32_t* __restrict__ tile_seq, int32_t* __restrict__ tile_q0,
+                                               int32_t* __restrict__ order, int32_t* __restrict__ pair_order) {
   constexpr int kBuckets = 2048;   // = 2 * blockDim.x (launched with 1024 threads)
   __shared__ int s_bad;
   __shared__ int s_carry;
@@ -47,7 +50,9 @@ schedule_kernel(const int32_t* __restrict__ cu, int nseq, int64_t Ttot, int max_
   __shared__ int s_off[kBuckets];
   const int tid = threadIdx.x;
   if (tid == 0) { s_bad = 0; s_carry = 0; }
-  for (int i = tid; i < cap; i += blockDim.x) { tile_seq[i] = -1; tile_q0[i] = -1; order[i] = -1; }
+  for (int i = tid; i < cap; i += blockDim.x) {
+    tile_seq[i] = -1; tile_q0[i] = -1; order[i] = -1; pair_order[i] = -1;
+  }
   for (int k = tid; k < kBuckets; k += blockDim.x) { s_cnt[k] = 0; s_off[k] = 0; }
   __syncthreads();
   // 1) per-sequence tile counts -> exclusive scan into seq_tile0
@@ -116,26 +121,78 @@ schedule_kernel(const int32_t* __restrict__ cu, int nseq, int64_t Ttot, int max_
       order[pos] = t0 + k;
     }
   }
+  // 4) the same for 256-row blocks, bucketed by block index
+  __syncthreads();
+  for (int k = tid; k < kBuckets; k += blockDim.x) s_cnt[k] = 0;
+  __syncthreads();
+  for (int s = tid; s < nseq; s += blockDim.x) {
+    const int nt = seq_tile0[s + 1] - seq_tile0[s];
+    for (int k = 0; k < nt; k += 2) atomicAdd(&s_cnt[min(k / 2, kBuckets - 1)], 1);
+  }
+  __syncthreads();
+  {
+    const int k0 = kBuckets - 1 - 2 * tid, k1 = k0 - 1;
+    const int c0 = s_cnt[k0], c1 = s_cnt[k1];
+    s_scan[tid] = c0 + c1;
+    __syncthreads();
+    for (int off = 1; off < (int)blockDim.x; off <<= 1) {
+      const int v = tid >= off ? s_scan[tid - off] : 0;
+      __syncthreads();
+      s_scan[tid] += v;
+      __syncthreads();
+    }
+    const int before = s_scan[tid] - (c0 + c1);
+    s_off[k0] = before;
+    s_off[k1] = before + c0;
+  }
+  __syncthreads();
+  for (int s = tid; s < nseq; s += blockDim.x) {
+    const int t0 = seq_tile0[s], nt = seq_tile0[s + 1] - t0;
+    for (int k = 0; k < nt; k += 2) {
+      const int pos = atomicAdd(&s_off[min(k / 2, kBuckets - 1)], 1);
+      pair_order[pos] = t0 + k;
+    }
+  }
 }
 
-// ---- fp16 copy of the kv_b_proj weight ------------------------------------------
-// 8 values per thread; a weight beyond the fp16 range sets the device error word.
-__global__ void __launch_bounds__(256)
-weight_to_f16_kernel(const __nv_bfloat16* __restrict__ w, __half* __restrict__ w16, int64_t n8) {
-  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (i >= n8) return;
-  const uint4 v = reinterpret_cast<const uint4*>(w)[i];
-  const uint32_t in[4] = {v.x, v.y, v.z, v.w};
-  uint32_t o[4];
+// ---- prefill preparation: tile schedule + fp16 copy of the kv_b_proj weight ----
+// Block 0 builds the schedule (schedule_block); blocks 1.. convert the weight,
+// 4 x 8 values per thread. A weight beyond the fp16 range sets the device
+// error word.
+constexpr int kPrepThreads = 1024;
+constexpr int kPrepUnroll = 4;
+__global__ void __launch_bounds__(kPrepThreads)
+prefill_prep_kernel(const int32_t* __restrict__ cu, int nseq, int64_t Ttot, int max_seqlen, int cap,
+                    int32_t* __restrict__ seq_tile0, int32_t* __restrict__ tile_seq,
+                    int32_t* __restrict__ tile_q0, int32_t* __restrict__ order, int32_t* __restrict__ pair_order,
+                    const __nv_bfloat16* __restrict__ w, __half* __restrict__ w16, int64_t n8) {
+  if (blockIdx.x == 0) {
+    schedule_block(cu, nseq, Ttot, max_seqlen, cap, seq_tile0, tile_seq, tile_q0, order, pair_order);
+    return;
+  }
+  const int64_t base = (int64_t)(blockIdx.x - 1) * kPrepThreads * kPrepUnroll + threadIdx.x;
+  uint4 v[kPrepUnroll];
+#pragma unroll
+  for (int u = 0; u < kPrepUnroll; ++u) {
+    const int64_t i = base + (int64_t)u * kPrepThreads;
+    if (i < n8) v[u] = reinterpret_cast<const uint4*>(w)[i];
+  }
   float mx = 0.f;
 #pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const float2 f = unpack_bf16x2(in[e]);
-    mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
-    o[e] = pack_f16x2(f.x, f.y);
+  for (int u = 0; u < kPrepUnroll; ++u) {
+    const int64_t i = base + (int64_t)u * kPrepThreads;
+    if (i >= n8) break;
+    const uint32_t in[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+    uint32_t o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = unpack_bf16x2(in[e]);
+      mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
+      o[e] = pack_f16x2(f.x, f.y);
+    }
+    reinterpret_cast<uint4*>(w16)[i] = make_uint4(o[0], o[1], o[2], o[3]);
   }
   if (!(mx <= kF16Max)) raise_device_error(kDevErrRange);
-  reinterpret_cast<uint4*>(w16)[i] = make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 // ---- fused RMSNorm + kv_b_proj GEMM ------------------------------------------
@@ -373,6 +430,273 @@ norm_kvb_gemm_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_c
 #pragma unroll
           for (int e = 0; e < 16; ++e) dst[(int64_t)e * p.Tpad] = __float2half_rn(__uint_as_float(v[e]));
         }
+      }
+      tc_fence_before();
+      mbar_arrive(&bars.acc_empty[acc]);
+    }
+    if (!(vmax <= kF16Max)) raise_device_error(kDevErrRange);
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+}
+
+}  // namespace tc
+}  // namespace mla
+
+namespace mla {
+namespace tc {
+
+// ---- fused RMSNorm + kv_b_proj GEMM, value half produced transposed --------
+// Heads with qk_nope = kN in {64, 128} and v_head = 128. Per head h and
+// 128-token tile, two tensor-core products share the resident normalized
+// latent tile c_hat [128 x R] and one streamed weight stage (the head's
+// kN + 128 rows of W, 64 K columns per stage):
+//   D1 = c_hat W_K^T   M = 128 tokens,   N = kN      -> k_nope rows
+//   D2 = W_V c_hat^T   M = 128 channels, N = 128 tokens -> value rows of vt
+// The products are the same sums as one c_hat [W_K; W_V]^T; swapping the
+// operands of the value half puts one value channel in each TMEM lane, so
+// the epilogue writes every transposed value row as 256 contiguous bytes.
+// Warps: 0 TMA, 1 MMA, 2-5 RMSNorm prologue then the k_nope epilogue,
+// 6-9 rotated shared key then the value epilogue.
+constexpr int kG2Threads = 320;
+constexpr int kG2Stages = 3;
+constexpr int kG2StageBytes = 256 * 128;
+constexpr size_t kG2SmemBytes = (size_t)kGemmMaxAtoms * kAtomBytes + (size_t)kG2Stages * kG2StageBytes + 1024;
+
+template <int kN>
+__global__ void __launch_bounds__(kG2Threads, 1)
+norm_kvb_gemm_vt_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant__ CUtensorMap map_w,
+                        GemmParams p) {
+  constexpr int kV = 128;
+  constexpr int kRows = kN + kV;                  // weight rows of one head
+  constexpr int kStage = kRows * 128;             // bytes of one stage
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  __shared__ GemmBarriers bars;
+  __shared__ uint4 s_wnorm[kGemmMaxAtoms * 8];   // the RMSNorm weight, 8 bf16 per entry
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tile = blockIdx.x;
+  const int seq = p.tile_seq[tile];
+  if (seq < 0) return;   // past the real tiles (uniform over the CTA)
+  // one vector load per thread, all in flight together (published by the
+  // __syncthreads below)
+  if (threadIdx.x < p.R / 8) s_wnorm[threadIdx.x] = reinterpret_cast<const uint4*>(p.w_norm)[threadIdx.x];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + kGemmMaxAtoms * kAtomBytes;
+  const int q0 = p.tile_q0[tile];
+  const int64_t seq0 = p.cu[seq];
+  const int L = (int)(p.cu[seq + 1] - seq0);
+  const int tp0 = tile * kTile;
+  const int natoms = p.R / 64;
+  const int h_begin = blockIdx.y * p.tiles_per_cta;
+  const int h_end = min(p.H, h_begin + p.tiles_per_cta);
+  const int my_heads = h_end - h_begin;
+  volatile int* abort_flag = &bars.abort_flag;
+
+  if (threadIdx.x == 0) {
+    mbar_init(&bars.a_full, 1);
+    mbar_init(&bars.a_ready, 128);
+    for (int s = 0; s < kG2Stages; ++s) { mbar_init(&bars.b_full[s], 1); mbar_init(&bars.b_empty[s], 1); }
+    for (int s = 0; s < 2; ++s) { mbar_init(&bars.acc_full[s], 1); mbar_init(&bars.acc_empty[s], 256); }
+    mbar_init(&bars.mma_done, 1);
+    bars.abort_flag = 0;
+    mbar_fence_init();
+  }
+  if (warp == 1) tmem_alloc(&bars.tmem_base, 512);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = bars.tmem_base;
+
+  if (warp == 0) {
+    // ---------------- TMA producer ----------------
+    if (lane == 0 && my_heads > 0) {
+      tma_prefetch_desc(&map_lat);
+      tma_prefetch_desc(&map_w);
+      mbar_arrive_expect_tx(&bars.a_full, natoms * kAtomBytes);
+      for (int a = 0; a < natoms; ++a)
+        tma_load_2d(sA + a * kAtomBytes, &map_lat, &bars.a_full, a * 64, (int)(seq0 + q0));
+      int it = 0;
+      bool ok = true;
+      for (int h = h_begin; h < h_end && ok; ++h) {
+        for (int kc = 0; kc < natoms; ++kc, ++it) {
+          const int s = it % kG2Stages;
+          if (!mbar_wait(&bars.b_empty[s], ((uint32_t)(it / kG2Stages) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&bars.b_full[s], kStage);
+          tma_load_2d(sB + s * kG2StageBytes, &map_w, &bars.b_full[s], kc * 64, h * kRows);
+        }
+      }
+      if (!ok) {
+        mbar_wait_drain(&bars.a_full, 0);
+        for (int j = (it > kG2Stages ? it - kG2Stages : 0); j < it; ++j)
+          mbar_wait_drain(&bars.b_full[j % kG2Stages], (uint32_t)(j / kG2Stages) & 1u);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issuer (whole warp; one elected lane issues) ----------------
+    if (my_heads > 0) {
+      const uint32_t idesc1 = idesc_f16_f32(kTile, kN);
+      const uint32_t idesc2 = idesc_f16_f32(kTile, kTile);
+      bool ok = mbar_wait_warp(&bars.a_ready, 0, abort_flag);
+      tc_fence_after();
+      int it = 0;
+      for (int i = 0; i < my_heads && ok; ++i) {
+        const int acc = i & 1;
+        if (!mbar_wait_warp(&bars.acc_empty[acc], ((uint32_t)(i >> 1) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        const uint32_t d1 = tmem + (uint32_t)(acc * 256);
+        const uint32_t d2 = d1 + (uint32_t)kN;
+        for (int kc = 0; kc < natoms; ++kc, ++it) {
+          const int s = it % kG2Stages;
+          if (!mbar_wait_warp(&bars.b_full[s], (uint32_t)(it / kG2Stages) & 1u, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t cd = desc_kmajor_sw128(smem_u32(sA + kc * kAtomBytes));
+          const uint64_t wk = desc_kmajor_sw128(smem_u32(sB + s * kG2StageBytes));
+          const uint64_t wv = desc_kmajor_sw128(smem_u32(sB + s * kG2StageBytes + kN * 128));
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            mma_ss_elect(d1, desc_advance(cd, k * 32), desc_advance(wk, k * 32), idesc1, (kc | k) != 0);
+            mma_ss_elect(d2, desc_advance(wv, k * 32), desc_advance(cd, k * 32), idesc2, (kc | k) != 0);
+          }
+          mma_commit_elect(&bars.b_empty[s]);
+        }
+        if (!ok) break;
+        mma_commit_elect(&bars.acc_full[acc]);
+      }
+      mma_commit_elect(&bars.mma_done);
+      if (lane == 0) mbar_wait_drain(&bars.mma_done, 0);
+      __syncwarp();
+    }
+  } else {
+    const int half = (warp - 2) >> 2;          // 0: norm + k_nope, 1: k_rot + values
+    const int grp = warp & 3;
+    const int lrow = grp * 32 + lane;          // TMEM lane of this thread
+    const uint32_t lane_base = (uint32_t)(grp * 32) << 16;
+    bool ok = my_heads > 0;
+    if (half == 0) {
+      // RMSNorm prologue: lane = token row of the tile
+      const bool valid = (q0 + lrow) < L;
+      if (ok) ok = mbar_wait_warp(&bars.a_full, 0, abort_flag);
+      if (ok) {
+        // sum of squares: eight independent partial sums; each atom's eight
+        // chunks are loaded before any is used
+        float ss8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+        for (int a = 0; a < natoms; ++a) {
+          const uint8_t* base = sA + a * kAtomBytes;
+          uint4 v[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) v[c] = *reinterpret_cast<const uint4*>(base + sw128_offset(lrow, c));
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint32_t w4[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = unpack_bf16x2(w4[e]);
+              ss8[c] = fmaf(f.x, f.x, fmaf(f.y, f.y, ss8[c]));
+            }
+          }
+        }
+        const float ss = ((ss8[0] + ss8[1]) + (ss8[2] + ss8[3])) + ((ss8[4] + ss8[5]) + (ss8[6] + ss8[7]));
+        const float r = valid ? 1.0f / sqrtf(ss / (float)p.R + p.eps) : 0.f;
+        // c_hat = w * x * r in place, as fp16 (rows past the sequence become
+        // zeros): per atom, all loads, then the arithmetic, then all stores
+        for (int a = 0; a < natoms; ++a) {
+          uint8_t* base = sA + a * kAtomBytes;
+          uint4 v[8];
+#pragma unroll
+          for (int c = 0; c < 8; ++c) v[c] = *reinterpret_cast<const uint4*>(base + sw128_offset(lrow, c));
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            const uint32_t w4[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
+            const uint4 wv = s_wnorm[a * 8 + c];
+            const uint32_t g4[4] = {wv.x, wv.y, wv.z, wv.w};
+            uint32_t o4[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float2 f = unpack_bf16x2(w4[e]);
+              const float2 g = unpack_bf16x2(g4[e]);
+              o4[e] = pack_f16x2(g.x * (f.x * r), g.y * (f.y * r));
+            }
+            v[c] = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+          }
+#pragma unroll
+          for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(base + sw128_offset(lrow, c)) = v[c];
+        }
+        fence_proxy_async_smem();
+      }
+      mbar_arrive(&bars.a_ready);
+    } else if (blockIdx.y == 0) {
+      // rotated shared key of token row lrow (one CTA column per tile writes
+      // it); P = 64: the row's 64 values and its 32 cos / sin entries come in
+      // as independent vector loads
+      const bool valid = (q0 + lrow) < L;
+      const int64_t t = seq0 + q0 + lrow;
+      uint4* dst = reinterpret_cast<uint4*>(p.k_rot + (int64_t)(tp0 + lrow) * 64);
+      if (valid) {
+        const uint4* src = reinterpret_cast<const uint4*>(p.latent + t * (p.R + 64) + p.R);
+        const int64_t pos = checked_pos(p.positions[t], p.max_pos);
+        const float4* c4 = reinterpret_cast<const float4*>(p.cos_t + pos * 32);
+        const float4* s4 = reinterpret_cast<const float4*>(p.sin_t + pos * 32);
+        uint4 raw[8];
+        float4 cv[8], sv[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) { raw[i] = src[i]; cv[i] = c4[i]; sv[i] = s4[i]; }
+        float x[64], y[64], cs[32], sn[32];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const uint32_t w4[4] = {raw[i].x, raw[i].y, raw[i].z, raw[i].w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = unpack_bf16x2(w4[e]);
+            x[i * 8 + 2 * e] = f.x;
+            x[i * 8 + 2 * e + 1] = f.y;
+          }
+          cs[4 * i] = cv[i].x; cs[4 * i + 1] = cv[i].y; cs[4 * i + 2] = cv[i].z; cs[4 * i + 3] = cv[i].w;
+          sn[4 * i] = sv[i].x; sn[4 * i + 1] = sv[i].y; sn[4 * i + 2] = sv[i].z; sn[4 * i + 3] = sv[i].w;
+        }
+        if (p.interleaved) {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) rope_turn(x[2 * i], x[2 * i + 1], cs[i], sn[i], y[2 * i], y[2 * i + 1]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 32; ++i) rope_turn(x[i], x[i + 32], cs[i], sn[i], y[i], y[i + 32]);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          dst[i] = make_uint4(pack_f16x2(y[8 * i], y[8 * i + 1]), pack_f16x2(y[8 * i + 2], y[8 * i + 3]),
+                              pack_f16x2(y[8 * i + 4], y[8 * i + 5]), pack_f16x2(y[8 * i + 6], y[8 * i + 7]));
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) dst[i] = make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+    // epilogue: half 0 writes k_nope rows (lane = token), half 1 value rows (lane = channel)
+    float vmax = 0.f;
+    for (int i = 0; i < my_heads && ok; ++i) {
+      const int acc = i & 1;
+      const int h = h_begin + i;
+      if (!mbar_wait_warp(&bars.acc_full[acc], (uint32_t)(i >> 1) & 1u, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      const uint32_t src = tmem + lane_base + (uint32_t)(acc * 256 + (half ? kN : 0));
+      uint4* dst = half ? reinterpret_cast<uint4*>(p.vt + ((int64_t)h * kV + lrow) * p.Tpad + tp0)
+                        : reinterpret_cast<uint4*>(p.k_nope + ((int64_t)h * p.Tpad + tp0 + lrow) * kN);
+      const int nchunks = half ? kTile / 32 : kN / 32;
+      for (int c = 0; c < nchunks; ++c) {
+        uint32_t v[32];
+        tmem_ld32(src + (uint32_t)(c * 32), v);
+        uint32_t pk[16];
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const float a = __uint_as_float(v[2 * e]), b = __uint_as_float(v[2 * e + 1]);
+          vmax = fmaxf(vmax, fmaxf(fabsf(a), fabsf(b)));
+          pk[e] = pack_f16x2(a, b);
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) dst[c * 4 + e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
       }
       tc_fence_before();
       mbar_arrive(&bars.acc_empty[acc]);

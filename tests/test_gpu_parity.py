@@ -65,6 +65,17 @@ def test_prefill_glm_heads_small(gpu_lib):
     compare(f64(got), oracle_prefill(wl, inp), "bf16", "glm small")
 
 
+@pytest.mark.parametrize("nv", [(64, 64), (64, 128), (128, 64), (64, 192)], ids=lambda nv: "N%dV%d" % nv)
+def test_prefill_bf16_other_head_geometry(gpu_lib, nv):
+    # tensor-core geometries unlike the configs: 4 heads, rank 256, ragged lengths
+    N, V = nv
+    wl = W.Workload("geom_bf16", "prefill", 4, 256, N, 64, V, "bf16", W.KIMI_ROPE, 31 + N + V,
+                    seqlens=(300, 129, 520, 1))
+    inp = W.prefill_inputs(wl)
+    got = run_prefill(wl, inp)
+    compare(f64(got), oracle_prefill(wl, inp), "bf16", "geometry N%d V%d" % nv)
+
+
 def test_prefill_fp32_other_geometry(gpu_lib):
     # fp32, half-split pairs, a geometry unlike the configs (H=3, N=32, P=16, V=24)
     wl = W.Workload("odd_fp32", "prefill", 3, 128, 32, 16, 24, "fp32", dict(W.KIMI_ROPE, rope_dim=16),
