@@ -67,6 +67,22 @@ def decode_bytes(wl, lens) -> dict:
 
 # ---------------------------------------------------------------- environment
 
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch of ``kernel`` from the committed ncu capture
+    (profiles/traffic.json), or None when there is none or the kernel's
+    source changed since it was taken."""
+    from decode_latent_rmsnorm_b200.kernel_sources import source_digest
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(kernel)
+    except (OSError, ValueError):
+        return None
+    if not isinstance(rec, dict) or rec.get("source_digest") != source_digest(kernel):
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
 def measured_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -327,7 +343,7 @@ def run_ours(args, rank, world, device):
         algo = by["cache"] if "attention" in top else by["total"]
         roof = dict(bound="hbm", achieved=algo / (top_ms * 1e-3) / 1e9, peak=peaks["hbm"], unit="GB/s")
     roof["frac"] = roof["achieved"] / roof["peak"]
-    roof["traffic"] = None
+    roof["traffic"] = recorded_traffic(top)
     roof["kernel"] = top
     roof["peak_source"] = peaks["source"]
 
