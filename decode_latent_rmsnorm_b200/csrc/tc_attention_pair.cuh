@@ -14,7 +14,7 @@
 // twice the tensor-core work. Warps:
 //   warp 0     TMA producer (Q tiles, then per step: the key atoms and the two
 //              transposed value boxes into a ring of 16 KB slots)
-//   warp 1     MMA issuer (one thread)
+//   warp 1     MMA issuer (whole warp, one elected lane issues)
 //   warps 2-5  softmax of tile A (one query row per thread, TMEM lane = row)
 //   warps 6-9  softmax of tile B
 // TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,256+V),
@@ -254,27 +254,13 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
     const int qi = min(qrow, L - 1);
     const int64_t t = seq0 + qrow;
     bool ok = nX > 0;
-    // this row's rotation angle: position, then its 32 cos / sin entries as
-    // independent vector loads, issued before the wait for the Q tile
-    float cs[32], sn[32];
-    if (ok) {
-      const int64_t pos = valid ? checked_pos(p.positions[t], p.max_pos) : 0;
-      const float4* c4 = reinterpret_cast<const float4*>(p.cos_t + pos * 32);
-      const float4* s4 = reinterpret_cast<const float4*>(p.sin_t + pos * 32);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float4 c = c4[i], s = s4[i];
-        cs[4 * i] = c.x; cs[4 * i + 1] = c.y; cs[4 * i + 2] = c.z; cs[4 * i + 3] = c.w;
-        sn[4 * i] = s.x; sn[4 * i + 1] = s.y; sn[4 * i + 2] = s.z; sn[4 * i + 3] = s.w;
-      }
-    }
     if (ok) ok = mbar_wait_warp(&bars.q_full, 0, abort_flag);
     if (ok) {
-      // this row of q: bf16 -> fp16 in place; the rotary part (last atom) is
-      // rotated at the token's position on the way
+      // this row of q: bf16 -> fp16 in place (per atom: all loads, the
+      // conversion, then all stores); the rotary atom is rotated at the
+      // token's position, its 32 pairs in two halves of 16
       uint8_t* sQx = sQ + x * C::kQTileBytes;
       float qmax = 0.f;
-      // per atom: all loads, then the conversion, then all stores
 #pragma unroll 1
       for (int a = 0; a < C::kQAtoms - 1; ++a) {
         uint8_t* qa = sQx + a * kTile * 128;
@@ -296,37 +282,62 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
 #pragma unroll
         for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(qa + sw128_offset(row, c)) = v[c];
       }
+      const int64_t pos = valid ? checked_pos(p.positions[t], p.max_pos) : 0;
       uint8_t* qr = sQx + (C::kQAtoms - 1) * kTile * 128;
-      float xr[64];
+#pragma unroll 1
+      for (int hp = 0; hp < 2; ++hp) {
+        // rotary pairs [16 hp, 16 hp + 16): 16 cos / sin entries as four vector
+        // loads each; the four 16-byte chunks holding the pairs' 32 values
+        // (half-split pairing: chunks 2hp, 2hp+1 and 4+2hp, 5+2hp;
+        // interleaved: chunks 4hp .. 4hp+3)
+        const float4* c4 = reinterpret_cast<const float4*>(p.cos_t + pos * 32 + hp * 16);
+        const float4* s4 = reinterpret_cast<const float4*>(p.sin_t + pos * 32 + hp * 16);
+        float cs[16], sn[16];
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint4 v = *reinterpret_cast<const uint4*>(qr + sw128_offset(row, c));
-        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = unpack_bf16x2(w4[e]);
-          xr[c * 8 + 2 * e] = f.x;
-          xr[c * 8 + 2 * e + 1] = f.y;
+        for (int i = 0; i < 4; ++i) {
+          const float4 cv = c4[i], sv = s4[i];
+          cs[4 * i] = cv.x; cs[4 * i + 1] = cv.y; cs[4 * i + 2] = cv.z; cs[4 * i + 3] = cv.w;
+          sn[4 * i] = sv.x; sn[4 * i + 1] = sv.y; sn[4 * i + 2] = sv.z; sn[4 * i + 3] = sv.w;
         }
-      }
-      float y[64];
-      if (p.interleaved) {
+        int ch[4];
+        if (p.interleaved) {
+          ch[0] = 4 * hp; ch[1] = 4 * hp + 1; ch[2] = 4 * hp + 2; ch[3] = 4 * hp + 3;
+        } else {
+          ch[0] = 2 * hp; ch[1] = 2 * hp + 1; ch[2] = 4 + 2 * hp; ch[3] = 5 + 2 * hp;
+        }
+        float xr[32];
 #pragma unroll
-        for (int i = 0; i < 32; ++i) rope_turn(xr[2 * i], xr[2 * i + 1], cs[i], sn[i], y[2 * i], y[2 * i + 1]);
-      } else {
+        for (int k = 0; k < 4; ++k) {
+          const uint4 v = *reinterpret_cast<const uint4*>(qr + sw128_offset(row, ch[k]));
+          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
 #pragma unroll
-        for (int i = 0; i < 32; ++i) rope_turn(xr[i], xr[i + 32], cs[i], sn[i], y[i], y[i + 32]);
-      }
+          for (int e = 0; e < 4; ++e) {
+            const float2 f = unpack_bf16x2(w4[e]);
+            xr[k * 8 + 2 * e] = f.x;
+            xr[k * 8 + 2 * e + 1] = f.y;
+          }
+        }
+        // xr holds, in order, chunks ch[0..3]; local pair i is (xr[2i],
+        // xr[2i+1]) when interleaved, (xr[i], xr[16+i]) otherwise
+        float y[32];
+        if (p.interleaved) {
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint4 v;
-        v.x = pack_f16x2(y[c * 8 + 0], y[c * 8 + 1]);
-        v.y = pack_f16x2(y[c * 8 + 2], y[c * 8 + 3]);
-        v.z = pack_f16x2(y[c * 8 + 4], y[c * 8 + 5]);
-        v.w = pack_f16x2(y[c * 8 + 6], y[c * 8 + 7]);
-        *reinterpret_cast<uint4*>(qr + sw128_offset(row, c)) = v;
+          for (int i = 0; i < 16; ++i) rope_turn(xr[2 * i], xr[2 * i + 1], cs[i], sn[i], y[2 * i], y[2 * i + 1]);
+        } else {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) qmax = fmaxf(qmax, fabsf(y[c * 8 + e]));
+          for (int i = 0; i < 16; ++i) rope_turn(xr[i], xr[16 + i], cs[i], sn[i], y[i], y[16 + i]);
+        }
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          uint4 v;
+          v.x = pack_f16x2(y[k * 8 + 0], y[k * 8 + 1]);
+          v.y = pack_f16x2(y[k * 8 + 2], y[k * 8 + 3]);
+          v.z = pack_f16x2(y[k * 8 + 4], y[k * 8 + 5]);
+          v.w = pack_f16x2(y[k * 8 + 6], y[k * 8 + 7]);
+          *reinterpret_cast<uint4*>(qr + sw128_offset(row, ch[k])) = v;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) qmax = fmaxf(qmax, fabsf(y[k * 8 + e]));
+        }
       }
       if (valid && !(qmax <= kF16Max)) raise_device_error(kDevErrRange);
       fence_proxy_async_smem();
@@ -341,13 +352,15 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
     for (int j = 0; j < nX && ok; ++j) {
       if (!mbar_wait_warp(&bars.s_full[x], (uint32_t)j & 1u, abort_flag)) { ok = false; break; }
       tc_fence_after();
+      // the row's 128 scores: four loads in flight, one wait
       float sc[kPrBKV];
+      {
+        uint32_t v[kPrBKV];
 #pragma unroll
-      for (int c = 0; c < kPrBKV / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tS + (uint32_t)(c * 32), v);
+        for (int c = 0; c < kPrBKV / 32; ++c) tmem_ld32_nowait(tS + (uint32_t)(c * 32), v + c * 32);
+        tmem_wait_ld128(v);
 #pragma unroll
-        for (int e = 0; e < 32; ++e) sc[c * 32 + e] = __uint_as_float(v[e]);
+        for (int e = 0; e < kPrBKV; ++e) sc[e] = __uint_as_float(v[e]);
       }
       if (j == nX - 1) {        // the diagonal step: causal mask (also masks padded keys)
         const int lim = qi - j * kPrBKV;
@@ -377,14 +390,17 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
           tmem_st16(ta, v);
         }
       }
+      // P = 2^(s scale log2(e) - m) in fp32, packed to fp16; the row sum adds
+      // the fp32 weights before their rounding to fp16.
       float rs4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c = 0; c < kPrBKV / 32; ++c) {
         uint32_t pk[16];
 #pragma unroll
         for (int e = 0; e < 16; ++e) {
-          const float p0 = ex2_approx(fmaf(sc[c * 32 + 2 * e], sl, -m));
-          const float p1 = ex2_approx(fmaf(sc[c * 32 + 2 * e + 1], sl, -m));
+          const float a0 = fmaf(sc[c * 32 + 2 * e], sl, -m);
+          const float a1 = fmaf(sc[c * 32 + 2 * e + 1], sl, -m);
+          const float p0 = ex2_approx(a0), p1 = ex2_approx(a1);
           rs4[e & 3] += p0 + p1;
           pk[e] = pack_f16x2(p0, p1);
         }
