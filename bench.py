@@ -239,6 +239,32 @@ def oracle_prefill_sample(wl, inp, budget_s: float):
 
 # ---------------------------------------------------------------- GPU bench
 
+def max_over_ranks(x: float, world: int) -> float:
+    """The largest value of ``x`` over the job's ranks (identity at one rank).
+    The reduction tensor lives where the process group's backend wants it."""
+    if world == 1:
+        return x
+    dist = torch.distributed
+    dev = torch.device("cuda", torch.cuda.current_device()) if dist.get_backend() == "nccl" else torch.device("cpu")
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(work_per_rank: float, world: int, slowest_ms: float) -> float:
+    """Whole-job rate: the work of all ranks (replicas) over the slowest rank's time."""
+    return world * work_per_rank / (slowest_ms * 1e-3)
+
+
+def workload_config(world, lens):
+    """The config object both arms print."""
+    return dict(workload="kimi_k2_prefill_bf16 + absorbed_decode_bf16",
+                prefill="B=1 T=2048 H=64 R=512 N=128 P=64 V=128 YaRN(base 5e4, factor 32)",
+                decode="B=64 H=64 R=512 N=128 P=64 V=128, cache lens U[1000,32768] sum=%d" % sum(lens),
+                global_batch=world * (1 + len(lens)), parallelism="replicas x%d" % world,
+                l2="flushed between steps (256 MiB write outside per-step events)")
+
+
 def run_ours(args, rank, world, device):
     torch.cuda.set_device(device)
     peaks = measured_peaks()
@@ -310,19 +336,15 @@ def run_ours(args, rank, world, device):
     step_ms = [a + b for a, b in zip(p_ms, d_ms)]
 
     def reduce_max(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        return float(t.item())
+        return max_over_ranks(x, world)
 
     p_mean = reduce_max(statistics.mean(p_ms))
     d_mean = reduce_max(statistics.mean(d_ms))
     s_mean = reduce_max(statistics.mean(step_ms))
     fl = prefill_flops(pwl)
     by = decode_bytes(dwl, lens)
-    p_tflops = world * fl["total"] / (p_mean * 1e-3) / 1e12
-    d_gbs = world * by["total"] / (d_mean * 1e-3) / 1e9
+    p_tflops = job_throughput(fl["total"], world, p_mean) / 1e12
+    d_gbs = job_throughput(by["total"], world, d_mean) / 1e9
 
     # per-kernel mean durations (kernel names reported by the library)
     def kernel_means(kev):
@@ -355,11 +377,7 @@ def run_ours(args, rank, world, device):
         metric=METRIC, value=p_tflops, unit="TFLOP/s", n_gpus=world, steps=args.steps,
         warmup=args.warmup, ms_per_step=s_mean, higher_is_better=True, scaling="weak",
         vs_baseline=None, dtype="bf16", data="synthetic (seeded N(0,1) inputs, N(0,1/R) kv_b_proj)",
-        config=dict(workload="kimi_k2_prefill_bf16 + absorbed_decode_bf16",
-                    prefill="B=1 T=2048 H=64 R=512 N=128 P=64 V=128 YaRN(base 5e4, factor 32)",
-                    decode="B=64 H=64 R=512 N=128 P=64 V=128, cache lens U[1000,32768] sum=%d" % sum(lens),
-                    global_batch=world * (1 + B), parallelism="replicas x%d" % world,
-                    l2="flushed between steps (256 MiB write outside per-step events)"),
+        config=workload_config(world, lens),
         prefill=dict(ms=p_mean, tflops=p_tflops, frac_of_bf16_peak=p_tflops / (world * peaks["bf16"]),
                      tokens_per_s=world * T / (p_mean * 1e-3), gflop=fl["total"] / 1e9),
         decode=dict(metric="absorbed decode HBM GB/s", value=d_gbs, unit="GB/s", ms=d_mean,
@@ -448,7 +466,7 @@ def run_reference(args, rank, world):
     return dict(metric=METRIC, value=v, unit="TFLOP/s", n_gpus=world, steps=args.steps, warmup=args.warmup,
                 ms_per_step=fl / (v * 1e12) * 1e3, higher_is_better=True, scaling="weak", vs_baseline=None,
                 dtype="f64", data="synthetic", impl="reference",
-                config=dict(workload="kimi_k2_prefill_bf16 (oracle on a sample of heads per step)"),
+                config=workload_config(world, [int(x) for x in W.decode_cache_lens(W.DECODE)]),
                 cpu_baseline=dict(kind="oracle", cores=threads, sample=sample, value=v, unit="TFLOP/s"),
                 e2e=dict(value=v, unit="TFLOP/s", h2d_bytes_per_step=0, d2h_bytes_per_step=0))
 

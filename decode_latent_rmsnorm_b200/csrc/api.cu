@@ -593,10 +593,6 @@ int launch_decode_tc(const mla_dims* d, const void* q, const void* cache, int64_
     int rc = make_map(&map_q, qf, 2, dims, strides, box);
     if (rc) return rc;
   }
-  prof_begin(st, "tc_decode_schedule");
-  T::decode_schedule_kernel<<<1, 1024, 0, st>>>(lens, offsets, B, max_len, cache_rows, L.G, prefix, meta);
-  prof_end(st);
-
   // q_lat[b, h, :] = q_nope[b, h, :] W_UK_h   (W_UK_h = rows j < N of head h: [N, R], R contiguous)
   CUtensorMap map_wk, map_qn, map_wv, map_ol;
   {
@@ -638,16 +634,25 @@ int launch_decode_tc(const mla_dims* d, const void* q, const void* cache, int64_
     hp.K = N;
     hp.a_row0 = 0;
     hp.a_hstride = N + V;
-    prof_begin(st, "tc_decode_qabsorb");
-    T::head_gemm_kernel<true><<<dim3(H, R / 128, (B + 63) / 64), 192, T::kHgSmem, st>>>(map_wk, map_qn, hp);
+    hp.q = static_cast<const bf16*>(q);
+    hp.positions = positions;
+    hp.cos_t = cos_t;
+    hp.sin_t = sin_t;
+    hp.max_pos = max_pos;
+    hp.N = N;
+    hp.interleaved = d->rope_interleaved;
+    hp.lens = lens;
+    hp.offsets = offsets;
+    hp.max_len = max_len;
+    hp.G = L.G;
+    hp.cache_rows = cache_rows;
+    hp.prefix = prefix;
+    hp.meta = meta;
+    // grid x: the H heads plus one column whose first CTA builds the split schedule
+    prof_begin(st, "tc_decode_qprep");
+    T::head_gemm_kernel<true><<<dim3(H + 1, R / 128, (B + 63) / 64), 192, T::kHgSmem, st>>>(map_wk, map_qn, hp);
     prof_end(st);
   }
-  const int64_t nrope = (int64_t)B * H * (P / 2);
-  prof_begin(st, "tc_decode_qrope");
-  T::decode_qrope_kernel<<<(unsigned)((nrope + 255) / 256), 256, 0, st>>>(static_cast<const bf16*>(q), positions,
-                                                                           cos_t, sin_t, max_pos, B, H, R, N, P,
-                                                                           d->rope_interleaved, qf);
-  prof_end(st);
 
   T::DecParams dp;
   dp.prefix = prefix;

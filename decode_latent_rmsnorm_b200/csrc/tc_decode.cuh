@@ -44,9 +44,11 @@ constexpr int kDecSCol = 256;                   // S^T: 64 columns
 // ---- split schedule -----------------------------------------------------------
 // prefix[b] = rows of sequences before b (invalid sequences count 0 rows);
 // prefix[B] = total; meta[0] = rows per CTA (ceil(total / G)).
-__global__ void __launch_bounds__(1024)
-decode_schedule_kernel(const int32_t* __restrict__ lens, const int64_t* __restrict__ offsets, int B, int max_len,
-                       int64_t cache_rows, int G, int64_t* __restrict__ prefix, int64_t* __restrict__ meta) {
+// Run by one whole block (any size up to 1024 threads).
+__device__ __forceinline__ void decode_schedule_block(const int32_t* __restrict__ lens,
+                                                      const int64_t* __restrict__ offsets, int B, int max_len,
+                                                      int64_t cache_rows, int G, int64_t* __restrict__ prefix,
+                                                      int64_t* __restrict__ meta) {
   __shared__ int64_t s_scan[1024];
   __shared__ int64_t s_carry;
   const int tid = threadIdx.x;
@@ -81,26 +83,60 @@ decode_schedule_kernel(const int32_t* __restrict__ lens, const int64_t* __restri
 }
 
 // q_pe rotated at the query position, into the last P columns of qf rows.
-__global__ void decode_qrope_kernel(const __nv_bfloat16* __restrict__ q, const int32_t* __restrict__ positions,
-                                    const float* __restrict__ cos_t, const float* __restrict__ sin_t, int max_pos,
-                                    int B, int H, int R, int N, int P, int interleaved,
-                                    __nv_bfloat16* __restrict__ qf) {
-  const int pairs = P / 2;
-  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  if (e >= (int64_t)B * H * pairs) return;
-  const int i = (int)(e % pairs);
-  const int64_t bh = e / pairs;
-  const int b = (int)(bh / H);
-  int ia, ib;
-  rope_pair_slots(i, P, interleaved, ia, ib);
+// q_pe of sequences [b0, b0 + nb) and head h, rotated at each sequence's
+// position, into qf[b, h, R:] (bf16). Rotary width P = 64: the 128 calling
+// threads take one sequence and half of its 32 pairs each, as vector loads
+// (half-split pairing: values [16 hp, 16 hp + 16) and [32 + 16 hp, 48 + 16 hp);
+// interleaved: values [32 hp, 32 hp + 32)).
+__device__ __forceinline__ void decode_qrope_rows(const __nv_bfloat16* __restrict__ q,
+                                                  const int32_t* __restrict__ positions,
+                                                  const float* __restrict__ cos_t, const float* __restrict__ sin_t,
+                                                  int max_pos, int h, int b0, int nb, int H, int R, int N,
+                                                  int interleaved, __nv_bfloat16* __restrict__ qf, int tid) {
+  const int b = b0 + (tid >> 1), hp = tid & 1;
+  if ((tid >> 1) >= nb) return;
   const int64_t pos = checked_pos(positions[b], max_pos);
-  const __nv_bfloat16* qr = q + bh * (N + P) + N;
-  float ox, oy;
-  rope_turn(__bfloat162float(qr[ia]), __bfloat162float(qr[ib]), cos_t[pos * pairs + i], sin_t[pos * pairs + i], ox,
-            oy);
-  __nv_bfloat16* dst = qf + bh * (R + P) + R;
-  dst[ia] = __float2bfloat16_rn(ox);
-  dst[ib] = __float2bfloat16_rn(oy);
+  const int64_t bh = (int64_t)b * H + h;
+  const uint4* src = reinterpret_cast<const uint4*>(q + bh * (N + 64) + N);
+  uint4* dst = reinterpret_cast<uint4*>(qf + bh * (R + 64) + R);
+  const float4* c4 = reinterpret_cast<const float4*>(cos_t + pos * 32 + hp * 16);
+  const float4* s4 = reinterpret_cast<const float4*>(sin_t + pos * 32 + hp * 16);
+  int ch[4];   // 16-byte chunks (8 values) of the row holding this thread's pairs
+  if (interleaved) {
+    ch[0] = 4 * hp; ch[1] = 4 * hp + 1; ch[2] = 4 * hp + 2; ch[3] = 4 * hp + 3;
+  } else {
+    ch[0] = 2 * hp; ch[1] = 2 * hp + 1; ch[2] = 4 + 2 * hp; ch[3] = 5 + 2 * hp;
+  }
+  uint4 raw[4];
+  float4 cv[4], sv[4];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) { raw[k] = src[ch[k]]; cv[k] = c4[k]; sv[k] = s4[k]; }
+  float x[32], cs[16], sn[16];
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const uint32_t w4[4] = {raw[k].x, raw[k].y, raw[k].z, raw[k].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = unpack_bf16x2(w4[e]);
+      x[k * 8 + 2 * e] = f.x;
+      x[k * 8 + 2 * e + 1] = f.y;
+    }
+    cs[4 * k] = cv[k].x; cs[4 * k + 1] = cv[k].y; cs[4 * k + 2] = cv[k].z; cs[4 * k + 3] = cv[k].w;
+    sn[4 * k] = sv[k].x; sn[4 * k + 1] = sv[k].y; sn[4 * k + 2] = sv[k].z; sn[4 * k + 3] = sv[k].w;
+  }
+  // local pair i: (x[2i], x[2i+1]) when interleaved, (x[i], x[16+i]) otherwise
+  float y[32];
+  if (interleaved) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) rope_turn(x[2 * i], x[2 * i + 1], cs[i], sn[i], y[2 * i], y[2 * i + 1]);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) rope_turn(x[i], x[16 + i], cs[i], sn[i], y[i], y[16 + i]);
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k)
+    dst[ch[k]] = make_uint4(pack_bf16x2(y[k * 8], y[k * 8 + 1]), pack_bf16x2(y[k * 8 + 2], y[k * 8 + 3]),
+                            pack_bf16x2(y[k * 8 + 4], y[k * 8 + 5]), pack_bf16x2(y[k * 8 + 6], y[k * 8 + 7]));
 }
 
 // ---- segments of one CTA's row range --------------------------------------------
@@ -598,6 +634,20 @@ struct HgParams {
   int B, Nout, K;
   int a_row0;            // first weight row of head h: a_row0 + h * a_hstride
   int a_hstride;
+  // q absorption only: the CTAs of the first output block also rotate q_pe
+  // into out[b, h, Nout:], and one extra CTA (x index H) builds the split
+  // schedule of the attention
+  const __nv_bfloat16* q;
+  const int32_t* positions;
+  const float* cos_t;
+  const float* sin_t;
+  int max_pos, N, interleaved;     // rotary width 64
+  const int32_t* lens;
+  const int64_t* offsets;
+  int max_len, G;
+  int64_t cache_rows;
+  int64_t* prefix;
+  int64_t* meta;
 };
 
 template <bool kAMN>
@@ -609,6 +659,11 @@ head_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
   __shared__ int abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int h = blockIdx.x, n0 = blockIdx.y * 128, b0 = blockIdx.z * 64;
+  if (kAMN && h == (int)gridDim.x - 1) {   // the extra CTA column (uniform over the CTA)
+    if (blockIdx.y == 0 && blockIdx.z == 0)
+      decode_schedule_block(p.lens, p.offsets, p.B, p.max_len, p.cache_rows, p.G, p.prefix, p.meta);
+    return;
+  }
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + kHgStages * kHgABytes;
@@ -683,6 +738,9 @@ head_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
         }
       }
     }
+    if (kAMN && blockIdx.y == 0)
+      decode_qrope_rows(p.q, p.positions, p.cos_t, p.sin_t, p.max_pos, h, b0, min(64, p.B - b0), gridDim.x - 1,
+                        p.Nout, p.N, p.interleaved, p.out, threadIdx.x - 64);
   }
   tc_fence_before();
   __syncthreads();
