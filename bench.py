@@ -306,9 +306,10 @@ def run_ours(args, rank, world, device):
     torch.cuda.synchronize()
     mla.mla_check_device_status()
 
-    # timed region: per-step events around prefill and decode, per-kernel events
+    # timed region: events around the prefill and the decode of each step (no
+    # events between the kernels of one call, which would keep the next
+    # kernel from starting while the previous one finishes)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    kev_p, kev_d = [], []
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
@@ -316,18 +317,25 @@ def run_ours(args, rank, world, device):
     with ClockSampler(device) as clocks:
         for i in range(args.steps):
             flush.fill_(i & 0xff)
-            kp, kd = mla.KernelEvents(16), mla.KernelEvents(16)
             ev[i][0].record()
-            with kp:
-                prefill()
+            prefill()
             ev[i][1].record()
-            with kd:
-                decode()
+            decode()
             ev[i][2].record()
-            kev_p.append(kp)
-            kev_d.append(kd)
         torch.cuda.synchronize()
     launches = mla.mla_launch_count() - launches0
+    # per-kernel breakdown: the same steps again, with events around every kernel
+    kev_p, kev_d = [], []
+    for i in range(args.steps):
+        flush.fill_(i & 0xff)
+        kp, kd = mla.KernelEvents(16), mla.KernelEvents(16)
+        with kp:
+            prefill()
+        with kd:
+            decode()
+        kev_p.append(kp)
+        kev_d.append(kd)
+    torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     mla.mla_check_device_status()

@@ -100,6 +100,26 @@ void prof_end(cudaStream_t st) {
   }
 }
 
+// Launch with programmatic stream serialization: the kernel may begin while
+// the previous kernel of the stream is finishing; it waits in device code
+// (pdl_wait) before it reads that kernel's results. Used for the second and
+// later kernels of one call.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_dependent(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                             Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 // ---- YaRN scalars (Kimi-K2 "RoPE coefficients" page, rope excerpt) -------
 double correction_dim(double rotations, int dim, double base, double max_pos) {
   return (dim * log(max_pos / (rotations * 2.0 * M_PI))) / (2.0 * log(base));
@@ -321,9 +341,9 @@ int launch_attention_tc_t(unsigned grid, const CUtensorMap& mq, const CUtensorMa
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
   if (e != cudaSuccess) return cuda_status(e, "attention smem attribute");
   prof_begin(st, "tc_attention");
-  kern<<<grid, mla::tc::kAttThreads, C::kSmem, st>>>(mq, mkn, mkr, mvt, ap);
+  e = launch_dependent(kern, dim3(grid), dim3(mla::tc::kAttThreads), C::kSmem, st, mq, mkn, mkr, mvt, ap);
   prof_end(st);
-  return cuda_status(cudaGetLastError(), "attention launch");
+  return cuda_status(e, "attention launch");
 }
 
 int launch_attention_tc(int N, int V, unsigned grid, const CUtensorMap& mq, const CUtensorMap& mkn,
@@ -350,9 +370,9 @@ int launch_attention_pair_t(unsigned grid, const CUtensorMap& mq, const CUtensor
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
   if (e != cudaSuccess) return cuda_status(e, "attention smem attribute");
   prof_begin(st, "tc_attention");
-  kern<<<grid, mla::tc::kPrThreads, C::kSmem, st>>>(mq, mkn, mkr, mvt, ap);
+  e = launch_dependent(kern, dim3(grid), dim3(mla::tc::kPrThreads), C::kSmem, st, mq, mkn, mkr, mvt, ap);
   prof_end(st);
-  return cuda_status(cudaGetLastError(), "attention launch");
+  return cuda_status(e, "attention launch");
 }
 
 int launch_attention_pair(int N, int V, unsigned grid, const CUtensorMap& mq, const CUtensorMap& mkn,
@@ -449,16 +469,19 @@ int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, cons
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mla::tc::kG2SmemBytes);
     if (e != cudaSuccess) return cuda_status(e, "gemm smem attribute");
     prof_begin(st, "tc_norm_kv_b_proj");
-    kern<<<dim3(cap, gy2), mla::tc::kG2Threads, mla::tc::kG2SmemBytes, st>>>(map_lat, map_w, gp);
+    e = launch_dependent(kern, dim3(cap, gy2), dim3(mla::tc::kG2Threads), mla::tc::kG2SmemBytes, st, map_lat, map_w,
+                         gp);
     prof_end(st);
+    if (e != cudaSuccess) return cuda_status(e, "gemm launch");
   } else {
     e = cudaFuncSetAttribute(mla::tc::norm_kvb_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)mla::tc::kGemmSmemBytes);
     if (e != cudaSuccess) return cuda_status(e, "gemm smem attribute");
     prof_begin(st, "tc_norm_kv_b_proj");
-    mla::tc::norm_kvb_gemm_kernel<<<dim3(cap, gy), mla::tc::kGemmThreads, mla::tc::kGemmSmemBytes, st>>>(
-        map_lat, map_w, gp);
+    e = launch_dependent(mla::tc::norm_kvb_gemm_kernel, dim3(cap, gy), dim3(mla::tc::kGemmThreads),
+                         mla::tc::kGemmSmemBytes, st, map_lat, map_w, gp);
     prof_end(st);
+    if (e != cudaSuccess) return cuda_status(e, "gemm launch");
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_status(e, "gemm launch");
@@ -668,12 +691,16 @@ int launch_decode_tc(const mla_dims* d, const void* q, const void* cache, int64_
   e = cudaFuncSetAttribute(T::decode_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)T::kDecSmem);
   if (e != cudaSuccess) return cuda_status(e, "decode smem attribute");
   prof_begin(st, "tc_decode_attention");
-  T::decode_attn_kernel<<<L.G, T::kDecThreads, T::kDecSmem, st>>>(map_cache, map_q, dp);
+  e = launch_dependent(T::decode_attn_kernel, dim3(L.G), dim3(T::kDecThreads), T::kDecSmem, st, map_cache, map_q, dp);
   prof_end(st);
+  if (e != cudaSuccess) return cuda_status(e, "decode attention launch");
 
   prof_begin(st, "tc_decode_combine");
-  T::decode_combine_kernel<<<dim3(B, (H + 3) / 4), 256, 0, st>>>(o_part, m_part, l_part, prefix, meta, H, R, o_lat);
+  e = launch_dependent(T::decode_combine_kernel, dim3(B, (H + 3) / 4), dim3(256), 0, st, (const float*)o_part,
+                       (const float*)m_part, (const float*)l_part, (const int64_t*)prefix, (const int64_t*)meta, H, R,
+                       o_lat);
   prof_end(st);
+  if (e != cudaSuccess) return cuda_status(e, "decode combine launch");
 
   // out[b, h, :] = W_UV_h o_lat[b, h, :]   (W_UV_h = rows N .. N+V-1 of head h: [V, R], R contiguous)
   {
@@ -687,8 +714,10 @@ int launch_decode_tc(const mla_dims* d, const void* q, const void* cache, int64_
     hp.a_row0 = N;
     hp.a_hstride = N + V;
     prof_begin(st, "tc_decode_unabsorb");
-    T::head_gemm_kernel<false><<<dim3(H, (V + 127) / 128, (B + 63) / 64), 192, T::kHgSmem, st>>>(map_wv, map_ol, hp);
+    e = launch_dependent(T::head_gemm_kernel<false>, dim3(H, (V + 127) / 128, (B + 63) / 64), dim3(192), T::kHgSmem,
+                         st, map_wv, map_ol, hp);
     prof_end(st);
+    if (e != cudaSuccess) return cuda_status(e, "decode un-absorb launch");
   }
   return cuda_status(cudaGetLastError(), "decode launch");
 }

@@ -79,6 +79,7 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ AttBarriers<kStages> bars;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_allow_next();
   const int rank = blockIdx.x / p.H, h = blockIdx.x % p.H;
   const int tile = p.order[rank];
   if (tile < 0) return;   // uniform over the CTA
@@ -122,6 +123,7 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       mbar_arrive_expect_tx(&bars.q_full, C::kQBytes);
       for (int a = 0; a < C::kQAtoms; ++a)
         tma_load_3d(sQ + a * kTile * 128, &map_q, &bars.q_full, a * 64, h, (int)(seq0 + q0));
+      pdl_wait();   // k_nope, the values and k_rot come from the previous kernel
       bool ok = true;
       int j = 0;
       for (; j < n_kv; ++j) {

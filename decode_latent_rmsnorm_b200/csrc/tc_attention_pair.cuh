@@ -89,6 +89,7 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ PairBarriers bars;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_allow_next();
   const int rank = blockIdx.x / p.H, h = blockIdx.x % p.H;
   const int tile = p.order[rank];       // first tile of the block
   if (tile < 0) return;                 // uniform over the CTA
@@ -148,6 +149,7 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
         uint64_t* bar = (gp % C::kBoxes) < C::kQAtoms ? &bars.kempty[jp & 3] : &bars.vempty[jp & 3];
         return mbar_wait(bar, (uint32_t)(jp >> 2) & 1u, abort_flag);
       };
+      pdl_wait();   // k_nope, the values and k_rot come from the previous kernel
       bool ok = true;
       int jk = -1, jv = -1;              // last key / value group issued
       for (int j = 0; j < n && ok; ++j) {

@@ -305,6 +305,8 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_c
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ DecBarriers bars;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_wait();         // the schedule and the absorbed queries come from the previous kernel
+  pdl_allow_next();
   const int c = blockIdx.x;
   const int64_t per = p.meta[0], total = p.meta[1];
   const int64_t r_lo = (int64_t)c * per;
@@ -579,6 +581,8 @@ __global__ void __launch_bounds__(256)
 decode_combine_kernel(const float* __restrict__ o_part, const float* __restrict__ m_part,
                       const float* __restrict__ l_part, const int64_t* __restrict__ prefix,
                       const int64_t* __restrict__ meta, int H, int R, __nv_bfloat16* __restrict__ o_lat) {
+  pdl_wait();         // the partials come from the previous kernel
+  pdl_allow_next();
   const int b = blockIdx.x;
   const int h = blockIdx.y * 4 + (threadIdx.x >> 6);
   const int d0 = (threadIdx.x & 63) * 8;
@@ -658,6 +662,8 @@ head_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (!kAMN) pdl_wait();   // un-absorption: o_lat comes from the previous kernel
+  pdl_allow_next();
   const int h = blockIdx.x, n0 = blockIdx.y * 128, b0 = blockIdx.z * 64;
   if (kAMN && h == (int)gridDim.x - 1) {   // the extra CTA column (uniform over the CTA)
     if (blockIdx.y == 0 && blockIdx.z == 0)

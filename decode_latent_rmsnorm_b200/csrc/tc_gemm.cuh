@@ -37,6 +37,29 @@ constexpr int kTile = 128;            // token rows per tile (M of the MMAs)
 // one sequence; the second may not exist), blocks sorted by decreasing k.
 // Entries past the real tile / block count are -1. Bad cu_seqlens set the
 // device error word and leave every entry at -1.
+// Inclusive prefix sum over the 1024 threads of a block (thread order):
+// a shuffle scan inside each warp, then one over the 32 warp totals.
+// Every thread of the block must call it.
+__device__ __forceinline__ int block_inclusive_scan_1024(int v, int* s_warp /* [32] */) {
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, v, o);
+    if (lane >= o) v += y;
+  }
+  __syncthreads();                       // s_warp free from any earlier use
+  if (lane == 31) s_warp[wid] = v;
+  __syncthreads();
+  int w = s_warp[lane];
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, w, o);
+    if (lane >= o) w += y;
+  }
+  const int before = __shfl_sync(0xffffffffu, w, (wid + 31) & 31);   // total of the earlier warps
+  return v + (wid > 0 ? before : 0);
+}
+
 // Run by one block of 1024 threads.
 __device__ __forceinline__ void schedule_block(const int32_t* __restrict__ cu, int nseq, int64_t Ttot,
                                                int max_seqlen, int cap, int32_t* __restrict__ seq_tile0,
@@ -64,17 +87,10 @@ __device__ __forceinline__ void schedule_block(const int32_t* __restrict__ cu, i
       if (a < 0 || b < a || b > Ttot || b - a > max_seqlen) s_bad = 1;
       else nt = (int)((b - a + kTile - 1) / kTile);
     }
-    s_scan[tid] = nt;
+    const int inc = block_inclusive_scan_1024(nt, s_scan);
+    if (s <= nseq) seq_tile0[s] = s_carry + inc - nt;
     __syncthreads();
-    for (int off = 1; off < (int)blockDim.x; off <<= 1) {
-      const int v = tid >= off ? s_scan[tid - off] : 0;
-      __syncthreads();
-      s_scan[tid] += v;
-      __syncthreads();
-    }
-    if (s <= nseq) seq_tile0[s] = s_carry + s_scan[tid] - nt;
-    __syncthreads();
-    if (tid == (int)blockDim.x - 1) s_carry += s_scan[tid];
+    if (tid == (int)blockDim.x - 1) s_carry += inc;
     __syncthreads();
   }
   if (s_bad) {
@@ -101,15 +117,7 @@ __device__ __forceinline__ void schedule_block(const int32_t* __restrict__ cu, i
     // Thread i owns reversed buckets 2i and 2i + 1 (bucket kBuckets-1-2i, ...).
     const int k0 = kBuckets - 1 - 2 * tid, k1 = k0 - 1;
     const int c0 = s_cnt[k0], c1 = s_cnt[k1];
-    s_scan[tid] = c0 + c1;
-    __syncthreads();
-    for (int off = 1; off < (int)blockDim.x; off <<= 1) {
-      const int v = tid >= off ? s_scan[tid - off] : 0;
-      __syncthreads();
-      s_scan[tid] += v;
-      __syncthreads();
-    }
-    const int before = s_scan[tid] - (c0 + c1);
+    const int before = block_inclusive_scan_1024(c0 + c1, s_scan) - (c0 + c1);
     s_off[k0] = before;
     s_off[k1] = before + c0;
   }
@@ -133,15 +141,7 @@ __device__ __forceinline__ void schedule_block(const int32_t* __restrict__ cu, i
   {
     const int k0 = kBuckets - 1 - 2 * tid, k1 = k0 - 1;
     const int c0 = s_cnt[k0], c1 = s_cnt[k1];
-    s_scan[tid] = c0 + c1;
-    __syncthreads();
-    for (int off = 1; off < (int)blockDim.x; off <<= 1) {
-      const int v = tid >= off ? s_scan[tid - off] : 0;
-      __syncthreads();
-      s_scan[tid] += v;
-      __syncthreads();
-    }
-    const int before = s_scan[tid] - (c0 + c1);
+    const int before = block_inclusive_scan_1024(c0 + c1, s_scan) - (c0 + c1);
     s_off[k0] = before;
     s_off[k1] = before + c0;
   }
@@ -166,6 +166,7 @@ prefill_prep_kernel(const int32_t* __restrict__ cu, int nseq, int64_t Ttot, int 
                     int32_t* __restrict__ seq_tile0, int32_t* __restrict__ tile_seq,
                     int32_t* __restrict__ tile_q0, int32_t* __restrict__ order, int32_t* __restrict__ pair_order,
                     const __nv_bfloat16* __restrict__ w, __half* __restrict__ w16, int64_t n8) {
+  pdl_allow_next();
   if (blockIdx.x == 0) {
     schedule_block(cu, nseq, Ttot, max_seqlen, cap, seq_tile0, tile_seq, tile_q0, order, pair_order);
     return;
@@ -245,6 +246,8 @@ norm_kvb_gemm_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_c
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ GemmBarriers bars;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_wait();         // the schedule and the fp16 weight come from the previous kernel
+  pdl_allow_next();
   const int tile = blockIdx.x;
   const int seq = p.tile_seq[tile];
   if (seq < 0) return;   // past the real tiles (uniform over the CTA)
@@ -478,6 +481,8 @@ norm_kvb_gemm_vt_kernel(const __grid_constant__ CUtensorMap map_lat, const __gri
   __shared__ GemmBarriers bars;
   __shared__ uint4 s_wnorm[kGemmMaxAtoms * 8];   // the RMSNorm weight, 8 bf16 per entry
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_wait();         // the schedule and the fp16 weight come from the previous kernel
+  pdl_allow_next();
   const int tile = blockIdx.x;
   const int seq = p.tile_seq[tile];
   if (seq < 0) return;   // past the real tiles (uniform over the CTA)
