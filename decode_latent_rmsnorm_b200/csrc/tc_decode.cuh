@@ -369,55 +369,54 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_c
       }
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
-      const uint32_t idesc_s = idesc_bf16_f32(kDecRows, kDecHeads);
-      const uint32_t idesc_o = idesc_bf16_f32(128, kDecHeads) | kIdescAMajorMN | kIdescBMajorMN;
-      bool ok = true;
-      int j = 0;
-      DecTileIter tiles;
-      tiles.init(p, r_lo, r_hi);
-      DecTile t;
-      while (ok && tiles.next(t)) {
-        const uint32_t ph = (uint32_t)j & 1u;
-        // ---- S^T(j) ----
-        if (t.first && !(ok = mbar_wait(&bars.q_full, (uint32_t)t.seg & 1u, abort_flag))) break;
-        if (!(ok = mbar_wait(&bars.s_free, ph ^ 1u, abort_flag))) break;
+    // ---------------- MMA issuer (whole warp; one elected lane issues) ----------------
+    const uint32_t idesc_s = idesc_bf16_f32(kDecRows, kDecHeads);
+    const uint32_t idesc_o = idesc_bf16_f32(128, kDecHeads) | kIdescAMajorMN | kIdescBMajorMN;
+    bool ok = true;
+    int j = 0;
+    DecTileIter tiles;
+    tiles.init(p, r_lo, r_hi);
+    DecTile t;
+    while (ok && tiles.next(t)) {
+      const uint32_t ph = (uint32_t)j & 1u;
+      // ---- S^T(j) ----
+      if (t.first && !(ok = mbar_wait_warp(&bars.q_full, (uint32_t)t.seg & 1u, abort_flag))) break;
+      if (!(ok = mbar_wait_warp(&bars.s_free, ph ^ 1u, abort_flag))) break;
+      tc_fence_after();
+      for (int a = 0; a < kDecBoxes && ok; ++a) {
+        if (!(ok = mbar_wait_warp(&bars.full[a], ph, abort_flag))) break;
         tc_fence_after();
-        for (int a = 0; a < kDecBoxes && ok; ++a) {
-          if (!(ok = mbar_wait(&bars.full[a], ph, abort_flag))) break;
-          tc_fence_after();
-          const uint64_t cd = desc_kmajor_sw128(smem_u32(sSlot + a * kDecBoxBytes));
-          const uint64_t qd = desc_kmajor_sw128(smem_u32(sQ + a * kDecHeads * 128));
+        const uint64_t cd = desc_kmajor_sw128(smem_u32(sSlot + a * kDecBoxBytes));
+        const uint64_t qd = desc_kmajor_sw128(smem_u32(sQ + a * kDecHeads * 128));
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            mma_bf16_ss(tmem + kDecSCol, desc_advance(cd, k * 32), desc_advance(qd, k * 32), idesc_s, (a | k) != 0);
-        }
-        if (!ok) break;
-        mma_commit(&bars.s_full);
-        if (t.last) mma_commit(&bars.q_empty);     // q may be replaced once these are done
-        // ---- O^T(j) += C^T P^T ----
-        if (t.first && t.seg > 0 && !(ok = mbar_wait(&bars.o_free, (uint32_t)(t.seg - 1) & 1u, abort_flag))) break;
-        if (!(ok = mbar_wait(&bars.p_full, ph, abort_flag))) break;
-        tc_fence_after();
-        const uint64_t pd = desc_mnmajor_sw128(smem_u32(sP), kDecBoxBytes, 1024);
-        for (int blk = 0; blk < 4; ++blk) {
-          // latent columns [128 blk, 128 blk + 128): slots 2 blk, 2 blk + 1, read MN-major
-          const uint64_t ad = desc_mnmajor_sw128(smem_u32(sSlot + 2 * blk * kDecBoxBytes), kDecBoxBytes, 1024);
-#pragma unroll
-          for (int k = 0; k < kDecRows / 16; ++k)
-            mma_bf16_ss(tmem + kDecOCol + blk * kDecHeads, desc_advance(ad, k * 2048), desc_advance(pd, k * 2048),
-                        idesc_o, (t.first && k == 0) ? 0u : 1u);
-          mma_commit(&bars.empty[2 * blk]);
-          mma_commit(&bars.empty[2 * blk + 1]);
-        }
-        mma_commit(&bars.empty[kDecSlots - 1]);    // P^T read: the rope slot is free
-        mma_commit(&bars.pv_done);
-        ++j;
+        for (int k = 0; k < 4; ++k)
+          mma_ss_elect(tmem + kDecSCol, desc_advance(cd, k * 32), desc_advance(qd, k * 32), idesc_s, (a | k) != 0);
       }
-      mma_commit(&bars.mma_done);          // every MMA done before TMEM is freed
-      mbar_wait_drain(&bars.mma_done, 0);
+      if (!ok) break;
+      mma_commit_elect(&bars.s_full);
+      if (t.last) mma_commit_elect(&bars.q_empty);     // q may be replaced once these are done
+      // ---- O^T(j) += C^T P^T ----
+      if (t.first && t.seg > 0 && !(ok = mbar_wait_warp(&bars.o_free, (uint32_t)(t.seg - 1) & 1u, abort_flag))) break;
+      if (!(ok = mbar_wait_warp(&bars.p_full, ph, abort_flag))) break;
+      tc_fence_after();
+      const uint64_t pd = desc_mnmajor_sw128(smem_u32(sP), kDecBoxBytes, 1024);
+      for (int blk = 0; blk < 4; ++blk) {
+        // latent columns [128 blk, 128 blk + 128): slots 2 blk, 2 blk + 1, read MN-major
+        const uint64_t ad = desc_mnmajor_sw128(smem_u32(sSlot + 2 * blk * kDecBoxBytes), kDecBoxBytes, 1024);
+#pragma unroll
+        for (int k = 0; k < kDecRows / 16; ++k)
+          mma_ss_elect(tmem + kDecOCol + blk * kDecHeads, desc_advance(ad, k * 2048), desc_advance(pd, k * 2048),
+                       idesc_o, (t.first && k == 0) ? 0u : 1u);
+        mma_commit_elect(&bars.empty[2 * blk]);
+        mma_commit_elect(&bars.empty[2 * blk + 1]);
+      }
+      mma_commit_elect(&bars.empty[kDecSlots - 1]);    // P^T read: the rope slot is free
+      mma_commit_elect(&bars.pv_done);
+      ++j;
     }
+    mma_commit_elect(&bars.mma_done);          // every MMA done before TMEM is freed
+    if (lane == 0) mbar_wait_drain(&bars.mma_done, 0);
+    __syncwarp();
   } else {
     // ---------------- softmax / correction / partial epilogue (warps 2-5) ----------------
     const int grp = warp & 3;                       // TMEM quadrant
