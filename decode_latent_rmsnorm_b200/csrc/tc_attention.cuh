@@ -145,48 +145,47 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       }
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0) {
-      const uint32_t idesc_s = idesc_f16_f32(kTile, kAttBKV);
-      const uint32_t idesc_o = idesc_f16_f32(kTile, kV);
-      const uint32_t o_tmem = tmem + C::kOCol;
-      bool ok = mbar_wait(&bars.q_ready, 0, abort_flag);
+    // ---------------- MMA issuer (whole warp; one elected lane issues) ----------------
+    const uint32_t idesc_s = idesc_f16_f32(kTile, kAttBKV);
+    const uint32_t idesc_o = idesc_f16_f32(kTile, kV);
+    const uint32_t o_tmem = tmem + C::kOCol;
+    bool ok = mbar_wait_warp(&bars.q_ready, 0, abort_flag);
+    tc_fence_after();
+    auto issue_pv = [&](int jj) -> bool {
+      if (!mbar_wait_warp(&bars.p_full, (uint32_t)jj & 1u, abort_flag)) return false;
       tc_fence_after();
-      auto issue_pv = [&](int jj) -> bool {
-        if (!mbar_wait(&bars.p_full, (uint32_t)jj & 1u, abort_flag)) return false;
-        tc_fence_after();
-        const int s = jj % kStages;
-        const uint64_t pd = desc_kmajor_sw128(smem_u32(sP));
-        const uint64_t vd = desc_kmajor_sw128(smem_u32(sKV + s * C::kStageBytes + C::kKBytes));
+      const int s = jj % kStages;
+      const uint64_t pd = desc_kmajor_sw128(smem_u32(sP));
+      const uint64_t vd = desc_kmajor_sw128(smem_u32(sKV + s * C::kStageBytes + C::kKBytes));
 #pragma unroll
-        for (int k = 0; k < kAttBKV / 16; ++k)
-          mma_bf16_ss(o_tmem, desc_advance(pd, k * 32), desc_advance(vd, k * 32), idesc_o, (jj | k) != 0);
-        mma_commit(&bars.kv_empty[s]);
-        mma_commit(&bars.pv_done);
-        return true;
-      };
-      for (int j = 0; j < n_kv && ok; ++j) {
-        const int s = j % kStages, b = j & 1;
-        if (!mbar_wait(&bars.kv_full[s], (uint32_t)(j / kStages) & 1u, abort_flag)) { ok = false; break; }
-        if (!mbar_wait(&bars.s_free[b], ((uint32_t)(j >> 1) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
-        tc_fence_after();
-        const uint8_t* sK = sKV + s * C::kStageBytes;
-        const uint32_t s_tmem = tmem + C::kSCol + b * kAttBKV;
+      for (int k = 0; k < kAttBKV / 16; ++k)
+        mma_ss_elect(o_tmem, desc_advance(pd, k * 32), desc_advance(vd, k * 32), idesc_o, (jj | k) != 0);
+      mma_commit_elect(&bars.kv_empty[s]);
+      mma_commit_elect(&bars.pv_done);
+      return true;
+    };
+    for (int j = 0; j < n_kv && ok; ++j) {
+      const int s = j % kStages, b = j & 1;
+      if (!mbar_wait_warp(&bars.kv_full[s], (uint32_t)(j / kStages) & 1u, abort_flag)) { ok = false; break; }
+      if (!mbar_wait_warp(&bars.s_free[b], ((uint32_t)(j >> 1) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+      tc_fence_after();
+      const uint8_t* sK = sKV + s * C::kStageBytes;
+      const uint32_t s_tmem = tmem + C::kSCol + b * kAttBKV;
 #pragma unroll
-        for (int a = 0; a < C::kQAtoms; ++a) {
-          const uint64_t qd = desc_kmajor_sw128(smem_u32(sQ + a * kTile * 128));
-          const uint64_t kd = desc_kmajor_sw128(smem_u32(sK + a * C::kKAtomBytes));
+      for (int a = 0; a < C::kQAtoms; ++a) {
+        const uint64_t qd = desc_kmajor_sw128(smem_u32(sQ + a * kTile * 128));
+        const uint64_t kd = desc_kmajor_sw128(smem_u32(sK + a * C::kKAtomBytes));
 #pragma unroll
-          for (int k = 0; k < 4; ++k)
-            mma_bf16_ss(s_tmem, desc_advance(qd, k * 32), desc_advance(kd, k * 32), idesc_s, (a | k) != 0);
-        }
-        mma_commit(&bars.s_full[b]);
-        if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
+        for (int k = 0; k < 4; ++k)
+          mma_ss_elect(s_tmem, desc_advance(qd, k * 32), desc_advance(kd, k * 32), idesc_s, (a | k) != 0);
       }
-      if (ok && n_kv > 0) issue_pv(n_kv - 1);
-      mma_commit(&bars.mma_done);     // every MMA done before TMEM is freed
-      mbar_wait_drain(&bars.mma_done, 0);
+      mma_commit_elect(&bars.s_full[b]);
+      if (j >= 1 && !issue_pv(j - 1)) { ok = false; break; }
     }
+    if (ok && n_kv > 0) issue_pv(n_kv - 1);
+    mma_commit_elect(&bars.mma_done);     // every MMA done before TMEM is freed
+    if (lane == 0) mbar_wait_drain(&bars.mma_done, 0);
+    __syncwarp();
   } else {
     // ---------------- softmax / correction / epilogue (warps 2-5) ----------------
     const int grp = warp & 3;

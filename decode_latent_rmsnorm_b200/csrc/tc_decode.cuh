@@ -707,24 +707,23 @@ head_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
           mbar_wait_drain(&full[i % kHgStages], (uint32_t)(i / kHgStages) & 1u);
     }
   } else if (warp == 1) {
-    if (lane == 0) {
-      const uint32_t idesc = idesc_bf16_f32(128, 64) | (kAMN ? kIdescAMajorMN : 0u);
-      for (int kc = 0; kc < nk; ++kc) {
-        const int s = kc % kHgStages;
-        if (!mbar_wait(&full[s], (uint32_t)(kc / kHgStages) & 1u, &abort_flag)) break;
-        tc_fence_after();
-        const uint32_t aaddr = smem_u32(sA + s * kHgABytes);
-        const uint64_t ad = kAMN ? desc_mnmajor_sw128(aaddr, kHgABytes / 2, 1024) : desc_kmajor_sw128(aaddr);
-        const uint64_t bd = desc_kmajor_sw128(smem_u32(sB + s * kHgBBytes));
+    // MMA issuer: whole warp, one elected lane issues
+    const uint32_t idesc = idesc_bf16_f32(128, 64) | (kAMN ? kIdescAMajorMN : 0u);
+    for (int kc = 0; kc < nk; ++kc) {
+      const int s = kc % kHgStages;
+      if (!mbar_wait_warp(&full[s], (uint32_t)(kc / kHgStages) & 1u, &abort_flag)) break;
+      tc_fence_after();
+      const uint32_t aaddr = smem_u32(sA + s * kHgABytes);
+      const uint64_t ad = kAMN ? desc_mnmajor_sw128(aaddr, kHgABytes / 2, 1024) : desc_kmajor_sw128(aaddr);
+      const uint64_t bd = desc_kmajor_sw128(smem_u32(sB + s * kHgBBytes));
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          mma_bf16_ss(tmem, desc_advance(ad, kAMN ? k * 2048 : k * 32), desc_advance(bd, k * 32), idesc,
-                      (kc | k) != 0);
-        mma_commit(&empty[s]);
-      }
-      mma_commit(&done);
-      mbar_wait_drain(&done, 0);
+      for (int k = 0; k < 4; ++k)
+        mma_ss_elect(tmem, desc_advance(ad, kAMN ? k * 2048 : k * 32), desc_advance(bd, k * 32), idesc, (kc | k) != 0);
+      mma_commit_elect(&empty[s]);
     }
+    mma_commit_elect(&done);
+    if (lane == 0) mbar_wait_drain(&done, 0);
+    __syncwarp();
   } else {
     const int grp = warp & 3;
     const int n = n0 + grp * 32 + lane;

@@ -307,33 +307,34 @@ norm_kvb_gemm_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_c
       }
     }
   } else if (warp == 1) {
-    // ---------------- MMA issuer ----------------
-    if (lane == 0 && my_tiles > 0) {
+    // ---------------- MMA issuer (whole warp; one elected lane issues) ----------------
+    if (my_tiles > 0) {
       const uint32_t idesc = idesc_f16_f32(kTile, kGemmBN);
-      bool ok = mbar_wait(&bars.a_ready, 0, abort_flag);
+      bool ok = mbar_wait_warp(&bars.a_ready, 0, abort_flag);
       tc_fence_after();
       int it = 0;
       for (int i = 0; i < my_tiles && ok; ++i) {
         const int acc = i & 1;
-        if (!mbar_wait(&bars.acc_empty[acc], ((uint32_t)(i >> 1) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+        if (!mbar_wait_warp(&bars.acc_empty[acc], ((uint32_t)(i >> 1) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
         const uint32_t d = tmem + (uint32_t)(acc * kGemmBN);
         for (int kc = 0; kc < natoms; ++kc, ++it) {
           const int s = it % kGemmStages;
-          if (!mbar_wait(&bars.b_full[s], (uint32_t)(it / kGemmStages) & 1u, abort_flag)) { ok = false; break; }
+          if (!mbar_wait_warp(&bars.b_full[s], (uint32_t)(it / kGemmStages) & 1u, abort_flag)) { ok = false; break; }
           tc_fence_after();
           const uint64_t ad = desc_kmajor_sw128(smem_u32(sA + kc * kAtomBytes));
           const uint64_t bd = desc_kmajor_sw128(smem_u32(sB + s * kStageBytes));
 #pragma unroll
           for (int k = 0; k < 4; ++k)
-            mma_bf16_ss(d, desc_advance(ad, k * 32), desc_advance(bd, k * 32), idesc, (kc | k) != 0);
-          mma_commit(&bars.b_empty[s]);
+            mma_ss_elect(d, desc_advance(ad, k * 32), desc_advance(bd, k * 32), idesc, (kc | k) != 0);
+          mma_commit_elect(&bars.b_empty[s]);
         }
         if (!ok) break;
-        mma_commit(&bars.acc_full[acc]);
+        mma_commit_elect(&bars.acc_full[acc]);
       }
-      mma_commit(&bars.mma_done);          // every MMA done before TMEM is freed
-      mbar_wait_drain(&bars.mma_done, 0);
+      mma_commit_elect(&bars.mma_done);          // every MMA done before TMEM is freed
+      if (lane == 0) mbar_wait_drain(&bars.mma_done, 0);
+      __syncwarp();
     }
   } else {
     // ---------------- RMSNorm prologue, then epilogue (warps 2-5) ----------------

@@ -143,32 +143,13 @@ __device__ __forceinline__ void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// D[tmem] (+)= A[smem] * B[smem]^T, bf16 inputs, fp32 accumulate, one thread.
-__device__ __forceinline__ void mma_bf16_ss(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                                            uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// D[tmem] (+)= A[tmem] * B[smem]^T, fp16 inputs, fp32 accumulate, one thread.
-// A (M = 128 rows) sits in TMEM lanes 0-127, row i in lane i; each 32-bit
-// column packs two consecutive K elements (low half first), so one K = 16
-// step spans 8 columns.
-__device__ __forceinline__ void mma_f16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc, uint32_t idesc,
-                                           uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-// Warp-uniform forms: every lane of the warp executes the call (so loop
-// state and descriptors stay warp-uniform) and one elected lane issues the
-// instruction.
+// Matrix products issued by a warp: D[tmem] (+)= A * B^T with A in shared
+// memory (ss) or in TMEM (ts), fp32 accumulate; the operand types come from
+// the instruction descriptor. For the ts form, A (M = 128 rows) sits in TMEM
+// lanes 0-127, row i in lane i, each 32-bit column packing two consecutive K
+// elements (low half first), so one K = 16 step spans 8 columns. Every lane
+// of the warp executes the call (so loop state and descriptors stay
+// warp-uniform) and one elected lane issues the instruction.
 __device__ __forceinline__ void mma_ss_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                              uint32_t accumulate) {
   asm volatile(
@@ -189,6 +170,7 @@ __device__ __forceinline__ void mma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, u
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// Arrive on `bar` once every tcgen05 op the warp issued so far is done.
 __device__ __forceinline__ void mma_commit_elect(uint64_t* bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t"
@@ -197,13 +179,6 @@ __device__ __forceinline__ void mma_commit_elect(uint64_t* bar) {
           smem_u32(bar))
       : "memory");
 }
-// Arrive on `bar` once every tcgen05 op this thread issued so far is done.
-__device__ __forceinline__ void mma_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_u32(bar))
-               : "memory");
-}
-
 // Warp-collective: lane i of the warp reads TMEM lane (taddr.lane + i),
 // 16 consecutive 32-bit columns starting at taddr.col. The load and its
 // tcgen05.wait::ld sit in one asm statement, so no use of the registers can
