@@ -442,12 +442,14 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_c
       if (!mbar_wait_warp(&bars.s_full, (uint32_t)j & 1u, abort_flag)) { ok = false; break; }
       tc_fence_after();
       float x[kDecHeads];
+      {   // the row's 64 scores: two loads in flight, one wait
+        uint32_t v[kDecHeads];
 #pragma unroll
-      for (int cc = 0; cc < kDecHeads / 16; ++cc) {
-        uint32_t v[16];
-        tmem_ld16(tmem + lane_base + (uint32_t)(kDecSCol + cc * 16), v);
+        for (int cc = 0; cc < kDecHeads / 32; ++cc)
+          tmem_ld32_nowait(tmem + lane_base + (uint32_t)(kDecSCol + cc * 32), v + cc * 32);
+        tmem_wait_ld64(v);
 #pragma unroll
-        for (int e = 0; e < 16; ++e) x[cc * 16 + e] = __uint_as_float(v[e]);
+        for (int h = 0; h < kDecHeads; ++h) x[h] = __uint_as_float(v[h]);
       }
       tc_fence_before();
       mbar_arrive(&bars.s_free);
