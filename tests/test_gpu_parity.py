@@ -150,6 +150,19 @@ def test_decode_small_all_heads(gpu_lib):
     compare(f64(got), ref, "bf16", "decode small")
 
 
+def test_decode_glm_heads_interleaved_b70(gpu_lib):
+    # GLM-5 heads (qk_nope 192, v_head 256, interleaved rotary pairs), 70
+    # sequences (a partial second batch block in the per-head GEMMs), lengths
+    # around the 128-row tile edges
+    lens = tuple((1, 127, 128, 129, 255, 256, 257)[i % 7] for i in range(70))
+    wl = W.Workload("glm_decode_bf16", "decode", 64, 512, 192, 64, 256, "bf16", W.GLM_ROPE, 16,
+                    interleaved=True, batch=70, cache_lens=lens)
+    inp = W.decode_inputs(wl)
+    got = run_decode(wl, inp)
+    ref = oracle_decode(wl, inp, batches=[0, 1, 2, 3, 4, 5, 6, 33, 64, 65, 69], absorbed=True)
+    compare(f64(got), ref, "bf16", "decode glm b70")
+
+
 def test_decode_fp32_tiny_geometry(gpu_lib):
     wl = W.Workload("tiny_decode_fp32", "decode", 2, 64, 16, 8, 16, "fp32", W.TINY_ROPE, 15,
                     batch=3, cache_lens=(1, 40, 333))
