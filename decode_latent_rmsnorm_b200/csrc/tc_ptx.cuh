@@ -120,10 +120,6 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
 __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
-// Generic-proxy global writes -> visible to later TMA reads.
-__device__ __forceinline__ void fence_proxy_async_global() {
-  asm volatile("fence.proxy.async.global;" ::: "memory");
-}
 
 // ---- tcgen05 ------------------------------------------------------------------
 // Allocation by one full warp; the TMEM base address is written to smem.
@@ -292,18 +288,6 @@ __device__ __forceinline__ uint64_t desc_mnmajor_sw128(uint32_t smem_addr, uint3
   d |= static_cast<uint64_t>(1) << 46;
   d |= static_cast<uint64_t>(2) << 61;
   return d;
-}
-
-// Shared-memory matrix descriptor of a K-major operand tile without swizzle:
-// 8 x 8 core matrices of 16-byte rows (128 bytes each); the two core matrices
-// of one 16-wide K step are `lbo_bytes` apart and 8-row groups `sbo_bytes`.
-__device__ __forceinline__ uint64_t desc_kmajor_noswz(uint32_t smem_addr, uint32_t lbo_bytes, uint32_t sbo_bytes) {
-  uint64_t d = 0;
-  d |= static_cast<uint64_t>((smem_addr & 0x3FFFFu) >> 4);
-  d |= static_cast<uint64_t>((lbo_bytes >> 4) & 0x3FFFu) << 16;
-  d |= static_cast<uint64_t>((sbo_bytes >> 4) & 0x3FFFu) << 32;
-  d |= static_cast<uint64_t>(1) << 46;
-  return d;   // swizzle mode 0
 }
 
 // Next 16-element (32-byte) K step inside a 128-byte swizzle row.
