@@ -181,7 +181,7 @@ bool prefill_tc_shape(const mla_dims* d) {
 struct PrefillWs {
   int64_t cap, Tpad;
   int gemm_tiles_per_cta, gemm_gy;
-  size_t seq_tile0, tile_seq, tile_q0, order, pair_order, w16;
+  size_t seq_tile0, tile_seq, tile_q0, order, pair_order, w16, c16;
   size_t k_nope, vals, k_rot, total;
 };
 PrefillWs prefill_ws_layout(const mla_dims* d, int64_t T, int nseq, bool tc) {
@@ -205,6 +205,7 @@ PrefillWs prefill_ws_layout(const mla_dims* d, int64_t T, int nseq, bool tc) {
     w.order = off;     off = align_up(off + 4 * (size_t)w.cap, 256);
     w.pair_order = off; off = align_up(off + 4 * (size_t)w.cap, 256);
     w.w16 = off;       off = align_up(off + 2 * (size_t)NOUT * d->kv_lora_rank, 256);
+    w.c16 = off;       off = align_up(off + 2 * (size_t)T * d->kv_lora_rank, 256);   // normalized latent, fp16
   } else {
     w.Tpad = T;
   }
@@ -428,14 +429,26 @@ int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, cons
   __half* w16 = reinterpret_cast<__half*>(ws + L.w16);
   const int gy = L.gemm_gy;
 
+  __half* c16 = reinterpret_cast<__half*>(ws + L.c16);
   const int64_t n8 = (int64_t)NOUT * R / 8;
   const int64_t per_block = (int64_t)mla::tc::kPrepThreads * mla::tc::kPrepUnroll;
-  const unsigned prep_blocks = (unsigned)(1 + (n8 + per_block - 1) / per_block);
+  const int w_blocks = (int)((n8 + per_block - 1) / per_block);
+  // the transposed-value GEMM reads c_hat prepared here: one warp per token row
+  const int norm_blocks = vt_gemm ? (int)((T_tot + mla::tc::kPrepThreads / 32 - 1) / (mla::tc::kPrepThreads / 32)) : 0;
   prof_begin(st, "tc_prep");
-  mla::tc::prefill_prep_kernel<<<prep_blocks, mla::tc::kPrepThreads, 0, st>>>(
+  mla::tc::prefill_prep_kernel<<<(unsigned)(1 + w_blocks + norm_blocks), mla::tc::kPrepThreads, 0, st>>>(
       cu_seqlens, num_seqs, T_tot, max_seqlen, cap, seq_tile0, tile_seq, tile_q0, order, pair_order,
-      static_cast<const bf16*>(w_kvb), w16, n8);
+      static_cast<const bf16*>(w_kvb), w16, n8, w_blocks, static_cast<const bf16*>(latent),
+      static_cast<const bf16*>(w_norm), R, d->eps, c16);
   prof_end(st);
+  CUtensorMap map_c16;   // the transposed-value GEMM's A operand: c_hat fp16 [Ttot, R]
+  {
+    const uint64_t dims[2] = {(uint64_t)R, (uint64_t)T_tot};
+    const uint64_t strides[1] = {(uint64_t)R * 2};
+    const uint32_t box[2] = {64, 128};
+    int rc = make_map(&map_c16, c16, 2, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+    if (rc) return rc;
+  }
 
   mla::tc::GemmParams gp;
   gp.latent = static_cast<const bf16*>(latent);
@@ -469,7 +482,7 @@ int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, cons
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)mla::tc::kG2SmemBytes);
     if (e != cudaSuccess) return cuda_status(e, "gemm smem attribute");
     prof_begin(st, "tc_norm_kv_b_proj");
-    e = launch_dependent(kern, dim3(cap, gy2), dim3(mla::tc::kG2Threads), mla::tc::kG2SmemBytes, st, map_lat, map_w,
+    e = launch_dependent(kern, dim3(cap, gy2), dim3(mla::tc::kG2Threads), mla::tc::kG2SmemBytes, st, map_c16, map_w,
                          gp);
     prof_end(st);
     if (e != cudaSuccess) return cuda_status(e, "gemm launch");

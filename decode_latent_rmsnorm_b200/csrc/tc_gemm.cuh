@@ -155,20 +155,75 @@ __device__ __forceinline__ void schedule_block(const int32_t* __restrict__ cu, i
   }
 }
 
-// ---- prefill preparation: tile schedule + fp16 copy of the kv_b_proj weight ----
-// Block 0 builds the schedule (schedule_block); blocks 1.. convert the weight,
-// 4 x 8 values per thread. A weight beyond the fp16 range sets the device
-// error word.
+// ---- prefill preparation: tile schedule, fp16 weight, normalized latent ----
+// Block 0 builds the schedule (schedule_block); blocks 1 .. w_blocks convert
+// the weight, 4 x 8 values per thread; the blocks after them (when launched)
+// write the normalized latent in fp16 for the transposed-value GEMM. A value
+// beyond the fp16 range sets the device error word.
 constexpr int kPrepThreads = 1024;
 constexpr int kPrepUnroll = 4;
 __global__ void __launch_bounds__(kPrepThreads)
 prefill_prep_kernel(const int32_t* __restrict__ cu, int nseq, int64_t Ttot, int max_seqlen, int cap,
                     int32_t* __restrict__ seq_tile0, int32_t* __restrict__ tile_seq,
                     int32_t* __restrict__ tile_q0, int32_t* __restrict__ order, int32_t* __restrict__ pair_order,
-                    const __nv_bfloat16* __restrict__ w, __half* __restrict__ w16, int64_t n8) {
+                    const __nv_bfloat16* __restrict__ w, __half* __restrict__ w16, int64_t n8, int w_blocks,
+                    const __nv_bfloat16* __restrict__ latent, const __nv_bfloat16* __restrict__ w_norm, int R,
+                    float eps, __half* __restrict__ c16) {
   pdl_allow_next();
   if (blockIdx.x == 0) {
     schedule_block(cu, nseq, Ttot, max_seqlen, cap, seq_tile0, tile_seq, tile_q0, order, pair_order);
+    return;
+  }
+  if ((int)blockIdx.x > w_blocks) {
+    // normalized latent c_hat = w * x / sqrt(mean(x^2) + eps) in fp16
+    // [Ttot, R]: one warp per token row; lane l holds the 8-value chunks l and
+    // l + 32 of the row (R <= 512)
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int64_t t = (int64_t)((int)blockIdx.x - 1 - w_blocks) * (kPrepThreads / 32) + warp;
+    if (t >= Ttot) return;
+    const int nch = R / 8;
+    const uint4* src = reinterpret_cast<const uint4*>(latent + t * (R + 64));
+    const uint4* wn = reinterpret_cast<const uint4*>(w_norm);
+    uint4 xv[2], gv[2];
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int c = lane + 32 * k;
+      xv[k] = c < nch ? src[c] : make_uint4(0u, 0u, 0u, 0u);
+      gv[k] = c < nch ? wn[c] : make_uint4(0u, 0u, 0u, 0u);
+    }
+    float ss = 0.f;
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const uint32_t w4[4] = {xv[k].x, xv[k].y, xv[k].z, xv[k].w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 v = unpack_bf16x2(w4[e]);
+        ss = fmaf(v.x, v.x, fmaf(v.y, v.y, ss));
+      }
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float r = 1.0f / sqrtf(ss / (float)R + eps);
+    float mx = 0.f;
+    uint4* dst = reinterpret_cast<uint4*>(c16 + t * R);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int c = lane + 32 * k;
+      if (c >= nch) break;
+      const uint32_t w4[4] = {xv[k].x, xv[k].y, xv[k].z, xv[k].w};
+      const uint32_t g4[4] = {gv[k].x, gv[k].y, gv[k].z, gv[k].w};
+      uint32_t o4[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 v = unpack_bf16x2(w4[e]);
+        const float2 g = unpack_bf16x2(g4[e]);
+        const float a = g.x * (v.x * r), b = g.y * (v.y * r);
+        mx = fmaxf(mx, fmaxf(fabsf(a), fabsf(b)));
+        o4[e] = pack_f16x2(a, b);
+      }
+      dst[c] = make_uint4(o4[0], o4[1], o4[2], o4[3]);
+    }
+    if (!(mx <= kF16Max)) raise_device_error(kDevErrRange);
     return;
   }
   const int64_t base = (int64_t)(blockIdx.x - 1) * kPrepThreads * kPrepUnroll + threadIdx.x;
@@ -457,15 +512,18 @@ namespace tc {
 // ---- fused RMSNorm + kv_b_proj GEMM, value half produced transposed --------
 // Heads with qk_nope = kN in {64, 128} and v_head = 128. Per head h and
 // 128-token tile, two tensor-core products share the resident normalized
-// latent tile c_hat [128 x R] and one streamed weight stage (the head's
-// kN + 128 rows of W, 64 K columns per stage):
+// latent tile c_hat [128 x R] (fp16, written by prefill_prep_kernel in token
+// order: the rows of a sequence's last tile past its end belong to the next
+// sequence, so their outputs are finite, and attention gives those keys zero
+// weight) and one streamed weight stage (the head's kN + 128 rows of W, 64 K
+// columns per stage):
 //   D1 = c_hat W_K^T   M = 128 tokens,   N = kN      -> k_nope rows
 //   D2 = W_V c_hat^T   M = 128 channels, N = 128 tokens -> value rows of vt
 // The products are the same sums as one c_hat [W_K; W_V]^T; swapping the
 // operands of the value half puts one value channel in each TMEM lane, so
 // the epilogue writes every transposed value row as 256 contiguous bytes.
-// Warps: 0 TMA, 1 MMA, 2-5 RMSNorm prologue then the k_nope epilogue,
-// 6-9 rotated shared key then the value epilogue.
+// Warps: 0 TMA, 1 MMA, 2-5 the k_nope epilogue, 6-9 the rotated shared key,
+// then the value epilogue.
 constexpr int kG2Threads = 320;
 constexpr int kG2Stages = 3;
 constexpr int kG2StageBytes = 256 * 128;
@@ -473,23 +531,19 @@ constexpr size_t kG2SmemBytes = (size_t)kGemmMaxAtoms * kAtomBytes + (size_t)kG2
 
 template <int kN>
 __global__ void __launch_bounds__(kG2Threads, 1)
-norm_kvb_gemm_vt_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_constant__ CUtensorMap map_w,
+norm_kvb_gemm_vt_kernel(const __grid_constant__ CUtensorMap map_chat, const __grid_constant__ CUtensorMap map_w,
                         GemmParams p) {
   constexpr int kV = 128;
   constexpr int kRows = kN + kV;                  // weight rows of one head
   constexpr int kStage = kRows * 128;             // bytes of one stage
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ GemmBarriers bars;
-  __shared__ uint4 s_wnorm[kGemmMaxAtoms * 8];   // the RMSNorm weight, 8 bf16 per entry
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  pdl_wait();         // the schedule and the fp16 weight come from the previous kernel
+  pdl_wait();         // the schedule, the fp16 weight and c_hat come from the previous kernel
   pdl_allow_next();
   const int tile = blockIdx.x;
   const int seq = p.tile_seq[tile];
   if (seq < 0) return;   // past the real tiles (uniform over the CTA)
-  // one vector load per thread, all in flight together (published by the
-  // __syncthreads below)
-  if (threadIdx.x < p.R / 8) s_wnorm[threadIdx.x] = reinterpret_cast<const uint4*>(p.w_norm)[threadIdx.x];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + kGemmMaxAtoms * kAtomBytes;
@@ -521,11 +575,11 @@ norm_kvb_gemm_vt_kernel(const __grid_constant__ CUtensorMap map_lat, const __gri
   if (warp == 0) {
     // ---------------- TMA producer ----------------
     if (lane == 0 && my_heads > 0) {
-      tma_prefetch_desc(&map_lat);
+      tma_prefetch_desc(&map_chat);
       tma_prefetch_desc(&map_w);
       mbar_arrive_expect_tx(&bars.a_full, natoms * kAtomBytes);
       for (int a = 0; a < natoms; ++a)
-        tma_load_2d(sA + a * kAtomBytes, &map_lat, &bars.a_full, a * 64, (int)(seq0 + q0));
+        tma_load_2d(sA + a * kAtomBytes, &map_chat, &bars.a_full, a * 64, (int)(seq0 + q0));
       int it = 0;
       bool ok = true;
       for (int h = h_begin; h < h_end && ok; ++h) {
@@ -584,56 +638,9 @@ norm_kvb_gemm_vt_kernel(const __grid_constant__ CUtensorMap map_lat, const __gri
     const uint32_t lane_base = (uint32_t)(grp * 32) << 16;
     bool ok = my_heads > 0;
     if (half == 0) {
-      // RMSNorm prologue: lane = token row of the tile
-      const bool valid = (q0 + lrow) < L;
+      // c_hat arrives in fp16 from the preparation kernel: nothing to do
+      // before the epilogue but pass the tile on
       if (ok) ok = mbar_wait_warp(&bars.a_full, 0, abort_flag);
-      if (ok) {
-        // sum of squares: eight independent partial sums; each atom's eight
-        // chunks are loaded before any is used
-        float ss8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-        for (int a = 0; a < natoms; ++a) {
-          const uint8_t* base = sA + a * kAtomBytes;
-          uint4 v[8];
-#pragma unroll
-          for (int c = 0; c < 8; ++c) v[c] = *reinterpret_cast<const uint4*>(base + sw128_offset(lrow, c));
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint32_t w4[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 f = unpack_bf16x2(w4[e]);
-              ss8[c] = fmaf(f.x, f.x, fmaf(f.y, f.y, ss8[c]));
-            }
-          }
-        }
-        const float ss = ((ss8[0] + ss8[1]) + (ss8[2] + ss8[3])) + ((ss8[4] + ss8[5]) + (ss8[6] + ss8[7]));
-        const float r = valid ? 1.0f / sqrtf(ss / (float)p.R + p.eps) : 0.f;
-        // c_hat = w * x * r in place, as fp16 (rows past the sequence become
-        // zeros): per atom, all loads, then the arithmetic, then all stores
-        for (int a = 0; a < natoms; ++a) {
-          uint8_t* base = sA + a * kAtomBytes;
-          uint4 v[8];
-#pragma unroll
-          for (int c = 0; c < 8; ++c) v[c] = *reinterpret_cast<const uint4*>(base + sw128_offset(lrow, c));
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            const uint32_t w4[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
-            const uint4 wv = s_wnorm[a * 8 + c];
-            const uint32_t g4[4] = {wv.x, wv.y, wv.z, wv.w};
-            uint32_t o4[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float2 f = unpack_bf16x2(w4[e]);
-              const float2 g = unpack_bf16x2(g4[e]);
-              o4[e] = pack_f16x2(g.x * (f.x * r), g.y * (f.y * r));
-            }
-            v[c] = make_uint4(o4[0], o4[1], o4[2], o4[3]);
-          }
-#pragma unroll
-          for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(base + sw128_offset(lrow, c)) = v[c];
-        }
-        fence_proxy_async_smem();
-      }
       mbar_arrive(&bars.a_ready);
     } else if (blockIdx.y == 0) {
       // rotated shared key of token row lrow (one CTA column per tile writes
