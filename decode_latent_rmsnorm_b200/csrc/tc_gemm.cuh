@@ -157,11 +157,11 @@ __device__ __forceinline__ void schedule_block(const int32_t* __restrict__ cu, i
 
 // ---- prefill preparation: tile schedule, fp16 weight, normalized latent ----
 // Block 0 builds the schedule (schedule_block); blocks 1 .. w_blocks convert
-// the weight, 4 x 8 values per thread; the blocks after them (when launched)
+// the weight, kPrepUnroll x 8 values per thread; the blocks after them (when launched)
 // write the normalized latent in fp16 for the transposed-value GEMM. A value
 // beyond the fp16 range sets the device error word.
 constexpr int kPrepThreads = 1024;
-constexpr int kPrepUnroll = 4;
+constexpr int kPrepUnroll = 8;
 __global__ void __launch_bounds__(kPrepThreads)
 prefill_prep_kernel(const int32_t* __restrict__ cu, int nseq, int64_t Ttot, int max_seqlen, int cap,
                     int32_t* __restrict__ seq_tile0, int32_t* __restrict__ tile_seq,
