@@ -44,6 +44,11 @@ Readings taken where the pages are silent (each is listed in the design doc):
 * Decode cache rows hold [normalized latent (R) || rotated k_pe (P)], as the
   GLM-5 "KV cache" section describes; heads are expanded from every cached
   row; the query sits at ``positions[b]`` and attends to all cached rows.
+* A chunk of new tokens that continues a cached sequence: the chunk's rows
+  are written into the cache first (the GLM-5 "KV cache" order: update,
+  then expand every cached row). Chunk token i of a sequence with p cached
+  rows sits at position p + i, goes to the sequence's cache row p + i, and
+  attends to cached rows 0 .. p + i (the causal mask in absolute positions).
 """
 
 from __future__ import annotations
@@ -60,7 +65,7 @@ __all__ = [
     "rope_inv_freq", "rope_table_mscale", "rope_tables", "softmax_scale",
     "rms_norm", "kv_up_projection", "apply_rope",
     "causal_attention_rows", "prefill", "decode_eager", "decode_absorbed",
-    "cache_append",
+    "cache_append", "prefill_cached",
 ]
 
 
@@ -420,3 +425,49 @@ def cache_append(latent, w_norm, positions, cos, sin, shape: MlaShape):
     pos = np.asarray(positions).astype(np.int64)
     k_rot = apply_rope(latent[:, R:], cos[pos], sin[pos], shape.interleaved)
     return np.concatenate([c_hat, k_rot], axis=-1)
+
+
+def prefill_cached(latent, q, cache, cache_offsets, prefix_lens, cu_seqlens, W, w_norm,
+                   cos, sin, shape: MlaShape, scale: float, heads=None):
+    """A chunk of new tokens per sequence, continuing a latent cache.
+
+    Sequence s owns cache rows ``cache_offsets[s]`` onwards; the first
+    ``prefix_lens[s]`` of them are cached already. Its chunk is rows
+    ``cu_seqlens[s] .. cu_seqlens[s+1] - 1`` of ``latent`` [Tq, R + P] (raw
+    compressed_kv) and ``q`` [Tq, H, N + P].
+
+    Steps per sequence, in the order of the [GLM] "KV cache" section:
+      1. the chunk's cache rows, cache_append at positions p .. p + n - 1,
+         are written to the sequence's rows p .. p + n - 1;
+      2. k_nope and V of every cached row 0 .. p + n - 1 are expanded with
+         kv_b_proj (expand_kv); the cached rotated key is shared by all heads;
+      3. q_pe of chunk token i is rotated at position p + i;
+      4. scores * scale, causal mask in absolute positions (token i sees
+         cached rows j <= p + i), softmax, P @ V.
+
+    Returns (out [Tq, H, V], the cache after step 1). ``heads``: subset of
+    heads to evaluate (others stay NaN). The input cache is not modified.
+    """
+    H, R, N, V = shape.num_heads, shape.kv_lora_rank, shape.qk_nope, shape.v_head
+    Tq = latent.shape[0]
+    heads = list(range(H)) if heads is None else heads
+    cache = np.array(cache, dtype=np.float64, copy=True)
+    out = np.full((Tq, H, V), np.nan)
+    for s in range(len(cu_seqlens) - 1):
+        a, b = int(cu_seqlens[s]), int(cu_seqlens[s + 1])
+        n, p, o = b - a, int(prefix_lens[s]), int(cache_offsets[s])
+        if n == 0:
+            continue
+        pos = p + np.arange(n)
+        cache[o + p:o + p + n] = cache_append(latent[a:b], w_norm, pos, cos, sin, shape)  # step 1
+        rows = cache[o:o + p + n]
+        c_hat, k_rot = rows[:, :R], rows[:, R:]
+        k_nope, v = kv_up_projection(c_hat, W, shape, heads)                             # step 2
+        q_sel = q[a:b][:, heads, :]
+        q_pe_rot = apply_rope(q_sel[:, :, N:], cos[pos][:, None, :], sin[pos][:, None, :],
+                              shape.interleaved)                                          # step 3
+        for hi, h in enumerate(heads):
+            Q = np.concatenate([q_sel[:, hi, :N], q_pe_rot[:, hi, :]], axis=-1)
+            K = np.concatenate([k_nope[hi], k_rot], axis=-1)
+            out[a:b, h, :] = causal_attention_rows(Q, K, v[hi], pos, scale)              # step 4
+    return out, cache

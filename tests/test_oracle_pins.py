@@ -401,3 +401,80 @@ def test_cache_append_row():
     np.testing.assert_array_equal(rows[0, 16:], x[0, 16:])       # position 0: unrotated
     np.testing.assert_allclose(np.linalg.norm(rows[:, 16:], axis=-1),
                                np.linalg.norm(x[:, 16:], axis=-1), rtol=1e-13)
+
+
+# ---------------------------------------------------------------- chunks over a cached prefix
+
+def _chunked_inputs(seqlens, splits, gap=3, **kw):
+    """A small case whose sequences are cut at ``splits`` (cached prefix
+    length per sequence). The cache holds each sequence in its own region,
+    ``gap`` unused rows apart, so offsets are not a packed prefix sum."""
+    shape, rope, d, cos, sin = _small_case(seqlens, **kw)
+    offs = np.zeros(len(seqlens), dtype=np.int64)
+    for s in range(1, len(seqlens)):
+        offs[s] = offs[s - 1] + seqlens[s - 1] + gap
+    rows = int(offs[-1] + seqlens[-1] + gap)
+    return shape, rope, d, cos, sin, offs, rows
+
+
+@pytest.mark.parametrize("interleaved", [False, True])
+def test_prefill_cached_two_chunks_equal_one_prefill(interleaved):
+    # Splitting each sequence into a cached prefix and a chunk changes nothing:
+    # chunk 1 (empty prefix) and chunk 2 (prefix = chunk 1) together give the
+    # prefill of the whole sequence. An error in the chunk's positions, its
+    # cache rows or the offset of the causal mask breaks this.
+    seqlens, splits = [11, 6, 17], [4, 0, 16]
+    shape, rope, d, cos, sin, offs, nrows = _chunked_inputs(seqlens, splits, H=3, R=16, N=8, P=4, V=6,
+                                                            interleaved=interleaved, seed=21)
+    scale = 0.35
+    full = O.prefill(d["latent"], d["q"], d["W"], d["w_norm"], d["positions"], d["cu"], cos, sin, shape, scale)
+    cu = d["cu"]
+    idx1 = np.concatenate([np.arange(cu[s], cu[s] + splits[s]) for s in range(3)])
+    idx2 = np.concatenate([np.arange(cu[s] + splits[s], cu[s + 1]) for s in range(3)])
+    cu1 = np.concatenate([[0], np.cumsum(splits)])
+    cu2 = np.concatenate([[0], np.cumsum(np.array(seqlens) - np.array(splits))])
+    cache0 = np.full((nrows, shape.kv_lora_rank + shape.qk_rope), 7.5)
+    out1, cache1 = O.prefill_cached(d["latent"][idx1], d["q"][idx1], cache0, offs, np.zeros(3, int), cu1,
+                                    d["W"], d["w_norm"], cos, sin, shape, scale)
+    out2, cache2 = O.prefill_cached(d["latent"][idx2], d["q"][idx2], cache1, offs, np.array(splits), cu2,
+                                    d["W"], d["w_norm"], cos, sin, shape, scale)
+    np.testing.assert_allclose(out1, full[idx1], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(out2, full[idx2], rtol=1e-12, atol=1e-13)
+    # every sequence's region now holds its whole cache; the gaps are untouched
+    appended = O.cache_append(d["latent"], d["w_norm"], d["positions"], cos, sin, shape)
+    used = np.zeros(nrows, bool)
+    for s in range(3):
+        np.testing.assert_allclose(cache2[offs[s]:offs[s] + seqlens[s]], appended[cu[s]:cu[s + 1]], rtol=1e-15)
+        used[offs[s]:offs[s] + seqlens[s]] = True
+    assert np.all(cache2[~used] == 7.5) and np.all(cache0 == 7.5)
+
+
+def test_prefill_cached_last_token_is_a_decode_step():
+    # The chunk's last token attends to all p + n cached rows from position
+    # p + n - 1: a decode step over the updated cache at that position.
+    seqlens, splits = [9, 14], [5, 2]
+    shape, rope, d, cos, sin, offs, nrows = _chunked_inputs(seqlens, splits, seed=22)
+    scale = 0.3
+    cu = d["cu"]
+    pre = O.cache_append(d["latent"], d["w_norm"], d["positions"], cos, sin, shape)
+    cache = np.zeros((nrows, pre.shape[1]))
+    for s in range(2):
+        cache[offs[s]:offs[s] + splits[s]] = pre[cu[s]:cu[s] + splits[s]]
+    idx = np.concatenate([np.arange(cu[s] + splits[s], cu[s + 1]) for s in range(2)])
+    cuq = np.concatenate([[0], np.cumsum(np.array(seqlens) - np.array(splits))])
+    out, after = O.prefill_cached(d["latent"][idx], d["q"][idx], cache, offs, np.array(splits), cuq,
+                                  d["W"], d["w_norm"], cos, sin, shape, scale)
+    last = cuq[1:] - 1
+    lens = np.array(seqlens)
+    dec = O.decode_eager(d["q"][idx][last], after, offs, lens, lens - 1, d["W"], cos, sin, shape, scale)
+    np.testing.assert_allclose(out[last], dec, rtol=1e-12, atol=1e-13)
+
+
+def test_prefill_cached_without_prefix_is_prefill():
+    seqlens = [7, 1, 12]
+    shape, rope, d, cos, sin, offs, nrows = _chunked_inputs(seqlens, [0, 0, 0], interleaved=True, seed=23)
+    scale = 0.45
+    full = O.prefill(d["latent"], d["q"], d["W"], d["w_norm"], d["positions"], d["cu"], cos, sin, shape, scale)
+    out, _ = O.prefill_cached(d["latent"], d["q"], np.zeros((nrows, shape.kv_lora_rank + shape.qk_rope)), offs,
+                              np.zeros(3, int), d["cu"], d["W"], d["w_norm"], cos, sin, shape, scale)
+    np.testing.assert_allclose(out, full, rtol=1e-12, atol=1e-13)
