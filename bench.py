@@ -65,6 +65,16 @@ def decode_bytes(wl, lens) -> dict:
     return dict(cache=cache, weight=weight, io=io, total=cache + weight + io, flops=flops)
 
 
+def chunk_bytes(wl, prefix, n_new) -> dict:
+    """Cache rows of a chunk call: each chunk token reads its sequence's rows
+    up to its own (the absorbed form runs one decode row per token), and the
+    unique rows are each sequence's prefix plus its chunk."""
+    row = (wl.kv_lora_rank + wl.qk_rope) * 2
+    attended = sum(p * n_new + n_new * (n_new + 1) // 2 for p in prefix)
+    unique = sum(p + n_new for p in prefix)
+    return dict(attended=float(attended) * row, unique=float(unique) * row)
+
+
 # ---------------------------------------------------------------- environment
 
 def recorded_traffic(kernel: str):
@@ -377,6 +387,8 @@ def run_ours(args, rank, world, device):
     roof["kernel"] = top
     roof["peak_source"] = peaks["source"]
 
+    chunk = run_chunk(args, din, D, device, world, reduce_max, peaks)
+
     # end to end through the same C-ABI with pinned host buffers
     e2e = run_e2e(args, pwl, dwl, pin, din, dims_p, dims_d, cos, sin, P, D, p_ws, d_ws, device, world,
                   reduce_max, fl, by)
@@ -391,7 +403,7 @@ def run_ours(args, rank, world, device):
         decode=dict(metric="absorbed decode HBM GB/s", value=d_gbs, unit="GB/s", ms=d_mean,
                     frac_of_hbm=d_gbs / (world * peaks["hbm"]), tokens_per_s=world * B / (d_mean * 1e-3),
                     tflops=world * by["flops"] / (d_mean * 1e-3) / 1e12, bytes=by["total"]),
-        kernels_ms=dict(prefill=kp_ms, decode=kd_ms),
+        kernels_ms=dict(prefill=kp_ms, decode=kd_ms), chunk=chunk,
         roofline=roof, e2e=e2e, gpu_launches=int(launches), clocks=clocks.summary(),
         peaks=dict(hbm_gbs=peaks["hbm"], bf16_tflops=peaks["bf16"], source=peaks["source"]),
     )
@@ -449,6 +461,62 @@ def run_e2e(args, pwl, dwl, pin, din, dims_p, dims_d, cos, sin, P, D, p_ws, d_ws
                 h2d_bytes_per_step=h2d_p + h2d_d, d2h_bytes_per_step=d2h_p + d2h_d,
                 prefill_ms=p_ms, decode_ms=d_ms,
                 decode_gbs=world * by["total"] / (d_ms * 1e-3) / 1e9)
+
+
+def run_chunk(args, din, D, device, world, reduce_max, peaks, n_new=4):
+    """Chunks of ``n_new`` new tokens continuing the decode workload's 64
+    cached sequences (mla_prefill_cached): the chunk's rows are appended and
+    every chunk token attends to its prefix, the chunk tokens before it and
+    itself. The prefix rows are the decode cache's rows, copied on the device
+    into regions with room for the chunk."""
+    lens = [int(x) for x in din["cache_lens"]]
+    offs_d = [int(x) for x in din["cache_offsets"]]
+    B = len(lens)
+    cwl = W.scaled(W.KIMI, seqlens=(n_new,) * B, seed=5, extra=dict(prefix_lens=(0,) * B))
+    cin = W.chunk_inputs(cwl)
+    dims = mla.dims_for(cwl, mla.mla_softmax_scale(mla.rope_for(cwl), cwl.qk_head_dim))
+    max_total = max(lens) + n_new
+    cos, sin = mla.mla_init_rope_tables(mla.rope_for(cwl), max_total)
+    offs = [0] * B
+    for b in range(1, B):
+        offs[b] = offs[b - 1] + lens[b - 1] + n_new
+    cache = torch.empty((offs[-1] + lens[-1] + n_new, D["cache"].shape[1]), dtype=torch.bfloat16, device=device)
+    for b in range(B):
+        cache[offs[b]:offs[b] + lens[b]].copy_(D["cache"][offs_d[b]:offs_d[b] + lens[b]])
+    C = {k: cin[k].to(device) for k in ("latent", "q", "w_kvb", "w_norm", "cu_seqlens")}
+    c_offs = torch.tensor(offs, dtype=torch.int64, device=device)
+    c_pre = torch.tensor(lens, dtype=torch.int32, device=device)
+    T = B * n_new
+    out = torch.empty((T, cwl.num_heads, cwl.v_head), dtype=torch.bfloat16, device=device)
+    ws = torch.empty(mla.mla_prefill_cached_workspace_size(dims, T, max_total), dtype=torch.uint8, device=device)
+
+    def call():
+        mla.mla_prefill_cached(dims, C["latent"], C["q"], C["w_kvb"], C["w_norm"], C["cu_seqlens"], c_offs, c_pre,
+                               max_total, cos, sin, cache, out=out, workspace=ws)
+
+    for _ in range(args.warmup):
+        call()
+    torch.cuda.synchronize()
+    mla.mla_check_device_status()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    for e in evs:
+        e[0].record()
+        call()
+        e[1].record()
+    torch.cuda.synchronize()
+    kev = mla.KernelEvents(16)
+    with kev:
+        call()
+    torch.cuda.synchronize()
+    mla.mla_check_device_status()
+    ms = reduce_max(statistics.mean(e[0].elapsed_time(e[1]) for e in evs))
+    by = chunk_bytes(cwl, lens, n_new)
+    att = world * by["attended"] / (ms * 1e-3) / 1e9
+    return dict(workload="64 sequences, cached prefixes = the decode cache lengths, %d new tokens each" % n_new,
+                ms=ms, tokens_per_s=world * T / (ms * 1e-3), attended_gbs=att,
+                attended_frac_of_hbm=att / (world * peaks["hbm"]),
+                unique_cache_gbs=world * by["unique"] / (ms * 1e-3) / 1e9,
+                kernels_ms=dict(zip(kev.names, kev.durations_ms())))
 
 
 def cpu_baseline(budget_s=15.0):

@@ -18,6 +18,7 @@
 #include "tc_attention.cuh"
 #include "tc_attention_pair.cuh"
 #include "tc_decode.cuh"
+#include "chunk.cuh"
 
 #include <cudaTypedefs.h>
 
@@ -926,6 +927,28 @@ int mla_cache_append(const mla_dims* dims, const void* latent, const void* w_nor
   return cuda_status(cudaGetLastError(), "cache append launch");
 }
 
+// ---- chunks over a cached prefix ------------------------------------------------
+// Workspace: the per-token bookkeeping of chunk_rows_kernel, then the decode's own.
+namespace {
+struct ChunkWs {
+  size_t positions, lens, rows, offsets, decode, total;
+};
+
+ChunkWs chunk_ws_layout(const mla_dims* d, int64_t n, int max_total_len) {
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  ChunkWs L;
+  size_t o = 0;
+  L.positions = o; o = up(o + (size_t)n * 4);
+  L.lens = o;      o = up(o + (size_t)n * 4);
+  L.rows = o;      o = up(o + (size_t)n * 8);
+  L.offsets = o;   o = up(o + (size_t)n * 8);
+  L.decode = o;    o = up(o + decode_ws_bytes(d, (int)n, max_total_len));
+  L.total = o;
+  return L;
+}
+constexpr int64_t kMaxChunkTokens = 65535;   // the decode's batch limit
+}  // namespace
+
 // Device address of g_noalloc_scratch, looked up once per device (host code
 // cannot use the array's name as a device address).
 namespace {
@@ -967,6 +990,62 @@ int mla_prefill_noalloc(const mla_dims* dims, const void* latent, const void* q,
   if (rc) return rc;
   return mla_prefill(dims, latent, q, w_kvb, w_norm, positions, cu_seqlens, num_seqs, max_seqlen, total_tokens,
                      cos_table, sin_table, max_pos, out, scratch, (size_t)MLA_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+int mla_prefill_cached_workspace_size(const mla_dims* dims, int64_t total_tokens, int32_t max_total_len,
+                                      size_t* bytes) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (total_tokens < 0 || max_total_len < 0) return fail(MLA_ERR_INVALID_ARG, "negative size");
+  if (total_tokens > kMaxChunkTokens)
+    return fail(MLA_ERR_UNSUPPORTED_SHAPE, "at most %lld chunk tokens per call", (long long)kMaxChunkTokens);
+  if (!bytes) return fail(MLA_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = chunk_ws_layout(dims, total_tokens, max_total_len).total;
+  return MLA_OK;
+}
+
+int mla_prefill_cached(const mla_dims* dims, const void* latent, const void* q, const void* w_kvb,
+                       const void* w_norm, const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                       const int64_t* cache_offsets, const int32_t* prefix_lens, int32_t max_total_len,
+                       const float* cos_table, const float* sin_table, int32_t max_pos, void* cache,
+                       int64_t cache_num_rows, void* out, void* workspace, size_t workspace_bytes,
+                       cudaStream_t stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (total_tokens < 0 || num_seqs < 0) return fail(MLA_ERR_INVALID_ARG, "negative size");
+  if (total_tokens == 0) return MLA_OK;
+  if (num_seqs < 1) return fail(MLA_ERR_INVALID_ARG, "num_seqs must be >= 1 when there are chunk tokens");
+  if (total_tokens > kMaxChunkTokens)
+    return fail(MLA_ERR_UNSUPPORTED_SHAPE, "at most %lld chunk tokens per call", (long long)kMaxChunkTokens);
+  if (max_total_len < 1) return fail(MLA_ERR_INVALID_ARG, "max_total_len must be >= 1");
+  if (max_pos < 1) return fail(MLA_ERR_INVALID_ARG, "max_pos must be >= 1");
+  if (cache_num_rows < 1) return fail(MLA_ERR_INVALID_ARG, "cache_num_rows must be >= 1");
+  if (!latent || !q || !w_kvb || !w_norm || !cu_seqlens || !cache_offsets || !prefix_lens || !cos_table ||
+      !sin_table || !cache || !out)
+    return fail(MLA_ERR_INVALID_ARG, "a tensor pointer is NULL");
+  const ChunkWs L = chunk_ws_layout(dims, total_tokens, max_total_len);
+  if (!workspace || workspace_bytes < L.total)
+    return fail(MLA_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes, got %zu", L.total, workspace_bytes);
+  char* ws = static_cast<char*>(workspace);
+  int32_t* positions = reinterpret_cast<int32_t*>(ws + L.positions);
+  int32_t* lens = reinterpret_cast<int32_t*>(ws + L.lens);
+  int64_t* rows = reinterpret_cast<int64_t*>(ws + L.rows);
+  int64_t* offsets = reinterpret_cast<int64_t*>(ws + L.offsets);
+  prof_begin(stream, "chunk_rows");
+  mla::chunk_rows_kernel<<<(unsigned)((total_tokens + mla::kChunkThreads - 1) / mla::kChunkThreads),
+                           mla::kChunkThreads, 0, stream>>>(cu_seqlens, num_seqs, total_tokens, cache_offsets,
+                                                            prefix_lens, max_total_len, max_pos, cache_num_rows,
+                                                            positions, rows, offsets, lens);
+  prof_end(stream);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_status(e, "chunk rows launch");
+  // 1. the chunk's rows go into the cache; 2. each chunk token attends to its
+  // sequence's rows up to and including its own, as one absorbed decode row
+  rc = mla_cache_append(dims, latent, w_norm, positions, total_tokens, cos_table, sin_table, max_pos, cache,
+                        cache_num_rows, rows, stream);
+  if (rc) return rc;
+  return mla_decode(dims, q, cache, cache_num_rows, offsets, lens, positions, (int32_t)total_tokens, max_total_len,
+                    w_kvb, cos_table, sin_table, max_pos, out, ws + L.decode, workspace_bytes - L.decode, stream);
 }
 
 int mla_check_device_status(cudaStream_t stream) {

@@ -35,6 +35,9 @@ SIGNATURES = {
                            c_vp, c_i32, c_vp, c_vp, c_sz, c_vp]),
     "mla_cache_append": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_i64, c_vp, c_vp, c_i32, c_vp, c_i64,
                                  c_vp, c_vp]),
+    "mla_prefill_cached_workspace_size": (c_i32, [c_vp, c_i64, c_i32, ctypes.POINTER(c_sz)]),
+    "mla_prefill_cached": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_i32, c_i64, c_vp, c_vp, c_i32,
+                                   c_vp, c_vp, c_i32, c_vp, c_i64, c_vp, c_vp, c_sz, c_vp]),
     "mla_check_device_status": (c_i32, [c_vp]),
     "mla_last_error_string": (ctypes.c_char_p, []),
     "mla_version": (c_i32, []),
@@ -230,6 +233,40 @@ def mla_cache_append(dims: Dims, latent, w_norm, positions, cos, sin, cache, cac
         _dev(sin, "sin", torch.float32), int(cos.shape[0]), _dev(cache, "cache", dt),
         int(cache.shape[0]), _dev(cache_rows, "cache_rows", torch.int64, (n,)), _stream()))
     return cache
+
+
+def mla_prefill_cached_workspace_size(dims: Dims, total_tokens: int, max_total_len: int) -> int:
+    out = c_sz()
+    _check(load().mla_prefill_cached_workspace_size(ctypes.byref(dims), int(total_tokens), int(max_total_len),
+                                                    ctypes.byref(out)))
+    return out.value
+
+
+def mla_prefill_cached(dims: Dims, latent, q, w_kvb, w_norm, cu_seqlens, cache_offsets, prefix_lens,
+                       max_total_len: int, cos, sin, cache, out=None, workspace=None):
+    """Chunks of new tokens continuing cached sequences: appends the chunk's
+    rows to ``cache`` and returns ``out`` [Tq, H, V] (allocated if None)."""
+    dt = dims.torch_dtype
+    H, R, N, P, V = dims.num_heads, dims.kv_lora_rank, dims.qk_nope, dims.qk_rope, dims.v_head
+    T = latent.shape[0]
+    nseq = cu_seqlens.numel() - 1
+    if out is None:
+        out = torch.empty((T, H, V), dtype=dt, device=latent.device)
+    if workspace is None:
+        workspace = torch.empty(max(mla_prefill_cached_workspace_size(dims, T, max_total_len), 1),
+                                dtype=torch.uint8, device=latent.device)
+    if cache.dim() != 2 or cache.shape[1] != R + P:
+        raise ValueError("cache must be [rows, R + P]")
+    _check(load().mla_prefill_cached(
+        ctypes.byref(dims), _dev(latent, "latent", dt, (T, R + P)), _dev(q, "q", dt, (T, H, N + P)),
+        _dev(w_kvb, "w_kvb", dt, (H * (N + V), R)), _dev(w_norm, "w_norm", dt, (R,)),
+        _dev(cu_seqlens, "cu_seqlens", torch.int32), int(nseq), int(T),
+        _dev(cache_offsets, "cache_offsets", torch.int64, (nseq,)),
+        _dev(prefix_lens, "prefix_lens", torch.int32, (nseq,)), int(max_total_len),
+        _dev(cos, "cos", torch.float32), _dev(sin, "sin", torch.float32), int(cos.shape[0]),
+        _dev(cache, "cache", dt), int(cache.shape[0]), _dev(out, "out", dt, (T, H, V)),
+        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream()))
+    return out
 
 
 def mla_check_device_status():

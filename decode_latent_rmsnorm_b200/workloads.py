@@ -146,6 +146,48 @@ def decode_inputs(wl: Workload) -> dict:
                 positions=lens.clone())
 
 
+def chunk_inputs(wl: Workload, gap: int = 0) -> dict:
+    """CPU tensors for one call of chunks that continue cached sequences.
+
+    ``wl.seqlens`` gives each sequence's chunk tokens and
+    ``wl.extra["prefix_lens"]`` its rows cached before the call. The cache
+    [rows, R + P] gives sequence s a region of prefix + chunk rows followed
+    by ``gap`` unused rows; the prefix rows are drawn N(0, 1) like the decode
+    cache (the statistics of a normalized latent and a rotated key), and the
+    chunk's rows and the unused rows start at zero. Also returns latent
+    [Tq, R + P] (raw compressed_kv of the chunk tokens), q [Tq, H, N + P],
+    w_kvb, w_norm, cu_seqlens int32 [nseq + 1], cache_offsets int64 [nseq],
+    prefix_lens int32 [nseq] and max_total_len.
+    """
+    g = torch.Generator().manual_seed(wl.seed + 2000)
+    dt = wl.torch_dtype
+    H, R, N, P, V = wl.num_heads, wl.kv_lora_rank, wl.qk_nope, wl.qk_rope, wl.v_head
+    chunks = [int(n) for n in wl.seqlens]
+    prefix = [int(p) for p in wl.extra["prefix_lens"]]
+    nseq = len(chunks)
+    offsets, rows = [], 0
+    for s in range(nseq):
+        offsets.append(rows)
+        rows += prefix[s] + chunks[s] + gap
+    cache = torch.zeros((max(rows, 1), R + P), dtype=dt)
+    for s in range(nseq):
+        if prefix[s]:
+            cache[offsets[s]:offsets[s] + prefix[s]] = _randn(g, (prefix[s], R + P), dt)
+    T = sum(chunks)
+    latent = _randn(g, (T, R + P), dt)
+    q = _randn(g, (T, H, N + P), dt)
+    w_kvb = (torch.randn((H * (N + V), R), generator=g) * (1.0 / R) ** 0.5).to(dt)
+    w_norm = (1.0 + 0.1 * torch.randn((R,), generator=g)).to(dt)
+    cu = [0]
+    for n in chunks:
+        cu.append(cu[-1] + n)
+    return dict(latent=latent, q=q, w_kvb=w_kvb, w_norm=w_norm, cache=cache,
+                cu_seqlens=torch.tensor(cu, dtype=torch.int32),
+                cache_offsets=torch.tensor(offsets, dtype=torch.int64),
+                prefix_lens=torch.tensor(prefix, dtype=torch.int32),
+                max_total_len=max([p + n for p, n in zip(prefix, chunks)] + [1]))
+
+
 def max_position(wl: Workload) -> int:
     """Smallest rotary-table length that covers every position used."""
     if wl.kind == "prefill":

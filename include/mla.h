@@ -171,6 +171,46 @@ int mla_cache_append(const mla_dims* dims, const void* latent, const void* w_nor
                      const float* sin_table, int32_t max_pos, void* cache,
                      int64_t cache_num_rows, const int64_t* cache_rows, cudaStream_t stream);
 
+/* Workspace bytes mla_prefill_cached needs for total_tokens chunk tokens
+ * whose sequences hold at most max_total_len rows once the chunk is in. */
+int mla_prefill_cached_workspace_size(const mla_dims* dims, int64_t total_tokens,
+                                      int32_t max_total_len, size_t* bytes);
+
+/* Chunks of new tokens that continue cached sequences ([GLM] "KV cache": the
+ * cache is updated with the new tokens' normalized latent and rotated key,
+ * then the heads are expanded from every cached row and attended).
+ *   latent        [Tq, R + P]   compressed_kv rows of the chunk tokens
+ *   q             [Tq, H, N + P]
+ *   cu_seqlens    int32 [num_seqs + 1]  chunk tokens per sequence, packed
+ *                 (cu_seqlens[0] = 0, cu_seqlens[num_seqs] = Tq = total_tokens;
+ *                 a sequence may have no chunk tokens)
+ *   cache_offsets int64 [num_seqs]  first cache row of sequence s
+ *   prefix_lens   int32 [num_seqs]  rows of sequence s cached before the call
+ *   max_total_len prefix_lens[s] + chunk length of s, at most, over s
+ *   cache         [cache_num_rows, R + P]  read and written (as mla_decode / mla_cache_append)
+ *   w_kvb, w_norm, cos/sin tables as for mla_prefill
+ *   out           [Tq, H, V]
+ * Chunk token i of sequence s sits at position p + i (p = prefix_lens[s]).
+ * Its row RMSNorm(latent[:R]) || rope(latent[R:], p + i) is written to cache
+ * row cache_offsets[s] + p + i, and it attends to the sequence's rows
+ * 0 .. p + i: its cached prefix, the chunk tokens before it, and itself (the
+ * causal mask in absolute positions). Each chunk token runs as one row of
+ * the absorbed decode (mla_decode), so the cost is the sum over chunk
+ * tokens of the rows each attends. At most 65535 chunk tokens per call
+ * (MLA_ERR_UNSUPPORTED_SHAPE above). The sequences' cache regions must not
+ * overlap. Device-resident arguments are range-checked on the device: a
+ * token whose sequence is inconsistent with cu_seqlens, whose rows leave the
+ * cache or exceed max_total_len, or whose position is outside the table is
+ * neither written to the cache nor attended (its output is zero) and the
+ * device error word is set. */
+int mla_prefill_cached(const mla_dims* dims, const void* latent, const void* q, const void* w_kvb,
+                       const void* w_norm, const int32_t* cu_seqlens, int32_t num_seqs,
+                       int64_t total_tokens, const int64_t* cache_offsets,
+                       const int32_t* prefix_lens, int32_t max_total_len,
+                       const float* cos_table, const float* sin_table, int32_t max_pos,
+                       void* cache, int64_t cache_num_rows, void* out, void* workspace,
+                       size_t workspace_bytes, cudaStream_t stream);
+
 /* Size of the scratch array behind mla_prefill_noalloc (32 MiB). */
 #define MLA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 

@@ -111,3 +111,23 @@ def oracle_decode(wl, inp, batches, heads=None, absorbed=False):
                  w, cos, sin, shape, scale, heads=heads)
         out[b] = res[0]
     return out
+
+
+def run_prefill_cached(wl, inp):
+    """The chunk call on the GPU; returns (out, cache after the call)."""
+    rope, shape, scale = oracle_cfg(wl)
+    dims = mla.dims_for(wl, mla.mla_softmax_scale(mla.rope_for(wl), shape.qk_head_dim))
+    cos, sin = gpu_tables(wl, inp["max_total_len"])
+    d = {k: v.to("cuda") for k, v in inp.items() if isinstance(v, torch.Tensor)}
+    out = mla.mla_prefill_cached(dims, d["latent"], d["q"], d["w_kvb"], d["w_norm"], d["cu_seqlens"],
+                                 d["cache_offsets"], d["prefix_lens"], inp["max_total_len"], cos, sin, d["cache"])
+    torch.cuda.synchronize()
+    return out, d["cache"]
+
+
+def oracle_prefill_cached(wl, inp, heads=None):
+    rope, shape, scale = oracle_cfg(wl)
+    cos, sin = O.rope_tables(rope, inp["max_total_len"])
+    return O.prefill_cached(f64(inp["latent"]), f64(inp["q"]), f64(inp["cache"]), inp["cache_offsets"].numpy(),
+                            inp["prefix_lens"].numpy(), inp["cu_seqlens"].numpy(), f64(inp["w_kvb"]),
+                            f64(inp["w_norm"]), cos, sin, shape, scale, heads=heads)

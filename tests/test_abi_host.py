@@ -123,3 +123,33 @@ def test_workspace_sizes_are_monotone():
     assert mla.mla_decode_workspace_size(d, 64, 32768) > mla.mla_decode_workspace_size(d, 8, 32768)
     with pytest.raises(mla.MlaError):
         mla.mla_prefill_workspace_size(d, -1, 1)
+
+
+def test_prefill_cached_host_validation():
+    lib = mla.load()
+    d = kimi_dims()
+
+    def call(**over):
+        a = dict(lat=FAKE, q=FAKE, w=FAKE, wn=FAKE, cu=FAKE, nseq=2, T=5, offs=FAKE, pre=FAKE, maxlen=100,
+                 cos=FAKE, sin=FAKE, maxpos=200, cache=FAKE, rows=10 ** 6, out=FAKE, ws=FAKE, wsb=1 << 40)
+        a.update(over)
+        return lib.mla_prefill_cached(ctypes.byref(d), a["lat"], a["q"], a["w"], a["wn"], a["cu"], a["nseq"], a["T"],
+                                      a["offs"], a["pre"], a["maxlen"], a["cos"], a["sin"], a["maxpos"], a["cache"],
+                                      a["rows"], a["out"], a["ws"], a["wsb"], None)
+
+    assert call(T=0) == 0                    # no chunk tokens: nothing to do
+    assert call(T=-1) == 1
+    assert call(nseq=0) == 1                 # tokens but no sequence
+    assert call(T=65536) == 2                # above the decode's batch limit
+    assert call(maxlen=0) == 1
+    assert call(maxpos=0) == 1
+    assert call(rows=0) == 1
+    assert call(pre=None) == 1
+    assert call(cache=None) == 1
+    assert call(wsb=16) == 3
+    # the workspace holds the per-token bookkeeping plus the decode's own
+    need = mla.mla_prefill_cached_workspace_size(d, 5, 100)
+    assert need >= mla.mla_decode_workspace_size(d, 5, 100) + 5 * 24
+    assert call(wsb=need - 1) == 3
+    with pytest.raises(mla.MlaError):
+        mla.mla_prefill_cached_workspace_size(d, 65536, 100)

@@ -215,3 +215,91 @@ def test_cache_append_then_decode_matches_prefill_row(gpu_lib):
 
 def test_device_status_clean(gpu_lib):
     mla.mla_check_device_status()
+
+
+# ---------------------------------------------------------------- chunks over a cached prefix
+
+def _chunk_wl(base, chunks, prefixes, seed, **kw):
+    return W.scaled(base, kind="prefill", seqlens=tuple(chunks), seed=seed,
+                    extra=dict(prefix_lens=tuple(prefixes)), **kw)
+
+
+def _check_chunk(wl, heads=None, gap=3):
+    inp = W.chunk_inputs(wl, gap=gap)
+    got, cache = run_prefill_cached(wl, inp)
+    mla.mla_check_device_status()
+    ref, ref_cache = oracle_prefill_cached(wl, inp, heads=heads)
+    dt = "fp32" if wl.dtype == "fp32" else "bf16"
+    compare(f64(got), ref, dt, "chunk out %s" % wl.name)
+    # the chunk's rows went into the cache; no other row changed
+    new = np.zeros(cache.shape[0], bool)
+    cu, offs, pre = inp["cu_seqlens"], inp["cache_offsets"], inp["prefix_lens"]
+    for s in range(len(wl.seqlens)):
+        r0 = int(offs[s]) + int(pre[s])
+        new[r0:r0 + int(cu[s + 1] - cu[s])] = True
+    if new.any():
+        compare(f64(cache)[new], ref_cache[new], dt, "chunk cache rows %s" % wl.name)
+    assert torch.equal(cache.cpu()[torch.from_numpy(~new)], inp["cache"][torch.from_numpy(~new)])
+
+
+def test_prefill_cached_kimi_heads(gpu_lib):
+    # prefixes from empty to several tiles, chunks from none to past a tile
+    wl = _chunk_wl(W.KIMI, chunks=(5, 1, 0, 17, 130), prefixes=(0, 1, 127, 1000, 2999), seed=41)
+    _check_chunk(wl, heads=[0, 5, 31, 63])
+
+
+def test_prefill_cached_glm_heads_interleaved(gpu_lib):
+    wl = _chunk_wl(W.GLM, chunks=(3, 64), prefixes=(700, 129), seed=42)
+    _check_chunk(wl, heads=[0, 1, 62, 63])
+
+
+def test_prefill_cached_fp32_tiny_geometry(gpu_lib):
+    wl = _chunk_wl(W.TINY, chunks=(4, 9, 1), prefixes=(0, 30, 5), seed=43)
+    _check_chunk(wl)
+
+
+def test_prefill_cached_continues_a_prefill(gpu_lib):
+    # Each sequence's first tokens go into the cache through mla_cache_append,
+    # the rest run as a chunk: the chunk's outputs equal the oracle's prefill
+    # of the whole sequences at those rows.
+    wl = W.scaled(W.KIMI, seqlens=(333, 1000, 260), seed=44)
+    inp = W.prefill_inputs(wl)
+    split = (300, 999, 128)
+    rope, shape, scale = oracle_cfg(wl)
+    dims = mla.dims_for(wl, mla.mla_softmax_scale(mla.rope_for(wl), 192))
+    cos, sin = mla.mla_init_rope_tables(mla.rope_for(wl), 1000)
+    d = {k: v.cuda() for k, v in inp.items()}
+    cu = inp["cu_seqlens"].tolist()
+    first = torch.cat([torch.arange(cu[s], cu[s] + split[s]) for s in range(3)])
+    rest = torch.cat([torch.arange(cu[s] + split[s], cu[s + 1]) for s in range(3)])
+    cache = torch.zeros((sum(wl.seqlens), 576), dtype=torch.bfloat16, device="cuda")
+    offs = torch.tensor(cu[:3], dtype=torch.int64)
+    rows = torch.cat([offs[s] + torch.arange(split[s]) for s in range(3)])
+    mla.mla_cache_append(dims, d["latent"][first.cuda()].contiguous(), d["w_norm"],
+                         d["positions"][first.cuda()].contiguous(), cos, sin, cache, rows.cuda())
+    cuq = torch.tensor([0] + list(np.cumsum([wl.seqlens[s] - split[s] for s in range(3)])), dtype=torch.int32)
+    got = mla.mla_prefill_cached(dims, d["latent"][rest.cuda()].contiguous(), d["q"][rest.cuda()].contiguous(),
+                                 d["w_kvb"], d["w_norm"], cuq.cuda(), offs.cuda(),
+                                 torch.tensor(split, dtype=torch.int32, device="cuda"), 1000, cos, sin, cache)
+    torch.cuda.synchronize()
+    mla.mla_check_device_status()
+    ref = oracle_prefill(wl, inp, heads=[0, 1, 31, 63])
+    compare(f64(got), ref[rest.numpy()], "bf16", "chunk after cache append")
+
+
+def test_prefill_cached_out_of_range_sequence_is_skipped(gpu_lib):
+    # The last sequence's region is cut short (its rows would leave the
+    # cache): its tokens are neither written nor attended, their outputs are
+    # zero, the error word is set, and the other sequences are unaffected.
+    wl = _chunk_wl(W.KIMI, chunks=(6, 4), prefixes=(50, 20), seed=45)
+    inp = W.chunk_inputs(wl, gap=0)
+    full_rows = inp["cache"].shape[0]
+    inp_cut = dict(inp, cache=inp["cache"][:full_rows - 2].clone())
+    got, cache = run_prefill_cached(wl, inp_cut)
+    with pytest.raises(mla.MlaError):
+        mla.mla_check_device_status()
+    mla.mla_check_device_status()   # the error word was cleared
+    assert torch.all(got[6:].float() == 0)
+    assert torch.equal(cache[56:].cpu(), inp_cut["cache"][56:])
+    ref, _ = oracle_prefill_cached(wl, inp, heads=[0, 63])
+    compare(f64(got)[:6], ref[:6], "bf16", "chunk kept sequence")
