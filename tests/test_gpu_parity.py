@@ -12,8 +12,8 @@ import torch
 import oracle as O
 from decode_latent_rmsnorm_b200 import mla
 from decode_latent_rmsnorm_b200 import workloads as W
-from _parity import (compare, f64, oracle_cfg, oracle_decode, oracle_prefill, run_decode,
-                     run_prefill)
+from _parity import (compare, f64, oracle_cfg, oracle_decode, oracle_prefill, oracle_prefill_cached,
+                     run_decode, run_prefill, run_prefill_cached)
 
 pytestmark = pytest.mark.gpu
 
