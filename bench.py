@@ -412,55 +412,111 @@ def run_ours(args, rank, world, device):
 
 def run_e2e(args, pwl, dwl, pin, din, dims_p, dims_d, cos, sin, P, D, p_ws, d_ws, device, world,
             reduce_max, fl, by):
-    """Same calls with the step's inputs copied from pinned host memory and the
-    result read back inside the timed region. Weights, rotary tables and the
-    latent cache stay resident (model state); the step inputs are the
-    prefill's latent/q/positions/cu_seqlens and the decode's
-    q/positions/lengths/offsets."""
+    """The same calls end to end: every step copies its inputs from pinned host
+    memory and reads its result back. Weights, rotary tables and the latent
+    cache stay resident (model state); the step inputs are the prefill's
+    latent/q/positions/cu_seqlens and the decode's q/positions/lengths/offsets.
+
+    Steps run as a serving pipeline on three streams with double-buffered
+    device inputs and outputs: the upload of step i+1 and the download of
+    step i-1 overlap the kernels of step i. The timed region spans all K
+    steps, from the first upload to the last download; the reported time per
+    step is that span over K. The same steps run one after another on one
+    stream are reported under ``serial``."""
     hp = {k: pin[k].pin_memory() for k in ("latent", "q", "positions", "cu_seqlens")}
     hd = {k: din[k].pin_memory() for k in ("q", "positions", "cache_lens", "cache_offsets")}
     T = sum(pwl.seqlens)
     B = dwl.batch
     max_len = int(din["cache_lens"].max())
-    p_out_h = torch.empty((T, pwl.num_heads, pwl.v_head), dtype=torch.bfloat16).pin_memory()
-    d_out_h = torch.empty((B, dwl.num_heads, dwl.v_head), dtype=torch.bfloat16).pin_memory()
-    dp = {k: torch.empty_like(v, device=device) for k, v in hp.items()}
-    dd = {k: torch.empty_like(v, device=device) for k, v in hd.items()}
-    p_out = torch.empty(p_out_h.shape, dtype=torch.bfloat16, device=device)
-    d_out = torch.empty(d_out_h.shape, dtype=torch.bfloat16, device=device)
-    h2d_p = sum(v.numel() * v.element_size() for v in hp.values())
-    h2d_d = sum(v.numel() * v.element_size() for v in hd.values())
-    d2h_p = p_out_h.numel() * 2
-    d2h_d = d_out_h.numel() * 2
+    nb = 2
+    p_shape, d_shape = (T, pwl.num_heads, pwl.v_head), (B, dwl.num_heads, dwl.v_head)
+    bufs = dict(
+        prefill=dict(host_in=hp, dev_in=[{k: torch.empty_like(v, device=device) for k, v in hp.items()}
+                                         for _ in range(nb)],
+                     dev_out=[torch.empty(p_shape, dtype=torch.bfloat16, device=device) for _ in range(nb)],
+                     host_out=[torch.empty(p_shape, dtype=torch.bfloat16).pin_memory() for _ in range(nb)]),
+        decode=dict(host_in=hd, dev_in=[{k: torch.empty_like(v, device=device) for k, v in hd.items()}
+                                        for _ in range(nb)],
+                    dev_out=[torch.empty(d_shape, dtype=torch.bfloat16, device=device) for _ in range(nb)],
+                    host_out=[torch.empty(d_shape, dtype=torch.bfloat16).pin_memory() for _ in range(nb)]))
+    h2d = {k: sum(v.numel() * v.element_size() for v in b["host_in"].values()) for k, b in bufs.items()}
+    d2h = {k: b["host_out"][0].numel() * 2 for k, b in bufs.items()}
 
-    def step(evs):
-        evs[0].record()
-        for k in hp:
-            dp[k].copy_(hp[k], non_blocking=True)
-        mla.mla_prefill(dims_p, dp["latent"], dp["q"], P["w_kvb"], P["w_norm"], dp["positions"],
-                        dp["cu_seqlens"], max(pwl.seqlens), cos, sin, out=p_out, workspace=p_ws)
-        p_out_h.copy_(p_out, non_blocking=True)
-        evs[1].record()
-        for k in hd:
-            dd[k].copy_(hd[k], non_blocking=True)
-        mla.mla_decode(dims_d, dd["q"], D["cache"], dd["cache_offsets"], dd["cache_lens"], dd["positions"],
-                       max_len, D["w_kvb"], cos, sin, out=d_out, workspace=d_ws)
-        d_out_h.copy_(d_out, non_blocking=True)
-        evs[2].record()
+    def compute(kind, s):
+        x, out = bufs[kind]["dev_in"][s], bufs[kind]["dev_out"][s]
+        if kind == "prefill":
+            mla.mla_prefill(dims_p, x["latent"], x["q"], P["w_kvb"], P["w_norm"], x["positions"],
+                            x["cu_seqlens"], max(pwl.seqlens), cos, sin, out=out, workspace=p_ws)
+        else:
+            mla.mla_decode(dims_d, x["q"], D["cache"], x["cache_offsets"], x["cache_lens"], x["positions"],
+                           max_len, D["w_kvb"], cos, sin, out=out, workspace=d_ws)
 
-    for _ in range(args.warmup):
-        step([torch.cuda.Event(enable_timing=True) for _ in range(3)])
-    torch.cuda.synchronize()
-    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
-    for i in range(args.steps):
-        step(evs[i])
-    torch.cuda.synchronize()
-    p_ms = reduce_max(statistics.mean(e[0].elapsed_time(e[1]) for e in evs))
-    d_ms = reduce_max(statistics.mean(e[1].elapsed_time(e[2]) for e in evs))
-    return dict(value=world * fl["total"] / (p_ms * 1e-3) / 1e12, unit="TFLOP/s",
-                h2d_bytes_per_step=h2d_p + h2d_d, d2h_bytes_per_step=d2h_p + d2h_d,
-                prefill_ms=p_ms, decode_ms=d_ms,
-                decode_gbs=world * by["total"] / (d_ms * 1e-3) / 1e9)
+    def upload(kind, s):
+        b = bufs[kind]
+        for k, v in b["host_in"].items():
+            b["dev_in"][s][k].copy_(v, non_blocking=True)
+
+    def download(kind, s):
+        bufs[kind]["host_out"][s].copy_(bufs[kind]["dev_out"][s], non_blocking=True)
+
+    def pipelined(kind, steps):
+        comp = torch.cuda.current_stream()
+        up, down = torch.cuda.Stream(device), torch.cuda.Stream(device)
+        in_free, out_free = [None] * nb, [None] * nb
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize()
+        start.record(up)
+        for i in range(steps):
+            sl = i % nb
+            if in_free[sl] is not None:
+                up.wait_event(in_free[sl])
+            with torch.cuda.stream(up):
+                upload(kind, sl)
+            uploaded = torch.cuda.Event()
+            uploaded.record(up)
+            comp.wait_event(uploaded)
+            if out_free[sl] is not None:
+                comp.wait_event(out_free[sl])
+            compute(kind, sl)
+            done = torch.cuda.Event()
+            done.record(comp)
+            in_free[sl] = done
+            down.wait_event(done)
+            with torch.cuda.stream(down):
+                download(kind, sl)
+            fetched = torch.cuda.Event()
+            fetched.record(down)
+            out_free[sl] = fetched
+        end.record(down)
+        torch.cuda.synchronize()
+        return start.elapsed_time(end) / steps
+
+    def serial(kind, steps):
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(steps)]
+        for e in evs:
+            e[0].record()
+            upload(kind, 0)
+            compute(kind, 0)
+            download(kind, 0)
+            e[1].record()
+        torch.cuda.synchronize()
+        return statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+
+    res = {}
+    for kind in ("prefill", "decode"):
+        pipelined(kind, args.warmup)
+        res[kind] = reduce_max(pipelined(kind, args.steps))
+        serial(kind, args.warmup)
+        res[kind + "_serial"] = reduce_max(serial(kind, args.steps))
+    return dict(value=world * fl["total"] / (res["prefill"] * 1e-3) / 1e12, unit="TFLOP/s",
+                h2d_bytes_per_step=h2d["prefill"] + h2d["decode"], d2h_bytes_per_step=d2h["prefill"] + d2h["decode"],
+                prefill_ms=res["prefill"], decode_ms=res["decode"],
+                decode_gbs=world * by["total"] / (res["decode"] * 1e-3) / 1e9,
+                timing="pipelined steps (upload i+1 and download i-1 overlap the kernels of step i); "
+                       "span of all steps over K",
+                serial=dict(value=world * fl["total"] / (res["prefill_serial"] * 1e-3) / 1e12,
+                            prefill_ms=res["prefill_serial"], decode_ms=res["decode_serial"],
+                            decode_gbs=world * by["total"] / (res["decode_serial"] * 1e-3) / 1e9))
 
 
 def run_chunk(args, din, D, device, world, reduce_max, peaks, n_new=4):
