@@ -38,8 +38,12 @@ int fail(int code, const char* fmt, ...) {
   return code;
 }
 
+// A failed launch also leaves its error in the runtime's last-error slot;
+// reading the slot here clears it, so that the error is reported once, by the
+// call that made it, and not again by the next call's launch check.
 int cuda_status(cudaError_t e, const char* what) {
   if (e == cudaSuccess) return MLA_OK;
+  (void)cudaGetLastError();
   return fail(MLA_ERR_CUDA, "%s: %s", what, cudaGetErrorString(e));
 }
 
