@@ -24,6 +24,12 @@ Sources (page title, then the section or excerpt on it):
          "Query heads" (mla-init, mla-queries) and "Key heads" (mla-kv,
          mla-prefill excerpts).
 
+The projections on either side of the path (q_a_proj, q_a_layernorm,
+q_b_proj, kv_a_proj_with_mqa, o_proj) follow the [ROT] mla-init excerpt
+(their nn.Linear shapes) and the mla-queries / mla-kv excerpts (their order).
+They are taken without bias: the attention-bias option is outside this
+build. The pages give no hidden size or query rank; both are arguments.
+
 Readings taken where the pages are silent (each is listed in the design doc):
 
 * RMSNorm body: y = w * x / sqrt(mean(x**2) + eps), no bias, no centring;
@@ -66,6 +72,7 @@ __all__ = [
     "rms_norm", "kv_up_projection", "apply_rope",
     "causal_attention_rows", "prefill", "decode_eager", "decode_absorbed",
     "cache_append", "prefill_cached",
+    "kv_down_projection", "q_projection", "o_projection",
 ]
 
 
@@ -471,3 +478,34 @@ def prefill_cached(latent, q, cache, cache_offsets, prefix_lens, cu_seqlens, W, 
             K = np.concatenate([k_nope[hi], k_rot], axis=-1)
             out[a:b, h, :] = causal_attention_rows(Q, K, v[hi], pos, scale)              # step 4
     return out, cache
+
+
+# --------------------------------------------------------------------------
+# Projections on either side of the path -- [ROT] "Query heads" mla-init and
+# mla-queries, "Key heads" mla-kv
+# --------------------------------------------------------------------------
+
+def kv_down_projection(hidden, W_kva):
+    """kv_a_proj_with_mqa: hidden [n, hidden_size] -> compressed_kv
+    [n, R + P] = hidden @ W_kva.T, with W_kva the nn.Linear weight
+    [R + P, hidden_size]. Its first R columns are the latent that
+    kv_a_layernorm normalizes; the last P are the shared rotary key."""
+    return hidden @ W_kva.T
+
+
+def q_projection(hidden, W_qa, w_qnorm, W_qb, shape: MlaShape):
+    """q = q_b_proj(q_a_layernorm(q_a_proj(hidden))), viewed [n, H, N + P].
+
+    W_qa [q_rank, hidden_size], w_qnorm [q_rank] (an RMSNorm over the query
+    rank, the same normalization as kv_a_layernorm), W_qb [H * (N + P),
+    q_rank]; the view is q.view(bsz, q_len, H, q_head_dim) of mla-queries."""
+    q_a = hidden @ W_qa.T
+    q_an = rms_norm(q_a, w_qnorm, shape.eps)
+    q = q_an @ W_qb.T
+    return q.reshape(hidden.shape[0], shape.num_heads, shape.qk_head_dim)
+
+
+def o_projection(attn, W_o):
+    """o_proj: the attention output [n, H * V] (heads joined, as the path
+    writes it) -> [n, hidden_size] = attn @ W_o.T, W_o [hidden_size, H * V]."""
+    return attn @ W_o.T

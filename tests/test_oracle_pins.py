@@ -478,3 +478,69 @@ def test_prefill_cached_without_prefix_is_prefill():
     out, _ = O.prefill_cached(d["latent"], d["q"], np.zeros((nrows, shape.kv_lora_rank + shape.qk_rope)), offs,
                               np.zeros(3, int), d["cu"], d["W"], d["w_norm"], cos, sin, shape, scale)
     np.testing.assert_allclose(out, full, rtol=1e-12, atol=1e-13)
+
+
+# ---------------------------------------------------------------- projections on either side
+
+def _loop_linear(x, W):
+    """x @ W.T with explicit loops (independent of numpy's matmul)."""
+    out = np.zeros((x.shape[0], W.shape[0]))
+    for t in range(x.shape[0]):
+        for j in range(W.shape[0]):
+            out[t, j] = math.fsum(x[t, k] * W[j, k] for k in range(x.shape[1]))
+    return out
+
+
+def test_projections_against_loops():
+    rng = np.random.default_rng(31)
+    shape = O.MlaShape(2, 8, 4, 2, 3)
+    hid, qr = 12, 5
+    x = rng.standard_normal((3, hid))
+    W_kva = rng.standard_normal((8 + 2, hid))
+    np.testing.assert_allclose(O.kv_down_projection(x, W_kva), _loop_linear(x, W_kva), rtol=1e-13, atol=1e-13)
+    W_qa, W_qb = rng.standard_normal((qr, hid)), rng.standard_normal((2 * 6, qr))
+    w_qn = 1 + 0.1 * rng.standard_normal(qr)
+    qa = _loop_linear(x, W_qa)
+    qan = np.array([[w_qn[k] * qa[t, k] / math.sqrt(sum(v * v for v in qa[t]) / qr + shape.eps)
+                     for k in range(qr)] for t in range(3)])
+    want = _loop_linear(qan, W_qb).reshape(3, 2, 6)
+    np.testing.assert_allclose(O.q_projection(x, W_qa, w_qn, W_qb, shape), want, rtol=1e-12, atol=1e-12)
+    attn = rng.standard_normal((3, 2 * 3))
+    W_o = rng.standard_normal((hid, 6))
+    np.testing.assert_allclose(O.o_projection(attn, W_o), _loop_linear(attn, W_o), rtol=1e-13, atol=1e-13)
+
+
+def test_q_projection_layout_and_scale_invariance():
+    # unit rows pick single inputs: q_a = the picked hidden values; the
+    # RMSNorm makes the result independent of the hidden state's scale;
+    # head h of the view is rows h*(N+P) .. (h+1)*(N+P) - 1 of W_qb
+    shape = O.MlaShape(3, 8, 2, 2, 1)
+    hid, qr = 10, 4
+    W_qa = np.zeros((qr, hid))
+    for k in range(qr):
+        W_qa[k, 2 * k] = 1.0
+    W_qb = np.zeros((3 * 4, qr))
+    W_qb[1 * 4 + 3, 2] = 1.0                 # head 1, slot 3 <- q_an[2]
+    x = np.arange(1.0, hid + 1.0)[None, :]
+    q = O.q_projection(x, W_qa, np.ones(qr), W_qb, shape)
+    qa = x[0, [0, 2, 4, 6]]
+    expect = qa[2] / math.sqrt(np.mean(qa ** 2) + shape.eps)
+    assert q.shape == (1, 3, 4)
+    assert abs(q[0, 1, 3] - expect) < 1e-14 and np.count_nonzero(q) == 1
+    q10 = O.q_projection(10 * x, W_qa, np.ones(qr), W_qb, shape)
+    np.testing.assert_allclose(q10, q, rtol=1e-6)   # eps only breaks exact invariance
+
+
+def test_kv_down_then_append_is_the_paths_cache_row():
+    # compressed_kv from the down-projection, split, normalized and rotated:
+    # the cache row the decode reads (GLM-5 "KV cache" order)
+    rng = np.random.default_rng(32)
+    shape = O.MlaShape(2, 16, 4, 4, 4)
+    x = rng.standard_normal((2, 20))
+    W = rng.standard_normal((20, 20)) / math.sqrt(20)
+    cos, sin = O.rope_tables(O.RopeConfig(rope_dim=4, base=10000.0), 8)
+    latent = O.kv_down_projection(x, W)
+    rows = O.cache_append(latent, np.ones(16), [3, 5], cos, sin, shape)
+    np.testing.assert_allclose(rows[:, :16], O.rms_norm(latent[:, :16], np.ones(16), shape.eps), rtol=1e-14)
+    np.testing.assert_allclose(np.linalg.norm(rows[:, 16:], axis=-1), np.linalg.norm(latent[:, 16:], axis=-1),
+                               rtol=1e-13)
