@@ -388,6 +388,7 @@ def run_ours(args, rank, world, device):
     roof["peak_source"] = peaks["source"]
 
     chunk = run_chunk(args, din, D, device, world, reduce_max, peaks)
+    projections = run_projections(args, device, world, reduce_max, peaks)
 
     # end to end through the same C-ABI with pinned host buffers
     e2e = run_e2e(args, pwl, dwl, pin, din, dims_p, dims_d, cos, sin, P, D, p_ws, d_ws, device, world,
@@ -403,7 +404,7 @@ def run_ours(args, rank, world, device):
         decode=dict(metric="absorbed decode HBM GB/s", value=d_gbs, unit="GB/s", ms=d_mean,
                     frac_of_hbm=d_gbs / (world * peaks["hbm"]), tokens_per_s=world * B / (d_mean * 1e-3),
                     tflops=world * by["flops"] / (d_mean * 1e-3) / 1e12, bytes=by["total"]),
-        kernels_ms=dict(prefill=kp_ms, decode=kd_ms), chunk=chunk,
+        kernels_ms=dict(prefill=kp_ms, decode=kd_ms), chunk=chunk, projections=projections,
         roofline=roof, e2e=e2e, gpu_launches=int(launches), clocks=clocks.summary(),
         peaks=dict(hbm_gbs=peaks["hbm"], bf16_tflops=peaks["bf16"], source=peaks["source"]),
     )
@@ -573,6 +574,51 @@ def run_chunk(args, din, D, device, world, reduce_max, peaks, n_new=4):
                 attended_frac_of_hbm=att / (world * peaks["hbm"]),
                 unique_cache_gbs=world * by["unique"] / (ms * 1e-3) / 1e9,
                 kernels_ms=dict(zip(kev.names, kev.durations_ms())))
+
+
+def run_projections(args, device, world, reduce_max, peaks, n=2048, hidden=7168, q_rank=1536):
+    """The projections on either side of the path at the Kimi-K2 prefill size
+    (hidden size 7168 and query rank 1536 of the Kimi-K2 model): the joint
+    down-projection with the cache append, the query path and o_proj, each
+    timed alone with CUDA events; a 256 MiB write before each timed call
+    (outside its events) flushes L2."""
+    wl = W.KIMI
+    inp = W.projection_inputs(wl, n, hidden, q_rank)
+    d = {k: v.to(device) for k, v in inp.items()}
+    dims = mla.dims_for(wl, mla.mla_softmax_scale(mla.rope_for(wl), wl.qk_head_dim))
+    cos, sin = mla.mla_init_rope_tables(mla.rope_for(wl), n)
+    H, R, N, P, V = wl.num_heads, wl.kv_lora_rank, wl.qk_nope, wl.qk_rope, wl.v_head
+    latent = torch.empty((n, R + P), dtype=torch.bfloat16, device=device)
+    cache = torch.empty((n, R + P), dtype=torch.bfloat16, device=device)
+    rows = torch.arange(n, dtype=torch.int64, device=device)
+    q = torch.empty((n, H, N + P), dtype=torch.bfloat16, device=device)
+    q_ws = torch.empty(mla.mla_q_proj_workspace_size(dims, q_rank, n), dtype=torch.uint8, device=device)
+    out = torch.empty((n, hidden), dtype=torch.bfloat16, device=device)
+    calls = dict(
+        kv_a_proj_and_append=(lambda: mla.mla_kv_down_append(dims, d["hidden"], d["w_kva"], latent, d["w_norm"],
+                                                             d["positions"], cos, sin, cache, rows),
+                              2.0 * n * hidden * (R + P)),
+        q_proj=(lambda: mla.mla_q_proj(dims, d["hidden"], d["w_qa"], d["w_qnorm"], d["w_qb"], q, q_ws),
+                2.0 * n * hidden * q_rank + 2.0 * n * q_rank * H * (N + P)),
+        o_proj=(lambda: mla.mla_o_proj(dims, d["attn"], d["w_o"], out), 2.0 * n * H * V * hidden))
+    res = dict(workload="Kimi-K2 heads, %d tokens, hidden %d, query rank %d" % (n, hidden, q_rank),
+               l2="flushed before each timed call")
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    for name, (fn, flops) in calls.items():
+        for _ in range(args.warmup):
+            fn()
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+        for i, e in enumerate(evs):
+            flush.fill_(i & 0xff)
+            e[0].record()
+            fn()
+            e[1].record()
+        torch.cuda.synchronize()
+        ms = reduce_max(statistics.mean(e[0].elapsed_time(e[1]) for e in evs))
+        tf = world * flops / (ms * 1e-3) / 1e12
+        res[name] = dict(ms=ms, tflops=tf, frac_of_bf16_peak=tf / (world * peaks["bf16"]), gflop=flops / 1e9)
+    mla.mla_check_device_status()
+    return res
 
 
 def cpu_baseline(budget_s=15.0):

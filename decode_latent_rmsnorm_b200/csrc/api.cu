@@ -19,6 +19,7 @@
 #include "tc_attention_pair.cuh"
 #include "tc_decode.cuh"
 #include "chunk.cuh"
+#include "proj.cuh"
 
 #include <cudaTypedefs.h>
 
@@ -953,6 +954,74 @@ ChunkWs chunk_ws_layout(const mla_dims* d, int64_t n, int max_total_len) {
 constexpr int64_t kMaxChunkTokens = 65535;   // the decode's batch limit
 }  // namespace
 
+// ---- projections on either side of the path ----------------------------------
+namespace {
+constexpr int64_t kMaxProjRows = (int64_t)1 << 20;   // grid limits of the Linear kernels
+
+// out[t, j] = sum_k x[t, k] w[j, k] for x [n, K], w [Nout, K], out [n, Nout]
+// (row-major). bf16 with K a multiple of 64 and 16-byte aligned operands:
+// tcgen05 (head_gemm_kernel with one head, M = 128 output features x N = 64
+// rows per CTA); otherwise the CUDA-core Linear.
+int launch_linear(const mla_dims* d, const void* x, const void* w, void* out, int64_t n, int K, int Nout,
+                  cudaStream_t st, const char* name) {
+  namespace T = mla::tc;
+  if (d->dtype == MLA_BF16 && K % 64 == 0 && aligned16(x) && aligned16(w)) {
+    CUtensorMap map_w, map_x;
+    {
+      const uint64_t dims[2] = {(uint64_t)K, (uint64_t)Nout};
+      const uint64_t strides[1] = {(uint64_t)K * 2};
+      const uint32_t box[2] = {64, 128};
+      int rc = make_map(&map_w, w, 2, dims, strides, box);
+      if (rc) return rc;
+    }
+    {
+      const uint64_t dims[3] = {(uint64_t)K, 1, (uint64_t)n};
+      const uint64_t strides[2] = {(uint64_t)K * 2, (uint64_t)K * 2};
+      const uint32_t box[3] = {64, 1, 64};
+      int rc = make_map(&map_x, x, 3, dims, strides, box);
+      if (rc) return rc;
+    }
+    cudaError_t e = cudaFuncSetAttribute(T::head_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)T::kHgSmem);
+    if (e != cudaSuccess) return cuda_status(e, "linear smem attribute");
+    T::HgParams hp{};
+    hp.out = static_cast<__nv_bfloat16*>(out);
+    hp.out_bs = Nout;
+    hp.out_hs = 0;
+    hp.B = (int)n;
+    hp.Nout = Nout;
+    hp.K = K;
+    hp.a_row0 = 0;
+    hp.a_hstride = 0;
+    prof_begin(st, name);
+    T::head_gemm_kernel<false><<<dim3(1, (unsigned)((Nout + 127) / 128), (unsigned)((n + 63) / 64)), 192,
+                                 T::kHgSmem, st>>>(map_w, map_x, hp);
+    prof_end(st);
+    return cuda_status(cudaGetLastError(), name);
+  }
+  const dim3 grid((unsigned)((Nout + mla::kLinTile - 1) / mla::kLinTile),
+                  (unsigned)((n + mla::kLinTile - 1) / mla::kLinTile));
+  prof_begin(st, name);
+  if (d->dtype == MLA_FP32)
+    mla::simt_linear_kernel<float><<<grid, mla::kLinTile * mla::kLinTile, 0, st>>>(
+        static_cast<const float*>(x), static_cast<const float*>(w), static_cast<float*>(out), n, K, Nout);
+  else
+    mla::simt_linear_kernel<__nv_bfloat16><<<grid, mla::kLinTile * mla::kLinTile, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w),
+        static_cast<__nv_bfloat16*>(out), n, K, Nout);
+  prof_end(st);
+  return cuda_status(cudaGetLastError(), name);
+}
+
+int check_proj_rows(int64_t n) {
+  if (n < 0) return fail(MLA_ERR_INVALID_ARG, "n must be >= 0");
+  if (n > kMaxProjRows) return fail(MLA_ERR_UNSUPPORTED_SHAPE, "at most %lld rows per call", (long long)kMaxProjRows);
+  return MLA_OK;
+}
+
+size_t elem_bytes(const mla_dims* d) { return d->dtype == MLA_FP32 ? 4 : 2; }
+}  // namespace
+
 // Device address of g_noalloc_scratch, looked up once per device (host code
 // cannot use the array's name as a device address).
 namespace {
@@ -1050,6 +1119,83 @@ int mla_prefill_cached(const mla_dims* dims, const void* latent, const void* q, 
   if (rc) return rc;
   return mla_decode(dims, q, cache, cache_num_rows, offsets, lens, positions, (int32_t)total_tokens, max_total_len,
                     w_kvb, cos_table, sin_table, max_pos, out, ws + L.decode, workspace_bytes - L.decode, stream);
+}
+
+int mla_kv_down_append(const mla_dims* dims, int32_t hidden_size, const void* hidden, const void* w_kva,
+                       const void* w_norm, const int32_t* positions, int64_t n, const float* cos_table,
+                       const float* sin_table, int32_t max_pos, void* latent, void* cache, int64_t cache_num_rows,
+                       const int64_t* cache_rows, cudaStream_t stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  rc = check_proj_rows(n);
+  if (rc) return rc;
+  if (hidden_size < 1) return fail(MLA_ERR_INVALID_ARG, "hidden_size must be >= 1");
+  if (!hidden || !w_kva || !latent) return fail(MLA_ERR_INVALID_ARG, "a tensor pointer is NULL");
+  const bool append = cache != nullptr || cache_rows != nullptr;
+  if (append && (!cache || !cache_rows || !w_norm || !positions || !cos_table || !sin_table))
+    return fail(MLA_ERR_INVALID_ARG, "appending needs cache, cache_rows, w_norm, positions and the tables");
+  if (n == 0) return MLA_OK;
+  rc = launch_linear(dims, hidden, w_kva, latent, n, hidden_size, dims->kv_lora_rank + dims->qk_rope, stream,
+                     "kv_a_proj");
+  if (rc || !append) return rc;
+  return mla_cache_append(dims, latent, w_norm, positions, n, cos_table, sin_table, max_pos, cache, cache_num_rows,
+                          cache_rows, stream);
+}
+
+int mla_q_proj_workspace_size(const mla_dims* dims, int32_t q_rank, int64_t n, size_t* bytes) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  rc = check_proj_rows(n);
+  if (rc) return rc;
+  if (q_rank < 1) return fail(MLA_ERR_INVALID_ARG, "q_rank must be >= 1");
+  if (!bytes) return fail(MLA_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = align_up((size_t)n * (size_t)q_rank * elem_bytes(dims), 256);
+  return MLA_OK;
+}
+
+int mla_q_proj(const mla_dims* dims, int32_t hidden_size, int32_t q_rank, const void* hidden, const void* w_qa,
+               const void* w_qnorm, const void* w_qb, int64_t n, void* q, void* workspace, size_t workspace_bytes,
+               cudaStream_t stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  rc = check_proj_rows(n);
+  if (rc) return rc;
+  if (hidden_size < 1 || q_rank < 1) return fail(MLA_ERR_INVALID_ARG, "hidden_size and q_rank must be >= 1");
+  if (!hidden || !w_qa || !w_qnorm || !w_qb || !q) return fail(MLA_ERR_INVALID_ARG, "a tensor pointer is NULL");
+  if (n == 0) return MLA_OK;
+  const size_t need = align_up((size_t)n * (size_t)q_rank * elem_bytes(dims), 256);
+  if (!workspace || workspace_bytes < need)
+    return fail(MLA_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes, got %zu", need, workspace_bytes);
+  // q_a = hidden W_qa^T, normalized in place, then q = q_a W_qb^T
+  rc = launch_linear(dims, hidden, w_qa, workspace, n, hidden_size, q_rank, stream, "q_a_proj");
+  if (rc) return rc;
+  const unsigned blocks = (unsigned)((n + mla::kRowsPerNormBlock - 1) / mla::kRowsPerNormBlock);
+  prof_begin(stream, "q_a_layernorm");
+  if (dims->dtype == MLA_FP32)
+    mla::rmsnorm_rows_kernel<float><<<blocks, 32 * mla::kRowsPerNormBlock, 0, stream>>>(
+        static_cast<const float*>(workspace), static_cast<const float*>(w_qnorm), static_cast<float*>(workspace), n,
+        q_rank, dims->eps);
+  else
+    mla::rmsnorm_rows_kernel<__nv_bfloat16><<<blocks, 32 * mla::kRowsPerNormBlock, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(workspace), static_cast<const __nv_bfloat16*>(w_qnorm),
+        static_cast<__nv_bfloat16*>(workspace), n, q_rank, dims->eps);
+  prof_end(stream);
+  rc = cuda_status(cudaGetLastError(), "q_a_layernorm launch");
+  if (rc) return rc;
+  return launch_linear(dims, workspace, w_qb, q, n, q_rank, dims->num_heads * (dims->qk_nope + dims->qk_rope),
+                       stream, "q_b_proj");
+}
+
+int mla_o_proj(const mla_dims* dims, int32_t hidden_size, const void* attn, const void* w_o, int64_t n, void* out,
+               cudaStream_t stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  rc = check_proj_rows(n);
+  if (rc) return rc;
+  if (hidden_size < 1) return fail(MLA_ERR_INVALID_ARG, "hidden_size must be >= 1");
+  if (!attn || !w_o || !out) return fail(MLA_ERR_INVALID_ARG, "a tensor pointer is NULL");
+  if (n == 0) return MLA_OK;
+  return launch_linear(dims, attn, w_o, out, n, dims->num_heads * dims->v_head, hidden_size, stream, "o_proj");
 }
 
 int mla_check_device_status(cudaStream_t stream) {

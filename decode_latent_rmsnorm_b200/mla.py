@@ -38,6 +38,11 @@ SIGNATURES = {
     "mla_prefill_cached_workspace_size": (c_i32, [c_vp, c_i64, c_i32, ctypes.POINTER(c_sz)]),
     "mla_prefill_cached": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_i32, c_i64, c_vp, c_vp, c_i32,
                                    c_vp, c_vp, c_i32, c_vp, c_i64, c_vp, c_vp, c_sz, c_vp]),
+    "mla_kv_down_append": (c_i32, [c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_i64, c_vp, c_vp, c_i32, c_vp, c_vp,
+                                   c_i64, c_vp, c_vp]),
+    "mla_q_proj_workspace_size": (c_i32, [c_vp, c_i32, c_i64, ctypes.POINTER(c_sz)]),
+    "mla_q_proj": (c_i32, [c_vp, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_i64, c_vp, c_vp, c_sz, c_vp]),
+    "mla_o_proj": (c_i32, [c_vp, c_i32, c_vp, c_vp, c_i64, c_vp, c_vp]),
     "mla_check_device_status": (c_i32, [c_vp]),
     "mla_last_error_string": (ctypes.c_char_p, []),
     "mla_version": (c_i32, []),
@@ -266,6 +271,74 @@ def mla_prefill_cached(dims: Dims, latent, q, w_kvb, w_norm, cu_seqlens, cache_o
         _dev(cos, "cos", torch.float32), _dev(sin, "sin", torch.float32), int(cos.shape[0]),
         _dev(cache, "cache", dt), int(cache.shape[0]), _dev(out, "out", dt, (T, H, V)),
         _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream()))
+    return out
+
+
+def mla_kv_down_append(dims: Dims, hidden, w_kva, latent=None, w_norm=None, positions=None, cos=None, sin=None,
+                       cache=None, cache_rows=None):
+    """kv_a_proj_with_mqa: returns ``latent`` [n, R + P]; with ``cache`` and
+    ``cache_rows`` also appends the normalized, rotated rows to the cache."""
+    dt = dims.torch_dtype
+    R, P = dims.kv_lora_rank, dims.qk_rope
+    n, hid = hidden.shape
+    if latent is None:
+        latent = torch.empty((n, R + P), dtype=dt, device=hidden.device)
+    append = cache is not None or cache_rows is not None
+    if append:
+        if cache is None or cache_rows is None or w_norm is None or positions is None or cos is None or sin is None:
+            raise ValueError("appending needs cache, cache_rows, w_norm, positions, cos and sin")
+        if cache.dim() != 2 or cache.shape[1] != R + P:
+            raise ValueError("cache must be [rows, R + P]")
+    none = ctypes.c_void_p(0)
+    _check(load().mla_kv_down_append(
+        ctypes.byref(dims), int(hid), _dev(hidden, "hidden", dt, (n, hid)), _dev(w_kva, "w_kva", dt, (R + P, hid)),
+        _dev(w_norm, "w_norm", dt, (R,)) if append else none,
+        _dev(positions, "positions", torch.int32, (n,)) if append else none, int(n),
+        _dev(cos, "cos", torch.float32) if append else none, _dev(sin, "sin", torch.float32) if append else none,
+        int(cos.shape[0]) if append else 0, _dev(latent, "latent", dt, (n, R + P)),
+        _dev(cache, "cache", dt) if append else none, int(cache.shape[0]) if append else 0,
+        _dev(cache_rows, "cache_rows", torch.int64, (n,)) if append else none, _stream()))
+    return latent
+
+
+def mla_q_proj_workspace_size(dims: Dims, q_rank: int, n: int) -> int:
+    out = c_sz()
+    _check(load().mla_q_proj_workspace_size(ctypes.byref(dims), int(q_rank), int(n), ctypes.byref(out)))
+    return out.value
+
+
+def mla_q_proj(dims: Dims, hidden, w_qa, w_qnorm, w_qb, q=None, workspace=None):
+    """q = q_b_proj(q_a_layernorm(q_a_proj(hidden))); returns q [n, H, N + P]."""
+    dt = dims.torch_dtype
+    H, N, P = dims.num_heads, dims.qk_nope, dims.qk_rope
+    n, hid = hidden.shape
+    q_rank = w_qa.shape[0]
+    if q is None:
+        q = torch.empty((n, H, N + P), dtype=dt, device=hidden.device)
+    if workspace is None:
+        workspace = torch.empty(max(mla_q_proj_workspace_size(dims, q_rank, n), 1), dtype=torch.uint8,
+                                device=hidden.device)
+    _check(load().mla_q_proj(
+        ctypes.byref(dims), int(hid), int(q_rank), _dev(hidden, "hidden", dt, (n, hid)),
+        _dev(w_qa, "w_qa", dt, (q_rank, hid)), _dev(w_qnorm, "w_qnorm", dt, (q_rank,)),
+        _dev(w_qb, "w_qb", dt, (H * (N + P), q_rank)), int(n), _dev(q, "q", dt, (n, H, N + P)),
+        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream()))
+    return q
+
+
+def mla_o_proj(dims: Dims, attn, w_o, out=None):
+    """o_proj: attn [n, H, V] or [n, H * V] -> out [n, hidden_size]."""
+    dt = dims.torch_dtype
+    H, V = dims.num_heads, dims.v_head
+    n = attn.shape[0]
+    hid = w_o.shape[0]
+    if tuple(attn.shape[1:]) not in ((H, V), (H * V,)):
+        raise ValueError("attn must be [n, H, V] or [n, H * V]")
+    if out is None:
+        out = torch.empty((n, hid), dtype=dt, device=attn.device)
+    _check(load().mla_o_proj(
+        ctypes.byref(dims), int(hid), _dev(attn, "attn", dt), _dev(w_o, "w_o", dt, (hid, H * V)), int(n),
+        _dev(out, "out", dt, (n, hid)), _stream()))
     return out
 
 

@@ -188,6 +188,32 @@ def chunk_inputs(wl: Workload, gap: int = 0) -> dict:
                 max_total_len=max([p + n for p, n in zip(prefix, chunks)] + [1]))
 
 
+def projection_inputs(wl: Workload, n: int, hidden_size: int, q_rank: int, seed: int = 0) -> dict:
+    """CPU tensors for the projections on either side of the path, in the
+    run dtype: hidden [n, hidden_size] and attn [n, H * V] ~ N(0, 1); the
+    weights ~ N(0, 1/in) so each Linear keeps unit variance: w_kva
+    [R + P, hidden_size], w_qa [q_rank, hidden_size], w_qb [H * (N + P),
+    q_rank], w_o [hidden_size, H * V]; the RMSNorm weights w_norm [R] and
+    w_qnorm [q_rank] = 1 + 0.1 * N(0, 1); positions [n] = 0 .. n - 1."""
+    g = torch.Generator().manual_seed(wl.seed + 3000 + seed)
+    dt = wl.torch_dtype
+    H, R, N, P, V = wl.num_heads, wl.kv_lora_rank, wl.qk_nope, wl.qk_rope, wl.v_head
+
+    def lin(out_f, in_f):
+        return (torch.randn((out_f, in_f), generator=g) * (1.0 / in_f) ** 0.5).to(dt)
+
+    hidden = _randn(g, (n, hidden_size), dt)
+    attn = _randn(g, (n, H * V), dt)
+    w_kva = lin(R + P, hidden_size)
+    w_qa = lin(q_rank, hidden_size)
+    w_qb = lin(H * (N + P), q_rank)
+    w_o = lin(hidden_size, H * V)
+    w_norm = (1.0 + 0.1 * torch.randn((R,), generator=g)).to(dt)
+    w_qnorm = (1.0 + 0.1 * torch.randn((q_rank,), generator=g)).to(dt)
+    return dict(hidden=hidden, attn=attn, w_kva=w_kva, w_qa=w_qa, w_qb=w_qb, w_o=w_o, w_norm=w_norm,
+                w_qnorm=w_qnorm, positions=torch.arange(n, dtype=torch.int32))
+
+
 def max_position(wl: Workload) -> int:
     """Smallest rotary-table length that covers every position used."""
     if wl.kind == "prefill":

@@ -211,6 +211,47 @@ int mla_prefill_cached(const mla_dims* dims, const void* latent, const void* q, 
                        void* cache, int64_t cache_num_rows, void* out, void* workspace,
                        size_t workspace_bytes, cudaStream_t stream);
 
+/* The projections on either side of the path ([ROT] "Query heads": mla-init
+ * gives the nn.Linear shapes, mla-queries the query order; "Key heads": mla-kv
+ * the joint down-projection). A Linear is out[t, j] = sum_k x[t, k] w[j, k],
+ * with w the nn.Linear weight [out, in]; no bias. In bf16 runs with the
+ * reduced dimension K a multiple of 64 and 16-byte aligned x and w it runs on
+ * the tensor cores (fp32 accumulation, bf16 result); otherwise on the CUDA
+ * cores. At most 2^20 rows (tokens) per call (MLA_ERR_UNSUPPORTED_SHAPE). */
+
+/* kv_a_proj_with_mqa, optionally followed by the cache append:
+ *   hidden     [n, hidden_size]
+ *   w_kva      [R + P, hidden_size]
+ *   latent     [n, R + P]  written: compressed_kv (the latent input of mla_prefill)
+ * If cache and cache_rows are both non-NULL, the rows of latent are then
+ * appended exactly as by mla_cache_append (w_norm, positions and the tables
+ * are then required); if both are NULL only latent is written. */
+int mla_kv_down_append(const mla_dims* dims, int32_t hidden_size, const void* hidden,
+                       const void* w_kva, const void* w_norm, const int32_t* positions, int64_t n,
+                       const float* cos_table, const float* sin_table, int32_t max_pos,
+                       void* latent, void* cache, int64_t cache_num_rows,
+                       const int64_t* cache_rows, cudaStream_t stream);
+
+/* Workspace bytes of mla_q_proj: the [n, q_rank] intermediate. */
+int mla_q_proj_workspace_size(const mla_dims* dims, int32_t q_rank, int64_t n, size_t* bytes);
+
+/* q = q_b_proj(q_a_layernorm(q_a_proj(hidden))):
+ *   hidden  [n, hidden_size]
+ *   w_qa    [q_rank, hidden_size]
+ *   w_qnorm [q_rank]  RMSNorm weight (eps = dims->eps)
+ *   w_qb    [H * (N + P), q_rank]
+ *   q       [n, H, N + P]  written (the q input of mla_prefill / mla_decode)
+ * The intermediate q_a is kept in the run dtype in the workspace (bf16 runs
+ * round it to bf16, as the model's bf16 Linear does). */
+int mla_q_proj(const mla_dims* dims, int32_t hidden_size, int32_t q_rank, const void* hidden,
+               const void* w_qa, const void* w_qnorm, const void* w_qb, int64_t n, void* q,
+               void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/* o_proj: attn [n, H * V] (the output of mla_prefill / mla_decode, heads
+ * joined) times w_o [hidden_size, H * V]^T -> out [n, hidden_size]. */
+int mla_o_proj(const mla_dims* dims, int32_t hidden_size, const void* attn, const void* w_o,
+               int64_t n, void* out, cudaStream_t stream);
+
 /* Size of the scratch array behind mla_prefill_noalloc (32 MiB). */
 #define MLA_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 

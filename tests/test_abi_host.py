@@ -153,3 +153,46 @@ def test_prefill_cached_host_validation():
     assert call(wsb=need - 1) == 3
     with pytest.raises(mla.MlaError):
         mla.mla_prefill_cached_workspace_size(d, 65536, 100)
+
+
+def test_projection_host_validation():
+    lib = mla.load()
+    d = kimi_dims()
+
+    def kv(**o):
+        a = dict(hid=7168, x=FAKE, w=FAKE, wn=FAKE, pos=FAKE, n=4, cos=FAKE, sin=FAKE, mp=10, lat=FAKE, cache=None,
+                 rows=0, crows=None)
+        a.update(o)
+        return lib.mla_kv_down_append(ctypes.byref(d), a["hid"], a["x"], a["w"], a["wn"], a["pos"], a["n"], a["cos"],
+                                      a["sin"], a["mp"], a["lat"], a["cache"], a["rows"], a["crows"], None)
+
+    assert kv(n=0) == 0
+    assert kv(n=-1) == 1
+    assert kv(n=(1 << 20) + 1) == 2
+    assert kv(hid=0) == 1
+    assert kv(x=None) == 1
+    assert kv(lat=None) == 1
+    assert kv(cache=FAKE) == 1                     # a cache without destination rows
+    assert kv(cache=FAKE, crows=FAKE, wn=None) == 1
+
+    def qp(**o):
+        a = dict(hid=7168, qr=1536, x=FAKE, wa=FAKE, wn=FAKE, wb=FAKE, n=4, q=FAKE, ws=FAKE, wsb=1 << 40)
+        a.update(o)
+        return lib.mla_q_proj(ctypes.byref(d), a["hid"], a["qr"], a["x"], a["wa"], a["wn"], a["wb"], a["n"], a["q"],
+                              a["ws"], a["wsb"], None)
+
+    assert qp(n=0) == 0
+    assert qp(qr=0) == 1
+    assert qp(wn=None) == 1
+    assert qp(wsb=16) == 3
+    assert mla.mla_q_proj_workspace_size(d, 1536, 100) >= 100 * 1536 * 2
+
+    def op(**o):
+        a = dict(hid=7168, x=FAKE, w=FAKE, n=4, out=FAKE)
+        a.update(o)
+        return lib.mla_o_proj(ctypes.byref(d), a["hid"], a["x"], a["w"], a["n"], a["out"], None)
+
+    assert op(n=0) == 0
+    assert op(hid=-3) == 1
+    assert op(out=None) == 1
+    assert op(n=(1 << 21)) == 2

@@ -12,8 +12,8 @@ import torch
 import oracle as O
 from decode_latent_rmsnorm_b200 import mla
 from decode_latent_rmsnorm_b200 import workloads as W
-from _parity import (compare, f64, oracle_cfg, oracle_decode, oracle_prefill, oracle_prefill_cached,
-                     run_decode, run_prefill, run_prefill_cached)
+from _parity import (compare, compare_rounded, f64, oracle_cfg, oracle_decode, oracle_prefill,
+                     oracle_prefill_cached, run_decode, run_prefill, run_prefill_cached)
 
 pytestmark = pytest.mark.gpu
 
@@ -303,3 +303,71 @@ def test_prefill_cached_out_of_range_sequence_is_skipped(gpu_lib):
     assert torch.equal(cache[56:].cpu(), inp_cut["cache"][56:])
     ref, _ = oracle_prefill_cached(wl, inp, heads=[0, 63])
     compare(f64(got)[:6], ref[:6], "bf16", "chunk kept sequence")
+
+
+# ---------------------------------------------------------------- projections on either side
+
+# hidden size and query rank of the Kimi-K2 model (the pages name the
+# projections but print neither size)
+KIMI_HIDDEN, KIMI_QRANK = 7168, 1536
+
+
+def _proj_case(wl, n, hid, qr, seed):
+    inp = W.projection_inputs(wl, n, hid, qr, seed)
+    rope, shape, _ = oracle_cfg(wl)
+    dims = mla.dims_for(wl, mla.mla_softmax_scale(mla.rope_for(wl), shape.qk_head_dim))
+    return inp, {k: v.cuda() for k, v in inp.items()}, dims, rope, shape
+
+
+@pytest.mark.parametrize("hid", [KIMI_HIDDEN, 1000], ids=["tensor_cores", "cuda_cores"])
+def test_kv_down_append_kimi_heads(gpu_lib, hid):
+    n = 130
+    inp, d, dims, rope, shape = _proj_case(W.KIMI, n, hid, 64, seed=1)
+    cos, sin = mla.mla_init_rope_tables(mla.rope_for(W.KIMI), n)
+    cache = torch.full((n + 9, 576), 3.0, dtype=torch.bfloat16, device="cuda")
+    rows = torch.arange(n, dtype=torch.int64, device="cuda") + 5
+    latent = mla.mla_kv_down_append(dims, d["hidden"], d["w_kva"], w_norm=d["w_norm"], positions=d["positions"],
+                                    cos=cos, sin=sin, cache=cache, cache_rows=rows)
+    torch.cuda.synchronize()
+    mla.mla_check_device_status()
+    lat_ref = O.kv_down_projection(f64(inp["hidden"]), f64(inp["w_kva"]))
+    compare(f64(latent), lat_ref, "bf16", "kv_a_proj K=%d" % hid)
+    ocos, osin = O.rope_tables(rope, n)
+    rows_ref = O.cache_append(lat_ref, f64(inp["w_norm"]), inp["positions"].numpy(), ocos, osin, shape)
+    compare_rounded(f64(cache[5:n + 5]), rows_ref, "kv_a_proj cache rows K=%d" % hid)
+    assert torch.all(cache[:5] == 3.0) and torch.all(cache[n + 5:] == 3.0)
+
+
+@pytest.mark.parametrize("hid,qr", [(KIMI_HIDDEN, KIMI_QRANK), (1000, 200)], ids=["tensor_cores", "cuda_cores"])
+def test_q_proj_kimi_heads(gpu_lib, hid, qr):
+    n = 130
+    inp, d, dims, rope, shape = _proj_case(W.KIMI, n, hid, qr, seed=2)
+    q = mla.mla_q_proj(dims, d["hidden"], d["w_qa"], d["w_qnorm"], d["w_qb"])
+    torch.cuda.synchronize()
+    mla.mla_check_device_status()
+    ref = O.q_projection(f64(inp["hidden"]), f64(inp["w_qa"]), f64(inp["w_qnorm"]), f64(inp["w_qb"]), shape)
+    compare_rounded(f64(q), ref, "q_proj K=%d/%d" % (hid, qr))
+
+
+def test_o_proj_kimi_heads(gpu_lib):
+    n = 130
+    inp, d, dims, rope, shape = _proj_case(W.KIMI, n, KIMI_HIDDEN, 64, seed=3)
+    out = mla.mla_o_proj(dims, d["attn"], d["w_o"])
+    torch.cuda.synchronize()
+    mla.mla_check_device_status()
+    compare(f64(out), O.o_projection(f64(inp["attn"]), f64(inp["w_o"])), "bf16", "o_proj")
+
+
+def test_projections_fp32_tiny(gpu_lib):
+    n, hid, qr = 37, 48, 24
+    inp, d, dims, rope, shape = _proj_case(W.TINY, n, hid, qr, seed=4)
+    latent = mla.mla_kv_down_append(dims, d["hidden"], d["w_kva"])
+    q = mla.mla_q_proj(dims, d["hidden"], d["w_qa"], d["w_qnorm"], d["w_qb"])
+    out = mla.mla_o_proj(dims, d["attn"], d["w_o"])
+    torch.cuda.synchronize()
+    mla.mla_check_device_status()
+    x = f64(inp["hidden"])
+    compare(f64(latent), O.kv_down_projection(x, f64(inp["w_kva"])), "fp32", "kv_a_proj fp32")
+    compare(f64(q), O.q_projection(x, f64(inp["w_qa"]), f64(inp["w_qnorm"]), f64(inp["w_qb"]), shape), "fp32",
+            "q_proj fp32")
+    compare(f64(out), O.o_projection(f64(inp["attn"]), f64(inp["w_o"])), "fp32", "o_proj fp32")
