@@ -30,7 +30,7 @@ q_b_proj, kv_a_proj_with_mqa, o_proj) follow the [ROT] mla-init excerpt
 They are taken without bias: the attention-bias option is outside this
 build. The pages give no hidden size or query rank; both are arguments.
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
 
 * RMSNorm body: y = w * x / sqrt(mean(x**2) + eps), no bias, no centring;
   eps = 1e-6 ([GLM] "Key-value compression" says the latent RMSNorms use the
