@@ -4,8 +4,12 @@
 
 Cases: ``kimi_prefill`` (B=1 T=2048 H=64, YaRN), ``glm_prefill`` (B=2 T=4096,
 N=192 V=256), ``decode`` (B=64 absorbed decode over latent caches of lengths
-uniform in [1000, 32768]), ``all`` (Kimi prefill then decode). Inputs are the
-seeded synthetic workloads; every call goes through the C-ABI library.
+uniform in [1000, 32768]), ``chunk`` (4 new tokens on each of 64 cached
+sequences of 16384 rows, about 1.2 GB of cache), ``projections`` (the joint
+down-projection with the cache append, the query path and o_proj at 2048
+tokens, hidden size 7168, query rank 1536), ``all`` (Kimi prefill then
+decode). Inputs are the seeded synthetic workloads; every call goes through
+the C-ABI library.
 The last line printed is the mean device time of the calls after the first.
 """
 
@@ -52,9 +56,50 @@ def _decode_call(wl, device):
     return call
 
 
+def _chunk_call(device, n_new=4, prefix=16384, batch=64):
+    wl = W.scaled(W.KIMI, seqlens=(n_new,) * batch, seed=5, extra=dict(prefix_lens=(prefix,) * batch))
+    inp = W.chunk_inputs(wl)
+    d = {k: v.to(device) for k, v in inp.items() if isinstance(v, torch.Tensor)}
+    rope = mla.rope_for(wl)
+    dims = mla.dims_for(wl, mla.mla_softmax_scale(rope, wl.qk_head_dim))
+    cos, sin = mla.mla_init_rope_tables(rope, inp["max_total_len"])
+    T = n_new * batch
+    out = torch.empty((T, wl.num_heads, wl.v_head), dtype=torch.bfloat16, device=device)
+    ws = torch.empty(mla.mla_prefill_cached_workspace_size(dims, T, inp["max_total_len"]), dtype=torch.uint8,
+                     device=device)
+
+    def call():
+        mla.mla_prefill_cached(dims, d["latent"], d["q"], d["w_kvb"], d["w_norm"], d["cu_seqlens"],
+                               d["cache_offsets"], d["prefix_lens"], inp["max_total_len"], cos, sin, d["cache"],
+                               out=out, workspace=ws)
+    return call
+
+
+def _projection_call(device, n=2048, hidden=7168, q_rank=1536):
+    wl = W.KIMI
+    d = {k: v.to(device) for k, v in W.projection_inputs(wl, n, hidden, q_rank).items()}
+    rope = mla.rope_for(wl)
+    dims = mla.dims_for(wl, mla.mla_softmax_scale(rope, wl.qk_head_dim))
+    cos, sin = mla.mla_init_rope_tables(rope, n)
+    latent = torch.empty((n, wl.kv_lora_rank + wl.qk_rope), dtype=torch.bfloat16, device=device)
+    cache = torch.empty_like(latent)
+    rows = torch.arange(n, dtype=torch.int64, device=device)
+    q = torch.empty((n, wl.num_heads, wl.qk_head_dim), dtype=torch.bfloat16, device=device)
+    q_ws = torch.empty(mla.mla_q_proj_workspace_size(dims, q_rank, n), dtype=torch.uint8, device=device)
+    out = torch.empty((n, hidden), dtype=torch.bfloat16, device=device)
+
+    def call():
+        mla.mla_kv_down_append(dims, d["hidden"], d["w_kva"], latent, d["w_norm"], d["positions"], cos, sin,
+                               cache, rows)
+        mla.mla_q_proj(dims, d["hidden"], d["w_qa"], d["w_qnorm"], d["w_qb"], q, q_ws)
+        mla.mla_o_proj(dims, d["attn"], d["w_o"], out)
+    return call
+
+
 def main():
     ap = argparse.ArgumentParser()
-    ap.add_argument("--case", default="all", choices=["kimi_prefill", "glm_prefill", "decode", "all"])
+    ap.add_argument("--case", default="all",
+                    choices=["kimi_prefill", "glm_prefill", "decode", "chunk", "projections", "all"])
     ap.add_argument("--reps", type=int, default=4)
     args = ap.parse_args()
     device = torch.device("cuda", 0)
@@ -66,6 +111,10 @@ def main():
         calls.append(_prefill_call(W.GLM, device))
     if args.case in ("decode", "all"):
         calls.append(_decode_call(W.DECODE, device))
+    if args.case == "chunk":
+        calls.append(_chunk_call(device))
+    if args.case == "projections":
+        calls.append(_projection_call(device))
     times = []
     for _ in range(max(args.reps, 1)):
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
