@@ -1019,7 +1019,6 @@ int check_proj_rows(int64_t n) {
   return MLA_OK;
 }
 
-size_t elem_bytes(const mla_dims* d) { return d->dtype == MLA_FP32 ? 4 : 2; }
 }  // namespace
 
 // Device address of g_noalloc_scratch, looked up once per device (host code
@@ -1091,6 +1090,9 @@ int mla_prefill_cached(const mla_dims* dims, const void* latent, const void* q, 
   if (total_tokens > kMaxChunkTokens)
     return fail(MLA_ERR_UNSUPPORTED_SHAPE, "at most %lld chunk tokens per call", (long long)kMaxChunkTokens);
   if (max_total_len < 1) return fail(MLA_ERR_INVALID_ARG, "max_total_len must be >= 1");
+  // the decode's own limit, checked here so that nothing is written to the cache first
+  if ((max_total_len + mla::simt::kDecChunk - 1) / mla::simt::kDecChunk > 256)
+    return fail(MLA_ERR_UNSUPPORTED_SHAPE, "max_total_len must be <= %d", 256 * mla::simt::kDecChunk);
   if (max_pos < 1) return fail(MLA_ERR_INVALID_ARG, "max_pos must be >= 1");
   if (cache_num_rows < 1) return fail(MLA_ERR_INVALID_ARG, "cache_num_rows must be >= 1");
   if (!latent || !q || !w_kvb || !w_norm || !cu_seqlens || !cache_offsets || !prefix_lens || !cos_table ||
@@ -1149,7 +1151,7 @@ int mla_q_proj_workspace_size(const mla_dims* dims, int32_t q_rank, int64_t n, s
   if (rc) return rc;
   if (q_rank < 1) return fail(MLA_ERR_INVALID_ARG, "q_rank must be >= 1");
   if (!bytes) return fail(MLA_ERR_INVALID_ARG, "bytes is NULL");
-  *bytes = align_up((size_t)n * (size_t)q_rank * elem_bytes(dims), 256);
+  *bytes = align_up((size_t)n * (size_t)q_rank * elem_size(dims), 256);
   return MLA_OK;
 }
 
@@ -1163,7 +1165,7 @@ int mla_q_proj(const mla_dims* dims, int32_t hidden_size, int32_t q_rank, const 
   if (hidden_size < 1 || q_rank < 1) return fail(MLA_ERR_INVALID_ARG, "hidden_size and q_rank must be >= 1");
   if (!hidden || !w_qa || !w_qnorm || !w_qb || !q) return fail(MLA_ERR_INVALID_ARG, "a tensor pointer is NULL");
   if (n == 0) return MLA_OK;
-  const size_t need = align_up((size_t)n * (size_t)q_rank * elem_bytes(dims), 256);
+  const size_t need = align_up((size_t)n * (size_t)q_rank * elem_size(dims), 256);
   if (!workspace || workspace_bytes < need)
     return fail(MLA_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes, got %zu", need, workspace_bytes);
   // q_a = hidden W_qa^T, normalized in place, then q = q_a W_qb^T

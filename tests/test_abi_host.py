@@ -147,6 +147,7 @@ def test_prefill_cached_host_validation():
     assert call(pre=None) == 1
     assert call(cache=None) == 1
     assert call(wsb=16) == 3
+    assert call(maxlen=256 * 2048 + 1) == 2  # the decode's length limit, before anything is launched
     # the workspace holds the per-token bookkeeping plus the decode's own
     need = mla.mla_prefill_cached_workspace_size(d, 5, 100)
     assert need >= mla.mla_decode_workspace_size(d, 5, 100) + 5 * 24
