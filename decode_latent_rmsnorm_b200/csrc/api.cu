@@ -1136,6 +1136,8 @@ int mla_kv_down_append(const mla_dims* dims, int32_t hidden_size, const void* hi
   const bool append = cache != nullptr || cache_rows != nullptr;
   if (append && (!cache || !cache_rows || !w_norm || !positions || !cos_table || !sin_table))
     return fail(MLA_ERR_INVALID_ARG, "appending needs cache, cache_rows, w_norm, positions and the tables");
+  if (append && (max_pos < 1 || cache_num_rows < 1))
+    return fail(MLA_ERR_INVALID_ARG, "appending needs max_pos >= 1 and cache_num_rows >= 1");
   if (n == 0) return MLA_OK;
   rc = launch_linear(dims, hidden, w_kva, latent, n, hidden_size, dims->kv_lora_rank + dims->qk_rope, stream,
                      "kv_a_proj");

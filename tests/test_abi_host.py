@@ -175,6 +175,8 @@ def test_projection_host_validation():
     assert kv(lat=None) == 1
     assert kv(cache=FAKE) == 1                     # a cache without destination rows
     assert kv(cache=FAKE, crows=FAKE, wn=None) == 1
+    assert kv(cache=FAKE, crows=FAKE, rows=0) == 1      # checked before the Linear runs
+    assert kv(cache=FAKE, crows=FAKE, rows=10, mp=0) == 1
 
     def qp(**o):
         a = dict(hid=7168, qr=1536, x=FAKE, wa=FAKE, wn=FAKE, wb=FAKE, n=4, q=FAKE, ws=FAKE, wsb=1 << 40)
