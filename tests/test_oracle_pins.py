@@ -417,15 +417,20 @@ def _chunked_inputs(seqlens, splits, gap=3, **kw):
     return shape, rope, d, cos, sin, offs, rows
 
 
+_YARN_SMALL = O.RopeConfig(rope_dim=4, base=50000.0, yarn=True, factor=4.0, original_max_pos=8,
+                           mscale=0.9, mscale_all_dim=0.5)
+
+
+@pytest.mark.parametrize("rope", [None, _YARN_SMALL], ids=["default_rope", "yarn"])
 @pytest.mark.parametrize("interleaved", [False, True])
-def test_prefill_cached_two_chunks_equal_one_prefill(interleaved):
+def test_prefill_cached_two_chunks_equal_one_prefill(interleaved, rope):
     # Splitting each sequence into a cached prefix and a chunk changes nothing:
     # chunk 1 (empty prefix) and chunk 2 (prefix = chunk 1) together give the
     # prefill of the whole sequence. An error in the chunk's positions, its
     # cache rows or the offset of the causal mask breaks this.
     seqlens, splits = [11, 6, 17], [4, 0, 16]
     shape, rope, d, cos, sin, offs, nrows = _chunked_inputs(seqlens, splits, H=3, R=16, N=8, P=4, V=6,
-                                                            interleaved=interleaved, seed=21)
+                                                            interleaved=interleaved, seed=21, rope=rope)
     scale = 0.35
     full = O.prefill(d["latent"], d["q"], d["W"], d["w_norm"], d["positions"], d["cu"], cos, sin, shape, scale)
     cu = d["cu"]
