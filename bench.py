@@ -269,7 +269,8 @@ def job_throughput(work_per_rank: float, world: int, slowest_ms: float) -> float
 def workload_config(world, lens):
     """The config object both arms print."""
     return dict(workload="kimi_k2_prefill_bf16 + absorbed_decode_bf16",
-                prefill="B=1 T=2048 H=64 R=512 N=128 P=64 V=128 YaRN(base 5e4, factor 32)",
+                prefill="B=1 T=2048 H=64 R=512 N=128 P=64 V=128 YaRN(base 5e4, factor 32); "
+                        "kv_b_proj prepared once",
                 decode="B=64 H=64 R=512 N=128 P=64 V=128, cache lens U[1000,32768] sum=%d" % sum(lens),
                 global_batch=world * (1 + len(lens)), parallelism="replicas x%d" % world,
                 l2="flushed between steps (256 MiB write outside per-step events)")
@@ -300,8 +301,14 @@ def run_ours(args, rank, world, device):
     d_out = torch.empty((B, dwl.num_heads, dwl.v_head), dtype=torch.bfloat16, device=device)
     d_ws = torch.empty(mla.mla_decode_workspace_size(dims_d, B, max_len), dtype=torch.uint8, device=device)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+    # kv_b_proj is converted for the tensor cores once, as at model load
+    w_prep = mla.mla_prepare_kv_b_proj(dims_p, P["w_kvb"])
 
     def prefill():
+        mla.mla_prefill_prepared(dims_p, P["latent"], P["q"], w_prep, P["w_norm"], P["positions"],
+                                 P["cu_seqlens"], max(pwl.seqlens), cos, sin, out=p_out, workspace=p_ws)
+
+    def prefill_unprepared():
         mla.mla_prefill(dims_p, P["latent"], P["q"], P["w_kvb"], P["w_norm"], P["positions"],
                         P["cu_seqlens"], max(pwl.seqlens), cos, sin, out=p_out, workspace=p_ws)
 
@@ -387,12 +394,15 @@ def run_ours(args, rank, world, device):
     roof["kernel"] = top
     roof["peak_source"] = peaks["source"]
 
+    # the prefill with kv_b_proj converted inside the call (mla_prefill)
+    unprep_ms = reduce_max(time_calls(args, prefill_unprepared, flush))
     chunk = run_chunk(args, din, D, device, world, reduce_max, peaks)
     projections = run_projections(args, device, world, reduce_max, peaks)
+    configs = run_configs(args, device, world, reduce_max, peaks, flush)
 
     # end to end through the same C-ABI with pinned host buffers
     e2e = run_e2e(args, pwl, dwl, pin, din, dims_p, dims_d, cos, sin, P, D, p_ws, d_ws, device, world,
-                  reduce_max, fl, by)
+                  reduce_max, fl, by, w_prep)
 
     res = dict(
         metric=METRIC, value=p_tflops, unit="TFLOP/s", n_gpus=world, steps=args.steps,
@@ -400,11 +410,14 @@ def run_ours(args, rank, world, device):
         vs_baseline=None, dtype="bf16", data="synthetic (seeded N(0,1) inputs, N(0,1/R) kv_b_proj)",
         config=workload_config(world, lens),
         prefill=dict(ms=p_mean, tflops=p_tflops, frac_of_bf16_peak=p_tflops / (world * peaks["bf16"]),
-                     tokens_per_s=world * T / (p_mean * 1e-3), gflop=fl["total"] / 1e9),
+                     tokens_per_s=world * T / (p_mean * 1e-3), gflop=fl["total"] / 1e9,
+                     weight="kv_b_proj prepared once (mla_prepare_kv_b_proj), mla_prefill_prepared timed",
+                     unprepared=dict(call="mla_prefill (kv_b_proj converted inside every call)",
+                                     ms=unprep_ms, tflops=world * fl["total"] / (unprep_ms * 1e-3) / 1e12)),
         decode=dict(metric="absorbed decode HBM GB/s", value=d_gbs, unit="GB/s", ms=d_mean,
                     frac_of_hbm=d_gbs / (world * peaks["hbm"]), tokens_per_s=world * B / (d_mean * 1e-3),
                     tflops=world * by["flops"] / (d_mean * 1e-3) / 1e12, bytes=by["total"]),
-        kernels_ms=dict(prefill=kp_ms, decode=kd_ms), chunk=chunk, projections=projections,
+        kernels_ms=dict(prefill=kp_ms, decode=kd_ms), configs=configs, chunk=chunk, projections=projections,
         roofline=roof, e2e=e2e, gpu_launches=int(launches), clocks=clocks.summary(),
         peaks=dict(hbm_gbs=peaks["hbm"], bf16_tflops=peaks["bf16"], source=peaks["source"]),
     )
@@ -412,7 +425,7 @@ def run_ours(args, rank, world, device):
 
 
 def run_e2e(args, pwl, dwl, pin, din, dims_p, dims_d, cos, sin, P, D, p_ws, d_ws, device, world,
-            reduce_max, fl, by):
+            reduce_max, fl, by, w_prep):
     """The same calls end to end: every step copies its inputs from pinned host
     memory and reads its result back. Weights, rotary tables and the latent
     cache stay resident (model state); the step inputs are the prefill's
@@ -446,8 +459,8 @@ def run_e2e(args, pwl, dwl, pin, din, dims_p, dims_d, cos, sin, P, D, p_ws, d_ws
     def compute(kind, s):
         x, out = bufs[kind]["dev_in"][s], bufs[kind]["dev_out"][s]
         if kind == "prefill":
-            mla.mla_prefill(dims_p, x["latent"], x["q"], P["w_kvb"], P["w_norm"], x["positions"],
-                            x["cu_seqlens"], max(pwl.seqlens), cos, sin, out=out, workspace=p_ws)
+            mla.mla_prefill_prepared(dims_p, x["latent"], x["q"], w_prep, P["w_norm"], x["positions"],
+                                     x["cu_seqlens"], max(pwl.seqlens), cos, sin, out=out, workspace=p_ws)
         else:
             mla.mla_decode(dims_d, x["q"], D["cache"], x["cache_offsets"], x["cache_lens"], x["positions"],
                            max_len, D["w_kvb"], cos, sin, out=out, workspace=d_ws)
@@ -518,6 +531,69 @@ def run_e2e(args, pwl, dwl, pin, din, dims_p, dims_d, cos, sin, P, D, p_ws, d_ws
                 serial=dict(value=world * fl["total"] / (res["prefill_serial"] * 1e-3) / 1e12,
                             prefill_ms=res["prefill_serial"], decode_ms=res["decode_serial"],
                             decode_gbs=world * by["total"] / (res["decode_serial"] * 1e-3) / 1e9))
+
+
+def time_calls(args, fn, flush):
+    """Mean CUDA-event time (ms) of ``fn`` over ``args.steps`` calls after
+    ``args.warmup`` untimed ones; L2 flushed (256 MiB write) before each
+    timed call, outside its events."""
+    for _ in range(args.warmup):
+        fn()
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    for i, e in enumerate(evs):
+        flush.fill_(i & 0xff)
+        e[0].record()
+        fn()
+        e[1].record()
+    torch.cuda.synchronize()
+    mla.mla_check_device_status()
+    return statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+
+
+def run_configs(args, device, world, reduce_max, peaks, flush):
+    """Throughput of the other prefill workloads of the pages' shapes (GLM-5
+    B2 T4096 N192 V256, the packed varlen batch 1024/3000/7777/16384 with
+    Kimi-K2 heads, and the tiny fp32 case), each timed alone through the
+    C-ABI with the prepared kv_b_proj: TFLOP/s over the algorithmic FLOPs,
+    tokens/s, and the fraction of the bf16 peak (the fp32 case runs the
+    CUDA-core kernels: no tensor-core fraction)."""
+    res = {}
+    for wl in (W.GLM, W.VARLEN, W.TINY):
+        inp = W.prefill_inputs(wl)
+        d = {k: v.to(device) for k, v in inp.items()}
+        dims = mla.dims_for(wl, mla.mla_softmax_scale(mla.rope_for(wl), wl.qk_head_dim))
+        cos, sin = mla.mla_init_rope_tables(mla.rope_for(wl), W.max_position(wl))
+        T = sum(wl.seqlens)
+        out = torch.empty((T, wl.num_heads, wl.v_head), dtype=wl.torch_dtype, device=device)
+        ws = torch.empty(mla.mla_prefill_workspace_size(dims, T, len(wl.seqlens)), dtype=torch.uint8, device=device)
+        w_prep = mla.mla_prepare_kv_b_proj(dims, d["w_kvb"])
+
+        def call():
+            mla.mla_prefill_prepared(dims, d["latent"], d["q"], w_prep, d["w_norm"], d["positions"],
+                                     d["cu_seqlens"], max(wl.seqlens), cos, sin, out=out, workspace=ws)
+
+        ms = reduce_max(time_calls(args, call, flush))
+        kev = mla.KernelEvents(16)
+        flush.fill_(7)
+        with kev:
+            call()
+        torch.cuda.synchronize()
+        fl = prefill_flops(wl)
+        tf = world * fl["total"] / (ms * 1e-3) / 1e12
+        r = dict(shape="H=%d R=%d N=%d P=%d V=%d seqlens=%s %s" % (wl.num_heads, wl.kv_lora_rank, wl.qk_nope,
+                                                                  wl.qk_rope, wl.v_head, list(wl.seqlens),
+                                                                  wl.dtype),
+                 ms=ms, tflops=tf, tokens_per_s=world * T / (ms * 1e-3), gflop=fl["total"] / 1e9,
+                 dispatch=mla.mla_last_dispatch(), kernels_ms=dict(zip(kev.names, kev.durations_ms())))
+        if wl.dtype == "bf16":
+            r["frac_of_bf16_peak"] = tf / (world * peaks["bf16"])
+            att = [t for n, t in r["kernels_ms"].items() if "attention" in n]
+            if att:
+                r["attention_tflops"] = fl["attn"] / (att[0] * 1e-3) / 1e12
+        res[wl.name] = r
+        del d, out, ws, w_prep
+        torch.cuda.empty_cache()
+    return res
 
 
 def run_chunk(args, din, D, device, world, reduce_max, peaks, n_new=4):
@@ -593,10 +669,12 @@ def run_projections(args, device, world, reduce_max, peaks, n=2048, hidden=7168,
     rows = torch.arange(n, dtype=torch.int64, device=device)
     q = torch.empty((n, H, N + P), dtype=torch.bfloat16, device=device)
     q_ws = torch.empty(mla.mla_q_proj_workspace_size(dims, q_rank, n), dtype=torch.uint8, device=device)
+    kv_ws = torch.empty(mla.mla_kv_down_append_workspace_size(dims, n), dtype=torch.uint8, device=device)
     out = torch.empty((n, hidden), dtype=torch.bfloat16, device=device)
     calls = dict(
         kv_a_proj_and_append=(lambda: mla.mla_kv_down_append(dims, d["hidden"], d["w_kva"], latent, d["w_norm"],
-                                                             d["positions"], cos, sin, cache, rows),
+                                                             d["positions"], cos, sin, cache, rows,
+                                                             workspace=kv_ws),
                               2.0 * n * hidden * (R + P)),
         q_proj=(lambda: mla.mla_q_proj(dims, d["hidden"], d["w_qa"], d["w_qnorm"], d["w_qb"], q, q_ws),
                 2.0 * n * hidden * q_rank + 2.0 * n * q_rank * H * (N + P)),
@@ -627,25 +705,68 @@ def cpu_baseline(budget_s=15.0):
     return dict(value=v, unit="TFLOP/s", cores=threads, kind="oracle", sample=sample)
 
 
+def oracle_decode_sample(wl, din, budget_s: float):
+    """Time the fp64 absorbed-decode oracle on whole sequences of the decode
+    workload until ``budget_s`` is spent; returns (GB/s of algorithmic bytes,
+    sample text, seconds spent)."""
+    import oracle as O
+    rope = O.RopeConfig(**wl.rope)
+    shape = O.MlaShape(wl.num_heads, wl.kv_lora_rank, wl.qk_nope, wl.qk_rope, wl.v_head,
+                       eps=wl.eps, interleaved=wl.interleaved)
+    scale = O.softmax_scale(rope, shape.qk_head_dim)
+    cos, sin = O.rope_tables(rope, W.max_position(wl))
+    q = din["q"].double().numpy()
+    w = din["w_kvb"].double().numpy()
+    lens = [int(x) for x in din["cache_lens"]]
+    offs = [int(x) for x in din["cache_offsets"]]
+    done, t_spent, rows = 0, 0.0, 0
+    for b in range(len(lens)):
+        if t_spent >= budget_s:
+            break
+        rows_b = din["cache"][offs[b]:offs[b] + lens[b]].double().numpy()
+        t0 = time.perf_counter()
+        O.decode_absorbed(q[b:b + 1], rows_b, [0], [lens[b]], din["positions"][b:b + 1].numpy(), w, cos, sin,
+                          shape, scale)
+        t_spent += time.perf_counter() - t0
+        done += 1
+        rows += lens[b]
+    by = decode_bytes(wl, lens[:done])
+    return by["total"] / t_spent / 1e9, "%s: %d of %d sequences (%d cache rows, %.1f s)" % (
+        wl.name, done, len(lens), rows, t_spent), t_spent
+
+
 def run_reference(args, rank, world):
-    """The reference arm: the fp64 oracle as it stands, on host cores."""
+    """The reference arm: the fp64 oracle as it stands, on host cores. Each
+    step times a bounded sample of the same two workloads: whole heads of the
+    Kimi-K2 prefill (about 2 s) and whole sequences of the absorbed decode
+    (about 1 s). ``value`` is the prefill's TFLOP/s (the headline metric), the
+    ``decode`` object its GB/s, and ``ms_per_step`` the wall time of the
+    sample one step runs (not an extrapolation to the full workload)."""
     if rank != 0:
         return None
     pin = W.prefill_inputs(W.KIMI)
-    vals = []
-    sample = ""
+    din = W.decode_inputs(W.DECODE)
+    vals, dvals, step_s = [], [], []
+    sample = dsample = ""
     threads = 1
     for i in range(args.warmup + args.steps):
-        v, sample, threads = oracle_prefill_sample(W.KIMI, pin, budget_s=3.0)
+        t0 = time.perf_counter()
+        v, sample, threads = oracle_prefill_sample(W.KIMI, pin, budget_s=2.0)
+        dv, dsample, _ = oracle_decode_sample(W.DECODE, din, budget_s=1.0)
         if i >= args.warmup:
             vals.append(v)
+            dvals.append(dv)
+            step_s.append(time.perf_counter() - t0)
     v = statistics.mean(vals)
-    fl = prefill_flops(W.KIMI)["total"]
     return dict(metric=METRIC, value=v, unit="TFLOP/s", n_gpus=world, steps=args.steps, warmup=args.warmup,
-                ms_per_step=fl / (v * 1e12) * 1e3, higher_is_better=True, scaling="weak", vs_baseline=None,
-                dtype="f64", data="synthetic", impl="reference",
+                ms_per_step=statistics.mean(step_s) * 1e3, higher_is_better=True, scaling="weak",
+                vs_baseline=None, dtype="f64", data="synthetic", impl="reference",
                 config=workload_config(world, [int(x) for x in W.decode_cache_lens(W.DECODE)]),
-                cpu_baseline=dict(kind="oracle", cores=threads, sample=sample, value=v, unit="TFLOP/s"),
+                step="a bounded sample of each workload per step: " + sample + "; " + dsample,
+                decode=dict(metric="absorbed decode HBM GB/s (algorithmic bytes)", value=statistics.mean(dvals),
+                            unit="GB/s"),
+                cpu_baseline=dict(kind="oracle", cores=threads, sample=sample + "; " + dsample, value=v,
+                                  unit="TFLOP/s"),
                 e2e=dict(value=v, unit="TFLOP/s", h2d_bytes_per_step=0, d2h_bytes_per_step=0))
 
 

@@ -7,7 +7,6 @@
 #include <string.h>
 
 #include <atomic>
-#include <mutex>
 
 #include "mla.h"
 #include "common.cuh"
@@ -19,7 +18,9 @@
 #include "tc_attention_pair.cuh"
 #include "tc_decode.cuh"
 #include "chunk.cuh"
+#include "tc_chunk.cuh"
 #include "proj.cuh"
+#include "selftest.cuh"
 
 #include <cudaTypedefs.h>
 
@@ -30,6 +31,10 @@ static __device__ __align__(256) uint8_t g_noalloc_scratch[MLA_NOALLOC_SCRATCH_B
 namespace {
 
 thread_local char g_err[1024] = "no error";
+// Which kernels the last prefill / decode call of this thread ran, and why
+// (mla_last_dispatch).
+thread_local const char* g_dispatch = "none";
+void set_dispatch(const char* what) { g_dispatch = what; }
 
 int fail(int code, const char* fmt, ...) {
   va_list ap;
@@ -187,7 +192,7 @@ bool prefill_tc_shape(const mla_dims* d) {
 struct PrefillWs {
   int64_t cap, Tpad;
   int gemm_tiles_per_cta, gemm_gy;
-  size_t seq_tile0, tile_seq, tile_q0, order, pair_order, w16, c16;
+  size_t seq_tile0, tile_seq, tile_q0, order, pair_order, item_counter, w16, c16;
   size_t k_nope, vals, k_rot, total;
 };
 PrefillWs prefill_ws_layout(const mla_dims* d, int64_t T, int nseq, bool tc) {
@@ -210,6 +215,7 @@ PrefillWs prefill_ws_layout(const mla_dims* d, int64_t T, int nseq, bool tc) {
     w.tile_q0 = off;   off = align_up(off + 4 * (size_t)w.cap, 256);
     w.order = off;     off = align_up(off + 4 * (size_t)w.cap, 256);
     w.pair_order = off; off = align_up(off + 4 * (size_t)w.cap, 256);
+    w.item_counter = off; off = align_up(off + 4, 256);
     w.w16 = off;       off = align_up(off + 2 * (size_t)NOUT * d->kv_lora_rank, 256);
     w.c16 = off;       off = align_up(off + 2 * (size_t)T * d->kv_lora_rank, 256);   // normalized latent, fp16
   } else {
@@ -394,7 +400,9 @@ int launch_attention_pair(int N, int V, unsigned grid, const CUtensorMap& mq, co
 
 // Tensor-core prefill: tile schedule -> fused RMSNorm + kv_b_proj (tcgen05)
 // -> causal attention over the padded layout.
-int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, const void* w_kvb,
+// w_f16: the fp16 copy of w_kvb made by mla_prepare_kv_b_proj, or NULL to make
+// it here (in the workspace) on every call.
+int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, const void* w_kvb, const void* w_f16,
                       const void* w_norm, const int32_t* positions, const int32_t* cu_seqlens, int num_seqs,
                       int max_seqlen, int64_t T_tot, const float* cos_t, const float* sin_t, int max_pos,
                       void* out, void* workspace, cudaStream_t st) {
@@ -407,6 +415,7 @@ int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, cons
   int32_t* tile_q0 = reinterpret_cast<int32_t*>(ws + L.tile_q0);
   int32_t* order = reinterpret_cast<int32_t*>(ws + L.order);
   int32_t* pair_order = reinterpret_cast<int32_t*>(ws + L.pair_order);
+  int32_t* item_counter = reinterpret_cast<int32_t*>(ws + L.item_counter);
   __half* k_nope = reinterpret_cast<__half*>(ws + L.k_nope);
   __half* vt = reinterpret_cast<__half*>(ws + L.vals);
   __half* k_rot = reinterpret_cast<__half*>(ws + L.k_rot);
@@ -428,7 +437,8 @@ int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, cons
     const uint64_t dims[2] = {(uint64_t)R, (uint64_t)NOUT};
     const uint64_t strides[1] = {(uint64_t)R * 2};
     const uint32_t box[2] = {64, vt_gemm ? (uint32_t)(N + V) : 256u};
-    int rc = make_map(&map_w, ws + L.w16, 2, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+    int rc = make_map(&map_w, w_f16 ? w_f16 : (const void*)(ws + L.w16), 2, dims, strides, box,
+                      CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
     if (rc) return rc;
   }
 
@@ -438,13 +448,13 @@ int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, cons
   __half* c16 = reinterpret_cast<__half*>(ws + L.c16);
   const int64_t n8 = (int64_t)NOUT * R / 8;
   const int64_t per_block = (int64_t)mla::tc::kPrepThreads * mla::tc::kPrepUnroll;
-  const int w_blocks = (int)((n8 + per_block - 1) / per_block);
+  const int w_blocks = w_f16 ? 0 : (int)((n8 + per_block - 1) / per_block);
   // the transposed-value GEMM reads c_hat prepared here: one warp per token row
   const int norm_blocks = vt_gemm ? (int)((T_tot + mla::tc::kPrepThreads / 32 - 1) / (mla::tc::kPrepThreads / 32)) : 0;
   prof_begin(st, "tc_prep");
   mla::tc::prefill_prep_kernel<<<(unsigned)(1 + w_blocks + norm_blocks), mla::tc::kPrepThreads, 0, st>>>(
       cu_seqlens, num_seqs, T_tot, max_seqlen, cap, seq_tile0, tile_seq, tile_q0, order, pair_order,
-      static_cast<const bf16*>(w_kvb), w16, n8, w_blocks, static_cast<const bf16*>(latent),
+      item_counter, static_cast<const bf16*>(w_kvb), w16, n8, w_blocks, static_cast<const bf16*>(latent),
       static_cast<const bf16*>(w_norm), R, d->eps, c16);
   prof_end(st);
   CUtensorMap map_c16;   // the transposed-value GEMM's A operand: c_hat fp16 [Ttot, R]
@@ -456,7 +466,7 @@ int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, cons
     if (rc) return rc;
   }
 
-  mla::tc::GemmParams gp;
+  mla::tc::GemmParams gp{};
   gp.latent = static_cast<const bf16*>(latent);
   gp.w_norm = static_cast<const bf16*>(w_norm);
   gp.positions = positions;
@@ -549,17 +559,23 @@ int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, cons
   ap.cos_t = cos_t;
   ap.sin_t = sin_t;
   ap.out = static_cast<bf16*>(out);
+  ap.item_counter = item_counter;
+  ap.q_off = nullptr;
+  ap.n_blocks = cap;
   ap.H = H;
   ap.Tpad = (int)L.Tpad;
   ap.max_pos = max_pos;
   ap.interleaved = d->rope_interleaved;
   ap.scale_log2 = d->softmax_scale * 1.4426950408889634f;
   if (pair) {
-    // blocks of two tiles: sum over sequences of ceil(tiles / 2) <= (tiles + nseq) / 2
+    // persistent grid: one CTA per SM, at most one per work item (blocks of
+    // two tiles: sum over sequences of ceil(tiles / 2) <= (tiles + nseq) / 2)
     const int64_t tiles_ub = (T_tot + 127) / 128 + num_seqs;
     int64_t blocks = (tiles_ub + num_seqs) / 2;
     if (blocks > L.cap) blocks = L.cap;
-    return launch_attention_pair(N, V, (unsigned)(blocks * H), map_q, map_kn, map_kr, map_vt, ap, st);
+    int64_t grid = blocks * H;
+    if (grid > num_sms()) grid = num_sms();
+    return launch_attention_pair(N, V, (unsigned)grid, map_q, map_kn, map_kr, map_vt, ap, st);
   }
   const unsigned grid = (unsigned)(cap * H);
   return launch_attention_tc(N, V, grid, map_q, map_kn, map_kr, map_vt, ap, st);
@@ -667,7 +683,7 @@ int launch_decode_tc(const mla_dims* d, const void* q, const void* cache, int64_
   e = cudaFuncSetAttribute(T::head_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)T::kHgSmem);
   if (e != cudaSuccess) return cuda_status(e, "head gemm smem attribute");
   {
-    T::HgParams hp;
+    T::HgParams hp{};
     hp.out = qf;
     hp.out_bs = (int64_t)H * (R + P);
     hp.out_hs = R + P;
@@ -723,7 +739,7 @@ int launch_decode_tc(const mla_dims* d, const void* q, const void* cache, int64_
 
   // out[b, h, :] = W_UV_h o_lat[b, h, :]   (W_UV_h = rows N .. N+V-1 of head h: [V, R], R contiguous)
   {
-    T::HgParams hp;
+    T::HgParams hp{};
     hp.out = static_cast<bf16*>(out);
     hp.out_bs = (int64_t)H * V;
     hp.out_hs = V;
@@ -769,6 +785,8 @@ int mla_recorded_kernel_events(int32_t* recorded) {
 }
 
 const char* mla_last_error_string(void) { return g_err; }
+
+const char* mla_last_dispatch(void) { return g_dispatch; }
 
 int mla_softmax_scale(const mla_rope_cfg* rope, int32_t qk_head_dim, float* scale_out) {
   int rc = check_rope(rope);
@@ -827,11 +845,22 @@ int mla_prefill_workspace_size(const mla_dims* dims, int64_t total_tokens, int32
   return MLA_OK;
 }
 
-int mla_prefill(const mla_dims* dims, const void* latent, const void* q, const void* w_kvb,
-                const void* w_norm, const int32_t* positions, const int32_t* cu_seqlens,
-                int32_t num_seqs, int32_t max_seqlen, int64_t total_tokens, const float* cos_table,
-                const float* sin_table, int32_t max_pos, void* out, void* workspace,
-                size_t workspace_bytes, cudaStream_t stream) {
+}  // extern "C"
+
+namespace {
+// Bytes of the prepared kv_b_proj copy: fp16 for the tensor-core prefill's
+// head shapes, otherwise the weight itself in the run dtype.
+size_t prepared_bytes(const mla_dims* d) {
+  const size_t n = (size_t)d->num_heads * (d->qk_nope + d->v_head) * d->kv_lora_rank;
+  return prefill_tc_shape(d) ? 2 * n : elem_size(d) * n;
+}
+
+// mla_prefill (prepared false: w is kv_b_proj, converted on every call) and
+// mla_prefill_prepared (prepared true: w comes from mla_prepare_kv_b_proj).
+int prefill_entry(const mla_dims* dims, const void* latent, const void* q, const void* w, bool prepared,
+                  const void* w_norm, const int32_t* positions, const int32_t* cu_seqlens, int32_t num_seqs,
+                  int32_t max_seqlen, int64_t total_tokens, const float* cos_table, const float* sin_table,
+                  int32_t max_pos, void* out, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   int rc = check_dims(dims);
   if (rc) return rc;
   if (num_seqs < 0 || total_tokens < 0 || max_seqlen < 0 || max_pos < 1)
@@ -841,22 +870,89 @@ int mla_prefill(const mla_dims* dims, const void* latent, const void* q, const v
   if (max_seqlen > total_tokens) return fail(MLA_ERR_INVALID_ARG, "max_seqlen exceeds total_tokens");
   if (!cu_seqlens) return fail(MLA_ERR_INVALID_ARG, "cu_seqlens is NULL");
   if (total_tokens == 0 || num_seqs == 0 || max_seqlen == 0) return MLA_OK;   // nothing to attend
-  if (!latent || !q || !w_kvb || !w_norm || !positions || !cos_table || !sin_table || !out)
+  if (!latent || !q || !w || !w_norm || !positions || !cos_table || !sin_table || !out)
     return fail(MLA_ERR_INVALID_ARG, "a tensor pointer is NULL");
   const size_t need = prefill_ws_bytes(dims, total_tokens, num_seqs);
   if (!workspace || workspace_bytes < need)
     return fail(MLA_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes, got %zu", need, workspace_bytes);
-  if (prefill_tc_shape(dims) && aligned16(latent) && aligned16(w_kvb) && aligned16(q) && aligned16(workspace) &&
-      aligned16(w_norm))
-    return launch_prefill_tc(dims, latent, q, w_kvb, w_norm, positions, cu_seqlens, num_seqs, max_seqlen,
-                             total_tokens, cos_table, sin_table, max_pos, out, workspace, stream);
+  const bool aligned = aligned16(latent) && aligned16(q) && aligned16(workspace) && aligned16(w_norm) &&
+                       aligned16(w);
+  if (prefill_tc_shape(dims)) {
+    if (aligned) {
+      set_dispatch("tensor-core");
+      return launch_prefill_tc(dims, latent, q, prepared ? nullptr : w, prepared ? w : nullptr, w_norm, positions,
+                               cu_seqlens, num_seqs, max_seqlen, total_tokens, cos_table, sin_table, max_pos, out,
+                               workspace, stream);
+    }
+    if (prepared)
+      return fail(MLA_ERR_INVALID_ARG, "mla_prefill_prepared needs 16-byte aligned tensors and workspace");
+    set_dispatch("simt: a tensor or the workspace is not 16-byte aligned");
+  } else {
+    set_dispatch("simt: head shape or dtype outside the tensor-core kernels");
+  }
+  // (the prepared copy of a shape outside the tensor-core kernels is the weight itself)
   if (dims->dtype == MLA_FP32)
-    return launch_prefill<float>(dims, latent, q, w_kvb, w_norm, positions, cu_seqlens, num_seqs,
+    return launch_prefill<float>(dims, latent, q, w, w_norm, positions, cu_seqlens, num_seqs,
                                  max_seqlen, total_tokens, cos_table, sin_table, max_pos, out, workspace,
                                  stream);
-  return launch_prefill<__nv_bfloat16>(dims, latent, q, w_kvb, w_norm, positions, cu_seqlens, num_seqs,
+  return launch_prefill<__nv_bfloat16>(dims, latent, q, w, w_norm, positions, cu_seqlens, num_seqs,
                                        max_seqlen, total_tokens, cos_table, sin_table, max_pos, out,
                                        workspace, stream);
+}
+}  // namespace
+
+extern "C" {
+
+int mla_prefill(const mla_dims* dims, const void* latent, const void* q, const void* w_kvb,
+                const void* w_norm, const int32_t* positions, const int32_t* cu_seqlens,
+                int32_t num_seqs, int32_t max_seqlen, int64_t total_tokens, const float* cos_table,
+                const float* sin_table, int32_t max_pos, void* out, void* workspace,
+                size_t workspace_bytes, cudaStream_t stream) {
+  return prefill_entry(dims, latent, q, w_kvb, false, w_norm, positions, cu_seqlens, num_seqs, max_seqlen,
+                       total_tokens, cos_table, sin_table, max_pos, out, workspace, workspace_bytes, stream);
+}
+
+int mla_kv_b_proj_prepared_size(const mla_dims* dims, size_t* bytes) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (!bytes) return fail(MLA_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = prepared_bytes(dims);
+  return MLA_OK;
+}
+
+int mla_prepare_kv_b_proj(const mla_dims* dims, const void* w_kvb, void* prepared, size_t prepared_bytes_given,
+                          cudaStream_t stream) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (!w_kvb || !prepared) return fail(MLA_ERR_INVALID_ARG, "a tensor pointer is NULL");
+  const size_t need = prepared_bytes(dims);
+  if (prepared_bytes_given < need)
+    return fail(MLA_ERR_WORKSPACE_TOO_SMALL, "the prepared weight needs %zu bytes, got %zu", need,
+                prepared_bytes_given);
+  if (!prefill_tc_shape(dims)) {
+    prof_begin(stream, "prepare_kv_b_proj_copy");
+    cudaError_t e = cudaMemcpyAsync(prepared, w_kvb, need, cudaMemcpyDeviceToDevice, stream);
+    prof_end(stream);
+    return cuda_status(e, "prepared weight copy");
+  }
+  if (!aligned16(w_kvb) || !aligned16(prepared))
+    return fail(MLA_ERR_INVALID_ARG, "w_kvb and the prepared buffer must be 16-byte aligned");
+  const int64_t n8 = (int64_t)dims->num_heads * (dims->qk_nope + dims->v_head) * dims->kv_lora_rank / 8;
+  const int64_t per_block = (int64_t)mla::tc::kPrepThreads * mla::tc::kPrepUnroll;
+  prof_begin(stream, "prepare_kv_b_proj");
+  mla::tc::weight_f16_kernel<<<(unsigned)((n8 + per_block - 1) / per_block), mla::tc::kPrepThreads, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(w_kvb), static_cast<__half*>(prepared), n8);
+  prof_end(stream);
+  return cuda_status(cudaGetLastError(), "prepare kv_b_proj launch");
+}
+
+int mla_prefill_prepared(const mla_dims* dims, const void* latent, const void* q, const void* w_prepared,
+                         const void* w_norm, const int32_t* positions, const int32_t* cu_seqlens,
+                         int32_t num_seqs, int32_t max_seqlen, int64_t total_tokens, const float* cos_table,
+                         const float* sin_table, int32_t max_pos, void* out, void* workspace,
+                         size_t workspace_bytes, cudaStream_t stream) {
+  return prefill_entry(dims, latent, q, w_prepared, true, w_norm, positions, cu_seqlens, num_seqs, max_seqlen,
+                       total_tokens, cos_table, sin_table, max_pos, out, workspace, workspace_bytes, stream);
 }
 
 int mla_decode_workspace_size(const mla_dims* dims, int32_t batch, int32_t max_cache_len, size_t* bytes) {
@@ -891,6 +987,10 @@ int mla_decode(const mla_dims* dims, const void* q, const void* cache, int64_t c
   const size_t need = decode_ws_bytes(dims, batch, max_cache_len);
   if (!workspace || workspace_bytes < need)
     return fail(MLA_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes, got %zu", need, workspace_bytes);
+  if (!decode_tc_shape(dims)) set_dispatch("simt: head shape or dtype outside the tensor-core decode");
+  else if (cache_num_rows >= ((int64_t)1 << 31)) set_dispatch("simt: more than 2^31 cache rows");
+  else if (!aligned16(cache) || !aligned16(workspace)) set_dispatch("simt: cache or workspace not 16-byte aligned");
+  else set_dispatch("tensor-core");
   if (decode_tc_shape(dims) && cache_num_rows < ((int64_t)1 << 31) && aligned16(cache) && aligned16(workspace))
     return launch_decode_tc(dims, q, cache, cache_num_rows, cache_offsets, cache_lens, positions, batch, max_cache_len,
                             w_kvb, cos_table, sin_table, max_pos, out, workspace, stream);
@@ -952,6 +1052,53 @@ ChunkWs chunk_ws_layout(const mla_dims* d, int64_t n, int max_total_len) {
   return L;
 }
 constexpr int64_t kMaxChunkTokens = 65535;   // the decode's batch limit
+
+// ---- eager form of the chunk call ---------------------------------------------
+// Head shapes it takes: those of the transposed-value GEMM and the two-tile
+// attention (bf16, qk_rope 64, v_head 128, qk_nope 64 or 128, rank a multiple
+// of 64 up to 512).
+bool chunk_eager_shape(const mla_dims* d) {
+  return d->dtype == MLA_BF16 && d->qk_rope == 64 && d->v_head == 128 && (d->qk_nope == 64 || d->qk_nope == 128) &&
+         d->kv_lora_rank % 64 == 0 && d->kv_lora_rank <= 512;
+}
+// Average chunk length from which the eager form runs (when the workspace
+// holds it): below it every chunk token reading its prefix as one absorbed
+// decode row costs less than expanding the prefix's keys and values.
+constexpr int64_t kChunkEagerMinAvg = 128;
+
+struct ChunkEagerWs {
+  int64_t kcap, qcap, Kpad;
+  size_t positions, rows, offsets, lens, seq_ok, kseq_tile0, ktile_seq, ktile_k0, qblk_seq, qblk_q0, qorder,
+      counter, w16, c16, k_nope, vt, k_rot, total;
+};
+ChunkEagerWs chunk_eager_ws_layout(const mla_dims* d, int64_t n, int nseq, int max_total_len) {
+  auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
+  ChunkEagerWs L{};
+  L.kcap = (int64_t)nseq * ((max_total_len + 127) / 128);
+  L.qcap = n / 256 + nseq;
+  L.Kpad = L.kcap * 128;
+  const size_t H = d->num_heads, R = d->kv_lora_rank, N = d->qk_nope, V = d->v_head;
+  size_t o = 0;
+  L.positions = o;  o = up(o + (size_t)n * 4);
+  L.rows = o;       o = up(o + (size_t)n * 8);
+  L.offsets = o;    o = up(o + (size_t)n * 8);
+  L.lens = o;       o = up(o + (size_t)n * 4);
+  L.seq_ok = o;     o = up(o + (size_t)nseq * 4);
+  L.kseq_tile0 = o; o = up(o + (size_t)(nseq + 1) * 4);
+  L.ktile_seq = o;  o = up(o + (size_t)L.kcap * 4);
+  L.ktile_k0 = o;   o = up(o + (size_t)L.kcap * 4);
+  L.qblk_seq = o;   o = up(o + (size_t)L.qcap * 4);
+  L.qblk_q0 = o;    o = up(o + (size_t)L.qcap * 4);
+  L.qorder = o;     o = up(o + (size_t)L.qcap * 4);
+  L.counter = o;    o = up(o + 4);
+  L.w16 = o;        o = up(o + 2 * H * (N + V) * R);
+  L.c16 = o;        o = up(o + 2 * (size_t)L.Kpad * R);
+  L.k_nope = o;     o = up(o + 2 * H * (size_t)L.Kpad * N);
+  L.vt = o;         o = up(o + 2 * H * V * (size_t)L.Kpad);
+  L.k_rot = o;      o = up(o + 2 * (size_t)L.Kpad * 64);
+  L.total = o;
+  return L;
+}
 }  // namespace
 
 // ---- projections on either side of the path ----------------------------------
@@ -959,33 +1106,41 @@ namespace {
 constexpr int64_t kMaxProjRows = (int64_t)1 << 20;   // grid limits of the Linear kernels
 
 // out[t, j] = sum_k x[t, k] w[j, k] for x [n, K], w [Nout, K], out [n, Nout]
-// (row-major). bf16 with K a multiple of 64 and 16-byte aligned operands:
-// tcgen05 (head_gemm_kernel with one head, M = 128 output features x N = 64
-// rows per CTA); otherwise the CUDA-core Linear.
+// (row-major). x and w are in the run dtype, or both fp16 when `f16_operands`;
+// out in the run dtype, or fp32 into out_f32 when that is set. bf16 / fp16 with
+// K a multiple of 64 and 16-byte aligned operands: tcgen05 (head_gemm_kernel
+// with one head, M = 128 output features x N = 64 rows per CTA); otherwise the
+// CUDA-core Linear.
+bool linear_tc(const mla_dims* d, const void* x, const void* w, int K) {
+  return d->dtype == MLA_BF16 && K % 64 == 0 && aligned16(x) && aligned16(w);
+}
+
 int launch_linear(const mla_dims* d, const void* x, const void* w, void* out, int64_t n, int K, int Nout,
-                  cudaStream_t st, const char* name) {
+                  cudaStream_t st, const char* name, float* out_f32 = nullptr, bool f16_operands = false) {
   namespace T = mla::tc;
-  if (d->dtype == MLA_BF16 && K % 64 == 0 && aligned16(x) && aligned16(w)) {
+  if (linear_tc(d, x, w, K)) {
+    const CUtensorMapDataType dt = f16_operands ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
     CUtensorMap map_w, map_x;
     {
       const uint64_t dims[2] = {(uint64_t)K, (uint64_t)Nout};
       const uint64_t strides[1] = {(uint64_t)K * 2};
       const uint32_t box[2] = {64, 128};
-      int rc = make_map(&map_w, w, 2, dims, strides, box);
+      int rc = make_map(&map_w, w, 2, dims, strides, box, dt);
       if (rc) return rc;
     }
     {
       const uint64_t dims[3] = {(uint64_t)K, 1, (uint64_t)n};
       const uint64_t strides[2] = {(uint64_t)K * 2, (uint64_t)K * 2};
       const uint32_t box[3] = {64, 1, 64};
-      int rc = make_map(&map_x, x, 3, dims, strides, box);
+      int rc = make_map(&map_x, x, 3, dims, strides, box, dt);
       if (rc) return rc;
     }
-    cudaError_t e = cudaFuncSetAttribute(T::head_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)T::kHgSmem);
+    auto kern = f16_operands ? T::head_gemm_kernel<false, true> : T::head_gemm_kernel<false, false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)T::kHgSmem);
     if (e != cudaSuccess) return cuda_status(e, "linear smem attribute");
     T::HgParams hp{};
     hp.out = static_cast<__nv_bfloat16*>(out);
+    hp.out_f32 = out_f32;
     hp.out_bs = Nout;
     hp.out_hs = 0;
     hp.B = (int)n;
@@ -994,23 +1149,63 @@ int launch_linear(const mla_dims* d, const void* x, const void* w, void* out, in
     hp.a_row0 = 0;
     hp.a_hstride = 0;
     prof_begin(st, name);
-    T::head_gemm_kernel<false><<<dim3(1, (unsigned)((Nout + 127) / 128), (unsigned)((n + 63) / 64)), 192,
-                                 T::kHgSmem, st>>>(map_w, map_x, hp);
+    kern<<<dim3(1, (unsigned)((Nout + 127) / 128), (unsigned)((n + 63) / 64)), 192, T::kHgSmem, st>>>(map_w, map_x,
+                                                                                                       hp);
     prof_end(st);
     return cuda_status(cudaGetLastError(), name);
   }
   const dim3 grid((unsigned)((Nout + mla::kLinTile - 1) / mla::kLinTile),
                   (unsigned)((n + mla::kLinTile - 1) / mla::kLinTile));
+  using bf16 = __nv_bfloat16;
   prof_begin(st, name);
   if (d->dtype == MLA_FP32)
     mla::simt_linear_kernel<float><<<grid, mla::kLinTile * mla::kLinTile, 0, st>>>(
         static_cast<const float*>(x), static_cast<const float*>(w), static_cast<float*>(out), n, K, Nout);
+  else if (out_f32)
+    mla::simt_linear_kernel<bf16, bf16, float><<<grid, mla::kLinTile * mla::kLinTile, 0, st>>>(
+        static_cast<const bf16*>(x), static_cast<const bf16*>(w), out_f32, n, K, Nout);
   else
-    mla::simt_linear_kernel<__nv_bfloat16><<<grid, mla::kLinTile * mla::kLinTile, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(w),
-        static_cast<__nv_bfloat16*>(out), n, K, Nout);
+    mla::simt_linear_kernel<bf16><<<grid, mla::kLinTile * mla::kLinTile, 0, st>>>(
+        static_cast<const bf16*>(x), static_cast<const bf16*>(w), static_cast<bf16*>(out), n, K, Nout);
   prof_end(st);
   return cuda_status(cudaGetLastError(), name);
+}
+
+// A CUDA-core Linear whose x is fp32 (the normalized q_a of a bf16 run whose
+// q_b_proj cannot take the tensor cores) and whose w and out are bf16.
+int launch_linear_f32x(const float* x, const void* w, void* out, int64_t n, int K, int Nout, cudaStream_t st,
+                       const char* name) {
+  using bf16 = __nv_bfloat16;
+  const dim3 grid((unsigned)((Nout + mla::kLinTile - 1) / mla::kLinTile),
+                  (unsigned)((n + mla::kLinTile - 1) / mla::kLinTile));
+  prof_begin(st, name);
+  mla::simt_linear_kernel<float, bf16, bf16><<<grid, mla::kLinTile * mla::kLinTile, 0, st>>>(
+      x, static_cast<const bf16*>(w), static_cast<bf16*>(out), n, K, Nout);
+  prof_end(st);
+  return cuda_status(cudaGetLastError(), name);
+}
+
+// Workspace of mla_kv_down_append: the fp32 result of the Linear (bf16 runs).
+size_t kv_down_ws_bytes(const mla_dims* d, int64_t n) {
+  return d->dtype == MLA_BF16 ? align_up((size_t)n * (d->kv_lora_rank + d->qk_rope) * 4, 256) : 0;
+}
+
+// Workspace of mla_q_proj. fp32 runs: q_a [n, q_rank] fp32, normalized in
+// place. bf16 runs: q_a [n, q_rank] fp32, its normalized copy [n, q_rank] (fp16
+// for the tensor-core q_b_proj), and the fp16 copy of w_qb.
+struct QProjWs {
+  size_t q_a, q_an, w16, total;
+};
+QProjWs q_proj_ws_layout(const mla_dims* d, int32_t q_rank, int64_t n) {
+  QProjWs L{};
+  size_t off = 0;
+  L.q_a = off; off = align_up(off + (size_t)n * q_rank * 4, 256);
+  if (d->dtype == MLA_BF16) {
+    L.q_an = off; off = align_up(off + (size_t)n * q_rank * 4, 256);   // fp16 (tensor cores) or fp32 (CUDA cores)
+    L.w16 = off;  off = align_up(off + (size_t)d->num_heads * (d->qk_nope + d->qk_rope) * q_rank * 2, 256);
+  }
+  L.total = off;
+  return L;
 }
 
 int check_proj_rows(int64_t n) {
@@ -1021,26 +1216,17 @@ int check_proj_rows(int64_t n) {
 
 }  // namespace
 
-// Device address of g_noalloc_scratch, looked up once per device (host code
-// cannot use the array's name as a device address).
+// Device address of g_noalloc_scratch on the current device. Host code cannot
+// use the array's name as a device address, so every call looks the address
+// up (a host-side lookup, no stream operation): after a device reset or in a
+// new context the array lives at a new address, and a kept pointer would be
+// stale. The first lookup on a device may load the library's device code.
 namespace {
-constexpr int kMaxDevices = 64;
-std::mutex g_noalloc_mu;
-void* g_noalloc_ptr[kMaxDevices] = {};
-
 int noalloc_scratch(void** ptr) {
-  int dev = 0;
-  cudaError_t e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return cuda_status(e, "cudaGetDevice");
-  if (dev < 0 || dev >= kMaxDevices) return fail(MLA_ERR_UNSUPPORTED_SHAPE, "device index %d too large", dev);
-  std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (!g_noalloc_ptr[dev]) {
-    void* p = nullptr;
-    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
-    if (e != cudaSuccess) return cuda_status(e, "cudaGetSymbolAddress of the static scratch");
-    g_noalloc_ptr[dev] = p;
-  }
-  *ptr = g_noalloc_ptr[dev];
+  void* p = nullptr;
+  cudaError_t e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+  if (e != cudaSuccess) return cuda_status(e, "cudaGetSymbolAddress of the static scratch");
+  *ptr = p;
   return MLA_OK;
 }
 }  // namespace
@@ -1076,12 +1262,222 @@ int mla_prefill_cached_workspace_size(const mla_dims* dims, int64_t total_tokens
   return MLA_OK;
 }
 
+}  // extern "C"
+
+namespace {
+// The eager form: bookkeeping and append as in the absorbed form, then the
+// schedule over key tiles and query blocks, the fp16 weight copy, the padded
+// key rows (cached normalized latent and rotated key), zeroed outputs of
+// invalid sequences, the up-projection of every key row, and the two-tile
+// attention of the chunk's queries with each sequence's prefix length as
+// the query offset.
+int launch_prefill_cached_eager(const mla_dims* d, const void* latent, const void* q, const void* w_kvb,
+                                const void* w_norm, const int32_t* cu_seqlens, int nseq, int64_t Tq,
+                                const int64_t* cache_offsets, const int32_t* prefix_lens, int max_total_len,
+                                const float* cos_t, const float* sin_t, int max_pos, void* cache,
+                                int64_t cache_num_rows, void* out, void* workspace, cudaStream_t st) {
+  using bf16 = __nv_bfloat16;
+  namespace T = mla::tc;
+  const int H = d->num_heads, R = d->kv_lora_rank, N = d->qk_nope, P = d->qk_rope, V = d->v_head;
+  const ChunkEagerWs L = chunk_eager_ws_layout(d, Tq, nseq, max_total_len);
+  char* ws = static_cast<char*>(workspace);
+  int32_t* positions = reinterpret_cast<int32_t*>(ws + L.positions);
+  int64_t* rows = reinterpret_cast<int64_t*>(ws + L.rows);
+  int64_t* offsets = reinterpret_cast<int64_t*>(ws + L.offsets);
+  int32_t* lens = reinterpret_cast<int32_t*>(ws + L.lens);
+  int32_t* seq_ok = reinterpret_cast<int32_t*>(ws + L.seq_ok);
+  int32_t* kseq_tile0 = reinterpret_cast<int32_t*>(ws + L.kseq_tile0);
+  int32_t* ktile_seq = reinterpret_cast<int32_t*>(ws + L.ktile_seq);
+  int32_t* ktile_k0 = reinterpret_cast<int32_t*>(ws + L.ktile_k0);
+  int32_t* qblk_seq = reinterpret_cast<int32_t*>(ws + L.qblk_seq);
+  int32_t* qblk_q0 = reinterpret_cast<int32_t*>(ws + L.qblk_q0);
+  int32_t* qorder = reinterpret_cast<int32_t*>(ws + L.qorder);
+  int32_t* counter = reinterpret_cast<int32_t*>(ws + L.counter);
+  __half* w16 = reinterpret_cast<__half*>(ws + L.w16);
+  __half* c16 = reinterpret_cast<__half*>(ws + L.c16);
+  __half* k_nope = reinterpret_cast<__half*>(ws + L.k_nope);
+  __half* vt = reinterpret_cast<__half*>(ws + L.vt);
+  __half* k_rot = reinterpret_cast<__half*>(ws + L.k_rot);
+  const int NOUT = H * (N + V);
+
+  // 1. per-token positions and cache rows; 2. the chunk's rows into the cache
+  prof_begin(st, "chunk_rows");
+  mla::chunk_rows_kernel<<<(unsigned)((Tq + mla::kChunkThreads - 1) / mla::kChunkThreads), mla::kChunkThreads, 0,
+                           st>>>(cu_seqlens, nseq, Tq, cache_offsets, prefix_lens, max_total_len, max_pos,
+                                 cache_num_rows, positions, rows, offsets, lens);
+  prof_end(st);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_status(e, "chunk rows launch");
+  int rc = mla_cache_append(d, latent, w_norm, positions, Tq, cos_t, sin_t, max_pos, cache, cache_num_rows, rows,
+                            st);
+  if (rc) return rc;
+  // 3. schedule (one block); 4. fp16 weight copy
+  prof_begin(st, "chunk_eager_schedule");
+  T::chunk_eager_schedule_kernel<<<1, T::kChunkSchedThreads, 0, st>>>(
+      cu_seqlens, nseq, Tq, cache_offsets, prefix_lens, max_total_len, max_pos, cache_num_rows, (int)L.kcap,
+      (int)L.qcap, seq_ok, kseq_tile0, ktile_seq, ktile_k0, qblk_seq, qblk_q0, qorder, counter);
+  prof_end(st);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_status(e, "chunk schedule launch");
+  const int64_t n8 = (int64_t)NOUT * R / 8;
+  const int64_t per_block = (int64_t)T::kPrepThreads * T::kPrepUnroll;
+  prof_begin(st, "chunk_weight_f16");
+  T::weight_f16_kernel<<<(unsigned)((n8 + per_block - 1) / per_block), T::kPrepThreads, 0, st>>>(
+      static_cast<const bf16*>(w_kvb), w16, n8);
+  prof_end(st);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_status(e, "chunk weight launch");
+  // 5. padded key rows from the cache; 6. zero outputs of invalid sequences
+  prof_begin(st, "chunk_eager_rows");
+  e = launch_dependent(T::chunk_eager_rows_kernel, dim3((unsigned)((L.Kpad + T::kChunkRowsPerBlock - 1) /
+                                                                    T::kChunkRowsPerBlock)),
+                       dim3(32 * T::kChunkRowsPerBlock), 0, st, (const bf16*)cache, R, cache_offsets, prefix_lens,
+                       cu_seqlens, (const int32_t*)ktile_seq, (const int32_t*)ktile_k0, (int64_t)L.Kpad, c16, k_rot);
+  prof_end(st);
+  if (e != cudaSuccess) return cuda_status(e, "chunk key rows launch");
+  prof_begin(st, "chunk_eager_zero");
+  e = launch_dependent(T::chunk_eager_zero_kernel, dim3((unsigned)((Tq + T::kChunkRowsPerBlock - 1) /
+                                                                   T::kChunkRowsPerBlock)),
+                       dim3(32 * T::kChunkRowsPerBlock), 0, st, cu_seqlens, nseq, Tq, (const int32_t*)seq_ok, H * V,
+                       static_cast<bf16*>(out));
+  prof_end(st);
+  if (e != cudaSuccess) return cuda_status(e, "chunk zero launch");
+
+  // 7. k_nope / transposed values of every key row
+  CUtensorMap map_w, map_c16;
+  {
+    const uint64_t dims[2] = {(uint64_t)R, (uint64_t)NOUT};
+    const uint64_t strides[1] = {(uint64_t)R * 2};
+    const uint32_t box[2] = {64, (uint32_t)(N + V)};
+    rc = make_map(&map_w, w16, 2, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+    if (rc) return rc;
+  }
+  {
+    const uint64_t dims[2] = {(uint64_t)R, (uint64_t)L.Kpad};
+    const uint64_t strides[1] = {(uint64_t)R * 2};
+    const uint32_t box[2] = {64, 128};
+    rc = make_map(&map_c16, c16, 2, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+    if (rc) return rc;
+  }
+  T::GemmParams gp{};
+  gp.cu = cu_seqlens;
+  gp.tile_seq = ktile_seq;
+  gp.tile_q0 = ktile_k0;
+  gp.k_nope = k_nope;
+  gp.vt = vt;
+  gp.k_rot = k_rot;
+  gp.Ttot = Tq;
+  gp.Tpad = (int)L.Kpad;
+  gp.R = R; gp.P = P; gp.H = H; gp.N = N; gp.V = V; gp.NOUT = NOUT;
+  gp.max_pos = max_pos;
+  gp.interleaved = d->rope_interleaved;
+  gp.eps = d->eps;
+  gp.a_padded = 1;
+  int groups = num_sms() / (int)(L.kcap > 0 ? L.kcap : 1);
+  if (groups < 1) groups = 1;
+  if (groups > H) groups = H;
+  gp.tiles_per_cta = (H + groups - 1) / groups;
+  const int gy = (H + gp.tiles_per_cta - 1) / gp.tiles_per_cta;
+  auto gemm = N == 64 ? T::norm_kvb_gemm_vt_kernel<64> : T::norm_kvb_gemm_vt_kernel<128>;
+  e = cudaFuncSetAttribute(gemm, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)T::kG2SmemBytes);
+  if (e != cudaSuccess) return cuda_status(e, "gemm smem attribute");
+  prof_begin(st, "tc_norm_kv_b_proj");
+  e = launch_dependent(gemm, dim3((unsigned)L.kcap, (unsigned)gy), dim3(T::kG2Threads), T::kG2SmemBytes, st, map_c16,
+                       map_w, gp);
+  prof_end(st);
+  if (e != cudaSuccess) return cuda_status(e, "gemm launch");
+
+  // 8. the chunk's queries against each sequence's keys
+  const int D = N + P;
+  CUtensorMap map_q, map_kn, map_kr, map_vt;
+  {
+    const uint64_t dims[3] = {(uint64_t)D, (uint64_t)H, (uint64_t)Tq};
+    const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)H * D * 2};
+    const uint32_t box[3] = {64, 1, 128};
+    rc = make_map(&map_q, q, 3, dims, strides, box);
+    if (rc) return rc;
+  }
+  {
+    const uint64_t dims[2] = {(uint64_t)N, (uint64_t)H * L.Kpad};
+    const uint64_t strides[1] = {(uint64_t)N * 2};
+    const uint32_t box[2] = {64, (uint32_t)T::kPrBKV};
+    rc = make_map(&map_kn, k_nope, 2, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+    if (rc) return rc;
+  }
+  {
+    const uint64_t dims[2] = {(uint64_t)P, (uint64_t)L.Kpad};
+    const uint64_t strides[1] = {(uint64_t)P * 2};
+    const uint32_t box[2] = {64, (uint32_t)T::kPrBKV};
+    rc = make_map(&map_kr, k_rot, 2, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+    if (rc) return rc;
+  }
+  {
+    const uint64_t dims[2] = {(uint64_t)L.Kpad, (uint64_t)H * V};
+    const uint64_t strides[1] = {(uint64_t)L.Kpad * 2};
+    const uint32_t box[2] = {64, (uint32_t)V};
+    rc = make_map(&map_vt, vt, 2, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+    if (rc) return rc;
+  }
+  T::AttParams ap{};
+  ap.cu = cu_seqlens;
+  ap.positions = positions;
+  ap.seq_tile0 = kseq_tile0;
+  ap.tile_seq = qblk_seq;
+  ap.tile_q0 = qblk_q0;
+  ap.order = qorder;
+  ap.cos_t = cos_t;
+  ap.sin_t = sin_t;
+  ap.out = static_cast<bf16*>(out);
+  ap.item_counter = counter;
+  ap.q_off = prefix_lens;
+  ap.n_blocks = (int)L.qcap;
+  ap.H = H;
+  ap.Tpad = (int)L.Kpad;
+  ap.max_pos = max_pos;
+  ap.interleaved = d->rope_interleaved;
+  ap.scale_log2 = d->softmax_scale * 1.4426950408889634f;
+  int64_t grid = L.qcap * H;
+  if (grid > num_sms()) grid = num_sms();
+  return launch_attention_pair(N, V, (unsigned)grid, map_q, map_kn, map_kr, map_vt, ap, st);
+}
+}  // namespace
+
+extern "C" {
+
+int mla_prefill_cached_eager_workspace_size(const mla_dims* dims, int64_t total_tokens, int32_t num_seqs,
+                                            int32_t max_total_len, size_t* bytes) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  if (total_tokens < 0 || num_seqs < 0 || max_total_len < 0) return fail(MLA_ERR_INVALID_ARG, "negative size");
+  if (total_tokens > kMaxChunkTokens)
+    return fail(MLA_ERR_UNSUPPORTED_SHAPE, "at most %lld chunk tokens per call", (long long)kMaxChunkTokens);
+  if (!bytes) return fail(MLA_ERR_INVALID_ARG, "bytes is NULL");
+  if (!chunk_eager_shape(dims)) return fail(MLA_ERR_UNSUPPORTED_SHAPE, "no eager chunk form for this head shape");
+  if ((int64_t)num_seqs * ((max_total_len + 127) / 128) > 0x7fffffff / 128)
+    return fail(MLA_ERR_UNSUPPORTED_SHAPE, "too many key rows for the eager chunk form");
+  *bytes = chunk_eager_ws_layout(dims, total_tokens, num_seqs, max_total_len).total;
+  return MLA_OK;
+}
+
 int mla_prefill_cached(const mla_dims* dims, const void* latent, const void* q, const void* w_kvb,
                        const void* w_norm, const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
                        const int64_t* cache_offsets, const int32_t* prefix_lens, int32_t max_total_len,
                        const float* cos_table, const float* sin_table, int32_t max_pos, void* cache,
                        int64_t cache_num_rows, void* out, void* workspace, size_t workspace_bytes,
                        cudaStream_t stream) {
+  return mla_prefill_cached_form(dims, latent, q, w_kvb, w_norm, cu_seqlens, num_seqs, total_tokens, cache_offsets,
+                                 prefix_lens, max_total_len, cos_table, sin_table, max_pos, cache, cache_num_rows, out,
+                                 workspace, workspace_bytes, MLA_CHUNK_AUTO, stream);
+}
+
+int mla_prefill_cached_form(const mla_dims* dims, const void* latent, const void* q, const void* w_kvb,
+                            const void* w_norm, const int32_t* cu_seqlens, int32_t num_seqs, int64_t total_tokens,
+                            const int64_t* cache_offsets, const int32_t* prefix_lens, int32_t max_total_len,
+                            const float* cos_table, const float* sin_table, int32_t max_pos, void* cache,
+                            int64_t cache_num_rows, void* out, void* workspace, size_t workspace_bytes,
+                            int32_t form, cudaStream_t stream) {
+  if (form != MLA_CHUNK_AUTO && form != MLA_CHUNK_ABSORBED && form != MLA_CHUNK_EAGER)
+    return fail(MLA_ERR_INVALID_ARG, "form must be MLA_CHUNK_AUTO, MLA_CHUNK_ABSORBED or MLA_CHUNK_EAGER");
   int rc = check_dims(dims);
   if (rc) return rc;
   if (total_tokens < 0 || num_seqs < 0) return fail(MLA_ERR_INVALID_ARG, "negative size");
@@ -1098,6 +1494,26 @@ int mla_prefill_cached(const mla_dims* dims, const void* latent, const void* q, 
   if (!latent || !q || !w_kvb || !w_norm || !cu_seqlens || !cache_offsets || !prefix_lens || !cos_table ||
       !sin_table || !cache || !out)
     return fail(MLA_ERR_INVALID_ARG, "a tensor pointer is NULL");
+  // automatic: long chunks (on average kChunkEagerMinAvg tokens or more per
+  // sequence) take the eager form when the workspace holds it
+  const bool eager_ok = chunk_eager_shape(dims) && aligned16(q) && aligned16(cache) && aligned16(w_kvb) &&
+                        aligned16(out) && aligned16(workspace) &&
+                        (int64_t)num_seqs * ((max_total_len + 127) / 128) <= 0x7fffffff / 128;
+  if (form == MLA_CHUNK_EAGER && !eager_ok)
+    return fail(MLA_ERR_UNSUPPORTED_SHAPE, "the eager form needs the tensor-core head shapes and 16-byte alignment");
+  if (form == MLA_CHUNK_EAGER ||
+      (form == MLA_CHUNK_AUTO && eager_ok && total_tokens >= kChunkEagerMinAvg * num_seqs)) {
+    const size_t need_eager = chunk_eager_ws_layout(dims, total_tokens, num_seqs, max_total_len).total;
+    if (form == MLA_CHUNK_EAGER && (!workspace || workspace_bytes < need_eager))
+      return fail(MLA_ERR_WORKSPACE_TOO_SMALL, "the eager form needs %zu bytes of workspace, got %zu", need_eager,
+                  workspace_bytes);
+    if (workspace && workspace_bytes >= need_eager) {
+      set_dispatch("eager: keys and values of every cached row expanded, two-tile attention");
+      return launch_prefill_cached_eager(dims, latent, q, w_kvb, w_norm, cu_seqlens, num_seqs, total_tokens,
+                                         cache_offsets, prefix_lens, max_total_len, cos_table, sin_table, max_pos,
+                                         cache, cache_num_rows, out, workspace, stream);
+    }
+  }
   const ChunkWs L = chunk_ws_layout(dims, total_tokens, max_total_len);
   if (!workspace || workspace_bytes < L.total)
     return fail(MLA_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes, got %zu", L.total, workspace_bytes);
@@ -1119,14 +1535,27 @@ int mla_prefill_cached(const mla_dims* dims, const void* latent, const void* q, 
   rc = mla_cache_append(dims, latent, w_norm, positions, total_tokens, cos_table, sin_table, max_pos, cache,
                         cache_num_rows, rows, stream);
   if (rc) return rc;
-  return mla_decode(dims, q, cache, cache_num_rows, offsets, lens, positions, (int32_t)total_tokens, max_total_len,
-                    w_kvb, cos_table, sin_table, max_pos, out, ws + L.decode, workspace_bytes - L.decode, stream);
+  rc = mla_decode(dims, q, cache, cache_num_rows, offsets, lens, positions, (int32_t)total_tokens, max_total_len,
+                  w_kvb, cos_table, sin_table, max_pos, out, ws + L.decode, workspace_bytes - L.decode, stream);
+  if (!rc) set_dispatch(strcmp(g_dispatch, "tensor-core") == 0 ? "absorbed: one tensor-core decode row per chunk token"
+                                                               : "absorbed: one CUDA-core decode row per chunk token");
+  return rc;
+}
+
+int mla_kv_down_append_workspace_size(const mla_dims* dims, int64_t n, size_t* bytes) {
+  int rc = check_dims(dims);
+  if (rc) return rc;
+  rc = check_proj_rows(n);
+  if (rc) return rc;
+  if (!bytes) return fail(MLA_ERR_INVALID_ARG, "bytes is NULL");
+  *bytes = kv_down_ws_bytes(dims, n);
+  return MLA_OK;
 }
 
 int mla_kv_down_append(const mla_dims* dims, int32_t hidden_size, const void* hidden, const void* w_kva,
                        const void* w_norm, const int32_t* positions, int64_t n, const float* cos_table,
                        const float* sin_table, int32_t max_pos, void* latent, void* cache, int64_t cache_num_rows,
-                       const int64_t* cache_rows, cudaStream_t stream) {
+                       const int64_t* cache_rows, void* workspace, size_t workspace_bytes, cudaStream_t stream) {
   int rc = check_dims(dims);
   if (rc) return rc;
   rc = check_proj_rows(n);
@@ -1139,11 +1568,28 @@ int mla_kv_down_append(const mla_dims* dims, int32_t hidden_size, const void* hi
   if (append && (max_pos < 1 || cache_num_rows < 1))
     return fail(MLA_ERR_INVALID_ARG, "appending needs max_pos >= 1 and cache_num_rows >= 1");
   if (n == 0) return MLA_OK;
-  rc = launch_linear(dims, hidden, w_kva, latent, n, hidden_size, dims->kv_lora_rank + dims->qk_rope, stream,
-                     "kv_a_proj");
-  if (rc || !append) return rc;
-  return mla_cache_append(dims, latent, w_norm, positions, n, cos_table, sin_table, max_pos, cache, cache_num_rows,
-                          cache_rows, stream);
+  const size_t need = kv_down_ws_bytes(dims, n);
+  if (need && (!workspace || workspace_bytes < need))
+    return fail(MLA_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes, got %zu", need, workspace_bytes);
+  const int W = dims->kv_lora_rank + dims->qk_rope;
+  if (dims->dtype == MLA_FP32) {
+    rc = launch_linear(dims, hidden, w_kva, latent, n, hidden_size, W, stream, "kv_a_proj");
+    if (rc || !append) return rc;
+    return mla_cache_append(dims, latent, w_norm, positions, n, cos_table, sin_table, max_pos, cache,
+                            cache_num_rows, cache_rows, stream);
+  }
+  // bf16: the Linear's fp32 result, then compressed_kv and the cache row from it
+  float* x32 = static_cast<float*>(workspace);
+  rc = launch_linear(dims, hidden, w_kva, nullptr, n, hidden_size, W, stream, "kv_a_proj", x32);
+  if (rc) return rc;
+  prof_begin(stream, "kv_latent_append");
+  mla::kv_latent_append_kernel<<<(unsigned)((n + mla::kKvRowsPerBlock - 1) / mla::kKvRowsPerBlock),
+                                 32 * mla::kKvRowsPerBlock, 0, stream>>>(
+      x32, static_cast<__nv_bfloat16*>(latent), n, dims->kv_lora_rank, dims->qk_rope,
+      static_cast<const __nv_bfloat16*>(w_norm), positions, cos_table, sin_table, max_pos, dims->rope_interleaved,
+      dims->eps, append ? static_cast<__nv_bfloat16*>(cache) : nullptr, cache_num_rows, cache_rows);
+  prof_end(stream);
+  return cuda_status(cudaGetLastError(), "kv latent append launch");
 }
 
 int mla_q_proj_workspace_size(const mla_dims* dims, int32_t q_rank, int64_t n, size_t* bytes) {
@@ -1153,7 +1599,7 @@ int mla_q_proj_workspace_size(const mla_dims* dims, int32_t q_rank, int64_t n, s
   if (rc) return rc;
   if (q_rank < 1) return fail(MLA_ERR_INVALID_ARG, "q_rank must be >= 1");
   if (!bytes) return fail(MLA_ERR_INVALID_ARG, "bytes is NULL");
-  *bytes = align_up((size_t)n * (size_t)q_rank * elem_size(dims), 256);
+  *bytes = q_proj_ws_layout(dims, q_rank, n).total;
   return MLA_OK;
 }
 
@@ -1167,27 +1613,61 @@ int mla_q_proj(const mla_dims* dims, int32_t hidden_size, int32_t q_rank, const 
   if (hidden_size < 1 || q_rank < 1) return fail(MLA_ERR_INVALID_ARG, "hidden_size and q_rank must be >= 1");
   if (!hidden || !w_qa || !w_qnorm || !w_qb || !q) return fail(MLA_ERR_INVALID_ARG, "a tensor pointer is NULL");
   if (n == 0) return MLA_OK;
-  const size_t need = align_up((size_t)n * (size_t)q_rank * elem_size(dims), 256);
-  if (!workspace || workspace_bytes < need)
-    return fail(MLA_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes, got %zu", need, workspace_bytes);
-  // q_a = hidden W_qa^T, normalized in place, then q = q_a W_qb^T
-  rc = launch_linear(dims, hidden, w_qa, workspace, n, hidden_size, q_rank, stream, "q_a_proj");
-  if (rc) return rc;
+  const QProjWs L = q_proj_ws_layout(dims, q_rank, n);
+  if (!workspace || workspace_bytes < L.total)
+    return fail(MLA_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes, got %zu", L.total, workspace_bytes);
+  char* ws = static_cast<char*>(workspace);
+  const int NQ = dims->num_heads * (dims->qk_nope + dims->qk_rope);
   const unsigned blocks = (unsigned)((n + mla::kRowsPerNormBlock - 1) / mla::kRowsPerNormBlock);
-  prof_begin(stream, "q_a_layernorm");
-  if (dims->dtype == MLA_FP32)
+  if (dims->dtype == MLA_FP32) {
+    // q_a = hidden W_qa^T, normalized in place, then q = q_a W_qb^T
+    float* qa = reinterpret_cast<float*>(ws + L.q_a);
+    rc = launch_linear(dims, hidden, w_qa, qa, n, hidden_size, q_rank, stream, "q_a_proj");
+    if (rc) return rc;
+    prof_begin(stream, "q_a_layernorm");
     mla::rmsnorm_rows_kernel<float><<<blocks, 32 * mla::kRowsPerNormBlock, 0, stream>>>(
-        static_cast<const float*>(workspace), static_cast<const float*>(w_qnorm), static_cast<float*>(workspace), n,
-        q_rank, dims->eps);
-  else
-    mla::rmsnorm_rows_kernel<__nv_bfloat16><<<blocks, 32 * mla::kRowsPerNormBlock, 0, stream>>>(
-        static_cast<const __nv_bfloat16*>(workspace), static_cast<const __nv_bfloat16*>(w_qnorm),
-        static_cast<__nv_bfloat16*>(workspace), n, q_rank, dims->eps);
+        qa, static_cast<const float*>(w_qnorm), qa, n, q_rank, dims->eps);
+    prof_end(stream);
+    rc = cuda_status(cudaGetLastError(), "q_a_layernorm launch");
+    if (rc) return rc;
+    return launch_linear(dims, qa, w_qb, q, n, q_rank, NQ, stream, "q_b_proj");
+  }
+  // bf16: q_a_proj's fp32 result is normalized without a rounding in between;
+  // the normalized q_a feeds q_b_proj in fp16 against an fp16 copy of w_qb
+  // (tensor cores), or in fp32 (CUDA cores)
+  float* qa32 = reinterpret_cast<float*>(ws + L.q_a);
+  rc = launch_linear(dims, hidden, w_qa, nullptr, n, hidden_size, q_rank, stream, "q_a_proj", qa32);
+  if (rc) return rc;
+  const bool tc_b = linear_tc(dims, ws + L.q_an, w_qb, q_rank) && aligned16(q);
+  if (tc_b) {
+    __half* qan = reinterpret_cast<__half*>(ws + L.q_an);
+    __half* w16 = reinterpret_cast<__half*>(ws + L.w16);
+    const int64_t n8 = (int64_t)NQ * q_rank / 8;
+    const int64_t per_block = (int64_t)mla::tc::kPrepThreads * mla::tc::kPrepUnroll;
+    if ((int64_t)NQ * q_rank % 8 == 0) {
+      prof_begin(stream, "q_b_proj_weight_f16");
+      mla::tc::weight_f16_kernel<<<(unsigned)((n8 + per_block - 1) / per_block), mla::tc::kPrepThreads, 0, stream>>>(
+          static_cast<const __nv_bfloat16*>(w_qb), w16, n8);
+      prof_end(stream);
+      rc = cuda_status(cudaGetLastError(), "q_b_proj weight launch");
+      if (rc) return rc;
+      prof_begin(stream, "q_a_layernorm");
+      mla::rmsnorm_f32_rows_kernel<__half><<<blocks, 32 * mla::kRowsPerNormBlock, 0, stream>>>(
+          qa32, static_cast<const __nv_bfloat16*>(w_qnorm), qan, n, q_rank, dims->eps);
+      prof_end(stream);
+      rc = cuda_status(cudaGetLastError(), "q_a_layernorm launch");
+      if (rc) return rc;
+      return launch_linear(dims, qan, w16, q, n, q_rank, NQ, stream, "q_b_proj", nullptr, true);
+    }
+  }
+  float* qan32 = reinterpret_cast<float*>(ws + L.q_an);
+  prof_begin(stream, "q_a_layernorm");
+  mla::rmsnorm_f32_rows_kernel<float><<<blocks, 32 * mla::kRowsPerNormBlock, 0, stream>>>(
+      qa32, static_cast<const __nv_bfloat16*>(w_qnorm), qan32, n, q_rank, dims->eps);
   prof_end(stream);
   rc = cuda_status(cudaGetLastError(), "q_a_layernorm launch");
   if (rc) return rc;
-  return launch_linear(dims, workspace, w_qb, q, n, q_rank, dims->num_heads * (dims->qk_nope + dims->qk_rope),
-                       stream, "q_b_proj");
+  return launch_linear_f32x(qan32, w_qb, q, n, q_rank, NQ, stream, "q_b_proj");
 }
 
 int mla_o_proj(const mla_dims* dims, int32_t hidden_size, const void* attn, const void* w_o, int64_t n, void* out,
@@ -1200,6 +1680,15 @@ int mla_o_proj(const mla_dims* dims, int32_t hidden_size, const void* attn, cons
   if (!attn || !w_o || !out) return fail(MLA_ERR_INVALID_ARG, "a tensor pointer is NULL");
   if (n == 0) return MLA_OK;
   return launch_linear(dims, attn, w_o, out, n, dims->num_heads * dims->v_head, hidden_size, stream, "o_proj");
+}
+
+int mla_selftest_wait_timeout(uint32_t limit_us, int32_t* gave_up, cudaStream_t stream) {
+  if (limit_us < 1 || limit_us > 1000000) return fail(MLA_ERR_INVALID_ARG, "limit_us must be in 1 .. 1000000");
+  if (!gave_up) return fail(MLA_ERR_INVALID_ARG, "gave_up is NULL");
+  prof_begin(stream, "selftest_wait_timeout");
+  mla::tc::wait_timeout_selftest_kernel<<<1, 32, 0, stream>>>((uint64_t)limit_us * 1000ull, gave_up);
+  prof_end(stream);
+  return cuda_status(cudaGetLastError(), "self-test launch");
 }
 
 int mla_check_device_status(cudaStream_t stream) {

@@ -38,13 +38,93 @@ rmsnorm_rows_kernel(const T* x, const T* __restrict__ w, T* y, int64_t rows, int
   for (int k = lane; k < width; k += 32) yr[k] = from_f32<T>(to_f32(w[k]) * (to_f32(xr[k]) * r));
 }
 
+// The query RMSNorm of a bf16 run, on q_a_proj's fp32 result (never rounded
+// before the norm): y[t, :] = w * x[t, :] / sqrt(mean(x[t, :]^2) + eps) in
+// TO (fp16 for the tensor-core q_b_proj, fp32 for the CUDA-core one).
+template <typename TO>
+__global__ void __launch_bounds__(32 * kRowsPerNormBlock)
+rmsnorm_f32_rows_kernel(const float* __restrict__ x, const __nv_bfloat16* __restrict__ w, TO* __restrict__ y,
+                        int64_t rows, int width, float eps) {
+  const int64_t t = (int64_t)blockIdx.x * kRowsPerNormBlock + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= rows) return;
+  const float* xr = x + t * width;
+  float ss = 0.f;
+  for (int k = lane; k < width; k += 32) ss = fmaf(xr[k], xr[k], ss);
+  ss = warp_sum(ss);
+  const float r = 1.0f / sqrtf(ss / (float)width + eps);
+  TO* yr = y + t * width;
+  bool over = false;
+  for (int k = lane; k < width; k += 32) {
+    const float v = __bfloat162float(w[k]) * (xr[k] * r);
+    if constexpr (sizeof(TO) == 2) {
+      over |= !(fabsf(v) <= 65504.f);
+      yr[k] = __float2half_rn(v);
+    } else {
+      yr[k] = v;
+    }
+  }
+  if (over) raise_device_error(kDevErrRange);
+}
+
+// The joint down-projection's fp32 result x [n, R + P] of a bf16 run, one
+// warp per token: latent[t] = bf16(x[t]) (compressed_kv, the prefill's latent
+// input), and when `cache` is set the cache row
+//   RMSNorm(x[t, :R]) || rope(x[t, R:], positions[t])
+// into cache[cache_rows[t]], both computed from the fp32 values (the cache
+// append of the GLM-5 "KV cache" section fused onto the Linear's result). A
+// destination row or position out of range skips the row's append and sets
+// the device error word.
+constexpr int kKvRowsPerBlock = 8;
+__global__ void __launch_bounds__(32 * kKvRowsPerBlock)
+kv_latent_append_kernel(const float* __restrict__ x, __nv_bfloat16* __restrict__ latent, int64_t n, int R, int P,
+                        const __nv_bfloat16* __restrict__ w_norm, const int32_t* __restrict__ positions,
+                        const float* __restrict__ cos_t, const float* __restrict__ sin_t, int max_pos, int interleaved,
+                        float eps, __nv_bfloat16* __restrict__ cache, int64_t cache_num_rows,
+                        const int64_t* __restrict__ cache_rows) {
+  const int64_t t = (int64_t)blockIdx.x * kKvRowsPerBlock + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
+  if (t >= n) return;
+  const int W = R + P;
+  const float* xr = x + t * W;
+  __nv_bfloat16* lr = latent + t * W;
+  float ss = 0.f;
+  for (int k = lane; k < W; k += 32) {
+    const float v = xr[k];
+    lr[k] = __float2bfloat16_rn(v);
+    if (k < R) ss = fmaf(v, v, ss);
+  }
+  if (!cache) return;
+  ss = warp_sum(ss);
+  const int64_t row = cache_rows[t];
+  const int64_t pos = positions[t];
+  if (row < 0 || row >= cache_num_rows || pos < 0 || pos >= max_pos) {
+    if (lane == 0) raise_device_error(kDevErrBadInput);
+    return;
+  }
+  const float r = 1.0f / sqrtf(ss / (float)R + eps);
+  __nv_bfloat16* dst = cache + row * W;
+  for (int k = lane; k < R; k += 32) dst[k] = __float2bfloat16_rn(__bfloat162float(w_norm[k]) * (xr[k] * r));
+  const int half = P / 2;
+  for (int i = lane; i < half; i += 32) {
+    int a, b;
+    rope_pair_slots(i, P, interleaved, a, b);
+    float ox, oy;
+    rope_turn(xr[R + a], xr[R + b], cos_t[pos * half + i], sin_t[pos * half + i], ox, oy);
+    dst[R + a] = __float2bfloat16_rn(ox);
+    dst[R + b] = __float2bfloat16_rn(oy);
+  }
+}
+
 // out[t, j] = sum_k x[t, k] w[j, k], fp32 accumulation: 16 x 16 output tiles,
-// K staged through shared memory 16 at a time. Every load is guarded.
+// K staged through shared memory 16 at a time. Every load is guarded. x, w
+// and out may have different types (bf16 runs keep the results that feed an
+// RMSNorm in fp32).
 constexpr int kLinTile = 16;
 
-template <typename T>
+template <typename T, typename TW = T, typename TO = T>
 __global__ void __launch_bounds__(kLinTile * kLinTile)
-simt_linear_kernel(const T* __restrict__ x, const T* __restrict__ w, T* __restrict__ out, int64_t n, int K,
+simt_linear_kernel(const T* __restrict__ x, const TW* __restrict__ w, TO* __restrict__ out, int64_t n, int K,
                    int Nout) {
   __shared__ float sx[kLinTile][kLinTile + 1];
   __shared__ float sw[kLinTile][kLinTile + 1];
@@ -63,7 +143,7 @@ simt_linear_kernel(const T* __restrict__ x, const T* __restrict__ w, T* __restri
     for (int kk = 0; kk < kLinTile; ++kk) acc = fmaf(sx[ty][kk], sw[tx][kk], acc);
     __syncthreads();
   }
-  if (t < n && j < Nout) out[t * Nout + j] = from_f32<T>(acc);
+  if (t < n && j < Nout) out[t * Nout + j] = from_f32<TO>(acc);
 }
 
 }  // namespace mla

@@ -56,7 +56,12 @@ struct AttParams {
   const float* cos_t;
   const float* sin_t;
   __nv_bfloat16* out;
+  int* item_counter;            // two-tile kernel: next work item (zeroed by the preparation kernel)
+  const int32_t* q_off;         // two-tile kernel: per sequence, the key index of its first query
+                                // (cached rows before it; NULL: 0). Keys come from the padded
+                                // layout of the sequence's q_off + length rows.
   int H, Tpad, max_pos, interleaved;
+  int n_blocks;                 // two-tile kernel: entries of `order` (256-row blocks, -1 past the last)
   float scale_log2;             // softmax scale * log2(e)
 };
 

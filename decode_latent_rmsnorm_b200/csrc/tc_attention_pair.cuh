@@ -1,4 +1,5 @@
-// Tensor-core (tcgen05) causal attention, two query tiles per CTA.
+// Tensor-core (tcgen05) causal attention, two query tiles per work item, on a
+// persistent grid.
 //
 // Sources: Kimi-K2 "Query content heads" page, "Join query parts", and the
 // Kimi-K2 "RoPE coefficients" page, "Key heads" (mla-prefill excerpt): each
@@ -8,29 +9,51 @@
 // values. The arithmetic is the one of attention_kernel; this kernel changes
 // how it is scheduled on the SM.
 //
-// One CTA = one head x one 256-row block of queries, split into tile A (rows
-// 0-127) and tile B (rows 128-255). Both tiles read the same key / value
-// tiles (128 keys per step), so each K/V byte staged in shared memory feeds
-// twice the tensor-core work. Warps:
-//   warp 0     TMA producer (Q tiles, then per step: the key atoms and the two
-//              transposed value boxes into a ring of 16 KB slots)
+// Work item = one head x one 256-row block of queries, split into tile A
+// (rows 0-127) and tile B (rows 128-255). Both tiles read the same key /
+// value tiles (128 keys per step), so each K/V byte staged in shared memory
+// feeds twice the tensor-core work. One CTA runs per SM and takes items from
+// a device-wide counter, heaviest blocks first (the block list is sorted by
+// causal work), so the grid balances itself. Warps (three warpgroups; the
+// first runs on 56 registers per thread so that the softmax warpgroups can
+// hold a whole row of scores in 216):
+//   warp 0     producer: takes the next item, publishes it to the other warps
+//              through a two-slot ring in shared memory, loads the tiles' Q
+//              and, per key step, the key atoms and the two transposed value
+//              boxes into a ring of 16 KB slots. The key/value stream runs on
+//              across items, and the next item's Q is loaded as soon as the
+//              current item's last score product on that tile has finished.
 //   warp 1     MMA issuer (whole warp, one elected lane issues)
-//   warps 2-5  softmax of tile A (one query row per thread, TMEM lane = row)
-//   warps 6-9  softmax of tile B
+//   warps 2-3  idle
+//   warps 4-7  softmax of tile A (one query row per thread, TMEM lane = row)
+//   warps 8-11 softmax of tile B
 // TMEM (512 columns): S_A [0,128), S_B [128,256), O_A [256,256+V),
 // O_B [384,384+V). P (fp16) is written back over the first 64 columns of its
 // own S buffer and read from there by the P V product (A operand in TMEM).
-// The MMA thread alternates the tiles so that one tile's softmax runs while
-// the tensor cores work on the other tile:
-//   ... PV_A(j)  S_A(j+1)  PV_B(j)  S_B(j+1)  PV_A(j+1) ...
-// Tensor-core instructions from one thread run in issue order, so S_X(j+1)
-// overwrites P_X(j) only after PV_X(j) has read it.
+// Per global key step g the MMA warp issues
+//   PV_A(g)  S_A(g+1)  PV_B(g)  S_B(g+1)
+// (each only when that tile uses the step; step g+1 may belong to the next
+// item), so one tile's softmax runs while the tensor cores work on the other
+// tile, and every key and value group is consumed in the order it was loaded.
+// Tensor-core instructions from one thread run in issue order, so S_X(g+1)
+// overwrites P_X(g) only after PV_X(g) has read it.
+//
+// At the end of an item a tile's softmax warps first convert the next item's
+// Q (so that its first score product can start) and then write the item's
+// output from O; the next item's first P V product (which overwrites O) waits
+// for that.
 //
 // Softmax reference: a row's reference m is its maximum over the first key
 // tile; it is raised (and O and the row sum rescaled) only when a later tile's
 // maximum exceeds it by more than kPrLazy (log2 units), so P <= 2^kPrLazy,
-// well inside fp16. The row sum adds the fp32 weights before their rounding
-// to fp16 (relative difference <= 2^-12 of the result).
+// well inside fp16. The weights are formed as e = 2^(s - m - kPrBias) (fp32,
+// always normal), their row sum is kept in fp32 at that scale, and their fp16
+// codes come from e * 2^-12 = P * 2^-112 by integer arithmetic
+// (f16x2_from_scaled), which keeps the conversion off the MUFU pipe that the
+// exponentials saturate. The codes equal round-to-nearest fp16 of P
+// (subnormals included; exact ties round away from zero). The row sum adds the
+// fp32 weights before their rounding to fp16 (relative difference <= 2^-12 of
+// the result).
 #pragma once
 #include "tc_attention.cuh"
 
@@ -38,11 +61,53 @@ namespace mla {
 namespace tc {
 
 constexpr int kPrBKV = 128;                 // keys per step
-constexpr int kPrThreads = 320;
+constexpr int kPrThreads = 384;
+// Registers per thread of the producer / MMA warpgroup and of the two softmax
+// warpgroups: 128 x 56 + 256 x 216 = 62464, within the 384 x 168 = 64512 the
+// launch holds (ptxas gives this kernel 168 per thread; checked at build).
+constexpr int kPrRegsCtl = 56;
+constexpr int kPrRegsSoftmax = 216;
+static_assert(128 * kPrRegsCtl + 256 * kPrRegsSoftmax <= kPrThreads * 168, "register split exceeds the launch");
 constexpr int kPrSlotBytes = 16384;
 constexpr int kPrMaxSlots = 12;
 constexpr float kPrLazy = 8.f;
 constexpr int kPrGroupDepth = 4;
+constexpr int kPrSched = 2;                 // item slots between the producer and the other warps
+constexpr int kPrSchedReaders = 9;          // the MMA warp and the eight softmax warps
+constexpr float kPrBias = 100.f;            // e = P * 2^-kPrBias stays a normal fp32 number
+constexpr float kPrTwoM12 = 2.44140625e-4f;         // 2^-12
+constexpr float kPrTwoMBias = 7.888609052210118e-31f;   // 2^-100
+// Of the four 32-key chunks of a row's step, the last kPrPolyChunks take
+// their exponentials from ex2_fma2 (FMA pipes) instead of the MUFU.
+#ifndef MLA_PR_POLY_CHUNKS
+#define MLA_PR_POLY_CHUNKS 0
+#endif
+constexpr int kPrPolyChunks = MLA_PR_POLY_CHUNKS;
+
+// 2^a for a pair of exponents a <= 2^22 on the FMA pipes (packed fp32): a is
+// clamped at -126 (smaller weights round to 0 in fp16 anyway), split as
+// a = j + f with j = round(a) (the 1.5 * 2^23 rounding trick) and f in
+// [-0.5, 0.5]; 2^f comes from a cubic fitted here to 2^f on [-0.5, 0.5]
+// for relative error (Lawson-weighted least squares; at most 7.5e-5, below
+// fp16's half-ulp), and j is added to its exponent field: the bits of
+// 1.5 * 2^23 shifted left by 23 vanish modulo 2^32, so (bits(t) << 23)
+// equals j << 23.
+__device__ __forceinline__ uint64_t ex2_fma2(uint64_t a2) {
+  float a0, a1;
+  f2_split(a2, a0, a1);
+  const uint64_t a = f2_make(fmaxf(a0, -126.f), fmaxf(a1, -126.f));
+  const uint64_t t = f2_add(a, f2_make(12582912.f, 12582912.f));
+  const uint64_t jf = f2_add(t, f2_make(-12582912.f, -12582912.f));
+  const uint64_t f = f2_fma(jf, f2_make(-1.f, -1.f), a);
+  uint64_t p = f2_fma(f2_make(5.517166853e-02f, 5.517166853e-02f), f, f2_make(2.426111400e-01f, 2.426111400e-01f));
+  p = f2_fma(p, f, f2_make(6.932609677e-01f, 6.932609677e-01f));
+  p = f2_fma(p, f, f2_make(9.999280572e-01f, 9.999280572e-01f));
+  float p0, p1, t0, t1;
+  f2_split(p, p0, p1);
+  f2_split(t, t0, t1);
+  return f2_make(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
+                 __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
+}
 
 template <int kN, int kV>
 struct PairCfg {
@@ -66,18 +131,68 @@ struct PairCfg {
 // atoms and the rotary key atom) and one value group (two boxes). Each group
 // has one "full" barrier (all its copies landed) and one "empty" barrier (the
 // MMAs reading it are done), so the MMA warp waits once per group instead of
-// once per box. The barriers rotate over kPrGroupDepth steps: a box's slot
-// was last used at most three steps earlier (static_assert below), and the
-// release the producer waits for before re-arming a step's barrier is issued
-// after the MMA warp's wait on that barrier four steps earlier.
+// once per box. The barriers rotate over kPrGroupDepth global steps: a box's
+// slot was last used at most three steps earlier (static_assert above), and
+// the release the producer waits for before re-arming a step's barrier is
+// issued after the MMA warp's wait on that barrier four steps earlier.
 struct PairBarriers {
-  uint64_t q_full, q_ready[2];
+  uint64_t q_full[2], q_ready[2], q_free[2];
   uint64_t kfull[kPrGroupDepth], kempty[kPrGroupDepth], vfull[kPrGroupDepth], vempty[kPrGroupDepth];
-  uint64_t s_full[2], p_full[2], pv_done[2];
+  uint64_t s_full[2], p_full[2], pv_done[2], o_free[2];
+  uint64_t sched_full[kPrSched], sched_empty[kPrSched];
   uint64_t mma_done;
+  int sched_item[kPrSched];
   uint32_t tmem_base;
   int abort_flag;
 };
+
+// One work item, decoded from its index: head h of the block whose first tile
+// is order[item / H].
+struct PairItem {
+  int valid;                  // 0: past the last item (or the counter ran past the list)
+  int h, q0, L, kv_pad0;
+  int off;                    // key index of the sequence's first query (0 without cached rows)
+  int nA, nB, n;              // key steps of tile A, tile B (0: all padding), the item
+  int64_t seq0;
+};
+
+__device__ __forceinline__ PairItem pair_item(const AttParams& p, int item) {
+  PairItem it;
+  it.valid = 0;
+  it.h = it.q0 = it.L = it.kv_pad0 = it.off = it.nA = it.nB = it.n = 0;
+  it.seq0 = 0;
+  if (item < 0) return it;
+  const int rank = item / p.H;
+  if (rank >= p.n_blocks) return it;
+  const int tile = p.order[rank];
+  if (tile < 0) return it;
+  const int seq = p.tile_seq[tile];
+  it.valid = 1;
+  it.h = item - rank * p.H;
+  it.q0 = p.tile_q0[tile];                                   // multiple of 256
+  it.seq0 = p.cu[seq];
+  it.L = (int)(p.cu[seq + 1] - it.seq0);
+  it.kv_pad0 = p.seq_tile0[seq] * kTile;
+  it.off = p.q_off ? p.q_off[seq] : 0;
+  // query row r attends keys 0 .. off + r; a tile's key steps reach its last valid row's
+  it.nA = (it.off + min(it.q0 + kTile - 1, it.L - 1)) / kPrBKV + 1;
+  it.nB = (it.q0 + kTile < it.L) ? (it.off + min(it.q0 + 2 * kTile - 1, it.L - 1)) / kPrBKV + 1 : 0;
+  it.n = it.nA > it.nB ? it.nA : it.nB;
+  return it;
+}
+
+// The k-th work item of the CTA, as published by the producer: every reader
+// warp reads every slot once, in order. Returns false on abort.
+__device__ __forceinline__ bool pair_read_item(PairBarriers& bars, const AttParams& p, int k, int lane,
+                                               volatile int* abort_flag, PairItem& it) {
+  const int s = k % kPrSched;
+  if (!mbar_wait_warp(&bars.sched_full[s], (uint32_t)(k / kPrSched) & 1u, abort_flag)) return false;
+  const int item = *reinterpret_cast<volatile int*>(&bars.sched_item[s]);
+  __syncwarp();
+  if (lane == 0) mbar_arrive(&bars.sched_empty[s]);
+  it = pair_item(p, item);
+  return true;
+}
 
 template <int kN, int kV>
 __global__ void __launch_bounds__(kPrThreads, 1)
@@ -90,33 +205,28 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
   __shared__ PairBarriers bars;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_allow_next();
-  const int rank = blockIdx.x / p.H, h = blockIdx.x % p.H;
-  const int tile = p.order[rank];       // first tile of the block
-  if (tile < 0) return;                 // uniform over the CTA
-  const int seq = p.tile_seq[tile];
-  const int q0 = p.tile_q0[tile];       // multiple of 256
-  const int64_t seq0 = p.cu[seq];
-  const int L = (int)(p.cu[seq + 1] - seq0);
-  const int kv_pad0 = p.seq_tile0[seq] * kTile;
-  const int nA = q0 / kPrBKV + 1;                              // key steps of tile A
-  const int nB = (q0 + kTile < L) ? q0 / kPrBKV + 2 : 0;      // 0: tile B is all padding
-  const int n = nA > nB ? nA : nB;
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
   uint8_t* sRing = smem + C::kQBytes;
   volatile int* abort_flag = &bars.abort_flag;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars.q_full, 1);
     for (int x = 0; x < 2; ++x) {
+      mbar_init(&bars.q_full[x], 1);
       mbar_init(&bars.q_ready[x], 128);
+      mbar_init(&bars.q_free[x], 1);
       mbar_init(&bars.s_full[x], 1);
       mbar_init(&bars.p_full[x], 128);
       mbar_init(&bars.pv_done[x], 1);
+      mbar_init(&bars.o_free[x], 128);
     }
     for (int b = 0; b < kPrGroupDepth; ++b) {
       mbar_init(&bars.kfull[b], 1); mbar_init(&bars.kempty[b], 1);
       mbar_init(&bars.vfull[b], 1); mbar_init(&bars.vempty[b], 1);
+    }
+    for (int s = 0; s < kPrSched; ++s) {
+      mbar_init(&bars.sched_full[s], 1);
+      mbar_init(&bars.sched_empty[s], kPrSchedReaders);
     }
     mbar_init(&bars.mma_done, 1);
     bars.abort_flag = 0;
@@ -128,140 +238,228 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
   tc_fence_after();
   const uint32_t tmem = bars.tmem_base;
 
-  if (warp == 0) {
-    // ---------------- TMA producer ----------------
-    if (lane == 0) {
-      tma_prefetch_desc(&map_q);
-      tma_prefetch_desc(&map_kn);
-      tma_prefetch_desc(&map_kr);
-      tma_prefetch_desc(&map_vt);
-      mbar_arrive_expect_tx(&bars.q_full, nB > 0 ? C::kQBytes : C::kQTileBytes);
-      for (int a = 0; a < C::kQAtoms; ++a)
-        tma_load_3d(sQ + a * kTile * 128, &map_q, &bars.q_full, a * 64, h, (int)(seq0 + q0));
-      if (nB > 0)
-        for (int a = 0; a < C::kQAtoms; ++a)
-          tma_load_3d(sQ + C::kQTileBytes + a * kTile * 128, &map_q, &bars.q_full, a * 64, h,
-                      (int)(seq0 + q0 + kTile));
-      // box g of the ring sits in slot g % S; before it is filled, the group
-      // that last used the slot (box g - S) must have been released
-      auto wait_released = [&](int gp) -> bool {
-        const int jp = gp / C::kBoxes;
-        uint64_t* bar = (gp % C::kBoxes) < C::kQAtoms ? &bars.kempty[jp & 3] : &bars.vempty[jp & 3];
-        return mbar_wait(bar, (uint32_t)(jp >> 2) & 1u, abort_flag);
-      };
-      pdl_wait();   // k_nope, the values and k_rot come from the previous kernel
-      bool ok = true;
-      int jk = -1, jv = -1;              // last key / value group issued
-      for (int j = 0; j < n && ok; ++j) {
-        const int kv_row = kv_pad0 + j * kPrBKV;
-        const int g0 = j * C::kBoxes;
-        for (int i = 0; i < C::kQAtoms && ok; ++i)
-          if (g0 + i >= S) ok = wait_released(g0 + i - S);
-        if (!ok) break;
-        mbar_arrive_expect_tx(&bars.kfull[j & 3], C::kQAtoms * kPrBKV * 128);
-        for (int i = 0; i < C::kKAtoms; ++i)
-          tma_load_2d(sRing + ((g0 + i) % S) * kPrSlotBytes, &map_kn, &bars.kfull[j & 3], i * 64,
-                      h * p.Tpad + kv_row);
-        tma_load_2d(sRing + ((g0 + C::kKAtoms) % S) * kPrSlotBytes, &map_kr, &bars.kfull[j & 3], 0, kv_row);
-        jk = j;
-        for (int v = 0; v < 2 && ok; ++v)
-          if (g0 + C::kQAtoms + v >= S) ok = wait_released(g0 + C::kQAtoms + v - S);
-        if (!ok) break;
-        mbar_arrive_expect_tx(&bars.vfull[j & 3], 2 * C::kVBoxBytes);
-        for (int v = 0; v < 2; ++v)
-          tma_load_2d(sRing + ((g0 + C::kQAtoms + v) % S) * kPrSlotBytes, &map_vt, &bars.vfull[j & 3],
-                      kv_row + v * 64, h * kV);
-        jv = j;
-      }
-      if (!ok) {   // let every copy already issued land before the CTA exits
-        mbar_wait_drain(&bars.q_full, 0);
-        for (int jj = (jk > 3 ? jk - 3 : 0); jj <= jk; ++jj)
-          mbar_wait_drain(&bars.kfull[jj & 3], (uint32_t)(jj >> 2) & 1u);
-        for (int jj = (jv > 3 ? jv - 3 : 0); jj <= jv; ++jj)
-          mbar_wait_drain(&bars.vfull[jj & 3], (uint32_t)(jj >> 2) & 1u);
-      }
-    }
-  } else if (warp == 1) {
-    // ---------------- MMA issuer (whole warp; one elected lane issues) ----------------
-    const uint32_t idesc_s = idesc_f16_f32(kTile, kPrBKV);
-    const uint32_t idesc_o = idesc_f16_f32(kTile, kV);
-    auto slot_addr = [&](int g) -> uint32_t { return smem_u32(sRing + (g % S) * kPrSlotBytes); };
-    int k_seen = -1, v_seen = -1;        // last step whose key / value group was waited for
-    // S_x(j) = Q_x K_j^T over all D columns
-    auto issue_s = [&](int x, int j) -> bool {
-      if (k_seen < j) {
-        if (!mbar_wait_warp(&bars.kfull[j & 3], (uint32_t)(j >> 2) & 1u, abort_flag)) return false;
-        k_seen = j;
-      }
-      tc_fence_after();
-      const uint32_t d = tmem + (uint32_t)(x * kPrBKV);
-#pragma unroll
-      for (int a = 0; a < C::kQAtoms; ++a) {
-        const uint64_t qd = desc_kmajor_sw128(smem_u32(sQ + x * C::kQTileBytes + a * kTile * 128));
-        const uint64_t kd = desc_kmajor_sw128(slot_addr(j * C::kBoxes + a));
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          mma_ss_elect(d, desc_advance(qd, k * 32), desc_advance(kd, k * 32), idesc_s, (a | k) != 0);
-      }
-      mma_commit_elect(&bars.s_full[x]);
-      return true;
-    };
-    // O_x += P_x(j) V_j, P_x(j) read from TMEM
-    auto issue_pv = [&](int x, int j) -> bool {
-      if (v_seen < j) {
-        if (!mbar_wait_warp(&bars.vfull[j & 3], (uint32_t)(j >> 2) & 1u, abort_flag)) return false;
-        v_seen = j;
-      }
-      if (!mbar_wait_warp(&bars.p_full[x], (uint32_t)j & 1u, abort_flag)) return false;
-      tc_fence_after();
-      const uint32_t pa = tmem + (uint32_t)(x * kPrBKV);
-      const uint32_t o = tmem + C::kOCol + (uint32_t)(x * 128);
-#pragma unroll
-      for (int v = 0; v < 2; ++v) {
-        const uint64_t vd = desc_kmajor_sw128(slot_addr(j * C::kBoxes + C::kQAtoms + v));
-#pragma unroll
-        for (int k = 0; k < 4; ++k)
-          mma_ts_elect(o, pa + (uint32_t)((v * 4 + k) * 8), desc_advance(vd, k * 32), idesc_o, (j | v | k) != 0);
-      }
-      mma_commit_elect(&bars.pv_done[x]);
-      return true;
-    };
 
-    bool ok = mbar_wait_warp(&bars.q_ready[0], 0, abort_flag);
-    if (ok && nB > 0) ok = mbar_wait_warp(&bars.q_ready[1], 0, abort_flag);
-    if (ok) ok = issue_s(0, 0);
-    if (ok && nB > 0) ok = issue_s(1, 0);
-    if (ok) mma_commit_elect(&bars.kempty[0]);
-    for (int j = 0; j < n && ok; ++j) {
-      const bool a_now = j < nA, b_now = j < nB, a_next = j + 1 < nA, b_next = j + 1 < nB;
-      if (a_now && !(ok = issue_pv(0, j))) break;
-      if (a_next && !(ok = issue_s(0, j + 1))) break;
-      if (b_now && !(ok = issue_pv(1, j))) break;
-      mma_commit_elect(&bars.vempty[j & 3]);                 // value group j released
-      if (b_next && !(ok = issue_s(1, j + 1))) break;
-      if (a_next || b_next) mma_commit_elect(&bars.kempty[(j + 1) & 3]);   // key group j + 1 released
+  if (warp < 4) {
+    warpgroup_reg_dec<kPrRegsCtl>();
+    if (warp == 0) {
+      // ---------------- producer ----------------
+      if (lane == 0) {
+        tma_prefetch_desc(&map_q);
+        tma_prefetch_desc(&map_kn);
+        tma_prefetch_desc(&map_kr);
+        tma_prefetch_desc(&map_vt);
+        // box gb of the ring sits in slot gb % S; before it is filled, the group
+        // that last used the slot (box gb - S) must have been released
+        auto wait_released = [&](int gp) -> bool {
+          const int jp = gp / C::kBoxes;
+          uint64_t* bar = (gp % C::kBoxes) < C::kQAtoms ? &bars.kempty[jp & 3] : &bars.vempty[jp & 3];
+          return mbar_wait(bar, (uint32_t)(jp >> 2) & 1u, abort_flag);
+        };
+        pdl_wait();   // k_nope, the values, k_rot and the schedule come from the previous kernels
+        bool ok = true;
+        int g = 0;                         // global key step
+        int gk = -1, gv = -1;              // last key / value group issued
+        int uq[2] = {0, 0};                // Q loads issued per tile
+        for (int k = 0; ok; ++k) {
+          const int s = k % kPrSched;
+          if (!(ok = mbar_wait(&bars.sched_empty[s], ((uint32_t)(k / kPrSched) & 1u) ^ 1u, abort_flag))) break;
+          const int item = atomicAdd(p.item_counter, 1);
+          const PairItem it = pair_item(p, item);
+          bars.sched_item[s] = it.valid ? item : -1;
+          mbar_arrive(&bars.sched_full[s]);
+          if (!it.valid) break;
+          auto load_q = [&](int x) -> bool {
+            if (uq[x] > 0 && !mbar_wait(&bars.q_free[x], (uint32_t)(uq[x] - 1) & 1u, abort_flag)) return false;
+            mbar_arrive_expect_tx(&bars.q_full[x], C::kQTileBytes);
+            for (int a = 0; a < C::kQAtoms; ++a)
+              tma_load_3d(sQ + x * C::kQTileBytes + a * kTile * 128, &map_q, &bars.q_full[x], a * 64, it.h,
+                          (int)(it.seq0 + it.q0 + x * kTile));
+            ++uq[x];
+            return true;
+          };
+          if (!(ok = load_q(0))) break;
+          for (int j = 0; j < it.n && ok; ++j, ++g) {
+            const int kv_row = it.kv_pad0 + j * kPrBKV;
+            const int g0 = g * C::kBoxes;
+            for (int i = 0; i < C::kQAtoms && ok; ++i)
+              if (g0 + i >= S) ok = wait_released(g0 + i - S);
+            if (!ok) break;
+            uint64_t* kb = &bars.kfull[g & 3];
+            mbar_arrive_expect_tx(kb, C::kQAtoms * kPrBKV * 128);
+            for (int i = 0; i < C::kKAtoms; ++i)
+              tma_load_2d(sRing + ((g0 + i) % S) * kPrSlotBytes, &map_kn, kb, i * 64, it.h * p.Tpad + kv_row);
+            tma_load_2d(sRing + ((g0 + C::kKAtoms) % S) * kPrSlotBytes, &map_kr, kb, 0, kv_row);
+            gk = g;
+            for (int v = 0; v < 2 && ok; ++v)
+              if (g0 + C::kQAtoms + v >= S) ok = wait_released(g0 + C::kQAtoms + v - S);
+            if (!ok) break;
+            uint64_t* vb = &bars.vfull[g & 3];
+            mbar_arrive_expect_tx(vb, 2 * C::kVBoxBytes);
+            for (int v = 0; v < 2; ++v)
+              tma_load_2d(sRing + ((g0 + C::kQAtoms + v) % S) * kPrSlotBytes, &map_vt, vb, kv_row + v * 64,
+                          it.h * kV);
+            gv = g;
+            // tile B's Q after the first step's keys and values, so that a
+            // wait for the previous item's last tile-B scores never holds up
+            // the keys tile A needs first
+            if (j == 0 && it.nB > 0 && !(ok = load_q(1))) break;
+          }
+        }
+        if (!ok) {   // let every copy already issued land before the CTA exits
+          for (int x = 0; x < 2; ++x)
+            if (uq[x] > 0) mbar_wait_drain(&bars.q_full[x], (uint32_t)(uq[x] - 1) & 1u);
+          for (int jj = (gk > 3 ? gk - 3 : 0); jj <= gk; ++jj)
+            mbar_wait_drain(&bars.kfull[jj & 3], (uint32_t)(jj >> 2) & 1u);
+          for (int jj = (gv > 3 ? gv - 3 : 0); jj <= gv; ++jj)
+            mbar_wait_drain(&bars.vfull[jj & 3], (uint32_t)(jj >> 2) & 1u);
+        }
+      }
+    } else if (warp == 1) {
+      // ---------------- MMA issuer (whole warp; one elected lane issues) ----------------
+      const uint32_t idesc_s = idesc_f16_f32(kTile, kPrBKV);
+      const uint32_t idesc_o = idesc_f16_f32(kTile, kV);
+      const uint32_t ring0 = smem_u32(sRing), q0addr = smem_u32(sQ);
+      auto slot_addr = [&](int gb) -> uint32_t { return ring0 + (uint32_t)(gb % S) * kPrSlotBytes; };
+      int k_seen = -1, v_seen = -1;       // last global step whose key / value group was waited for
+      int uq[2] = {0, 0};                 // Q uses per tile (q_ready phases)
+      int uo[2] = {0, 0};                 // items per tile whose P V has started (o_free phases)
+      int ts[2] = {0, 0};                 // tile-steps per tile (p_full phases)
+      // S_x(step g) = Q_x K_g^T over all D columns
+      auto issue_s = [&](int x, int g) -> bool {
+        if (k_seen < g) {
+          if (!mbar_wait_warp(&bars.kfull[g & 3], (uint32_t)(g >> 2) & 1u, abort_flag)) return false;
+          k_seen = g;
+        }
+        tc_fence_after();
+        const uint32_t d = tmem + (uint32_t)(x * kPrBKV);
+  #pragma unroll 1
+        for (int a = 0; a < C::kQAtoms; ++a) {
+          const uint64_t qd = desc_kmajor_sw128(q0addr + (uint32_t)(x * C::kQTileBytes + a * kTile * 128));
+          const uint64_t kd = desc_kmajor_sw128(slot_addr(g * C::kBoxes + a));
+  #pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_ss_elect(d, desc_advance(qd, k * 32), desc_advance(kd, k * 32), idesc_s, (a | k) != 0);
+        }
+        mma_commit_elect(&bars.s_full[x]);
+        return true;
+      };
+      // first S of tile x in a new item: its Q must be converted
+      auto issue_s_first = [&](int x, int g, int nx) -> bool {
+        if (!mbar_wait_warp(&bars.q_ready[x], (uint32_t)uq[x] & 1u, abort_flag)) return false;
+        ++uq[x];
+        if (!issue_s(x, g)) return false;
+        if (nx == 1) mma_commit_elect(&bars.q_free[x]);
+        return true;
+      };
+      // O_x (+)= P_x(step g) V_g, P_x read from TMEM; `first`: the item's first step
+      auto issue_pv = [&](int x, int g, bool first) -> bool {
+        if (v_seen < g) {
+          if (!mbar_wait_warp(&bars.vfull[g & 3], (uint32_t)(g >> 2) & 1u, abort_flag)) return false;
+          v_seen = g;
+        }
+        if (first) {
+          if (uo[x] > 0 && !mbar_wait_warp(&bars.o_free[x], (uint32_t)(uo[x] - 1) & 1u, abort_flag)) return false;
+          ++uo[x];
+        }
+        if (!mbar_wait_warp(&bars.p_full[x], (uint32_t)ts[x] & 1u, abort_flag)) return false;
+        ++ts[x];
+        tc_fence_after();
+        const uint32_t pa = tmem + (uint32_t)(x * kPrBKV);
+        const uint32_t o = tmem + C::kOCol + (uint32_t)(x * 128);
+  #pragma unroll 1
+        for (int v = 0; v < 2; ++v) {
+          const uint64_t vd = desc_kmajor_sw128(slot_addr(g * C::kBoxes + C::kQAtoms + v));
+  #pragma unroll
+          for (int k = 0; k < 4; ++k)
+            mma_ts_elect(o, pa + (uint32_t)((v * 4 + k) * 8), desc_advance(vd, k * 32), idesc_o,
+                         (!first || (v | k) != 0) ? 1u : 0u);
+        }
+        mma_commit_elect(&bars.pv_done[x]);
+        return true;
+      };
+
+      // the MMA warp needs only the step counts of an item
+      struct Steps { int valid, nA, nB, n; };
+      auto read_steps = [&](int k, Steps& st) -> bool {
+        PairItem it;
+        if (!pair_read_item(bars, p, k, lane, abort_flag, it)) return false;
+        st.valid = it.valid; st.nA = it.nA; st.nB = it.nB; st.n = it.n;
+        return true;
+      };
+      int kread = 0;
+      Steps cur;
+      bool ok = read_steps(kread++, cur);
+      int g = 0;                          // global step of cur's first key step
+      if (ok && cur.valid) {
+        ok = issue_s_first(0, 0, cur.nA);
+        if (ok && cur.nB > 0) ok = issue_s_first(1, 0, cur.nB);
+        if (ok) mma_commit_elect(&bars.kempty[0]);
+      }
+      while (ok && cur.valid) {
+        Steps nxt;
+        nxt.valid = 0; nxt.nA = nxt.nB = nxt.n = 0;
+        for (int j = 0; j < cur.n && ok; ++j) {
+          const int gs = g + j;
+          const bool last = j == cur.n - 1;
+          if (last && !(ok = read_steps(kread++, nxt))) break;
+          if (j < cur.nA && !(ok = issue_pv(0, gs, j == 0))) break;
+          if (!last) {
+            if (j + 1 < cur.nA) {
+              if (!(ok = issue_s(0, gs + 1))) break;
+              if (j + 1 == cur.nA - 1) mma_commit_elect(&bars.q_free[0]);
+            }
+          } else if (nxt.valid && !(ok = issue_s_first(0, gs + 1, nxt.nA))) {
+            break;
+          }
+          if (j < cur.nB && !(ok = issue_pv(1, gs, j == 0))) break;
+          mma_commit_elect(&bars.vempty[gs & 3]);                 // value group gs released
+          if (!last) {
+            if (j + 1 < cur.nB) {
+              if (!(ok = issue_s(1, gs + 1))) break;
+              if (j + 1 == cur.nB - 1) mma_commit_elect(&bars.q_free[1]);
+            }
+          } else if (nxt.valid && nxt.nB > 0 && !(ok = issue_s_first(1, gs + 1, nxt.nB))) {
+            break;
+          }
+          if (!last || nxt.valid) mma_commit_elect(&bars.kempty[(gs + 1) & 3]);   // key group gs + 1 released
+        }
+        g += cur.n;
+        cur = nxt;
+      }
+      mma_commit_elect(&bars.mma_done);     // every MMA done before TMEM is freed
+      if (lane == 0) mbar_wait_drain(&bars.mma_done, 0);
+      __syncwarp();
     }
-    mma_commit_elect(&bars.mma_done);     // every MMA done before TMEM is freed
-    if (lane == 0) mbar_wait_drain(&bars.mma_done, 0);
-    __syncwarp();
   } else {
-    // ---------------- softmax and epilogue (warps 2-5: tile A, 6-9: tile B) ----------------
-    const int x = (warp - 2) >> 2;
-    const int nX = x ? nB : nA;
+    warpgroup_reg_inc<kPrRegsSoftmax>();
+    // ---------------- softmax and epilogue (warps 4-7: tile A, 8-11: tile B) ----------------
+    const int x = (warp - 4) >> 2;
     const int grp = warp & 3;                     // TMEM lane quadrant of this warp
     const int row = grp * 32 + lane;
     const uint32_t lane_base = (uint32_t)(grp * 32) << 16;
-    const int qrow = q0 + x * kTile + row;        // in-sequence query index
-    const bool valid = qrow < L;
-    const int qi = min(qrow, L - 1);
-    const int64_t t = seq0 + qrow;
-    bool ok = nX > 0;
-    if (ok) ok = mbar_wait_warp(&bars.q_full, 0, abort_flag);
-    if (ok) {
-      // this row of q: bf16 -> fp16 in place (per atom: all loads, the
-      // conversion, then all stores); the rotary atom is rotated at the
-      // token's position, its 32 pairs in two halves of 16
-      uint8_t* sQx = sQ + x * C::kQTileBytes;
+    const uint32_t tS = tmem + lane_base + (uint32_t)(x * kPrBKV);
+    const uint32_t tO = tmem + lane_base + C::kOCol + (uint32_t)(x * 128);
+    const float sl = p.scale_log2;
+    uint8_t* sQx = sQ + x * C::kQTileBytes;
+    int kread = 0;
+    int uq = 0;                                   // items of this tile (q_full phases)
+    int ts = 0;                                   // tile-steps (s_full / pv_done phases)
+    // next item in which this tile has rows
+    auto next_item = [&](PairItem& it) -> bool {
+      for (;;) {
+        if (!pair_read_item(bars, p, kread++, lane, abort_flag, it)) return false;
+        if (!it.valid || (x ? it.nB : it.nA) > 0) return true;
+      }
+    };
+    // this row of the item's Q: bf16 -> fp16 in place (per atom: all loads,
+    // the conversion, then all stores); the rotary atom is rotated at the
+    // token's position, its 32 pairs in two halves of 16
+    auto prep_q = [&](const PairItem& it) -> bool {
+      if (!mbar_wait_warp(&bars.q_full[x], (uint32_t)uq & 1u, abort_flag)) return false;
+      ++uq;
+      const int qrow = it.q0 + x * kTile + row;
+      const bool valid = qrow < it.L;
+      const int64_t t = it.seq0 + qrow;
       float qmax = 0.f;
 #pragma unroll 1
       for (int a = 0; a < C::kQAtoms - 1; ++a) {
@@ -344,93 +542,137 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
       if (valid && !(qmax <= kF16Max)) raise_device_error(kDevErrRange);
       fence_proxy_async_smem();
       mbar_arrive(&bars.q_ready[x]);
-    }
+      return true;
+    };
 
-    const uint32_t tS = tmem + lane_base + (uint32_t)(x * kPrBKV);
-    const uint32_t tO = tmem + lane_base + C::kOCol + (uint32_t)(x * 128);
-    const float sl = p.scale_log2;
-    float m = 0.f;            // reference max (log2 units, scaled)
-    float l = 0.f;            // running sum of the weights at that reference
-    for (int j = 0; j < nX && ok; ++j) {
-      if (!mbar_wait_warp(&bars.s_full[x], (uint32_t)j & 1u, abort_flag)) { ok = false; break; }
-      tc_fence_after();
-      // the row's 128 scores: four loads in flight, one wait
-      float sc[kPrBKV];
-      {
-        uint32_t v[kPrBKV];
-#pragma unroll
-        for (int c = 0; c < kPrBKV / 32; ++c) tmem_ld32_nowait(tS + (uint32_t)(c * 32), v + c * 32);
-        tmem_wait_ld128(v);
-#pragma unroll
-        for (int e = 0; e < kPrBKV; ++e) sc[e] = __uint_as_float(v[e]);
-      }
-      if (j == nX - 1) {        // the diagonal step: causal mask (also masks padded keys)
-        const int lim = qi - j * kPrBKV;
-#pragma unroll
-        for (int e = 0; e < kPrBKV; ++e)
-          if (e > lim) sc[e] = -INFINITY;
-      }
-      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
-#pragma unroll
-      for (int e = 0; e < kPrBKV; ++e) mx4[e & 3] = fmaxf(mx4[e & 3], sc[e]);
-      const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])) * sl;
-      bool raise = false;
-      if (j == 0) m = mx;
-      else raise = mx > m + kPrLazy;
-      if (__any_sync(0xffffffffu, raise)) {
-        // rare: raise the reference; O must hold P V of every earlier step first
-        if (!mbar_wait_warp(&bars.pv_done[x], (uint32_t)(j - 1) & 1u, abort_flag)) { ok = false; break; }
+    PairItem cur;
+    bool ok = next_item(cur);
+    if (ok && cur.valid) ok = prep_q(cur);
+    while (ok && cur.valid) {
+      const int nX = x ? cur.nB : cur.nA;
+      const int qrow = cur.q0 + x * kTile + row;  // in-sequence query index
+      const bool valid = qrow < cur.L;
+      const int qi = min(qrow, cur.L - 1);
+      const int lim_row = cur.off + qi;             // last key this row attends
+      // steps from jm on reach past the tile's first row's last key: the
+      // causal mask applies there (one step without cached rows; with an
+      // offset that is not a multiple of 128, two)
+      const int jm = (cur.off + cur.q0 + x * kTile) / kPrBKV;
+      const int64_t t = cur.seq0 + qrow;
+      float m = 0.f;                              // reference max (log2 units, scaled)
+      uint64_t l2[2] = {0ull, 0ull};              // row sum of e, as two fp32 pairs
+      for (int j = 0; j < nX && ok; ++j) {
+        if (!mbar_wait_warp(&bars.s_full[x], (uint32_t)ts & 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        const float alpha = raise ? ex2_approx(m - mx) : 1.f;
-        if (raise) { m = mx; l *= alpha; }
-        for (int c = 0; c < kV / 16; ++c) {
-          uint32_t v[16];
-          const uint32_t ta = tO + (uint32_t)(c * 16);
-          tmem_ld16(ta, v);
+        // the row's 128 scores: four loads in flight, one wait
+        float sc[kPrBKV];
+        {
+          uint32_t v[kPrBKV];
 #pragma unroll
-          for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
-          tmem_st16(ta, v);
+          for (int c = 0; c < kPrBKV / 32; ++c) tmem_ld32_nowait(tS + (uint32_t)(c * 32), v + c * 32);
+          tmem_wait_ld128(v);
+#pragma unroll
+          for (int e = 0; e < kPrBKV; ++e) sc[e] = __uint_as_float(v[e]);
         }
-      }
-      // P = 2^(s scale log2(e) - m) in fp32, packed to fp16; the row sum adds
-      // the fp32 weights before their rounding to fp16.
-      float rs4[4] = {0.f, 0.f, 0.f, 0.f};
+        if (j >= jm) {            // the diagonal steps: causal mask (also masks padded keys)
+          const int lim = lim_row - j * kPrBKV;
 #pragma unroll
-      for (int c = 0; c < kPrBKV / 32; ++c) {
-        uint32_t pk[16];
-#pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float a0 = fmaf(sc[c * 32 + 2 * e], sl, -m);
-          const float a1 = fmaf(sc[c * 32 + 2 * e + 1], sl, -m);
-          const float p0 = ex2_approx(a0), p1 = ex2_approx(a1);
-          rs4[e & 3] += p0 + p1;
-          pk[e] = pack_f16x2(p0, p1);
+          for (int e = 0; e < kPrBKV; ++e)
+            if (e > lim) sc[e] = -INFINITY;
         }
-        tmem_st16(tS + (uint32_t)(c * 16), pk);
+        float mx4[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          float a = fmax3(sc[32 * q], sc[32 * q + 1], sc[32 * q + 2]);
+#pragma unroll
+          for (int e = 3; e + 1 < 32; e += 2) a = fmax3(a, sc[32 * q + e], sc[32 * q + e + 1]);
+          mx4[q] = fmaxf(a, sc[32 * q + 31]);
+        }
+        const float mx = fmaxf(fmax3(mx4[0], mx4[1], mx4[2]), mx4[3]) * sl;
+        bool raise = false;
+        if (j == 0) m = mx;
+        else raise = mx > m + kPrLazy;
+        if (__any_sync(0xffffffffu, raise)) {
+          // rare: raise the reference; O must hold P V of every earlier step first
+          if (!mbar_wait_warp(&bars.pv_done[x], (uint32_t)(ts - 1) & 1u, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          const float alpha = raise ? ex2_approx(m - mx) : 1.f;
+          if (raise) {
+            m = mx;
+            const uint64_t a2 = f2_make(alpha, alpha);
+            l2[0] = f2_mul(l2[0], a2);
+            l2[1] = f2_mul(l2[1], a2);
+          }
+          for (int c = 0; c < kV / 16; ++c) {
+            uint32_t v[16];
+            const uint32_t ta = tO + (uint32_t)(c * 16);
+            tmem_ld16(ta, v);
+#pragma unroll
+            for (int e = 0; e < 16; ++e) v[e] = __float_as_uint(__uint_as_float(v[e]) * alpha);
+            tmem_st16(ta, v);
+          }
+        }
+        // e = 2^(s scale log2(e) - m - bias) in fp32; P's fp16 codes from e 2^-12
+        const uint64_t sl2 = f2_make(sl, sl);
+        const float nb = -(m + kPrBias);
+        const uint64_t nb2 = f2_make(nb, nb);
+        const uint64_t k12 = f2_make(kPrTwoM12, kPrTwoM12);
+#pragma unroll
+        for (int c = 0; c < kPrBKV / 32; ++c) {
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const uint64_t a = f2_fma(f2_make(sc[c * 32 + 2 * e], sc[c * 32 + 2 * e + 1]), sl2, nb2);
+            uint64_t w;
+            if (c >= kPrBKV / 32 - kPrPolyChunks) {
+              w = ex2_fma2(a);
+            } else {
+              float a0, a1;
+              f2_split(a, a0, a1);
+              w = f2_make(ex2_approx(a0), ex2_approx(a1));
+            }
+            l2[e & 1] = f2_add(l2[e & 1], w);
+            float v0, v1;
+            f2_split(f2_mul(w, k12), v0, v1);
+            pk[e] = f16x2_from_scaled(v0, v1);
+          }
+          tmem_st16(tS + (uint32_t)(c * 16), pk);
+        }
+        tmem_st_wait();
+        tc_fence_before();
+        mbar_arrive(&bars.p_full[x]);
+        ++ts;
       }
-      l += (rs4[0] + rs4[1]) + (rs4[2] + rs4[3]);
-      tmem_st_wait();
-      tc_fence_before();
-      mbar_arrive(&bars.p_full[x]);
-    }
-    if (ok && nX > 0) ok = mbar_wait_warp(&bars.pv_done[x], (uint32_t)(nX - 1) & 1u, abort_flag);
-    if (ok && nX > 0) {
+      if (!ok) break;
+      // the next item's Q first (its first score product can start), then
+      // this item's output
+      PairItem nxt;
+      if (!(ok = next_item(nxt))) break;
+      if (nxt.valid && !(ok = prep_q(nxt))) break;
+      if (!(ok = mbar_wait_warp(&bars.pv_done[x], (uint32_t)(ts - 1) & 1u, abort_flag))) break;
       tc_fence_after();
-      const float inv = 1.f / l;
-      __nv_bfloat16* dst = p.out + (t * p.H + h) * kV;
-      for (int c = 0; c < kV / 16; ++c) {
-        uint32_t v[16];
-        tmem_ld16(tO + (uint32_t)(c * 16), v);
+      float la, lb, lc, ld;
+      f2_split(l2[0], la, lb);
+      f2_split(l2[1], lc, ld);
+      const float inv = (1.f / ((la + lb) + (lc + ld))) * kPrTwoMBias;
+      __nv_bfloat16* dst = p.out + (t * p.H + cur.h) * kV;
+#pragma unroll 1
+      for (int c = 0; c < kV / 32; ++c) {
+        uint32_t v[32];
+        tmem_ld32(tO + (uint32_t)(c * 32), v);
         if (valid) {
-          uint32_t o[8];
+          uint32_t o[16];
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
+          for (int e = 0; e < 16; ++e)
             o[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * inv, __uint_as_float(v[2 * e + 1]) * inv);
-          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 16);
-          d4[0] = make_uint4(o[0], o[1], o[2], o[3]);
-          d4[1] = make_uint4(o[4], o[5], o[6], o[7]);
+          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
+#pragma unroll
+          for (int e = 0; e < 4; ++e) d4[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
         }
       }
+      tc_fence_before();
+      mbar_arrive(&bars.o_free[x]);
+      cur = nxt;
     }
   }
   tc_fence_before();

@@ -627,7 +627,9 @@ decode_combine_kernel(const float* __restrict__ o_part, const float* __restrict_
 //   kAMN = false: A is read K-major (the weight stored [n][k]: W_UV_h), its box
 //                 [128 n x 64 k] per K chunk.
 // Bm comes through a 3D map {K, H, B} as [64 b x 64 k] boxes. The output row
-// of b is out[b * out_bs + h * out_hs + n] (bf16).
+// of b is out[b * out_bs + h * out_hs + n]: bf16, or fp32 into out_f32 when
+// that is set (the Linears whose result feeds an RMSNorm). kF16: both
+// operands fp16 instead of bf16.
 constexpr int kHgStages = 4;
 constexpr int kHgABytes = 128 * 128;            // 128 n x 64 k bf16
 constexpr int kHgBBytes = 64 * 128;             // 64 b x 64 k bf16
@@ -635,6 +637,7 @@ constexpr size_t kHgSmem = (size_t)kHgStages * (kHgABytes + kHgBBytes) + 1024;
 
 struct HgParams {
   __nv_bfloat16* out;
+  float* out_f32;        // when set: fp32 results here instead of `out`
   int64_t out_bs, out_hs;
   int B, Nout, K;
   int a_row0;            // first weight row of head h: a_row0 + h * a_hstride
@@ -655,7 +658,7 @@ struct HgParams {
   int64_t* meta;
 };
 
-template <bool kAMN>
+template <bool kAMN, bool kF16 = false>
 __global__ void __launch_bounds__(192, 1)
 head_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b, HgParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -663,7 +666,6 @@ head_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
   __shared__ uint32_t tmem_base;
   __shared__ int abort_flag;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (!kAMN) pdl_wait();   // un-absorption: o_lat comes from the previous kernel
   pdl_allow_next();
   const int h = blockIdx.x, n0 = blockIdx.y * 128, b0 = blockIdx.z * 64;
   if (kAMN && h == (int)gridDim.x - 1) {   // the extra CTA column (uniform over the CTA)
@@ -691,16 +693,31 @@ head_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     if (lane == 0) {
       int kc = 0;
       bool ok = true;
-      for (; kc < nk; ++kc) {
-        const int s = kc % kHgStages;
-        if (!mbar_wait(&empty[s], ((uint32_t)(kc / kHgStages) & 1u) ^ 1u, &abort_flag)) { ok = false; break; }
-        mbar_arrive_expect_tx(&full[s], kHgABytes + kHgBBytes);
+      auto load_a = [&](int k, int s) {
         uint8_t* a = sA + s * kHgABytes;
         if (kAMN) {   // rows k, columns n: two [64 k x 64 n] boxes
-          tma_load_2d(a, &map_a, &full[s], n0, arow + kc * 64);
-          tma_load_2d(a + kHgABytes / 2, &map_a, &full[s], n0 + 64, arow + kc * 64);
+          tma_load_2d(a, &map_a, &full[s], n0, arow + k * 64);
+          tma_load_2d(a + kHgABytes / 2, &map_a, &full[s], n0 + 64, arow + k * 64);
         } else {      // rows n, columns k: one [128 n x 64 k] box
-          tma_load_2d(a, &map_a, &full[s], kc * 64, arow + n0);
+          tma_load_2d(a, &map_a, &full[s], k * 64, arow + n0);
+        }
+      };
+      // un-absorption: the weight halves of the first stages do not depend on
+      // the previous kernel (o_lat does), so they load before the wait. (A
+      // launch with programmatic serialization must therefore never follow
+      // a kernel that writes the weight; the Linears launch the plain way.)
+      const int npre = kAMN ? 0 : min(nk, kHgStages);
+      for (int k = 0; k < npre; ++k) {
+        mbar_arrive_expect_tx(&full[k], kHgABytes + kHgBBytes);
+        load_a(k, k);
+      }
+      if (!kAMN) pdl_wait();
+      for (; kc < nk; ++kc) {
+        const int s = kc % kHgStages;
+        if (kc >= npre) {
+          if (!mbar_wait(&empty[s], ((uint32_t)(kc / kHgStages) & 1u) ^ 1u, &abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&full[s], kHgABytes + kHgBBytes);
+          load_a(kc, s);
         }
         tma_load_3d(sB + s * kHgBBytes, &map_b, &full[s], kc * 64, h, b0);
       }
@@ -710,7 +727,7 @@ head_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     }
   } else if (warp == 1) {
     // MMA issuer: whole warp, one elected lane issues
-    const uint32_t idesc = idesc_bf16_f32(128, 64) | (kAMN ? kIdescAMajorMN : 0u);
+    const uint32_t idesc = (kF16 ? idesc_f16_f32(128, 64) : idesc_bf16_f32(128, 64)) | (kAMN ? kIdescAMajorMN : 0u);
     for (int kc = 0; kc < nk; ++kc) {
       const int s = kc % kHgStages;
       if (!mbar_wait_warp(&full[s], (uint32_t)(kc / kHgStages) & 1u, &abort_flag)) break;
@@ -739,7 +756,11 @@ head_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int b = b0 + cc * 16 + e;
-            if (b < p.B) p.out[(int64_t)b * p.out_bs + (int64_t)h * p.out_hs + n] = __float2bfloat16_rn(__uint_as_float(v[e]));
+            const int64_t o = (int64_t)b * p.out_bs + (int64_t)h * p.out_hs + n;
+            if (b < p.B) {
+              if (p.out_f32) p.out_f32[o] = __uint_as_float(v[e]);
+              else p.out[o] = __float2bfloat16_rn(__uint_as_float(v[e]));
+            }
           }
         }
       }

@@ -36,7 +36,8 @@ constexpr int kTile = 128;            // token rows per tile (M of the MMAs)
 // pair_order[j]: the first tile of each 256-row block (tiles 2k and 2k + 1 of
 // one sequence; the second may not exist), blocks sorted by decreasing k.
 // Entries past the real tile / block count are -1. Bad cu_seqlens set the
-// device error word and leave every entry at -1.
+// device error word and leave every entry at -1. item_counter (the two-tile
+// attention's work counter) is reset to 0.
 // Inclusive prefix sum over the 1024 threads of a block (thread order):
 // a shuffle scan inside each warp, then one over the 32 warp totals.
 // Every thread of the block must call it.
@@ -64,7 +65,8 @@ __device__ __forceinline__ int block_inclusive_scan_1024(int v, int* s_warp /* [
 __device__ __forceinline__ void schedule_block(const int32_t* __restrict__ cu, int nseq, int64_t Ttot,
                                                int max_seqlen, int cap, int32_t* __restrict__ seq_tile0,
                                                int32_t* __restrict__ tile_seq, int32_t* __restrict__ tile_q0,
-                                               int32_t* __restrict__ order, int32_t* __restrict__ pair_order) {
+                                               int32_t* __restrict__ order, int32_t* __restrict__ pair_order,
+                                               int32_t* __restrict__ item_counter) {
   constexpr int kBuckets = 2048;   // = 2 * blockDim.x (launched with 1024 threads)
   __shared__ int s_bad;
   __shared__ int s_carry;
@@ -72,7 +74,7 @@ __device__ __forceinline__ void schedule_block(const int32_t* __restrict__ cu, i
   __shared__ int s_cnt[kBuckets];
   __shared__ int s_off[kBuckets];
   const int tid = threadIdx.x;
-  if (tid == 0) { s_bad = 0; s_carry = 0; }
+  if (tid == 0) { s_bad = 0; s_carry = 0; *item_counter = 0; }
   for (int i = tid; i < cap; i += blockDim.x) {
     tile_seq[i] = -1; tile_q0[i] = -1; order[i] = -1; pair_order[i] = -1;
   }
@@ -162,16 +164,48 @@ __device__ __forceinline__ void schedule_block(const int32_t* __restrict__ cu, i
 // beyond the fp16 range sets the device error word.
 constexpr int kPrepThreads = 1024;
 constexpr int kPrepUnroll = 8;
+
+// Block `blk` of the fp16 weight copy: kPrepUnroll x 8 values per thread
+// (n8 groups of 8 values in all). A value beyond the fp16 range sets the
+// device error word.
+__device__ __forceinline__ void weight_f16_block(const __nv_bfloat16* __restrict__ w, __half* __restrict__ w16,
+                                                 int64_t n8, int64_t blk) {
+  const int64_t base = blk * kPrepThreads * kPrepUnroll + threadIdx.x;
+  uint4 v[kPrepUnroll];
+#pragma unroll
+  for (int u = 0; u < kPrepUnroll; ++u) {
+    const int64_t i = base + (int64_t)u * kPrepThreads;
+    if (i < n8) v[u] = reinterpret_cast<const uint4*>(w)[i];
+  }
+  float mx = 0.f;
+#pragma unroll
+  for (int u = 0; u < kPrepUnroll; ++u) {
+    const int64_t i = base + (int64_t)u * kPrepThreads;
+    if (i >= n8) break;
+    const uint32_t in[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+    uint32_t o[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      const float2 f = unpack_bf16x2(in[e]);
+      mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
+      o[e] = pack_f16x2(f.x, f.y);
+    }
+    reinterpret_cast<uint4*>(w16)[i] = make_uint4(o[0], o[1], o[2], o[3]);
+  }
+  if (!(mx <= kF16Max)) raise_device_error(kDevErrRange);
+}
 __global__ void __launch_bounds__(kPrepThreads)
 prefill_prep_kernel(const int32_t* __restrict__ cu, int nseq, int64_t Ttot, int max_seqlen, int cap,
                     int32_t* __restrict__ seq_tile0, int32_t* __restrict__ tile_seq,
                     int32_t* __restrict__ tile_q0, int32_t* __restrict__ order, int32_t* __restrict__ pair_order,
+                    int32_t* __restrict__ item_counter,
                     const __nv_bfloat16* __restrict__ w, __half* __restrict__ w16, int64_t n8, int w_blocks,
                     const __nv_bfloat16* __restrict__ latent, const __nv_bfloat16* __restrict__ w_norm, int R,
                     float eps, __half* __restrict__ c16) {
   pdl_allow_next();
   if (blockIdx.x == 0) {
-    schedule_block(cu, nseq, Ttot, max_seqlen, cap, seq_tile0, tile_seq, tile_q0, order, pair_order);
+    schedule_block(cu, nseq, Ttot, max_seqlen, cap, seq_tile0, tile_seq, tile_q0, order, pair_order,
+                   item_counter);
     return;
   }
   if ((int)blockIdx.x > w_blocks) {
@@ -226,29 +260,14 @@ prefill_prep_kernel(const int32_t* __restrict__ cu, int nseq, int64_t Ttot, int 
     if (!(mx <= kF16Max)) raise_device_error(kDevErrRange);
     return;
   }
-  const int64_t base = (int64_t)(blockIdx.x - 1) * kPrepThreads * kPrepUnroll + threadIdx.x;
-  uint4 v[kPrepUnroll];
-#pragma unroll
-  for (int u = 0; u < kPrepUnroll; ++u) {
-    const int64_t i = base + (int64_t)u * kPrepThreads;
-    if (i < n8) v[u] = reinterpret_cast<const uint4*>(w)[i];
-  }
-  float mx = 0.f;
-#pragma unroll
-  for (int u = 0; u < kPrepUnroll; ++u) {
-    const int64_t i = base + (int64_t)u * kPrepThreads;
-    if (i >= n8) break;
-    const uint32_t in[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-    uint32_t o[4];
-#pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const float2 f = unpack_bf16x2(in[e]);
-      mx = fmaxf(mx, fmaxf(fabsf(f.x), fabsf(f.y)));
-      o[e] = pack_f16x2(f.x, f.y);
-    }
-    reinterpret_cast<uint4*>(w16)[i] = make_uint4(o[0], o[1], o[2], o[3]);
-  }
-  if (!(mx <= kF16Max)) raise_device_error(kDevErrRange);
+  weight_f16_block(w, w16, n8, (int64_t)(blockIdx.x - 1));
+}
+
+// The fp16 copy of kv_b_proj on its own (mla_prepare_kv_b_proj), one block
+// per kPrepThreads x kPrepUnroll groups of 8 values.
+__global__ void __launch_bounds__(kPrepThreads)
+weight_f16_kernel(const __nv_bfloat16* __restrict__ w, __half* __restrict__ w16, int64_t n8) {
+  weight_f16_block(w, w16, n8, (int64_t)blockIdx.x);
 }
 
 // ---- fused RMSNorm + kv_b_proj GEMM ------------------------------------------
@@ -278,6 +297,10 @@ struct GemmParams {
   int tiles_per_cta;             // n tiles (256 columns) per CTA
   int max_pos, interleaved;
   float eps;
+  // transposed-value GEMM over cached rows (the eager chunk form): c_hat is
+  // already in the padded layout (tile t = rows 128 t ..) and k_rot has been
+  // written with it, so the tile's A rows are padded rows and k_rot is left
+  int a_padded;
 };
 
 struct GemmBarriers {
@@ -578,8 +601,9 @@ norm_kvb_gemm_vt_kernel(const __grid_constant__ CUtensorMap map_chat, const __gr
       tma_prefetch_desc(&map_chat);
       tma_prefetch_desc(&map_w);
       mbar_arrive_expect_tx(&bars.a_full, natoms * kAtomBytes);
+      const int arow = p.a_padded ? tp0 : (int)(seq0 + q0);
       for (int a = 0; a < natoms; ++a)
-        tma_load_2d(sA + a * kAtomBytes, &map_chat, &bars.a_full, a * 64, (int)(seq0 + q0));
+        tma_load_2d(sA + a * kAtomBytes, &map_chat, &bars.a_full, a * 64, arow);
       int it = 0;
       bool ok = true;
       for (int h = h_begin; h < h_end && ok; ++h) {
@@ -642,7 +666,7 @@ norm_kvb_gemm_vt_kernel(const __grid_constant__ CUtensorMap map_chat, const __gr
       // before the epilogue but pass the tile on
       if (ok) ok = mbar_wait_warp(&bars.a_full, 0, abort_flag);
       mbar_arrive(&bars.a_ready);
-    } else if (blockIdx.y == 0) {
+    } else if (blockIdx.y == 0 && !p.a_padded) {
       // rotated shared key of token row lrow (one CTA column per tile writes
       // it); P = 64: the row's 64 values and its 32 cos / sin entries come in
       // as independent vector loads

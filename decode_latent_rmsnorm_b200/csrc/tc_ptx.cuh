@@ -28,6 +28,21 @@ __device__ __forceinline__ uint64_t global_timer_ns() {
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_allow_next() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
+// ---- per-warpgroup register budgets -----------------------------------------
+// Executed by all four warps of a warpgroup: lowers / raises the registers
+// per thread of that warpgroup. An increase waits until enough registers have
+// been released by decreases of other warpgroups of the CTA, so the budgets
+// of all warpgroups must add up to at most the registers the CTA was launched
+// with (threads x registers per thread).
+template <int kRegs>
+__device__ __forceinline__ void warpgroup_reg_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+template <int kRegs>
+__device__ __forceinline__ void warpgroup_reg_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegs));
+}
+
 // ---- mbarrier ---------------------------------------------------------------
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
@@ -60,20 +75,27 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 // soon as another thread of the CTA has aborted.
 constexpr uint64_t kWaitLimitNs = 2000000000ull;   // 2 s
 
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+// The wait with an explicit limit; mbar_wait is this helper at kWaitLimitNs
+// (a self-test runs it with a short limit on a barrier nothing arrives at).
+__device__ __forceinline__ bool mbar_wait_for(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                              uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((i & 127u) == 0) {
       if (*abort_flag) return false;
-      if (global_timer_ns() - t0 > kWaitLimitNs) {
+      if (global_timer_ns() - t0 > limit_ns) {
         *abort_flag = 1;
         raise_device_error(kDevErrTimeout);
         return false;
       }
     }
   }
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  return mbar_wait_for(bar, parity, abort_flag, kWaitLimitNs);
 }
 
 // Warp-uniform wait: every lane waits (bounded), then the warp votes, so a
@@ -338,6 +360,55 @@ constexpr float kF16Max = 65504.f;
 __device__ __forceinline__ float2 unpack_bf16x2(uint32_t v) {
   __nv_bfloat162 b = *reinterpret_cast<__nv_bfloat162*>(&v);
   return __bfloat1622float2(b);
+}
+
+// ---- packed fp32 pairs (sm_100: one instruction for two fp32 lanes) ----------
+// A pair travels as one 64-bit register (low word = first value).
+__device__ __forceinline__ uint64_t f2_make(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// Rounds to nearest and keeps subnormal results (no flush to zero).
+__device__ __forceinline__ uint64_t f2_mul(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// max(a, b, c) in one instruction.
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+
+// fp16 encoding of softmax weights without the conversion unit. The caller
+// passes v = w * 2^-112 (fp32, computed without flush to zero), where w is the
+// weight (0 <= w < 2^16). For such v the fp32 exponent field is the fp16
+// exponent field of w (bias 127 - 112 = 15), and fp32 subnormals map onto fp16
+// subnormals, so the fp16 bits of w are the fp32 bits of v shifted right by
+// 13, rounded to nearest (ties away from zero) by adding half of the dropped
+// range first. Two such codes are returned packed (lo in the low half).
+__device__ __forceinline__ uint32_t f16x2_from_scaled(float lo, float hi) {
+  // (bits + 2^12) << 3 keeps the wanted 16 bits in the upper half of each word
+  const uint32_t a = __float_as_uint(lo) * 8u + 0x8000u;
+  const uint32_t b = __float_as_uint(hi) * 8u + 0x8000u;
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, 0x7632;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
 }
 
 }  // namespace tc

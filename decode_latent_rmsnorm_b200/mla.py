@@ -38,8 +38,9 @@ SIGNATURES = {
     "mla_prefill_cached_workspace_size": (c_i32, [c_vp, c_i64, c_i32, ctypes.POINTER(c_sz)]),
     "mla_prefill_cached": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_i32, c_i64, c_vp, c_vp, c_i32,
                                    c_vp, c_vp, c_i32, c_vp, c_i64, c_vp, c_vp, c_sz, c_vp]),
+    "mla_kv_down_append_workspace_size": (c_i32, [c_vp, c_i64, ctypes.POINTER(c_sz)]),
     "mla_kv_down_append": (c_i32, [c_vp, c_i32, c_vp, c_vp, c_vp, c_vp, c_i64, c_vp, c_vp, c_i32, c_vp, c_vp,
-                                   c_i64, c_vp, c_vp]),
+                                   c_i64, c_vp, c_vp, c_sz, c_vp]),
     "mla_q_proj_workspace_size": (c_i32, [c_vp, c_i32, c_i64, ctypes.POINTER(c_sz)]),
     "mla_q_proj": (c_i32, [c_vp, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_i64, c_vp, c_vp, c_sz, c_vp]),
     "mla_o_proj": (c_i32, [c_vp, c_i32, c_vp, c_vp, c_i64, c_vp, c_vp]),
@@ -52,6 +53,15 @@ SIGNATURES = {
     "mla_recorded_kernel_name": (ctypes.c_char_p, [c_i32]),
     "mla_prefill_noalloc": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_i32, c_i32, c_i64,
                                     c_vp, c_vp, c_i32, c_vp, c_vp]),
+    "mla_kv_b_proj_prepared_size": (c_i32, [c_vp, ctypes.POINTER(c_sz)]),
+    "mla_prepare_kv_b_proj": (c_i32, [c_vp, c_vp, c_vp, c_sz, c_vp]),
+    "mla_prefill_prepared": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_i32, c_i32, c_i64,
+                                     c_vp, c_vp, c_i32, c_vp, c_vp, c_sz, c_vp]),
+    "mla_last_dispatch": (ctypes.c_char_p, []),
+    "mla_selftest_wait_timeout": (c_i32, [ctypes.c_uint32, c_vp, c_vp]),
+    "mla_prefill_cached_eager_workspace_size": (c_i32, [c_vp, c_i64, c_i32, c_i32, ctypes.POINTER(c_sz)]),
+    "mla_prefill_cached_form": (c_i32, [c_vp, c_vp, c_vp, c_vp, c_vp, c_vp, c_i32, c_i64, c_vp, c_vp, c_i32,
+                                        c_vp, c_vp, c_i32, c_vp, c_i64, c_vp, c_vp, c_sz, c_i32, c_vp]),
 }
 
 # Bytes of the static scratch behind mla_prefill_noalloc (MLA_NOALLOC_SCRATCH_BYTES).
@@ -176,6 +186,63 @@ def mla_prefill(dims: Dims, latent, q, w_kvb, w_norm, positions, cu_seqlens, max
     return out
 
 
+def mla_kv_b_proj_prepared_size(dims: Dims) -> int:
+    out = c_sz()
+    _check(load().mla_kv_b_proj_prepared_size(ctypes.byref(dims), ctypes.byref(out)))
+    return out.value
+
+
+def mla_prepare_kv_b_proj(dims: Dims, w_kvb, prepared=None):
+    """The prepared copy of kv_b_proj for mla_prefill_prepared (a uint8
+    device tensor; allocated if None). Done once per weight."""
+    H, R, N, V = dims.num_heads, dims.kv_lora_rank, dims.qk_nope, dims.v_head
+    n = mla_kv_b_proj_prepared_size(dims)
+    if prepared is None:
+        prepared = torch.empty(n, dtype=torch.uint8, device=w_kvb.device)
+    _check(load().mla_prepare_kv_b_proj(
+        ctypes.byref(dims), _dev(w_kvb, "w_kvb", dims.torch_dtype, (H * (N + V), R)), _dev(prepared, "prepared"),
+        prepared.numel() * prepared.element_size(), _stream()))
+    return prepared
+
+
+def mla_prefill_prepared(dims: Dims, latent, q, w_prepared, w_norm, positions, cu_seqlens, max_seqlen: int,
+                         cos, sin, out=None, workspace=None):
+    """mla_prefill with the kv_b_proj copy from mla_prepare_kv_b_proj."""
+    dt = dims.torch_dtype
+    H, R, N, P, V = dims.num_heads, dims.kv_lora_rank, dims.qk_nope, dims.qk_rope, dims.v_head
+    T = latent.shape[0]
+    nseq = cu_seqlens.numel() - 1
+    if out is None:
+        out = torch.empty((T, H, V), dtype=dt, device=latent.device)
+    if workspace is None:
+        workspace = torch.empty(max(mla_prefill_workspace_size(dims, T, nseq), 1), dtype=torch.uint8,
+                                device=latent.device)
+    if w_prepared.numel() * w_prepared.element_size() < mla_kv_b_proj_prepared_size(dims):
+        raise ValueError("w_prepared is smaller than mla_kv_b_proj_prepared_size")
+    _check(load().mla_prefill_prepared(
+        ctypes.byref(dims), _dev(latent, "latent", dt, (T, R + P)), _dev(q, "q", dt, (T, H, N + P)),
+        _dev(w_prepared, "w_prepared"), _dev(w_norm, "w_norm", dt, (R,)),
+        _dev(positions, "positions", torch.int32, (T,)), _dev(cu_seqlens, "cu_seqlens", torch.int32),
+        int(nseq), int(max_seqlen), int(T), _dev(cos, "cos", torch.float32),
+        _dev(sin, "sin", torch.float32), int(cos.shape[0]), _dev(out, "out", dt, (T, H, V)),
+        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream()))
+    return out
+
+
+def mla_selftest_wait_timeout(limit_us: int = 1000):
+    """Runs the bounded-wait self-test kernel; returns the device int32 flag
+    (1 once the wait has given up). Read the error word afterwards with
+    mla_check_device_status (it reports MLA_ERR_DEVICE_TIMEOUT)."""
+    flag = torch.full((1,), -1, dtype=torch.int32, device="cuda")
+    _check(load().mla_selftest_wait_timeout(int(limit_us), _dev(flag, "gave_up", torch.int32), _stream()))
+    return flag
+
+
+def mla_last_dispatch() -> str:
+    """Which kernels this thread's last prefill / decode call ran."""
+    return load().mla_last_dispatch().decode()
+
+
 def mla_prefill_noalloc(dims: Dims, latent, q, w_kvb, w_norm, positions, cu_seqlens, max_seqlen: int,
                         cos, sin, out):
     """mla_prefill without a workspace, for callers that cannot allocate
@@ -247,10 +314,23 @@ def mla_prefill_cached_workspace_size(dims: Dims, total_tokens: int, max_total_l
     return out.value
 
 
+def mla_prefill_cached_eager_workspace_size(dims: Dims, total_tokens: int, num_seqs: int, max_total_len: int) -> int:
+    out = c_sz()
+    _check(load().mla_prefill_cached_eager_workspace_size(ctypes.byref(dims), int(total_tokens), int(num_seqs),
+                                                          int(max_total_len), ctypes.byref(out)))
+    return out.value
+
+
+CHUNK_FORMS = {"auto": 0, "absorbed": 1, "eager": 2}
+
+
 def mla_prefill_cached(dims: Dims, latent, q, w_kvb, w_norm, cu_seqlens, cache_offsets, prefix_lens,
-                       max_total_len: int, cos, sin, cache, out=None, workspace=None):
+                       max_total_len: int, cos, sin, cache, out=None, workspace=None, form="auto"):
     """Chunks of new tokens continuing cached sequences: appends the chunk's
-    rows to ``cache`` and returns ``out`` [Tq, H, V] (allocated if None)."""
+    rows to ``cache`` and returns ``out`` [Tq, H, V] (allocated if None).
+    ``form``: "auto" (the library picks by chunk length), "absorbed" or
+    "eager". When ``workspace`` is None it is allocated for the forms the
+    call may take."""
     dt = dims.torch_dtype
     H, R, N, P, V = dims.num_heads, dims.kv_lora_rank, dims.qk_nope, dims.qk_rope, dims.v_head
     T = latent.shape[0]
@@ -258,11 +338,17 @@ def mla_prefill_cached(dims: Dims, latent, q, w_kvb, w_norm, cu_seqlens, cache_o
     if out is None:
         out = torch.empty((T, H, V), dtype=dt, device=latent.device)
     if workspace is None:
-        workspace = torch.empty(max(mla_prefill_cached_workspace_size(dims, T, max_total_len), 1),
-                                dtype=torch.uint8, device=latent.device)
+        n = mla_prefill_cached_workspace_size(dims, T, max_total_len)
+        if form == "eager" or (form == "auto" and nseq > 0 and T >= 128 * nseq):
+            try:
+                n = max(n, mla_prefill_cached_eager_workspace_size(dims, T, nseq, max_total_len))
+            except MlaError:
+                if form == "eager":
+                    raise
+        workspace = torch.empty(max(n, 1), dtype=torch.uint8, device=latent.device)
     if cache.dim() != 2 or cache.shape[1] != R + P:
         raise ValueError("cache must be [rows, R + P]")
-    _check(load().mla_prefill_cached(
+    _check(load().mla_prefill_cached_form(
         ctypes.byref(dims), _dev(latent, "latent", dt, (T, R + P)), _dev(q, "q", dt, (T, H, N + P)),
         _dev(w_kvb, "w_kvb", dt, (H * (N + V), R)), _dev(w_norm, "w_norm", dt, (R,)),
         _dev(cu_seqlens, "cu_seqlens", torch.int32), int(nseq), int(T),
@@ -270,12 +356,19 @@ def mla_prefill_cached(dims: Dims, latent, q, w_kvb, w_norm, cu_seqlens, cache_o
         _dev(prefix_lens, "prefix_lens", torch.int32, (nseq,)), int(max_total_len),
         _dev(cos, "cos", torch.float32), _dev(sin, "sin", torch.float32), int(cos.shape[0]),
         _dev(cache, "cache", dt), int(cache.shape[0]), _dev(out, "out", dt, (T, H, V)),
-        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), _stream()))
+        _dev(workspace, "workspace"), workspace.numel() * workspace.element_size(), CHUNK_FORMS[form],
+        _stream()))
     return out
 
 
+def mla_kv_down_append_workspace_size(dims: Dims, n: int) -> int:
+    out = c_sz()
+    _check(load().mla_kv_down_append_workspace_size(ctypes.byref(dims), int(n), ctypes.byref(out)))
+    return out.value
+
+
 def mla_kv_down_append(dims: Dims, hidden, w_kva, latent=None, w_norm=None, positions=None, cos=None, sin=None,
-                       cache=None, cache_rows=None):
+                       cache=None, cache_rows=None, workspace=None):
     """kv_a_proj_with_mqa: returns ``latent`` [n, R + P]; with ``cache`` and
     ``cache_rows`` also appends the normalized, rotated rows to the cache."""
     dt = dims.torch_dtype
@@ -283,6 +376,9 @@ def mla_kv_down_append(dims: Dims, hidden, w_kva, latent=None, w_norm=None, posi
     n, hid = hidden.shape
     if latent is None:
         latent = torch.empty((n, R + P), dtype=dt, device=hidden.device)
+    if workspace is None:
+        workspace = torch.empty(max(mla_kv_down_append_workspace_size(dims, n), 1), dtype=torch.uint8,
+                                device=hidden.device)
     append = cache is not None or cache_rows is not None
     if append:
         if cache is None or cache_rows is None or w_norm is None or positions is None or cos is None or sin is None:
@@ -297,7 +393,8 @@ def mla_kv_down_append(dims: Dims, hidden, w_kva, latent=None, w_norm=None, posi
         _dev(cos, "cos", torch.float32) if append else none, _dev(sin, "sin", torch.float32) if append else none,
         int(cos.shape[0]) if append else 0, _dev(latent, "latent", dt, (n, R + P)),
         _dev(cache, "cache", dt) if append else none, int(cache.shape[0]) if append else 0,
-        _dev(cache_rows, "cache_rows", torch.int64, (n,)) if append else none, _stream()))
+        _dev(cache_rows, "cache_rows", torch.int64, (n,)) if append else none, _dev(workspace, "workspace"),
+        workspace.numel() * workspace.element_size(), _stream()))
     return latent
 
 

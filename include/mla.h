@@ -124,6 +124,35 @@ int mla_prefill(const mla_dims* dims,
                 const float* cos_table, const float* sin_table, int32_t max_pos,
                 void* out, void* workspace, size_t workspace_bytes, cudaStream_t stream);
 
+/* kv_b_proj is a model constant, so its conversion for the tensor cores can
+ * be done once when the weights are loaded instead of inside every prefill.
+ * mla_kv_b_proj_prepared_size gives the bytes of the prepared copy for
+ * `dims`; mla_prepare_kv_b_proj writes it (device buffer owned by the caller,
+ * w_kvb as for mla_prefill). For the tensor-core head shapes (bf16, qk_rope =
+ * 64, qk_nope and v_head multiples of 64 with qk_nope + qk_rope <= 256,
+ * kv_lora_rank a multiple of 64 up to 512) the copy is w_kvb in fp16 (exact
+ * for weights in fp16's normal range; a weight beyond the fp16 range sets the
+ * device error word, MLA_ERR_INVALID_ARG at mla_check_device_status); for
+ * other shapes it is w_kvb itself. Both pointers 16-byte aligned for the
+ * tensor-core shapes (MLA_ERR_INVALID_ARG otherwise); a buffer smaller than
+ * the size returns MLA_ERR_WORKSPACE_TOO_SMALL. */
+int mla_kv_b_proj_prepared_size(const mla_dims* dims, size_t* bytes);
+int mla_prepare_kv_b_proj(const mla_dims* dims, const void* w_kvb, void* prepared,
+                          size_t prepared_bytes, cudaStream_t stream);
+
+/* mla_prefill with the prepared kv_b_proj (w_prepared, written by
+ * mla_prepare_kv_b_proj for the same dims) in place of w_kvb: the same
+ * kernels and the same results (bit for bit), minus the per-call conversion.
+ * For the tensor-core head shapes every tensor and the workspace must be
+ * 16-byte aligned (MLA_ERR_INVALID_ARG otherwise: this entry point has no
+ * fallback to the CUDA-core kernels for them). */
+int mla_prefill_prepared(const mla_dims* dims,
+                         const void* latent, const void* q, const void* w_prepared, const void* w_norm,
+                         const int32_t* positions, const int32_t* cu_seqlens,
+                         int32_t num_seqs, int32_t max_seqlen, int64_t total_tokens,
+                         const float* cos_table, const float* sin_table, int32_t max_pos,
+                         void* out, void* workspace, size_t workspace_bytes, cudaStream_t stream);
+
 /* Workspace bytes mla_decode needs for `batch` sequences whose longest
  * cache has max_cache_len rows. */
 int mla_decode_workspace_size(const mla_dims* dims, int32_t batch, int32_t max_cache_len,
@@ -196,13 +225,40 @@ int mla_prefill_cached_workspace_size(const mla_dims* dims, int64_t total_tokens
  * 0 .. p + i: its cached prefix, the chunk tokens before it, and itself (the
  * causal mask in absolute positions). Each chunk token runs as one row of
  * the absorbed decode (mla_decode), so the cost is the sum over chunk
- * tokens of the rows each attends. At most 65535 chunk tokens per call
+ * tokens of the rows each attends (the absorbed form). Long chunks take the
+ * eager form instead when it applies: bf16 with qk_rope 64, v_head 128,
+ * qk_nope 64 or 128, at least 128 chunk tokens per sequence on average,
+ * 16-byte aligned q, cache, w_kvb, out and workspace, and a workspace of at
+ * least mla_prefill_cached_eager_workspace_size bytes. It expands the keys and
+ * values of every row of each sequence (prefix and chunk) with the
+ * up-projection and runs the prefill's attention over them, so its cost
+ * grows with the rows once plus the chunk x rows attention on the tensor
+ * cores; a smaller workspace keeps the absorbed form. Both give the same
+ * results up to rounding; mla_last_dispatch names the form used. At most
+ * 65535 chunk tokens per call
  * (MLA_ERR_UNSUPPORTED_SHAPE above). The sequences' cache regions must not
  * overlap. Device-resident arguments are range-checked on the device: a
  * token whose sequence is inconsistent with cu_seqlens, whose rows leave the
  * cache or exceed max_total_len, or whose position is outside the table is
  * neither written to the cache nor attended (its output is zero) and the
  * device error word is set. */
+/* Workspace bytes of the eager form of mla_prefill_cached for num_seqs
+ * sequences of total_tokens chunk tokens whose sequences hold at most
+ * max_total_len rows once the chunk is in (padded key layout of
+ * num_seqs x ceil(max_total_len / 128) tiles of 128 rows: keys and values of
+ * every row, fp16). MLA_ERR_UNSUPPORTED_SHAPE for head shapes without the
+ * eager form. */
+int mla_prefill_cached_eager_workspace_size(const mla_dims* dims, int64_t total_tokens, int32_t num_seqs,
+                                            int32_t max_total_len, size_t* bytes);
+
+/* The form of a chunk call (mla_prefill_cached_form). */
+typedef enum mla_chunk_form {
+  MLA_CHUNK_AUTO = 0,      /* eager for long chunks when it applies and fits, else absorbed */
+  MLA_CHUNK_ABSORBED = 1,  /* one absorbed decode row per chunk token */
+  MLA_CHUNK_EAGER = 2      /* keys and values of every row expanded; MLA_ERR_UNSUPPORTED_SHAPE or
+                              MLA_ERR_WORKSPACE_TOO_SMALL when it does not apply */
+} mla_chunk_form;
+
 int mla_prefill_cached(const mla_dims* dims, const void* latent, const void* q, const void* w_kvb,
                        const void* w_norm, const int32_t* cu_seqlens, int32_t num_seqs,
                        int64_t total_tokens, const int64_t* cache_offsets,
@@ -210,6 +266,16 @@ int mla_prefill_cached(const mla_dims* dims, const void* latent, const void* q, 
                        const float* cos_table, const float* sin_table, int32_t max_pos,
                        void* cache, int64_t cache_num_rows, void* out, void* workspace,
                        size_t workspace_bytes, cudaStream_t stream);
+
+/* mla_prefill_cached with the form chosen by the caller (`form`, an
+ * mla_chunk_form); mla_prefill_cached is this call with MLA_CHUNK_AUTO. */
+int mla_prefill_cached_form(const mla_dims* dims, const void* latent, const void* q, const void* w_kvb,
+                            const void* w_norm, const int32_t* cu_seqlens, int32_t num_seqs,
+                            int64_t total_tokens, const int64_t* cache_offsets,
+                            const int32_t* prefix_lens, int32_t max_total_len,
+                            const float* cos_table, const float* sin_table, int32_t max_pos,
+                            void* cache, int64_t cache_num_rows, void* out, void* workspace,
+                            size_t workspace_bytes, int32_t form, cudaStream_t stream);
 
 /* The projections on either side of the path ([ROT] "Query heads": mla-init
  * gives the nn.Linear shapes, mla-queries the query order; "Key heads": mla-kv
@@ -219,20 +285,29 @@ int mla_prefill_cached(const mla_dims* dims, const void* latent, const void* q, 
  * the tensor cores (fp32 accumulation, bf16 result); otherwise on the CUDA
  * cores. At most 2^20 rows (tokens) per call (MLA_ERR_UNSUPPORTED_SHAPE). */
 
+/* Workspace bytes of mla_kv_down_append for n rows: the Linear's fp32
+ * result [n, R + P] in bf16 runs, 0 in fp32 runs. */
+int mla_kv_down_append_workspace_size(const mla_dims* dims, int64_t n, size_t* bytes);
+
 /* kv_a_proj_with_mqa, optionally followed by the cache append:
  *   hidden     [n, hidden_size]
  *   w_kva      [R + P, hidden_size]
  *   latent     [n, R + P]  written: compressed_kv (the latent input of mla_prefill)
- * If cache and cache_rows are both non-NULL, the rows of latent are then
- * appended exactly as by mla_cache_append (w_norm, positions and the tables
- * are then required); if both are NULL only latent is written. */
+ * If cache and cache_rows are both non-NULL, each row is also appended as by
+ * mla_cache_append (w_norm, positions and the tables are then required); if
+ * both are NULL only latent is written. In bf16 runs the Linear's result stays
+ * fp32 in the workspace: latent is its rounding to bf16, and the cache row's
+ * RMSNorm and rotation are computed from the fp32 values (no rounding before
+ * the norm); workspace may be NULL in fp32 runs. */
 int mla_kv_down_append(const mla_dims* dims, int32_t hidden_size, const void* hidden,
                        const void* w_kva, const void* w_norm, const int32_t* positions, int64_t n,
                        const float* cos_table, const float* sin_table, int32_t max_pos,
                        void* latent, void* cache, int64_t cache_num_rows,
-                       const int64_t* cache_rows, cudaStream_t stream);
+                       const int64_t* cache_rows, void* workspace, size_t workspace_bytes,
+                       cudaStream_t stream);
 
-/* Workspace bytes of mla_q_proj: the [n, q_rank] intermediate. */
+/* Workspace bytes of mla_q_proj: the [n, q_rank] fp32 intermediate; in bf16
+ * runs also its normalized copy and an fp16 copy of w_qb. */
 int mla_q_proj_workspace_size(const mla_dims* dims, int32_t q_rank, int64_t n, size_t* bytes);
 
 /* q = q_b_proj(q_a_layernorm(q_a_proj(hidden))):
@@ -241,8 +316,11 @@ int mla_q_proj_workspace_size(const mla_dims* dims, int32_t q_rank, int64_t n, s
  *   w_qnorm [q_rank]  RMSNorm weight (eps = dims->eps)
  *   w_qb    [H * (N + P), q_rank]
  *   q       [n, H, N + P]  written (the q input of mla_prefill / mla_decode)
- * The intermediate q_a is kept in the run dtype in the workspace (bf16 runs
- * round it to bf16, as the model's bf16 Linear does). */
+ * q_a stays fp32 until its RMSNorm. In bf16 runs the normalized q_a enters
+ * q_b_proj in fp16 against an fp16 copy of w_qb made in the workspace (tensor
+ * cores: q_rank a multiple of 64, 16-byte aligned tensors; a w_qb value beyond
+ * the fp16 range sets the device error word), or in fp32 (CUDA cores);
+ * accumulation is fp32 and q is bf16. */
 int mla_q_proj(const mla_dims* dims, int32_t hidden_size, int32_t q_rank, const void* hidden,
                const void* w_qa, const void* w_qnorm, const void* w_qb, int64_t n, void* q,
                void* workspace, size_t workspace_bytes, cudaStream_t stream);
@@ -266,9 +344,11 @@ int mla_o_proj(const mla_dims* dims, int32_t hidden_size, const void* attn, cons
  * GPU that loads this library, until the process exits. The pages have no
  * counterpart to this entry point; it changes how scratch is provided, not
  * what is computed (the results equal mla_prefill's).
- *   - The first call on a device, with that device current, looks up the
- *     array's device address (cudaGetSymbolAddress) and keeps it; make that
- *     first call before any stream capture.
+ *   - Every call looks up the array's device address on the current device
+ *     (cudaGetSymbolAddress, a host-side lookup), so a call after
+ *     cudaDeviceReset finds the array in the new context. The first call on
+ *     a device may load the library's device code: make it before any
+ *     stream capture.
  *   - A call whose workspace need (mla_prefill_workspace_size) exceeds
  *     MLA_NOALLOC_SCRATCH_BYTES returns MLA_ERR_WORKSPACE_TOO_SMALL and
  *     launches nothing. For the Kimi-K2 head geometry half of the array
@@ -292,8 +372,27 @@ int mla_prefill_noalloc(const mla_dims* dims,
  * up since the last check, MLA_ERR_CUDA on a CUDA error, else MLA_OK. */
 int mla_check_device_status(cudaStream_t stream);
 
+/* Self-test of the failure detection (the pages have no counterpart: their
+ * only error convention is the shape checks of the eager code). Every wait in
+ * the library's kernels is bounded: after its time limit it sets the device
+ * error word and lets the kernel return, so a lost arrival never hangs the
+ * GPU. This call launches one CTA whose wait, through the same helper but with
+ * a limit of `limit_us` microseconds (1 .. 1000000), is on an mbarrier that
+ * nothing arrives at. It runs out, sets the device error word and writes 1 to
+ * *gave_up (device int32, owned by the caller; 0 had the barrier completed).
+ * The next mla_check_device_status then returns MLA_ERR_DEVICE_TIMEOUT and
+ * clears the word; the context stays usable. */
+int mla_selftest_wait_timeout(uint32_t limit_us, int32_t* gave_up, cudaStream_t stream);
+
 /* Text of the calling thread's last error (static storage, never NULL). */
 const char* mla_last_error_string(void);
+
+/* Which kernels the calling thread's last prefill or decode call launched:
+ * "tensor-core", or "simt: <reason>" when it ran the exact CUDA-core kernels
+ * instead (a head shape or dtype outside the tensor-core kernels, or a tensor
+ * that is not 16-byte aligned). Static storage, never NULL; "none" before the
+ * first call. */
+const char* mla_last_dispatch(void);
 
 /* Profiling support. Registers `pairs` pairs of host cudaEvent_t handles
  * (`events` points to 2 * pairs handles created by the caller). Every kernel

@@ -131,35 +131,3 @@ def oracle_prefill_cached(wl, inp, heads=None):
     return O.prefill_cached(f64(inp["latent"]), f64(inp["q"]), f64(inp["cache"]), inp["cache_offsets"].numpy(),
                             inp["prefix_lens"].numpy(), inp["cu_seqlens"].numpy(), f64(inp["w_kvb"]),
                             f64(inp["w_norm"]), cos, sin, shape, scale, heads=heads)
-
-
-ROUNDED_REL = 2.0 ** -7
-ROUNDED_RMS = 2.0 ** -5
-
-
-def compare_rounded(got, ref, what=""):
-    """bf16 results computed from an intermediate that the model rounds to
-    bf16 (the latent before its RMSNorm, q_a before its RMSNorm), against the
-    oracle's unrounded fp64 chain. Per element |got - ref| <= 2^-7 |ref| +
-    2^-5 rms(ref). The intermediate's rounding (at most 2^-9 relative per
-    element) reaches a result either element-wise (the RMSNorm scales each
-    element: at most 2^-9 |ref|) or through the next Linear's sum, which
-    spreads it into an error of about 0.003 rms(ref) per element (q's
-    measured rel-L2), about 2^-6 rms(ref) at the extremes of millions of
-    elements; the result's own rounding adds at most 2^-9 |ref|. The bound
-    is about twice the worst case of each part. rel-L2 <= 5e-3 as for every
-    bf16 result."""
-    got = np.asarray(got, dtype=np.float64)
-    ref = np.asarray(ref, dtype=np.float64)
-    err = np.abs(got - ref)
-    rms = float(np.sqrt(np.mean(ref ** 2)))
-    ratio = float((err / (ROUNDED_REL * np.abs(ref) + ROUNDED_RMS * rms)).max())
-    rel_l2 = float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300))
-    m = dict(max_abs=float(err.max()), rel_l2=rel_l2, bound_ratio=ratio, n=int(ref.size))
-    log = os.environ.get("MLA_PARITY_LOG")
-    if log:
-        with open(log, "a") as f:
-            f.write(json.dumps(dict(what=what, dtype="bf16-rounded", **m)) + "\n")
-    assert np.isfinite(got).all(), "%s: non-finite output" % what
-    assert ratio <= 1.0 and rel_l2 <= BF16_REL_L2, "%s %s" % (what, m)
-    return m

@@ -162,10 +162,11 @@ def test_projection_host_validation():
 
     def kv(**o):
         a = dict(hid=7168, x=FAKE, w=FAKE, wn=FAKE, pos=FAKE, n=4, cos=FAKE, sin=FAKE, mp=10, lat=FAKE, cache=None,
-                 rows=0, crows=None)
+                 rows=0, crows=None, ws=FAKE, wsb=1 << 40)
         a.update(o)
         return lib.mla_kv_down_append(ctypes.byref(d), a["hid"], a["x"], a["w"], a["wn"], a["pos"], a["n"], a["cos"],
-                                      a["sin"], a["mp"], a["lat"], a["cache"], a["rows"], a["crows"], None)
+                                      a["sin"], a["mp"], a["lat"], a["cache"], a["rows"], a["crows"], a["ws"],
+                                      a["wsb"], None)
 
     assert kv(n=0) == 0
     assert kv(n=-1) == 1
@@ -177,6 +178,10 @@ def test_projection_host_validation():
     assert kv(cache=FAKE, crows=FAKE, wn=None) == 1
     assert kv(cache=FAKE, crows=FAKE, rows=0) == 1      # checked before the Linear runs
     assert kv(cache=FAKE, crows=FAKE, rows=10, mp=0) == 1
+    assert kv(wsb=16) == 3                         # bf16 runs keep the Linear's result in fp32
+    assert kv(ws=None) == 3
+    assert mla.mla_kv_down_append_workspace_size(d, 100) >= 100 * 576 * 4
+    assert mla.mla_kv_down_append_workspace_size(kimi_dims(dtype=1), 100) == 0
 
     def qp(**o):
         a = dict(hid=7168, qr=1536, x=FAKE, wa=FAKE, wn=FAKE, wb=FAKE, n=4, q=FAKE, ws=FAKE, wsb=1 << 40)
@@ -188,7 +193,7 @@ def test_projection_host_validation():
     assert qp(qr=0) == 1
     assert qp(wn=None) == 1
     assert qp(wsb=16) == 3
-    assert mla.mla_q_proj_workspace_size(d, 1536, 100) >= 100 * 1536 * 2
+    assert mla.mla_q_proj_workspace_size(d, 1536, 100) >= 100 * 1536 * (4 + 2) + 64 * 192 * 1536 * 2
 
     def op(**o):
         a = dict(hid=7168, x=FAKE, w=FAKE, n=4, out=FAKE)
@@ -199,3 +204,22 @@ def test_projection_host_validation():
     assert op(hid=-3) == 1
     assert op(out=None) == 1
     assert op(n=(1 << 21)) == 2
+
+
+def test_prepared_weight_and_selftest_host_validation():
+    lib = mla.load()
+    d = kimi_dims()
+    assert mla.mla_kv_b_proj_prepared_size(d) == 2 * 64 * 256 * 512
+    # outside the tensor-core shapes the prepared copy is the weight itself
+    assert mla.mla_kv_b_proj_prepared_size(kimi_dims(dtype=1)) == 4 * 64 * 256 * 512
+    assert lib.mla_prepare_kv_b_proj(ctypes.byref(d), FAKE, FAKE, 16, None) == 3
+    assert lib.mla_prepare_kv_b_proj(ctypes.byref(d), None, FAKE, 1 << 40, None) == 1
+    assert lib.mla_prepare_kv_b_proj(ctypes.byref(d), ctypes.c_void_p(0x1002), FAKE, 1 << 40, None) == 1  # alignment
+    # mla_prefill_prepared: a NULL weight is an argument error
+    rc = lib.mla_prefill_prepared(ctypes.byref(d), FAKE, FAKE, None, FAKE, FAKE, FAKE, 1, 10, 10, FAKE, FAKE, 10,
+                                  FAKE, FAKE, 1 << 40, None)
+    assert rc == 1
+    assert lib.mla_selftest_wait_timeout(0, FAKE, None) == 1
+    assert lib.mla_selftest_wait_timeout(2000000, FAKE, None) == 1
+    assert lib.mla_selftest_wait_timeout(1000, None, None) == 1
+    assert isinstance(mla.mla_last_dispatch(), str)

@@ -12,7 +12,7 @@ import torch
 import oracle as O
 from decode_latent_rmsnorm_b200 import mla
 from decode_latent_rmsnorm_b200 import workloads as W
-from _parity import (compare, compare_rounded, f64, oracle_cfg, oracle_decode, oracle_prefill,
+from _parity import (compare, f64, oracle_cfg, oracle_decode, oracle_prefill,
                      oracle_prefill_cached, run_decode, run_prefill, run_prefill_cached)
 
 pytestmark = pytest.mark.gpu
@@ -334,7 +334,7 @@ def test_kv_down_append_kimi_heads(gpu_lib, hid):
     compare(f64(latent), lat_ref, "bf16", "kv_a_proj K=%d" % hid)
     ocos, osin = O.rope_tables(rope, n)
     rows_ref = O.cache_append(lat_ref, f64(inp["w_norm"]), inp["positions"].numpy(), ocos, osin, shape)
-    compare_rounded(f64(cache[5:n + 5]), rows_ref, "kv_a_proj cache rows K=%d" % hid)
+    compare(f64(cache[5:n + 5]), rows_ref, "bf16", "kv_a_proj cache rows K=%d" % hid)
     assert torch.all(cache[:5] == 3.0) and torch.all(cache[n + 5:] == 3.0)
 
 
@@ -346,7 +346,30 @@ def test_q_proj_kimi_heads(gpu_lib, hid, qr):
     torch.cuda.synchronize()
     mla.mla_check_device_status()
     ref = O.q_projection(f64(inp["hidden"]), f64(inp["w_qa"]), f64(inp["w_qnorm"]), f64(inp["w_qb"]), shape)
-    compare_rounded(f64(q), ref, "q_proj K=%d/%d" % (hid, qr))
+    compare(f64(q), ref, "bf16", "q_proj K=%d/%d" % (hid, qr))
+
+
+def test_projections_bench_size(gpu_lib):
+    # the bench's 2048 tokens: the cache rows and q over millions of elements,
+    # where the bf16 output's half-ulp (0.0156 at |x| >= 4) leaves the least room
+    n = 2048
+    inp, d, dims, rope, shape = _proj_case(W.KIMI, n, KIMI_HIDDEN, KIMI_QRANK, seed=0)
+    cos, sin = mla.mla_init_rope_tables(mla.rope_for(W.KIMI), n)
+    cache = torch.empty((n, 576), dtype=torch.bfloat16, device="cuda")
+    rows = torch.arange(n, dtype=torch.int64, device="cuda")
+    latent = mla.mla_kv_down_append(dims, d["hidden"], d["w_kva"], w_norm=d["w_norm"], positions=d["positions"],
+                                    cos=cos, sin=sin, cache=cache, cache_rows=rows)
+    q = mla.mla_q_proj(dims, d["hidden"], d["w_qa"], d["w_qnorm"], d["w_qb"])
+    torch.cuda.synchronize()
+    mla.mla_check_device_status()
+    x = f64(inp["hidden"])
+    lat_ref = O.kv_down_projection(x, f64(inp["w_kva"]))
+    compare(f64(latent), lat_ref, "bf16", "kv_a_proj n=2048")
+    ocos, osin = O.rope_tables(rope, n)
+    compare(f64(cache), O.cache_append(lat_ref, f64(inp["w_norm"]), inp["positions"].numpy(), ocos, osin, shape),
+            "bf16", "kv_a_proj cache rows n=2048")
+    compare(f64(q), O.q_projection(x, f64(inp["w_qa"]), f64(inp["w_qnorm"]), f64(inp["w_qb"]), shape), "bf16",
+            "q_proj n=2048")
 
 
 def test_o_proj_kimi_heads(gpu_lib):
