@@ -87,6 +87,7 @@ int make_map(CUtensorMap* m, const void* base, int rank, const uint64_t* dims, c
 }
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned32(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 31u) == 0; }
 
 // ---- launch accounting and optional per-kernel events ---------------------
 std::atomic<uint64_t> g_launches{0};
@@ -192,7 +193,7 @@ bool prefill_tc_shape(const mla_dims* d) {
 struct PrefillWs {
   int64_t cap, Tpad;
   int gemm_tiles_per_cta, gemm_gy;
-  size_t seq_tile0, tile_seq, tile_q0, order, pair_order, item_counter, w16, c16;
+  size_t seq_tile0, tile_seq, tile_q0, order, pair_order, item_counter, w16, c16, q_rope;
   size_t k_nope, vals, k_rot, total;
 };
 PrefillWs prefill_ws_layout(const mla_dims* d, int64_t T, int nseq, bool tc) {
@@ -218,6 +219,7 @@ PrefillWs prefill_ws_layout(const mla_dims* d, int64_t T, int nseq, bool tc) {
     w.item_counter = off; off = align_up(off + 4, 256);
     w.w16 = off;       off = align_up(off + 2 * (size_t)NOUT * d->kv_lora_rank, 256);
     w.c16 = off;       off = align_up(off + 2 * (size_t)T * d->kv_lora_rank, 256);   // normalized latent, fp16
+    w.q_rope = off;    off = align_up(off + 2 * (size_t)T * d->num_heads * d->qk_rope, 256);   // rotated q, fp16
   } else {
     w.Tpad = T;
   }
@@ -376,23 +378,24 @@ int launch_attention_tc(int N, int V, unsigned grid, const CUtensorMap& mq, cons
 bool attention_pair_shape(int N, int V) { return (N == 64 || N == 128) && (V == 64 || V == 128); }
 
 template <int kN, int kV>
-int launch_attention_pair_t(unsigned grid, const CUtensorMap& mq, const CUtensorMap& mkn, const CUtensorMap& mkr,
-                            const CUtensorMap& mvt, const mla::tc::AttParams& ap, cudaStream_t st) {
+int launch_attention_pair_t(unsigned grid, const CUtensorMap& mq, const CUtensorMap& mqr, const CUtensorMap& mkn,
+                            const CUtensorMap& mkr, const CUtensorMap& mvt, const mla::tc::AttParams& ap,
+                            cudaStream_t st) {
   using C = mla::tc::PairCfg<kN, kV>;
   auto kern = mla::tc::attention_pair_kernel<kN, kV>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
   if (e != cudaSuccess) return cuda_status(e, "attention smem attribute");
   prof_begin(st, "tc_attention");
-  e = launch_dependent(kern, dim3(grid), dim3(mla::tc::kPrThreads), C::kSmem, st, mq, mkn, mkr, mvt, ap);
+  e = launch_dependent(kern, dim3(grid), dim3(mla::tc::kPrThreads), C::kSmem, st, mq, mqr, mkn, mkr, mvt, ap);
   prof_end(st);
   return cuda_status(e, "attention launch");
 }
 
-int launch_attention_pair(int N, int V, unsigned grid, const CUtensorMap& mq, const CUtensorMap& mkn,
-                          const CUtensorMap& mkr, const CUtensorMap& mvt, const mla::tc::AttParams& ap,
-                          cudaStream_t st) {
+int launch_attention_pair(int N, int V, unsigned grid, const CUtensorMap& mq, const CUtensorMap& mqr,
+                          const CUtensorMap& mkn, const CUtensorMap& mkr, const CUtensorMap& mvt,
+                          const mla::tc::AttParams& ap, cudaStream_t st) {
 #define MLA_PAIR_CASE(n, v) \
-  if (N == n && V == v) return launch_attention_pair_t<n, v>(grid, mq, mkn, mkr, mvt, ap, st);
+  if (N == n && V == v) return launch_attention_pair_t<n, v>(grid, mq, mqr, mkn, mkr, mvt, ap, st);
   MLA_PAIR_CASE(64, 64) MLA_PAIR_CASE(64, 128) MLA_PAIR_CASE(128, 64) MLA_PAIR_CASE(128, 128)
 #undef MLA_PAIR_CASE
   return fail(MLA_ERR_UNSUPPORTED_SHAPE, "no two-tile attention for qk_nope=%d v_head=%d", N, V);
@@ -419,8 +422,12 @@ int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, cons
   __half* k_nope = reinterpret_cast<__half*>(ws + L.k_nope);
   __half* vt = reinterpret_cast<__half*>(ws + L.vals);
   __half* k_rot = reinterpret_cast<__half*>(ws + L.k_rot);
+  __half* q_rope = reinterpret_cast<__half*>(ws + L.q_rope);
   const int cap = (int)L.cap;
   const int NOUT = H * (N + V);
+  // the two-tile attention takes k_nope in bf16 and the queries' rotated part
+  // from the preparation kernel
+  const bool pair = attention_pair_shape(N, V) && d->softmax_scale > 0.f;
 
   CUtensorMap map_lat, map_w;
   {
@@ -451,11 +458,21 @@ int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, cons
   const int w_blocks = w_f16 ? 0 : (int)((n8 + per_block - 1) / per_block);
   // the transposed-value GEMM reads c_hat prepared here: one warp per token row
   const int norm_blocks = vt_gemm ? (int)((T_tot + mla::tc::kPrepThreads / 32 - 1) / (mla::tc::kPrepThreads / 32)) : 0;
+  mla::tc::QRopeParams qrp{};
+  qrp.q = static_cast<const bf16*>(q);
+  qrp.positions = positions;
+  qrp.cos_t = cos_t;
+  qrp.sin_t = sin_t;
+  qrp.qr = q_rope;
+  qrp.rows = pair ? T_tot * H : 0;
+  qrp.H = H; qrp.D = N + P; qrp.N = N; qrp.max_pos = max_pos; qrp.interleaved = d->rope_interleaved;
+  const int qr_blocks = (int)((4 * qrp.rows + mla::tc::kPrepThreads - 1) / mla::tc::kPrepThreads);
   prof_begin(st, "tc_prep");
-  mla::tc::prefill_prep_kernel<<<(unsigned)(1 + w_blocks + norm_blocks), mla::tc::kPrepThreads, 0, st>>>(
+  mla::tc::prefill_prep_kernel<<<(unsigned)(1 + w_blocks + norm_blocks + qr_blocks), mla::tc::kPrepThreads, 0,
+                                 st>>>(
       cu_seqlens, num_seqs, T_tot, max_seqlen, cap, seq_tile0, tile_seq, tile_q0, order, pair_order,
       item_counter, static_cast<const bf16*>(w_kvb), w16, n8, w_blocks, static_cast<const bf16*>(latent),
-      static_cast<const bf16*>(w_norm), R, d->eps, c16);
+      static_cast<const bf16*>(w_norm), R, d->eps, c16, norm_blocks, qrp);
   prof_end(st);
   CUtensorMap map_c16;   // the transposed-value GEMM's A operand: c_hat fp16 [Ttot, R]
   {
@@ -485,6 +502,7 @@ int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, cons
   gp.interleaved = d->rope_interleaved;
   gp.eps = d->eps;
   gp.tiles_per_cta = L.gemm_tiles_per_cta;
+  gp.knope_bf16 = pair ? 1 : 0;
   cudaError_t e;
   if (vt_gemm) {
     // grid: (tiles, head groups); about one CTA per SM over the real tiles
@@ -515,12 +533,12 @@ int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, cons
   e = cudaGetLastError();
   if (e != cudaSuccess) return cuda_status(e, "gemm launch");
 
-  // attention tensor maps over the padded workspace and q [Ttot, H, D]; the
-  // two-tile kernel reads 128 keys per step, the one-tile kernel 64
-  const bool pair = attention_pair_shape(N, V) && d->softmax_scale > 0.f;
+  // attention tensor maps over the padded workspace, q [Ttot, H, D] and the
+  // rotated q [Ttot, H, P]; the two-tile kernel reads 128 keys per step, the
+  // one-tile kernel 64
   const uint32_t kv_box = pair ? (uint32_t)mla::tc::kPrBKV : (uint32_t)mla::tc::kAttBKV;
   const int D = N + P;
-  CUtensorMap map_q, map_kn, map_kr, map_vt;
+  CUtensorMap map_q, map_qr, map_kn, map_kr, map_vt;
   {
     const uint64_t dims[3] = {(uint64_t)D, (uint64_t)H, (uint64_t)T_tot};
     const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)H * D * 2};
@@ -528,11 +546,19 @@ int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, cons
     int rc = make_map(&map_q, q, 3, dims, strides, box);
     if (rc) return rc;
   }
+  if (pair) {
+    const uint64_t dims[3] = {(uint64_t)P, (uint64_t)H, (uint64_t)T_tot};
+    const uint64_t strides[2] = {(uint64_t)P * 2, (uint64_t)H * P * 2};
+    const uint32_t box[3] = {64, 1, 128};
+    int rc = make_map(&map_qr, q_rope, 3, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+    if (rc) return rc;
+  }
   {
     const uint64_t dims[2] = {(uint64_t)N, (uint64_t)H * L.Tpad};
     const uint64_t strides[1] = {(uint64_t)N * 2};
     const uint32_t box[2] = {64, kv_box};
-    int rc = make_map(&map_kn, k_nope, 2, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+    int rc = make_map(&map_kn, k_nope, 2, dims, strides, box,
+                      pair ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
     if (rc) return rc;
   }
   {
@@ -575,7 +601,7 @@ int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, cons
     if (blocks > L.cap) blocks = L.cap;
     int64_t grid = blocks * H;
     if (grid > num_sms()) grid = num_sms();
-    return launch_attention_pair(N, V, (unsigned)grid, map_q, map_kn, map_kr, map_vt, ap, st);
+    return launch_attention_pair(N, V, (unsigned)grid, map_q, map_qr, map_kn, map_kr, map_vt, ap, st);
   }
   const unsigned grid = (unsigned)(cap * H);
   return launch_attention_tc(N, V, grid, map_q, map_kn, map_kr, map_vt, ap, st);
@@ -875,8 +901,9 @@ int prefill_entry(const mla_dims* dims, const void* latent, const void* q, const
   const size_t need = prefill_ws_bytes(dims, total_tokens, num_seqs);
   if (!workspace || workspace_bytes < need)
     return fail(MLA_ERR_WORKSPACE_TOO_SMALL, "workspace needs %zu bytes, got %zu", need, workspace_bytes);
+  // (the attention writes each output row with 32-byte stores)
   const bool aligned = aligned16(latent) && aligned16(q) && aligned16(workspace) && aligned16(w_norm) &&
-                       aligned16(w);
+                       aligned16(w) && aligned32(out);
   if (prefill_tc_shape(dims)) {
     if (aligned) {
       set_dispatch("tensor-core");
@@ -885,8 +912,9 @@ int prefill_entry(const mla_dims* dims, const void* latent, const void* q, const
                                workspace, stream);
     }
     if (prepared)
-      return fail(MLA_ERR_INVALID_ARG, "mla_prefill_prepared needs 16-byte aligned tensors and workspace");
-    set_dispatch("simt: a tensor or the workspace is not 16-byte aligned");
+      return fail(MLA_ERR_INVALID_ARG,
+                  "mla_prefill_prepared needs 16-byte aligned tensors and workspace and a 32-byte aligned out");
+    set_dispatch("simt: a tensor or the workspace is not 16-byte aligned, or out not 32-byte aligned");
   } else {
     set_dispatch("simt: head shape or dtype outside the tensor-core kernels");
   }
@@ -1069,7 +1097,7 @@ constexpr int64_t kChunkEagerMinAvg = 128;
 struct ChunkEagerWs {
   int64_t kcap, qcap, Kpad;
   size_t positions, rows, offsets, lens, seq_ok, kseq_tile0, ktile_seq, ktile_k0, qblk_seq, qblk_q0, qorder,
-      counter, w16, c16, k_nope, vt, k_rot, total;
+      counter, w16, c16, k_nope, vt, k_rot, q_rope, total;
 };
 ChunkEagerWs chunk_eager_ws_layout(const mla_dims* d, int64_t n, int nseq, int max_total_len) {
   auto up = [](size_t x) { return (x + 255) & ~(size_t)255; };
@@ -1096,6 +1124,7 @@ ChunkEagerWs chunk_eager_ws_layout(const mla_dims* d, int64_t n, int nseq, int m
   L.k_nope = o;     o = up(o + 2 * H * (size_t)L.Kpad * N);
   L.vt = o;         o = up(o + 2 * H * V * (size_t)L.Kpad);
   L.k_rot = o;      o = up(o + 2 * (size_t)L.Kpad * 64);
+  L.q_rope = o;     o = up(o + 2 * (size_t)n * H * 64);
   L.total = o;
   return L;
 }
@@ -1342,6 +1371,22 @@ int launch_prefill_cached_eager(const mla_dims* d, const void* latent, const voi
                        static_cast<bf16*>(out));
   prof_end(st);
   if (e != cudaSuccess) return cuda_status(e, "chunk zero launch");
+  // the queries' rotary parts, turned at their positions (fp16)
+  T::QRopeParams qrp{};
+  qrp.q = static_cast<const bf16*>(q);
+  qrp.positions = positions;
+  qrp.cos_t = cos_t;
+  qrp.sin_t = sin_t;
+  qrp.qr = reinterpret_cast<__half*>(ws + L.q_rope);
+  qrp.rows = Tq * H;
+  qrp.H = H; qrp.D = N + P; qrp.N = N; qrp.max_pos = max_pos; qrp.interleaved = d->rope_interleaved;
+  if (qrp.rows > 0) {
+    prof_begin(st, "tc_q_rope");
+    e = launch_dependent(T::q_rope_kernel, dim3((unsigned)((4 * qrp.rows + T::kPrepThreads - 1) / T::kPrepThreads)),
+                         dim3(T::kPrepThreads), 0, st, qrp);
+    prof_end(st);
+    if (e != cudaSuccess) return cuda_status(e, "q rope launch");
+  }
 
   // 7. k_nope / transposed values of every key row
   CUtensorMap map_w, map_c16;
@@ -1373,6 +1418,7 @@ int launch_prefill_cached_eager(const mla_dims* d, const void* latent, const voi
   gp.interleaved = d->rope_interleaved;
   gp.eps = d->eps;
   gp.a_padded = 1;
+  gp.knope_bf16 = 1;
   int groups = num_sms() / (int)(L.kcap > 0 ? L.kcap : 1);
   if (groups < 1) groups = 1;
   if (groups > H) groups = H;
@@ -1389,7 +1435,7 @@ int launch_prefill_cached_eager(const mla_dims* d, const void* latent, const voi
 
   // 8. the chunk's queries against each sequence's keys
   const int D = N + P;
-  CUtensorMap map_q, map_kn, map_kr, map_vt;
+  CUtensorMap map_q, map_qr, map_kn, map_kr, map_vt;
   {
     const uint64_t dims[3] = {(uint64_t)D, (uint64_t)H, (uint64_t)Tq};
     const uint64_t strides[2] = {(uint64_t)D * 2, (uint64_t)H * D * 2};
@@ -1398,10 +1444,17 @@ int launch_prefill_cached_eager(const mla_dims* d, const void* latent, const voi
     if (rc) return rc;
   }
   {
+    const uint64_t dims[3] = {(uint64_t)P, (uint64_t)H, (uint64_t)Tq};
+    const uint64_t strides[2] = {(uint64_t)P * 2, (uint64_t)H * P * 2};
+    const uint32_t box[3] = {64, 1, 128};
+    rc = make_map(&map_qr, ws + L.q_rope, 3, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+    if (rc) return rc;
+  }
+  {
     const uint64_t dims[2] = {(uint64_t)N, (uint64_t)H * L.Kpad};
     const uint64_t strides[1] = {(uint64_t)N * 2};
     const uint32_t box[2] = {64, (uint32_t)T::kPrBKV};
-    rc = make_map(&map_kn, k_nope, 2, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+    rc = make_map(&map_kn, k_nope, 2, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
     if (rc) return rc;
   }
   {
@@ -1438,7 +1491,7 @@ int launch_prefill_cached_eager(const mla_dims* d, const void* latent, const voi
   ap.scale_log2 = d->softmax_scale * 1.4426950408889634f;
   int64_t grid = L.qcap * H;
   if (grid > num_sms()) grid = num_sms();
-  return launch_attention_pair(N, V, (unsigned)grid, map_q, map_kn, map_kr, map_vt, ap, st);
+  return launch_attention_pair(N, V, (unsigned)grid, map_q, map_qr, map_kn, map_kr, map_vt, ap, st);
 }
 }  // namespace
 
@@ -1497,7 +1550,7 @@ int mla_prefill_cached_form(const mla_dims* dims, const void* latent, const void
   // automatic: long chunks (on average kChunkEagerMinAvg tokens or more per
   // sequence) take the eager form when the workspace holds it
   const bool eager_ok = chunk_eager_shape(dims) && aligned16(q) && aligned16(cache) && aligned16(w_kvb) &&
-                        aligned16(out) && aligned16(workspace) &&
+                        aligned32(out) && aligned16(workspace) &&
                         (int64_t)num_seqs * ((max_total_len + 127) / 128) <= 0x7fffffff / 128;
   if (form == MLA_CHUNK_EAGER && !eager_ok)
     return fail(MLA_ERR_UNSUPPORTED_SHAPE, "the eager form needs the tensor-core head shapes and 16-byte alignment");

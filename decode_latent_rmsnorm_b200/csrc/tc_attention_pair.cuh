@@ -6,8 +6,9 @@
 // head's query and key join their non-rotary and rotary parts (the key's
 // rotary part is the one rotary key shared by all heads), the scores are
 // scaled, causally masked, normalized with a softmax in fp32 and mix the
-// values. The arithmetic is the one of attention_kernel; this kernel changes
-// how it is scheduled on the SM.
+// values. The arithmetic is the one of attention_kernel except for the types
+// of the score product's operands (below); this kernel changes how it is
+// scheduled on the SM.
 //
 // Work item = one head x one 256-row block of queries, split into tile A
 // (rows 0-127) and tile B (rows 128-255). Both tiles read the same key /
@@ -17,12 +18,16 @@
 // causal work), so the grid balances itself. Warps (three warpgroups; the
 // first runs on 56 registers per thread so that the softmax warpgroups can
 // hold a whole row of scores in 216):
-//   warp 0     producer: takes the next item, publishes it to the other warps
-//              through a two-slot ring in shared memory, loads the tiles' Q
-//              and, per key step, the key atoms and the two transposed value
-//              boxes into a ring of 16 KB slots. The key/value stream runs on
-//              across items, and the next item's Q is loaded as soon as the
-//              current item's last score product on that tile has finished.
+//   warp 0     producer: claims the next item two key steps before the
+//              current item's end (the claim and the lookup of the item's
+//              sequence, rows and step counts happen while key steps are in
+//              flight, and the next item's Q rows are prefetched into L2
+//              then), publishes each decoded item to the other warps through
+//              a two-slot ring in shared memory, loads the tiles' Q and, per
+//              key step, the key atoms and the two transposed value boxes into
+//              a ring of 16 KB slots. The key/value stream runs on across
+//              items, and the next item's Q is loaded as soon as the current
+//              item's last score product on that tile has finished.
 //   warp 1     MMA issuer (whole warp, one elected lane issues)
 //   warps 2-3  idle
 //   warps 4-7  softmax of tile A (one query row per thread, TMEM lane = row)
@@ -38,10 +43,15 @@
 // Tensor-core instructions from one thread run in issue order, so S_X(g+1)
 // overwrites P_X(g) only after PV_X(g) has read it.
 //
-// At the end of an item a tile's softmax warps first convert the next item's
-// Q (so that its first score product can start) and then write the item's
-// output from O; the next item's first P V product (which overwrites O) waits
-// for that.
+// Score operands: the non-rotary atoms multiply q as given (bf16) with k_nope
+// stored in bf16; the rotary atom multiplies the query's rotary part, turned
+// at its position once before this kernel (q_rope_group, run by the
+// up-projection GEMM's epilogue warps or a preparation kernel), with the
+// rotated shared key, both fp16; all products accumulate in one fp32 TMEM
+// tile. So Q needs no work on this SM: its first score product starts when
+// its copy lands. At the end of an item a tile's softmax warps write the
+// item's output from O; the next item's first P V product (which overwrites
+// O) waits for that.
 //
 // Softmax reference: a row's reference m is its maximum over the first key
 // tile; it is raised (and O and the row sum rescaled) only when a later tile's
@@ -77,38 +87,6 @@ constexpr int kPrSchedReaders = 9;          // the MMA warp and the eight softma
 constexpr float kPrBias = 100.f;            // e = P * 2^-kPrBias stays a normal fp32 number
 constexpr float kPrTwoM12 = 2.44140625e-4f;         // 2^-12
 constexpr float kPrTwoMBias = 7.888609052210118e-31f;   // 2^-100
-// Of the four 32-key chunks of a row's step, the last kPrPolyChunks take
-// their exponentials from ex2_fma2 (FMA pipes) instead of the MUFU.
-#ifndef MLA_PR_POLY_CHUNKS
-#define MLA_PR_POLY_CHUNKS 0
-#endif
-constexpr int kPrPolyChunks = MLA_PR_POLY_CHUNKS;
-
-// 2^a for a pair of exponents a <= 2^22 on the FMA pipes (packed fp32): a is
-// clamped at -126 (smaller weights round to 0 in fp16 anyway), split as
-// a = j + f with j = round(a) (the 1.5 * 2^23 rounding trick) and f in
-// [-0.5, 0.5]; 2^f comes from a cubic fitted here to 2^f on [-0.5, 0.5]
-// for relative error (Lawson-weighted least squares; at most 7.5e-5, below
-// fp16's half-ulp), and j is added to its exponent field: the bits of
-// 1.5 * 2^23 shifted left by 23 vanish modulo 2^32, so (bits(t) << 23)
-// equals j << 23.
-__device__ __forceinline__ uint64_t ex2_fma2(uint64_t a2) {
-  float a0, a1;
-  f2_split(a2, a0, a1);
-  const uint64_t a = f2_make(fmaxf(a0, -126.f), fmaxf(a1, -126.f));
-  const uint64_t t = f2_add(a, f2_make(12582912.f, 12582912.f));
-  const uint64_t jf = f2_add(t, f2_make(-12582912.f, -12582912.f));
-  const uint64_t f = f2_fma(jf, f2_make(-1.f, -1.f), a);
-  uint64_t p = f2_fma(f2_make(5.517166853e-02f, 5.517166853e-02f), f, f2_make(2.426111400e-01f, 2.426111400e-01f));
-  p = f2_fma(p, f, f2_make(6.932609677e-01f, 6.932609677e-01f));
-  p = f2_fma(p, f, f2_make(9.999280572e-01f, 9.999280572e-01f));
-  float p0, p1, t0, t1;
-  f2_split(p, p0, p1);
-  f2_split(t, t0, t1);
-  return f2_make(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(t0) << 23)),
-                 __uint_as_float(__float_as_uint(p1) + (__float_as_uint(t1) << 23)));
-}
-
 template <int kN, int kV>
 struct PairCfg {
   static constexpr int D = kN + 64;
@@ -136,12 +114,11 @@ struct PairCfg {
 // the release the producer waits for before re-arming a step's barrier is
 // issued after the MMA warp's wait on that barrier four steps earlier.
 struct PairBarriers {
-  uint64_t q_full[2], q_ready[2], q_free[2];
+  uint64_t q_full[2], q_free[2];
   uint64_t kfull[kPrGroupDepth], kempty[kPrGroupDepth], vfull[kPrGroupDepth], vempty[kPrGroupDepth];
   uint64_t s_full[2], p_full[2], pv_done[2], o_free[2];
   uint64_t sched_full[kPrSched], sched_empty[kPrSched];
   uint64_t mma_done;
-  int sched_item[kPrSched];
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -165,8 +142,9 @@ __device__ __forceinline__ PairItem pair_item(const AttParams& p, int item) {
   const int rank = item / p.H;
   if (rank >= p.n_blocks) return it;
   const int tile = p.order[rank];
-  if (tile < 0) return it;
+  if (tile < 0 || tile >= p.n_blocks) return it;   // n_blocks bounds the tile tables too
   const int seq = p.tile_seq[tile];
+  if (seq < 0) return it;
   it.valid = 1;
   it.h = item - rank * p.H;
   it.q0 = p.tile_q0[tile];                                   // multiple of 256
@@ -181,28 +159,31 @@ __device__ __forceinline__ PairItem pair_item(const AttParams& p, int item) {
   return it;
 }
 
-// The k-th work item of the CTA, as published by the producer: every reader
-// warp reads every slot once, in order. Returns false on abort.
-__device__ __forceinline__ bool pair_read_item(PairBarriers& bars, const AttParams& p, int k, int lane,
+// The k-th work item of the CTA, as published (decoded) by the producer in
+// the shared-memory ring `ring`: every reader warp reads every slot once, in
+// order. Returns false on abort.
+__device__ __forceinline__ bool pair_read_item(PairBarriers& bars, const PairItem* ring, int k, int lane,
                                                volatile int* abort_flag, PairItem& it) {
   const int s = k % kPrSched;
   if (!mbar_wait_warp(&bars.sched_full[s], (uint32_t)(k / kPrSched) & 1u, abort_flag)) return false;
-  const int item = *reinterpret_cast<volatile int*>(&bars.sched_item[s]);
+  const volatile PairItem& r = ring[s];
+  it.valid = r.valid; it.h = r.h; it.q0 = r.q0; it.L = r.L; it.kv_pad0 = r.kv_pad0; it.off = r.off;
+  it.nA = r.nA; it.nB = r.nB; it.n = r.n; it.seq0 = r.seq0;
   __syncwarp();
   if (lane == 0) mbar_arrive(&bars.sched_empty[s]);
-  it = pair_item(p, item);
   return true;
 }
 
 template <int kN, int kV>
 __global__ void __launch_bounds__(kPrThreads, 1)
-attention_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_kn,
-                      const __grid_constant__ CUtensorMap map_kr, const __grid_constant__ CUtensorMap map_vt,
-                      AttParams p) {
+attention_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_qr,
+                      const __grid_constant__ CUtensorMap map_kn, const __grid_constant__ CUtensorMap map_kr,
+                      const __grid_constant__ CUtensorMap map_vt, AttParams p) {
   using C = PairCfg<kN, kV>;
   constexpr int S = C::kSlots;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ PairBarriers bars;
+  __shared__ PairItem sched_ring[kPrSched];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_allow_next();
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -213,7 +194,6 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
   if (threadIdx.x == 0) {
     for (int x = 0; x < 2; ++x) {
       mbar_init(&bars.q_full[x], 1);
-      mbar_init(&bars.q_ready[x], 128);
       mbar_init(&bars.q_free[x], 1);
       mbar_init(&bars.s_full[x], 1);
       mbar_init(&bars.p_full[x], 128);
@@ -245,6 +225,7 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
       // ---------------- producer ----------------
       if (lane == 0) {
         tma_prefetch_desc(&map_q);
+        tma_prefetch_desc(&map_qr);
         tma_prefetch_desc(&map_kn);
         tma_prefetch_desc(&map_kr);
         tma_prefetch_desc(&map_vt);
@@ -260,20 +241,26 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
         int g = 0;                         // global key step
         int gk = -1, gv = -1;              // last key / value group issued
         int uq[2] = {0, 0};                // Q loads issued per tile
+        // the first item of every CTA is its own index (the grid never exceeds
+        // the item count); the counter hands out the rest
+        PairItem next = pair_item(p, (int)blockIdx.x);
         for (int k = 0; ok; ++k) {
           const int s = k % kPrSched;
           if (!(ok = mbar_wait(&bars.sched_empty[s], ((uint32_t)(k / kPrSched) & 1u) ^ 1u, abort_flag))) break;
-          const int item = atomicAdd(p.item_counter, 1);
-          const PairItem it = pair_item(p, item);
-          bars.sched_item[s] = it.valid ? item : -1;
+          const PairItem it = next;
+          volatile PairItem& r = sched_ring[s];
+          r.valid = it.valid; r.h = it.h; r.q0 = it.q0; r.L = it.L; r.kv_pad0 = it.kv_pad0; r.off = it.off;
+          r.nA = it.nA; r.nB = it.nB; r.n = it.n; r.seq0 = it.seq0;
           mbar_arrive(&bars.sched_full[s]);
           if (!it.valid) break;
+          bool claimed = false;              // the item after this one claimed yet
           auto load_q = [&](int x) -> bool {
             if (uq[x] > 0 && !mbar_wait(&bars.q_free[x], (uint32_t)(uq[x] - 1) & 1u, abort_flag)) return false;
             mbar_arrive_expect_tx(&bars.q_full[x], C::kQTileBytes);
-            for (int a = 0; a < C::kQAtoms; ++a)
-              tma_load_3d(sQ + x * C::kQTileBytes + a * kTile * 128, &map_q, &bars.q_full[x], a * 64, it.h,
-                          (int)(it.seq0 + it.q0 + x * kTile));
+            const int qrow0 = (int)(it.seq0 + it.q0 + x * kTile);
+            for (int a = 0; a < C::kKAtoms; ++a)
+              tma_load_3d(sQ + x * C::kQTileBytes + a * kTile * 128, &map_q, &bars.q_full[x], a * 64, it.h, qrow0);
+            tma_load_3d(sQ + x * C::kQTileBytes + C::kKAtoms * kTile * 128, &map_qr, &bars.q_full[x], 0, it.h, qrow0);
             ++uq[x];
             return true;
           };
@@ -303,7 +290,23 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
             // wait for the previous item's last tile-B scores never holds up
             // the keys tile A needs first
             if (j == 0 && it.nB > 0 && !(ok = load_q(1))) break;
+            if (!claimed && j == max(it.n - 2, 0)) {
+              // two steps before the item's end (the ring is full, so the
+              // lookups' latency costs nothing): claim and decode the next
+              // item, and start its Q rows on their way to L2. Claiming this
+              // late keeps the heaviest-first order of the claims close to the
+              // order in which the CTAs run out of work.
+              claimed = true;
+              next = pair_item(p, (int)gridDim.x + atomicAdd(p.item_counter, 1));
+              if (next.valid)
+                for (int x = 0; x < (next.nB > 0 ? 2 : 1); ++x) {
+                  const int r0 = (int)(next.seq0 + next.q0 + x * kTile);
+                  for (int a = 0; a < C::kKAtoms; ++a) tma_prefetch_l2_3d(&map_q, a * 64, next.h, r0);
+                  tma_prefetch_l2_3d(&map_qr, 0, next.h, r0);
+                }
+            }
           }
+          if (ok && !claimed) next = pair_item(p, (int)gridDim.x + atomicAdd(p.item_counter, 1));
         }
         if (!ok) {   // let every copy already issued land before the CTA exits
           for (int x = 0; x < 2; ++x)
@@ -316,12 +319,13 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
       }
     } else if (warp == 1) {
       // ---------------- MMA issuer (whole warp; one elected lane issues) ----------------
-      const uint32_t idesc_s = idesc_f16_f32(kTile, kPrBKV);
+      const uint32_t idesc_s_nope = idesc_bf16_f32(kTile, kPrBKV);   // q as given, k_nope in bf16
+      const uint32_t idesc_s_rope = idesc_f16_f32(kTile, kPrBKV);    // rotated q and key in fp16
       const uint32_t idesc_o = idesc_f16_f32(kTile, kV);
       const uint32_t ring0 = smem_u32(sRing), q0addr = smem_u32(sQ);
       auto slot_addr = [&](int gb) -> uint32_t { return ring0 + (uint32_t)(gb % S) * kPrSlotBytes; };
       int k_seen = -1, v_seen = -1;       // last global step whose key / value group was waited for
-      int uq[2] = {0, 0};                 // Q uses per tile (q_ready phases)
+      int uq[2] = {0, 0};                 // Q uses per tile (q_full phases)
       int uo[2] = {0, 0};                 // items per tile whose P V has started (o_free phases)
       int ts[2] = {0, 0};                 // tile-steps per tile (p_full phases)
       // S_x(step g) = Q_x K_g^T over all D columns
@@ -336,6 +340,7 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
         for (int a = 0; a < C::kQAtoms; ++a) {
           const uint64_t qd = desc_kmajor_sw128(q0addr + (uint32_t)(x * C::kQTileBytes + a * kTile * 128));
           const uint64_t kd = desc_kmajor_sw128(slot_addr(g * C::kBoxes + a));
+          const uint32_t idesc_s = a < C::kKAtoms ? idesc_s_nope : idesc_s_rope;
   #pragma unroll
           for (int k = 0; k < 4; ++k)
             mma_ss_elect(d, desc_advance(qd, k * 32), desc_advance(kd, k * 32), idesc_s, (a | k) != 0);
@@ -343,9 +348,9 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
         mma_commit_elect(&bars.s_full[x]);
         return true;
       };
-      // first S of tile x in a new item: its Q must be converted
+      // first S of tile x in a new item: its Q must have landed
       auto issue_s_first = [&](int x, int g, int nx) -> bool {
-        if (!mbar_wait_warp(&bars.q_ready[x], (uint32_t)uq[x] & 1u, abort_flag)) return false;
+        if (!mbar_wait_warp(&bars.q_full[x], (uint32_t)uq[x] & 1u, abort_flag)) return false;
         ++uq[x];
         if (!issue_s(x, g)) return false;
         if (nx == 1) mma_commit_elect(&bars.q_free[x]);
@@ -382,7 +387,7 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
       struct Steps { int valid, nA, nB, n; };
       auto read_steps = [&](int k, Steps& st) -> bool {
         PairItem it;
-        if (!pair_read_item(bars, p, k, lane, abort_flag, it)) return false;
+        if (!pair_read_item(bars, sched_ring, k, lane, abort_flag, it)) return false;
         st.valid = it.valid; st.nA = it.nA; st.nB = it.nB; st.n = it.n;
         return true;
       };
@@ -440,115 +445,59 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
     const uint32_t tS = tmem + lane_base + (uint32_t)(x * kPrBKV);
     const uint32_t tO = tmem + lane_base + C::kOCol + (uint32_t)(x * 128);
     const float sl = p.scale_log2;
-    uint8_t* sQx = sQ + x * C::kQTileBytes;
     int kread = 0;
-    int uq = 0;                                   // items of this tile (q_full phases)
     int ts = 0;                                   // tile-steps (s_full / pv_done phases)
     // next item in which this tile has rows
     auto next_item = [&](PairItem& it) -> bool {
       for (;;) {
-        if (!pair_read_item(bars, p, kread++, lane, abort_flag, it)) return false;
+        if (!pair_read_item(bars, sched_ring, kread++, lane, abort_flag, it)) return false;
         if (!it.valid || (x ? it.nB : it.nA) > 0) return true;
       }
     };
-    // this row of the item's Q: bf16 -> fp16 in place (per atom: all loads,
-    // the conversion, then all stores); the rotary atom is rotated at the
-    // token's position, its 32 pairs in two halves of 16
-    auto prep_q = [&](const PairItem& it) -> bool {
-      if (!mbar_wait_warp(&bars.q_full[x], (uint32_t)uq & 1u, abort_flag)) return false;
-      ++uq;
-      const int qrow = it.q0 + x * kTile + row;
-      const bool valid = qrow < it.L;
-      const int64_t t = it.seq0 + qrow;
-      float qmax = 0.f;
-#pragma unroll 1
-      for (int a = 0; a < C::kQAtoms - 1; ++a) {
-        uint8_t* qa = sQx + a * kTile * 128;
-        uint4 v[8];
+    // the previous item's output: O / row sum, bf16, row t of head h
+    auto epilogue = [&](bool valid, int64_t t, int h, const uint64_t (&l2)[2]) -> bool {
+      if (!mbar_wait_warp(&bars.pv_done[x], (uint32_t)(ts - 1) & 1u, abort_flag)) return false;
+      tc_fence_after();
+      float la, lb, lc, ld;
+      f2_split(l2[0], la, lb);
+      f2_split(l2[1], lc, ld);
+      const float inv = (1.f / ((la + lb) + (lc + ld))) * kPrTwoMBias;
+      __nv_bfloat16* dst = p.out + (t * p.H + h) * kV;
 #pragma unroll
-        for (int c = 0; c < 8; ++c) v[c] = *reinterpret_cast<const uint4*>(qa + sw128_offset(row, c));
+      for (int hh = 0; hh < kV / 64; ++hh) {   // 64 columns at a time: two loads in flight, one wait
+        uint32_t v[64];
+        tmem_ld32_nowait(tO + (uint32_t)(hh * 64), v);
+        tmem_ld32_nowait(tO + (uint32_t)(hh * 64 + 32), v + 32);
+        tmem_wait_ld64(v);
+        if (valid) {
 #pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          const uint32_t w4[4] = {v[c].x, v[c].y, v[c].z, v[c].w};
-          uint32_t o4[4];
+          for (int c = 0; c < 4; ++c) {
+            uint32_t o[8];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = unpack_bf16x2(w4[e]);
-            qmax = fmaxf(qmax, fmaxf(fabsf(f.x), fabsf(f.y)));
-            o4[e] = pack_f16x2(f.x, f.y);
-          }
-          v[c] = make_uint4(o4[0], o4[1], o4[2], o4[3]);
-        }
-#pragma unroll
-        for (int c = 0; c < 8; ++c) *reinterpret_cast<uint4*>(qa + sw128_offset(row, c)) = v[c];
-      }
-      const int64_t pos = valid ? checked_pos(p.positions[t], p.max_pos) : 0;
-      uint8_t* qr = sQx + (C::kQAtoms - 1) * kTile * 128;
-#pragma unroll 1
-      for (int hp = 0; hp < 2; ++hp) {
-        // rotary pairs [16 hp, 16 hp + 16): 16 cos / sin entries as four vector
-        // loads each; the four 16-byte chunks holding the pairs' 32 values
-        // (half-split pairing: chunks 2hp, 2hp+1 and 4+2hp, 5+2hp;
-        // interleaved: chunks 4hp .. 4hp+3)
-        const float4* c4 = reinterpret_cast<const float4*>(p.cos_t + pos * 32 + hp * 16);
-        const float4* s4 = reinterpret_cast<const float4*>(p.sin_t + pos * 32 + hp * 16);
-        float cs[16], sn[16];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float4 cv = c4[i], sv = s4[i];
-          cs[4 * i] = cv.x; cs[4 * i + 1] = cv.y; cs[4 * i + 2] = cv.z; cs[4 * i + 3] = cv.w;
-          sn[4 * i] = sv.x; sn[4 * i + 1] = sv.y; sn[4 * i + 2] = sv.z; sn[4 * i + 3] = sv.w;
-        }
-        int ch[4];
-        if (p.interleaved) {
-          ch[0] = 4 * hp; ch[1] = 4 * hp + 1; ch[2] = 4 * hp + 2; ch[3] = 4 * hp + 3;
-        } else {
-          ch[0] = 2 * hp; ch[1] = 2 * hp + 1; ch[2] = 4 + 2 * hp; ch[3] = 5 + 2 * hp;
-        }
-        float xr[32];
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint4 v = *reinterpret_cast<const uint4*>(qr + sw128_offset(row, ch[k]));
-          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = unpack_bf16x2(w4[e]);
-            xr[k * 8 + 2 * e] = f.x;
-            xr[k * 8 + 2 * e + 1] = f.y;
+            for (int e = 0; e < 8; ++e)
+              o[e] = pack_bf16x2(__uint_as_float(v[c * 16 + 2 * e]) * inv, __uint_as_float(v[c * 16 + 2 * e + 1]) * inv);
+            st_global_v8(dst + hh * 64 + c * 16, o);
           }
         }
-        // xr holds, in order, chunks ch[0..3]; local pair i is (xr[2i],
-        // xr[2i+1]) when interleaved, (xr[i], xr[16+i]) otherwise
-        float y[32];
-        if (p.interleaved) {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) rope_turn(xr[2 * i], xr[2 * i + 1], cs[i], sn[i], y[2 * i], y[2 * i + 1]);
-        } else {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) rope_turn(xr[i], xr[16 + i], cs[i], sn[i], y[i], y[16 + i]);
-        }
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          uint4 v;
-          v.x = pack_f16x2(y[k * 8 + 0], y[k * 8 + 1]);
-          v.y = pack_f16x2(y[k * 8 + 2], y[k * 8 + 3]);
-          v.z = pack_f16x2(y[k * 8 + 4], y[k * 8 + 5]);
-          v.w = pack_f16x2(y[k * 8 + 6], y[k * 8 + 7]);
-          *reinterpret_cast<uint4*>(qr + sw128_offset(row, ch[k])) = v;
-#pragma unroll
-          for (int e = 0; e < 8; ++e) qmax = fmaxf(qmax, fabsf(y[k * 8 + e]));
-        }
       }
-      if (valid && !(qmax <= kF16Max)) raise_device_error(kDevErrRange);
-      fence_proxy_async_smem();
-      mbar_arrive(&bars.q_ready[x]);
+      tc_fence_before();
+      mbar_arrive(&bars.o_free[x]);
       return true;
     };
 
-    PairItem cur;
-    bool ok = next_item(cur);
-    if (ok && cur.valid) ok = prep_q(cur);
-    while (ok && cur.valid) {
+    // the item's output rows are written after the next item has been read,
+    // while its first score product (whose Q needed no preparation) runs
+    PairItem nxt;
+    bool ok = next_item(nxt);
+    bool have = false;                            // an item's output is pending
+    bool prev_valid = false;
+    int64_t prev_t = 0;
+    int prev_h = 0;
+    uint64_t l2[2] = {0ull, 0ull};                // row sum of e, as two fp32 pairs
+    while (ok) {
+      if (have && !(ok = epilogue(prev_valid, prev_t, prev_h, l2))) break;
+      if (!nxt.valid) break;
+      const PairItem cur = nxt;
       const int nX = x ? cur.nB : cur.nA;
       const int qrow = cur.q0 + x * kTile + row;  // in-sequence query index
       const bool valid = qrow < cur.L;
@@ -558,9 +507,9 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
       // causal mask applies there (one step without cached rows; with an
       // offset that is not a multiple of 128, two)
       const int jm = (cur.off + cur.q0 + x * kTile) / kPrBKV;
-      const int64_t t = cur.seq0 + qrow;
       float m = 0.f;                              // reference max (log2 units, scaled)
-      uint64_t l2[2] = {0ull, 0ull};              // row sum of e, as two fp32 pairs
+      l2[0] = 0ull;
+      l2[1] = 0ull;
       for (int j = 0; j < nX && ok; ++j) {
         if (!mbar_wait_warp(&bars.s_full[x], (uint32_t)ts & 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
@@ -623,14 +572,9 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const uint64_t a = f2_fma(f2_make(sc[c * 32 + 2 * e], sc[c * 32 + 2 * e + 1]), sl2, nb2);
-            uint64_t w;
-            if (c >= kPrBKV / 32 - kPrPolyChunks) {
-              w = ex2_fma2(a);
-            } else {
-              float a0, a1;
-              f2_split(a, a0, a1);
-              w = f2_make(ex2_approx(a0), ex2_approx(a1));
-            }
+            float a0, a1;
+            f2_split(a, a0, a1);
+            const uint64_t w = f2_make(ex2_approx(a0), ex2_approx(a1));
             l2[e & 1] = f2_add(l2[e & 1], w);
             float v0, v1;
             f2_split(f2_mul(w, k12), v0, v1);
@@ -644,35 +588,11 @@ attention_pair_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_co
         ++ts;
       }
       if (!ok) break;
-      // the next item's Q first (its first score product can start), then
-      // this item's output
-      PairItem nxt;
-      if (!(ok = next_item(nxt))) break;
-      if (nxt.valid && !(ok = prep_q(nxt))) break;
-      if (!(ok = mbar_wait_warp(&bars.pv_done[x], (uint32_t)(ts - 1) & 1u, abort_flag))) break;
-      tc_fence_after();
-      float la, lb, lc, ld;
-      f2_split(l2[0], la, lb);
-      f2_split(l2[1], lc, ld);
-      const float inv = (1.f / ((la + lb) + (lc + ld))) * kPrTwoMBias;
-      __nv_bfloat16* dst = p.out + (t * p.H + cur.h) * kV;
-#pragma unroll 1
-      for (int c = 0; c < kV / 32; ++c) {
-        uint32_t v[32];
-        tmem_ld32(tO + (uint32_t)(c * 32), v);
-        if (valid) {
-          uint32_t o[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e)
-            o[e] = pack_bf16x2(__uint_as_float(v[2 * e]) * inv, __uint_as_float(v[2 * e + 1]) * inv);
-          uint4* d4 = reinterpret_cast<uint4*>(dst + c * 32);
-#pragma unroll
-          for (int e = 0; e < 4; ++e) d4[e] = make_uint4(o[4 * e], o[4 * e + 1], o[4 * e + 2], o[4 * e + 3]);
-        }
-      }
-      tc_fence_before();
-      mbar_arrive(&bars.o_free[x]);
-      cur = nxt;
+      have = true;
+      prev_valid = valid;
+      prev_t = cur.seq0 + qrow;
+      prev_h = cur.h;
+      ok = next_item(nxt);
     }
   }
   tc_fence_before();

@@ -10,15 +10,16 @@
 // Precision: the normalized latent c_hat = w * x / rms(x) is formed in fp32
 // and handed to the tensor cores in fp16 (11 significant bits), against an
 // fp16 copy of the weight (exact for weights in fp16's normal range), with
-// fp32 accumulation; k_nope and the values are stored in fp16 (attention runs
-// its tensor-core products on fp16 operands). A value beyond the fp16 range
-// sets the device error word.
+// fp32 accumulation; the values are stored in fp16, k_nope in bf16 for the
+// two-tile attention (whose non-rotary score atoms take q as given, in bf16)
+// and in fp16 for the one-tile attention. A value beyond the fp16 range sets
+// the device error word.
 //
 // Workspace layout ("padded token space"): every sequence starts on a
 // 128-row boundary, so a 128-token tile never straddles two sequences and
 // every TMA coordinate along tokens is a multiple of 64 elements. Rows past a
 // sequence's end are written as zeros.
-//   k_nope [H, Tpad, N]  fp16   (row tp, N contiguous)
+//   k_nope [H, Tpad, N]  bf16 / fp16   (row tp, N contiguous)
 //   vt     [H, V, Tpad]  fp16   (values transposed: tokens contiguous)
 //   k_rot  [Tpad, P]     fp16   (the shared rotary key, rotated)
 #pragma once
@@ -61,6 +62,9 @@ __device__ __forceinline__ int block_inclusive_scan_1024(int v, int* s_warp /* [
   return v + (wid > 0 ? before : 0);
 }
 
+// Largest sequence count whose bounds the schedule keeps in shared memory.
+constexpr int kSchedSmemSeqs = 2048;
+
 // Run by one block of 1024 threads.
 __device__ __forceinline__ void schedule_block(const int32_t* __restrict__ cu, int nseq, int64_t Ttot,
                                                int max_seqlen, int cap, int32_t* __restrict__ seq_tile0,
@@ -74,6 +78,109 @@ __device__ __forceinline__ void schedule_block(const int32_t* __restrict__ cu, i
   __shared__ int s_cnt[kBuckets];
   __shared__ int s_off[kBuckets];
   const int tid = threadIdx.x;
+  if (nseq <= kSchedSmemSeqs) {
+    // fast path: cu_seqlens is read once into shared memory and every table
+    // is derived there (each of the general path's dependent global round
+    // trips costs a memory latency on the prefill's critical path)
+    __shared__ int s_t0[kSchedSmemSeqs + 1];     // first tile of each sequence
+    if (tid == 0) { s_bad = 0; s_carry = 0; *item_counter = 0; }
+    for (int k = tid; k < kBuckets; k += blockDim.x) { s_cnt[k] = 0; s_off[k] = 0; }
+    __syncthreads();
+    // per-sequence tile counts (1024 sequences per pass) -> exclusive scan
+    for (int base = 0; base < nseq; base += blockDim.x) {
+      const int sq = base + tid;
+      int n_here = 0;
+      if (sq < nseq) {
+        const int64_t a = cu[sq], b = cu[sq + 1];
+        if (a < 0 || b < a || b > Ttot || b - a > max_seqlen) s_bad = 1;
+        else n_here = (int)((b - a + kTile - 1) / kTile);
+      }
+      const int inc = block_inclusive_scan_1024(n_here, s_scan);
+      if (sq < nseq) s_t0[sq] = s_carry + inc - n_here;
+      __syncthreads();
+      if (tid == (int)blockDim.x - 1) s_carry += inc;
+      __syncthreads();
+    }
+    if (tid == 0) s_t0[nseq] = s_carry;
+    __syncthreads();
+    const int total = s_t0[nseq];
+    if (s_bad || total > cap) {
+      for (int i = tid; i < cap; i += blockDim.x) { tile_seq[i] = -1; tile_q0[i] = -1; order[i] = -1; pair_order[i] = -1; }
+      if (tid == 0) raise_device_error(kDevErrBadInput);
+      return;
+    }
+    for (int i = tid; i <= nseq; i += blockDim.x) seq_tile0[i] = s_t0[i];
+    // tiles in natural order; bucket counts of causal work (tile index in
+    // its sequence) for single tiles and for 256-row blocks. Every entry of
+    // pair_order starts at -1 here: the blocks fill only its first entries
+    // (one per two tiles), after the barriers below.
+    for (int t = tid; t < cap; t += blockDim.x) {
+      pair_order[t] = -1;
+      if (t >= total) { tile_seq[t] = -1; tile_q0[t] = -1; order[t] = -1; continue; }
+      int lo = 0, hi = nseq - 1;               // the sequence whose tiles hold t
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_t0[mid] <= t) lo = mid;
+        else hi = mid - 1;
+      }
+      const int k = t - s_t0[lo];
+      tile_seq[t] = lo;
+      tile_q0[t] = k * kTile;
+      atomicAdd(&s_cnt[min(k, kBuckets - 1)], 1);
+    }
+    __syncthreads();
+    {
+      const int k0 = kBuckets - 1 - 2 * tid, k1 = k0 - 1;
+      const int c0 = s_cnt[k0], c1 = s_cnt[k1];
+      const int before = block_inclusive_scan_1024(c0 + c1, s_scan) - (c0 + c1);
+      s_off[k0] = before;
+      s_off[k1] = before + c0;
+    }
+    __syncthreads();
+    for (int t = tid; t < total; t += blockDim.x) {
+      int lo = 0, hi = nseq - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_t0[mid] <= t) lo = mid;
+        else hi = mid - 1;
+      }
+      const int pos = atomicAdd(&s_off[min(t - s_t0[lo], kBuckets - 1)], 1);
+      order[pos] = t;
+    }
+    __syncthreads();
+    for (int k = tid; k < kBuckets; k += blockDim.x) s_cnt[k] = 0;
+    __syncthreads();
+    for (int t = tid; t < total; t += blockDim.x) {
+      int lo = 0, hi = nseq - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_t0[mid] <= t) lo = mid;
+        else hi = mid - 1;
+      }
+      const int k = t - s_t0[lo];
+      if ((k & 1) == 0) atomicAdd(&s_cnt[min(k / 2, kBuckets - 1)], 1);
+    }
+    __syncthreads();
+    {
+      const int k0 = kBuckets - 1 - 2 * tid, k1 = k0 - 1;
+      const int c0 = s_cnt[k0], c1 = s_cnt[k1];
+      const int before = block_inclusive_scan_1024(c0 + c1, s_scan) - (c0 + c1);
+      s_off[k0] = before;
+      s_off[k1] = before + c0;
+    }
+    __syncthreads();
+    for (int t = tid; t < total; t += blockDim.x) {
+      int lo = 0, hi = nseq - 1;
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (s_t0[mid] <= t) lo = mid;
+        else hi = mid - 1;
+      }
+      const int k = t - s_t0[lo];
+      if ((k & 1) == 0) pair_order[atomicAdd(&s_off[min(k / 2, kBuckets - 1)], 1)] = t;
+    }
+    return;
+  }
   if (tid == 0) { s_bad = 0; s_carry = 0; *item_counter = 0; }
   for (int i = tid; i < cap; i += blockDim.x) {
     tile_seq[i] = -1; tile_q0[i] = -1; order[i] = -1; pair_order[i] = -1;
@@ -159,11 +266,88 @@ __device__ __forceinline__ void schedule_block(const int32_t* __restrict__ cu, i
 
 // ---- prefill preparation: tile schedule, fp16 weight, normalized latent ----
 // Block 0 builds the schedule (schedule_block); blocks 1 .. w_blocks convert
-// the weight, kPrepUnroll x 8 values per thread; the blocks after them (when launched)
-// write the normalized latent in fp16 for the transposed-value GEMM. A value
-// beyond the fp16 range sets the device error word.
+// the weight, kPrepUnroll x 8 values per thread; the next norm_blocks (when
+// launched) write the normalized latent in fp16 for the transposed-value
+// GEMM, and the blocks after those the rotated query rows (q_rope_group,
+// four threads per row). A value beyond the fp16 range sets the device error
+// word.
 constexpr int kPrepThreads = 1024;
 constexpr int kPrepUnroll = 8;
+
+// The rotary part of every query head, turned at its token's position once
+// for all key steps: qr [Ttot, H, 64] fp16 (the two-tile attention's last
+// score atom). Source: Kimi-K2 "RoPE coefficients" page, "Query heads": each
+// head's rotary query part is rotated at the token's position like the key's.
+struct QRopeParams {
+  const __nv_bfloat16* q;       // [Ttot, H, D], the rotary part in columns N .. N + 63
+  const int32_t* positions;     // [Ttot]
+  const float* cos_t;           // [max_pos, 32]
+  const float* sin_t;
+  __half* qr;                   // [Ttot, H, 64]
+  int64_t rows;                 // Ttot * H
+  int H, D, N, max_pos, interleaved;
+};
+
+// Pairs 8g .. 8g + 7 (g < 4) of row `row` = (t, h) of qr: pair i is
+// (x_i, x_{i+32}) (half-split) or (x_{2i}, x_{2i+1}) (interleaved), turned by
+// the angle of pair i at positions[t], each result rounded once to fp16.
+// Their values are the row's 16-byte chunks g and g + 4 (half-split) or 2g and
+// 2g + 1 (interleaved), so four threads with g = 0 .. 3 write a row's 128
+// bytes. mx takes the largest magnitude written (the caller checks the fp16
+// range).
+__device__ __forceinline__ void q_rope_group(const QRopeParams& p, int64_t row, int g, float& mx) {
+  const int64_t t = row / p.H;
+  const int64_t pos = checked_pos(p.positions[t], p.max_pos);
+  const uint4* src = reinterpret_cast<const uint4*>(p.q + row * p.D + p.N);
+  uint4* dst = reinterpret_cast<uint4*>(p.qr + row * 64);
+  const float4* c4 = reinterpret_cast<const float4*>(p.cos_t + pos * 32);
+  const float4* s4 = reinterpret_cast<const float4*>(p.sin_t + pos * 32);
+  const int ca = p.interleaved ? 2 * g : g, cb = p.interleaved ? 2 * g + 1 : g + 4;
+  const uint4 va = src[ca], vb = src[cb];
+  const float4 c0 = c4[2 * g], c1 = c4[2 * g + 1], s0 = s4[2 * g], s1 = s4[2 * g + 1];
+  const float cs[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
+  const float sn[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
+  const uint32_t wa[4] = {va.x, va.y, va.z, va.w}, wb[4] = {vb.x, vb.y, vb.z, vb.w};
+  float x[16];                        // chunk a, then chunk b
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    const float2 fa = unpack_bf16x2(wa[e]), fb = unpack_bf16x2(wb[e]);
+    x[2 * e] = fa.x; x[2 * e + 1] = fa.y;
+    x[8 + 2 * e] = fb.x; x[8 + 2 * e + 1] = fb.y;
+  }
+  float y[16];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    if (p.interleaved) rope_turn(x[2 * i], x[2 * i + 1], cs[i], sn[i], y[2 * i], y[2 * i + 1]);
+    else rope_turn(x[i], x[8 + i], cs[i], sn[i], y[i], y[8 + i]);
+  }
+  uint32_t oa[4], ob[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    mx = fmaxf(mx, fmaxf(fmaxf(fabsf(y[2 * e]), fabsf(y[2 * e + 1])), fmaxf(fabsf(y[8 + 2 * e]), fabsf(y[9 + 2 * e]))));
+    oa[e] = pack_f16x2(y[2 * e], y[2 * e + 1]);
+    ob[e] = pack_f16x2(y[8 + 2 * e], y[9 + 2 * e]);
+  }
+  dst[ca] = make_uint4(oa[0], oa[1], oa[2], oa[3]);
+  dst[cb] = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+}
+
+// Thread i of a grid-stride range: group i % 4 of row i / 4; a value beyond
+// the fp16 range sets the device error word.
+__device__ __forceinline__ void q_rope_unit(const QRopeParams& p, int64_t i) {
+  float mx = 0.f;
+  if (i < 4 * p.rows) q_rope_group(p, i >> 2, (int)(i & 3), mx);
+  if (!(mx <= kF16Max)) raise_device_error(kDevErrRange);
+}
+
+// The rotated query rows on their own (chunks over a cached prefix, whose
+// positions the previous kernel writes), four threads per row.
+__global__ void __launch_bounds__(kPrepThreads)
+q_rope_kernel(QRopeParams p) {
+  pdl_wait();
+  pdl_allow_next();
+  q_rope_unit(p, (int64_t)blockIdx.x * kPrepThreads + threadIdx.x);
+}
 
 // Block `blk` of the fp16 weight copy: kPrepUnroll x 8 values per thread
 // (n8 groups of 8 values in all). A value beyond the fp16 range sets the
@@ -201,11 +385,15 @@ prefill_prep_kernel(const int32_t* __restrict__ cu, int nseq, int64_t Ttot, int 
                     int32_t* __restrict__ item_counter,
                     const __nv_bfloat16* __restrict__ w, __half* __restrict__ w16, int64_t n8, int w_blocks,
                     const __nv_bfloat16* __restrict__ latent, const __nv_bfloat16* __restrict__ w_norm, int R,
-                    float eps, __half* __restrict__ c16) {
+                    float eps, __half* __restrict__ c16, int norm_blocks, QRopeParams qrp) {
   pdl_allow_next();
   if (blockIdx.x == 0) {
     schedule_block(cu, nseq, Ttot, max_seqlen, cap, seq_tile0, tile_seq, tile_q0, order, pair_order,
                    item_counter);
+    return;
+  }
+  if ((int)blockIdx.x > w_blocks + norm_blocks) {
+    q_rope_unit(qrp, (int64_t)((int)blockIdx.x - 1 - w_blocks - norm_blocks) * kPrepThreads + threadIdx.x);
     return;
   }
   if ((int)blockIdx.x > w_blocks) {
@@ -301,6 +489,9 @@ struct GemmParams {
   // already in the padded layout (tile t = rows 128 t ..) and k_rot has been
   // written with it, so the tile's A rows are padded rows and k_rot is left
   int a_padded;
+  // 1: k_nope is stored as bf16 (the two-tile attention's score operand),
+  // 0: as fp16 (the one-tile attention's); the buffer holds 16-bit codes
+  int knope_bf16;
 };
 
 struct GemmBarriers {
@@ -483,7 +674,7 @@ norm_kvb_gemm_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_c
         for (int i = 0; i < p.P; ++i) dst[i] = __float2half_rn(0.f);
       }
     }
-    // epilogue: TMEM -> bf16 k_nope / transposed values
+    // epilogue: TMEM -> k_nope (fp16 or bf16) / transposed values (fp16)
     const int NV = p.N + p.V;
     float vmax = 0.f;
     for (int i = 0; i < my_tiles && ok; ++i) {
@@ -497,13 +688,21 @@ norm_kvb_gemm_kernel(const __grid_constant__ CUtensorMap map_lat, const __grid_c
         const int o0 = o_base + ch * 16;
         if (o0 >= p.NOUT) continue;
         const int h = o0 / NV, c0 = o0 % NV;
+        if (c0 >= p.N || !p.knope_bf16) {
 #pragma unroll
-        for (int e = 0; e < 16; ++e) vmax = fmaxf(vmax, fabsf(__uint_as_float(v[e])));
+          for (int e = 0; e < 16; ++e) vmax = fmaxf(vmax, fabsf(__uint_as_float(v[e])));
+        }
         if (c0 < p.N) {
           uint32_t pk[8];
+          if (p.knope_bf16) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            pk[e] = pack_f16x2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+            for (int e = 0; e < 8; ++e)
+              pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e)
+              pk[e] = pack_f16x2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+          }
           uint4* dst = reinterpret_cast<uint4*>(p.k_nope + ((int64_t)h * p.Tpad + tp) * p.N + c0);
           dst[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
           dst[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
@@ -722,18 +921,24 @@ norm_kvb_gemm_vt_kernel(const __grid_constant__ CUtensorMap map_chat, const __gr
       uint4* dst = half ? reinterpret_cast<uint4*>(p.vt + ((int64_t)h * kV + lrow) * p.Tpad + tp0)
                         : reinterpret_cast<uint4*>(p.k_nope + ((int64_t)h * p.Tpad + tp0 + lrow) * kN);
       const int nchunks = half ? kTile / 32 : kN / 32;
+      const bool kb = !half && p.knope_bf16;   // warp-uniform
       for (int c = 0; c < nchunks; ++c) {
         uint32_t v[32];
         tmem_ld32(src + (uint32_t)(c * 32), v);
         uint32_t pk[16];
+        if (kb) {
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const float a = __uint_as_float(v[2 * e]), b = __uint_as_float(v[2 * e + 1]);
-          vmax = fmaxf(vmax, fmaxf(fabsf(a), fabsf(b)));
-          pk[e] = pack_f16x2(a, b);
+          for (int e = 0; e < 16; ++e) pk[e] = pack_bf16x2(__uint_as_float(v[2 * e]), __uint_as_float(v[2 * e + 1]));
+        } else {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const float a = __uint_as_float(v[2 * e]), b = __uint_as_float(v[2 * e + 1]);
+            vmax = fmaxf(vmax, fmaxf(fabsf(a), fabsf(b)));
+            pk[e] = pack_f16x2(a, b);
+          }
         }
-#pragma unroll
-        for (int e = 0; e < 4; ++e) dst[c * 4 + e] = make_uint4(pk[4 * e], pk[4 * e + 1], pk[4 * e + 2], pk[4 * e + 3]);
+        st_global_v8(dst + c * 4, pk);
+        st_global_v8(dst + c * 4 + 2, pk + 8);
       }
       tc_fence_before();
       mbar_arrive(&bars.acc_empty[acc]);

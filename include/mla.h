@@ -145,7 +145,7 @@ int mla_prepare_kv_b_proj(const mla_dims* dims, const void* w_kvb, void* prepare
  * kernels and the same results (bit for bit), minus the per-call conversion.
  * For the tensor-core head shapes every tensor and the workspace must be
  * 16-byte aligned (MLA_ERR_INVALID_ARG otherwise: this entry point has no
- * fallback to the CUDA-core kernels for them). */
+ * fallback to the CUDA-core kernels for them), and out 32-byte aligned. */
 int mla_prefill_prepared(const mla_dims* dims,
                          const void* latent, const void* q, const void* w_prepared, const void* w_norm,
                          const int32_t* positions, const int32_t* cu_seqlens,
@@ -228,7 +228,7 @@ int mla_prefill_cached_workspace_size(const mla_dims* dims, int64_t total_tokens
  * tokens of the rows each attends (the absorbed form). Long chunks take the
  * eager form instead when it applies: bf16 with qk_rope 64, v_head 128,
  * qk_nope 64 or 128, at least 128 chunk tokens per sequence on average,
- * 16-byte aligned q, cache, w_kvb, out and workspace, and a workspace of at
+ * 16-byte aligned q, cache, w_kvb and workspace, 32-byte aligned out, and a workspace of at
  * least mla_prefill_cached_eager_workspace_size bytes. It expands the keys and
  * values of every row of each sequence (prefix and chunk) with the
  * up-projection and runs the prefill's attention over them, so its cost
@@ -389,9 +389,9 @@ const char* mla_last_error_string(void);
 
 /* Which kernels the calling thread's last prefill or decode call launched:
  * "tensor-core", or "simt: <reason>" when it ran the exact CUDA-core kernels
- * instead (a head shape or dtype outside the tensor-core kernels, or a tensor
- * that is not 16-byte aligned). Static storage, never NULL; "none" before the
- * first call. */
+ * instead (a head shape or dtype outside the tensor-core kernels, a tensor
+ * that is not 16-byte aligned, or a prefill output that is not 32-byte
+ * aligned). Static storage, never NULL; "none" before the first call. */
 const char* mla_last_dispatch(void);
 
 /* Profiling support. Registers `pairs` pairs of host cudaEvent_t handles
