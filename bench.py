@@ -397,6 +397,7 @@ def run_ours(args, rank, world, device):
     # the prefill with kv_b_proj converted inside the call (mla_prefill)
     unprep_ms = reduce_max(time_calls(args, prefill_unprepared, flush))
     chunk = run_chunk(args, din, D, device, world, reduce_max, peaks)
+    chunk["long"] = run_chunk_long(args, device, world, reduce_max, peaks, flush)
     projections = run_projections(args, device, world, reduce_max, peaks)
     configs = run_configs(args, device, world, reduce_max, peaks, flush)
 
@@ -649,6 +650,52 @@ def run_chunk(args, din, D, device, world, reduce_max, peaks, n_new=4):
                 ms=ms, tokens_per_s=world * T / (ms * 1e-3), attended_gbs=att,
                 attended_frac_of_hbm=att / (world * peaks["hbm"]),
                 unique_cache_gbs=world * by["unique"] / (ms * 1e-3) / 1e9,
+                kernels_ms=dict(zip(kev.names, kev.durations_ms())))
+
+
+def run_chunk_long(args, device, world, reduce_max, peaks, flush, nseq=4, prefix=16384, n_new=2048):
+    """Long chunks over long cached prefixes: ``nseq`` sequences of ``prefix``
+    cached rows, each continued by ``n_new`` new tokens in one
+    mla_prefill_cached call (the library picks the eager form: every cached
+    row's keys and values are expanded once by the up-projection GEMM and the
+    chunk's queries attend to them causally in absolute positions). FLOPs:
+    the up-projection of every key row plus the attention of every chunk token
+    to its prefix, the chunk tokens before it and itself."""
+    cwl = W.scaled(W.KIMI, kind="prefill", seqlens=(n_new,) * nseq, seed=7,
+                   extra=dict(prefix_lens=(prefix,) * nseq))
+    cin = W.chunk_inputs(cwl)
+    dims = mla.dims_for(cwl, mla.mla_softmax_scale(mla.rope_for(cwl), cwl.qk_head_dim))
+    max_total = int(cin["max_total_len"])
+    cos, sin = mla.mla_init_rope_tables(mla.rope_for(cwl), max_total)
+    C = {k: v.to(device) for k, v in cin.items() if isinstance(v, torch.Tensor)}
+    T = nseq * n_new
+    out = torch.empty((T, cwl.num_heads, cwl.v_head), dtype=torch.bfloat16, device=device)
+    ws = torch.empty(mla.mla_prefill_cached_eager_workspace_size(dims, T, nseq, max_total), dtype=torch.uint8,
+                     device=device)
+
+    def call():
+        mla.mla_prefill_cached(dims, C["latent"], C["q"], C["w_kvb"], C["w_norm"], C["cu_seqlens"],
+                               C["cache_offsets"], C["prefix_lens"], max_total, cos, sin, C["cache"], out=out,
+                               workspace=ws)
+
+    ms = reduce_max(time_calls(args, call, flush))
+    form = mla.mla_last_dispatch()
+    kev = mla.KernelEvents(16)
+    with kev:
+        call()
+    torch.cuda.synchronize()
+    mla.mla_check_device_status()
+    H, R, N, V = cwl.num_heads, cwl.kv_lora_rank, cwl.qk_nope, cwl.v_head
+    D = N + cwl.qk_rope
+    keys = nseq * (prefix + n_new)
+    pairs = nseq * (n_new * prefix + n_new * (n_new + 1) // 2)
+    flops = 2.0 * keys * R * H * (N + V) + 2.0 * pairs * H * (D + V)
+    tflops = world * flops / (ms * 1e-3) / 1e12
+    unique = keys * (R + cwl.qk_rope) * 2
+    return dict(workload="%d sequences of %d cached rows, %d new tokens each" % (nseq, prefix, n_new),
+                form=form, ms=ms, tokens_per_s=world * T / (ms * 1e-3), gflop=flops / 1e9, tflops=tflops,
+                frac_of_bf16_peak=tflops / (world * peaks["bf16"]),
+                unique_cache_gbs=world * unique / (ms * 1e-3) / 1e9,
                 kernels_ms=dict(zip(kev.names, kev.durations_ms())))
 
 

@@ -181,6 +181,21 @@ def test_decode_full_sampled(gpu_lib):
     compare(got, absorbed, "bf16", "decode vs absorbed")
 
 
+def test_decode_longest_all_heads(gpu_lib):
+    # the longest cache length of the decode workload (32768 rows) next to a
+    # short one, every head checked against the oracle (its absorbed form,
+    # which is the same fp64 value up to rounding at a fraction of the cost);
+    # the long row spans many CTAs' row ranges, so its output merges many
+    # partials
+    wl = W.scaled(W.DECODE, batch=2, cache_lens=(32768, 3), seed=17)
+    inp = W.decode_inputs(wl)
+    got = f64(run_decode(wl, inp))
+    ref = oracle_decode(wl, inp, batches=[0, 1], absorbed=True)
+    compare(got, ref, "bf16", "decode L=32768 all heads")
+    eager = oracle_decode(wl, inp, batches=[0], heads=[0, 63])
+    compare(got, eager, "bf16", "decode L=32768 vs eager")
+
+
 def test_cache_append_then_decode_matches_prefill_row(gpu_lib):
     # Append every token of two sequences to a latent cache on the GPU, then a
     # decode step for each sequence's last token must reproduce the oracle's
