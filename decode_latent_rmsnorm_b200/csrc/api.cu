@@ -240,8 +240,11 @@ size_t prefill_ws_bytes(const mla_dims* d, int64_t T, int nseq) {
 }
 
 // Shapes the tensor-core decode takes (bf16, 64 heads, 512 + 64 latent row).
+// Up to 64 heads: fewer heads (a head-sharded decode) are padded to 64 with
+// zero queries, whose outputs are never un-absorbed; the kernel streams the
+// same cache bytes either way.
 bool decode_tc_shape(const mla_dims* d) {
-  return d->dtype == MLA_BF16 && d->num_heads == mla::tc::kDecHeads && d->kv_lora_rank == 512 &&
+  return d->dtype == MLA_BF16 && d->num_heads >= 1 && d->num_heads <= mla::tc::kDecHeads && d->kv_lora_rank == 512 &&
          d->qk_rope == 64 && d->qk_nope % 64 == 0 && d->qk_nope >= 64;
 }
 
@@ -271,15 +274,16 @@ DecodeWs decode_ws_layout(const mla_dims* d, int B, int max_len, bool tc) {
   const size_t H = d->num_heads, R = d->kv_lora_rank, P = d->qk_rope;
   size_t off = 0;
   if (tc) {
+    const size_t Hp = mla::tc::kDecHeads;   // heads padded to the kernel's 64
     w.G = num_sms();
     const size_t slots = (size_t)B + w.G;
     w.prefix = off; off = align_up(off + 8 * (size_t)(B + 1), 256);
     w.meta = off;   off = align_up(off + 16, 256);
-    w.qf = off;     off = align_up(off + 2 * (size_t)B * H * (R + P), 256);
-    w.o_part = off; off = align_up(off + 4 * slots * H * R, 256);
-    w.m_part = off; off = align_up(off + 4 * slots * H, 256);
-    w.l_part = off; off = align_up(off + 4 * slots * H, 256);
-    w.o_lat = off;  off = align_up(off + 2 * (size_t)B * H * R, 256);
+    w.qf = off;     off = align_up(off + 2 * (size_t)B * Hp * (R + P), 256);
+    w.o_part = off; off = align_up(off + 4 * slots * Hp * R, 256);
+    w.m_part = off; off = align_up(off + 4 * slots * Hp, 256);
+    w.l_part = off; off = align_up(off + 4 * slots * Hp, 256);
+    w.o_lat = off;  off = align_up(off + 2 * (size_t)B * Hp * R, 256);
     w.total = off;
     return w;
   }
@@ -652,6 +656,7 @@ int launch_decode_tc(const mla_dims* d, const void* q, const void* cache, int64_
   using bf16 = __nv_bfloat16;
   namespace T = mla::tc;
   const int H = d->num_heads, R = d->kv_lora_rank, N = d->qk_nope, P = d->qk_rope, V = d->v_head;
+  const int Hp = T::kDecHeads;   // the workspace's head count: H padded with zero queries
   const DecodeWs L = decode_ws_layout(d, B, max_len, true);
   char* ws = static_cast<char*>(workspace);
   int64_t* prefix = reinterpret_cast<int64_t*>(ws + L.prefix);
@@ -671,9 +676,9 @@ int launch_decode_tc(const mla_dims* d, const void* q, const void* cache, int64_
     if (rc) return rc;
   }
   {
-    const uint64_t dims[2] = {(uint64_t)(R + P), (uint64_t)B * H};
+    const uint64_t dims[2] = {(uint64_t)(R + P), (uint64_t)B * Hp};
     const uint64_t strides[1] = {(uint64_t)(R + P) * 2};
-    const uint32_t box[2] = {64, (uint32_t)T::kDecHeads};
+    const uint32_t box[2] = {64, (uint32_t)Hp};
     int rc = make_map(&map_q, qf, 2, dims, strides, box);
     if (rc) return rc;
   }
@@ -697,8 +702,8 @@ int launch_decode_tc(const mla_dims* d, const void* q, const void* cache, int64_
     if (rc) return rc;
   }
   {
-    const uint64_t dims[3] = {(uint64_t)R, (uint64_t)H, (uint64_t)B};
-    const uint64_t strides[2] = {(uint64_t)R * 2, (uint64_t)H * R * 2};
+    const uint64_t dims[3] = {(uint64_t)R, (uint64_t)Hp, (uint64_t)B};
+    const uint64_t strides[2] = {(uint64_t)R * 2, (uint64_t)Hp * R * 2};
     const uint32_t box[3] = {64, 1, 64};
     int rc = make_map(&map_ol, o_lat, 3, dims, strides, box);
     if (rc) return rc;
@@ -709,10 +714,16 @@ int launch_decode_tc(const mla_dims* d, const void* q, const void* cache, int64_
   e = cudaFuncSetAttribute(T::head_gemm_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)T::kHgSmem);
   if (e != cudaSuccess) return cuda_status(e, "head gemm smem attribute");
   {
+    if (H < Hp) {   // the padded heads' queries are zero (their scores are zero; their outputs unused)
+      e = cudaMemset2DAsync(qf + (size_t)H * (R + P), (size_t)Hp * (R + P) * 2, 0, (size_t)(Hp - H) * (R + P) * 2,
+                            (size_t)B, st);
+      if (e != cudaSuccess) return cuda_status(e, "decode query padding");
+    }
     T::HgParams hp{};
     hp.out = qf;
-    hp.out_bs = (int64_t)H * (R + P);
+    hp.out_bs = (int64_t)Hp * (R + P);
     hp.out_hs = R + P;
+    hp.qf_heads = Hp;
     hp.B = B;
     hp.Nout = R;
     hp.K = N;
@@ -746,7 +757,7 @@ int launch_decode_tc(const mla_dims* d, const void* q, const void* cache, int64_
   dp.m_part = m_part;
   dp.l_part = l_part;
   dp.B = B;
-  dp.H = H;
+  dp.H = Hp;
   dp.R = R;
   dp.scale_log2 = d->softmax_scale * 1.4426950408889634f;
   e = cudaFuncSetAttribute(T::decode_attn_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)T::kDecSmem);
@@ -758,7 +769,7 @@ int launch_decode_tc(const mla_dims* d, const void* q, const void* cache, int64_
 
   prof_begin(st, "tc_decode_combine");
   e = launch_dependent(T::decode_combine_kernel, dim3(B, (H + 3) / 4), dim3(256), 0, st, (const float*)o_part,
-                       (const float*)m_part, (const float*)l_part, (const int64_t*)prefix, (const int64_t*)meta, H, R,
+                       (const float*)m_part, (const float*)l_part, (const int64_t*)prefix, (const int64_t*)meta, Hp, R,
                        o_lat);
   prof_end(st);
   if (e != cudaSuccess) return cuda_status(e, "decode combine launch");

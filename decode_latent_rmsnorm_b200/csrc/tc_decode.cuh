@@ -83,22 +83,23 @@ __device__ __forceinline__ void decode_schedule_block(const int32_t* __restrict_
 }
 
 // q_pe rotated at the query position, into the last P columns of qf rows.
-// q_pe of sequences [b0, b0 + nb) and head h, rotated at each sequence's
-// position, into qf[b, h, R:] (bf16). Rotary width P = 64: the 128 calling
+// q_pe of sequences [b0, b0 + nb) and head h (q holds H heads per sequence),
+// rotated at each sequence's position, into qf[b, h, R:] (bf16; qf holds Hq
+// heads per sequence). Rotary width P = 64: the 128 calling
 // threads take one sequence and half of its 32 pairs each, as vector loads
 // (half-split pairing: values [16 hp, 16 hp + 16) and [32 + 16 hp, 48 + 16 hp);
 // interleaved: values [32 hp, 32 hp + 32)).
 __device__ __forceinline__ void decode_qrope_rows(const __nv_bfloat16* __restrict__ q,
                                                   const int32_t* __restrict__ positions,
                                                   const float* __restrict__ cos_t, const float* __restrict__ sin_t,
-                                                  int max_pos, int h, int b0, int nb, int H, int R, int N,
-                                                  int interleaved, __nv_bfloat16* __restrict__ qf, int tid) {
+                                                  int max_pos, int h, int b0, int nb, int H, int Hq, int R,
+                                                  int N, int interleaved, __nv_bfloat16* __restrict__ qf,
+                                                  int tid) {
   const int b = b0 + (tid >> 1), hp = tid & 1;
   if ((tid >> 1) >= nb) return;
   const int64_t pos = checked_pos(positions[b], max_pos);
-  const int64_t bh = (int64_t)b * H + h;
-  const uint4* src = reinterpret_cast<const uint4*>(q + bh * (N + 64) + N);
-  uint4* dst = reinterpret_cast<uint4*>(qf + bh * (R + 64) + R);
+  const uint4* src = reinterpret_cast<const uint4*>(q + ((int64_t)b * H + h) * (N + 64) + N);
+  uint4* dst = reinterpret_cast<uint4*>(qf + ((int64_t)b * Hq + h) * (R + 64) + R);
   const float4* c4 = reinterpret_cast<const float4*>(cos_t + pos * 32 + hp * 16);
   const float4* s4 = reinterpret_cast<const float4*>(sin_t + pos * 32 + hp * 16);
   int ch[4];   // 16-byte chunks (8 values) of the row holding this thread's pairs
@@ -650,6 +651,7 @@ struct HgParams {
   const float* cos_t;
   const float* sin_t;
   int max_pos, N, interleaved;     // rotary width 64
+  int qf_heads;                    // heads per sequence in the output rows (the padded count)
   const int32_t* lens;
   const int64_t* offsets;
   int max_len, G;
@@ -767,7 +769,7 @@ head_gemm_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constan
     }
     if (kAMN && blockIdx.y == 0)
       decode_qrope_rows(p.q, p.positions, p.cos_t, p.sin_t, p.max_pos, h, b0, min(64, p.B - b0), gridDim.x - 1,
-                        p.Nout, p.N, p.interleaved, p.out, threadIdx.x - 64);
+                        p.qf_heads, p.Nout, p.N, p.interleaved, p.out, threadIdx.x - 64);
   }
   tc_fence_before();
   __syncthreads();

@@ -23,7 +23,14 @@
  *   - The return value is an mla_status. mla_last_error_string() gives a
  *     text for the last non-zero status of the calling thread.
  *   - MLA_BF16 runs read and write bfloat16 tensors and accumulate in fp32;
- *     MLA_FP32 runs are fp32 throughout (exact-fp32 SIMT kernels).
+ *     MLA_FP32 runs are fp32 throughout (exact-fp32 SIMT kernels). Inside a
+ *     bf16 prefill on the tensor cores the normalized latent and kv_b_proj
+ *     enter the up-projection in fp16; the two-tile attention (qk_nope and
+ *     v_head 64 or 128) multiplies q as given with k_nope rounded to bf16 for
+ *     the non-rotary scores and the rotated q_pe and k_pe rounded to fp16 for
+ *     the rotary ones, and the softmax weights with the values in fp16; the
+ *     other head shapes use fp16 for all of these. Values beyond the fp16
+ *     range in those fp16 buffers set the device error word.
  */
 #ifndef MLA_H_
 #define MLA_H_
@@ -174,6 +181,12 @@ int mla_decode_workspace_size(const mla_dims* dims, int32_t batch, int32_t max_c
  * o_lat = softmax(s) . c_hat, out = W_UV_h o_lat, where W_UK_h / W_UV_h are
  * the k_nope / value rows of head h in w_kvb. Attention is split over rows
  * and the pieces are merged by their log-sum-exp.
+ * The tensor-core kernels take bf16 runs with R = 512, P = 64, N a multiple
+ * of 64 and 1..64 heads (fewer than 64, e.g. one GPU's share of a
+ * head-sharded model, are padded to 64 with zero queries whose outputs are
+ * dropped: the call streams the same cache bytes as with 64 heads), 16-byte
+ * aligned cache and workspace, and fewer than 2^31 cache rows; other calls
+ * run on the CUDA cores (mla_last_dispatch says which and why).
  * Device-resident arguments are range-checked on the device: a sequence whose
  * rows fall outside the cache, whose length is outside 1..max_cache_len or
  * whose position is outside the table is skipped (its output is zero) and the

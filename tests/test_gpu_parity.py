@@ -163,6 +163,19 @@ def test_decode_glm_heads_interleaved_b70(gpu_lib):
     compare(f64(got), ref, "bf16", "decode glm b70")
 
 
+@pytest.mark.parametrize("heads", [8, 16, 32])
+def test_decode_fewer_heads_tensor_core(gpu_lib, heads):
+    # one GPU's share of a head-sharded Kimi-K2 decode: the tensor-core
+    # kernels pad the heads to 64 with zero queries and drop their outputs
+    wl = W.Workload("kimi_decode_h%d" % heads, "decode", heads, 512, 128, 64, 128, "bf16", W.KIMI_ROPE,
+                    20 + heads, batch=6, cache_lens=(1, 127, 129, 700, 2049, 5000))
+    inp = W.decode_inputs(wl)
+    got = run_decode(wl, inp)
+    assert mla.mla_last_dispatch().startswith("tensor-core"), mla.mla_last_dispatch()
+    ref = oracle_decode(wl, inp, batches=range(6))
+    compare(f64(got), ref, "bf16", "decode %d heads" % heads)
+
+
 def test_decode_fp32_tiny_geometry(gpu_lib):
     wl = W.Workload("tiny_decode_fp32", "decode", 2, 64, 16, 8, 16, "fp32", W.TINY_ROPE, 15,
                     batch=3, cache_lens=(1, 40, 333))
