@@ -85,7 +85,11 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   __shared__ AttBarriers<kStages> bars;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_allow_next();
-  const int rank = blockIdx.x / p.H, h = blockIdx.x % p.H;
+  // head-major grid: the CTAs that run at the same time share a head's keys
+  // and values, which stay in L2 (heads interleaved, every CTA streamed its
+  // keys and values from DRAM); within a head, heaviest tiles first
+  const int n_rank = (int)gridDim.x / p.H;
+  const int rank = (int)blockIdx.x % n_rank, h = (int)blockIdx.x / n_rank;
   const int tile = p.order[rank];
   if (tile < 0) return;   // uniform over the CTA
   const int seq = p.tile_seq[tile];
