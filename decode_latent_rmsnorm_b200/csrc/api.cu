@@ -347,8 +347,9 @@ int launch_prefill(const mla_dims* d, const void* latent, const void* q, const v
 }
 
 template <int kN, int kV>
-int launch_attention_tc_t(unsigned grid, const CUtensorMap& mq, const CUtensorMap& mkn, const CUtensorMap& mkr,
-                          const CUtensorMap& mvt, const mla::tc::AttParams& ap, cudaStream_t st) {
+int launch_attention_tc_t(unsigned grid, const CUtensorMap& mq, const CUtensorMap& mqr, const CUtensorMap& mkn,
+                          const CUtensorMap& mkr, const CUtensorMap& mvt, const mla::tc::AttParams& ap,
+                          cudaStream_t st) {
   // deepest K/V pipeline that fits next to Q and P in 227 KB of shared memory
   constexpr size_t kBase = mla::tc::AttCfg<kN, kV, 1>::kSmem - mla::tc::AttCfg<kN, kV, 1>::kStageBytes;
   constexpr size_t kStage = mla::tc::AttCfg<kN, kV, 1>::kStageBytes;
@@ -360,16 +361,16 @@ int launch_attention_tc_t(unsigned grid, const CUtensorMap& mq, const CUtensorMa
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
   if (e != cudaSuccess) return cuda_status(e, "attention smem attribute");
   prof_begin(st, "tc_attention");
-  e = launch_dependent(kern, dim3(grid), dim3(mla::tc::kAttThreads), C::kSmem, st, mq, mkn, mkr, mvt, ap);
+  e = launch_dependent(kern, dim3(grid), dim3(mla::tc::kAttThreads), C::kSmem, st, mq, mqr, mkn, mkr, mvt, ap);
   prof_end(st);
   return cuda_status(e, "attention launch");
 }
 
-int launch_attention_tc(int N, int V, unsigned grid, const CUtensorMap& mq, const CUtensorMap& mkn,
-                        const CUtensorMap& mkr, const CUtensorMap& mvt, const mla::tc::AttParams& ap,
-                        cudaStream_t st) {
+int launch_attention_tc(int N, int V, unsigned grid, const CUtensorMap& mq, const CUtensorMap& mqr,
+                        const CUtensorMap& mkn, const CUtensorMap& mkr, const CUtensorMap& mvt,
+                        const mla::tc::AttParams& ap, cudaStream_t st) {
 #define MLA_ATT_CASE(n, v) \
-  if (N == n && V == v) return launch_attention_tc_t<n, v>(grid, mq, mkn, mkr, mvt, ap, st);
+  if (N == n && V == v) return launch_attention_tc_t<n, v>(grid, mq, mqr, mkn, mkr, mvt, ap, st);
   MLA_ATT_CASE(64, 64) MLA_ATT_CASE(64, 128) MLA_ATT_CASE(64, 192) MLA_ATT_CASE(64, 256)
   MLA_ATT_CASE(128, 64) MLA_ATT_CASE(128, 128) MLA_ATT_CASE(128, 192) MLA_ATT_CASE(128, 256)
   MLA_ATT_CASE(192, 64) MLA_ATT_CASE(192, 128) MLA_ATT_CASE(192, 192) MLA_ATT_CASE(192, 256)
@@ -429,7 +430,7 @@ int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, cons
   __half* q_rope = reinterpret_cast<__half*>(ws + L.q_rope);
   const int cap = (int)L.cap;
   const int NOUT = H * (N + V);
-  // the two-tile attention takes k_nope in bf16 and the queries' rotated part
+  // both attention kernels take k_nope in bf16 and the queries' rotated part
   // from the preparation kernel
   const bool pair = attention_pair_shape(N, V) && d->softmax_scale > 0.f;
 
@@ -468,7 +469,7 @@ int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, cons
   qrp.cos_t = cos_t;
   qrp.sin_t = sin_t;
   qrp.qr = q_rope;
-  qrp.rows = pair ? T_tot * H : 0;
+  qrp.rows = T_tot * H;
   qrp.H = H; qrp.D = N + P; qrp.N = N; qrp.max_pos = max_pos; qrp.interleaved = d->rope_interleaved;
   const int qr_blocks = (int)((4 * qrp.rows + mla::tc::kPrepThreads - 1) / mla::tc::kPrepThreads);
   prof_begin(st, "tc_prep");
@@ -506,7 +507,7 @@ int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, cons
   gp.interleaved = d->rope_interleaved;
   gp.eps = d->eps;
   gp.tiles_per_cta = L.gemm_tiles_per_cta;
-  gp.knope_bf16 = pair ? 1 : 0;
+  gp.knope_bf16 = 1;
   cudaError_t e;
   if (vt_gemm) {
     // grid: (tiles, head groups); about one CTA per SM over the real tiles
@@ -550,7 +551,7 @@ int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, cons
     int rc = make_map(&map_q, q, 3, dims, strides, box);
     if (rc) return rc;
   }
-  if (pair) {
+  {
     const uint64_t dims[3] = {(uint64_t)P, (uint64_t)H, (uint64_t)T_tot};
     const uint64_t strides[2] = {(uint64_t)P * 2, (uint64_t)H * P * 2};
     const uint32_t box[3] = {64, 1, 128};
@@ -561,8 +562,7 @@ int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, cons
     const uint64_t dims[2] = {(uint64_t)N, (uint64_t)H * L.Tpad};
     const uint64_t strides[1] = {(uint64_t)N * 2};
     const uint32_t box[2] = {64, kv_box};
-    int rc = make_map(&map_kn, k_nope, 2, dims, strides, box,
-                      pair ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16);
+    int rc = make_map(&map_kn, k_nope, 2, dims, strides, box, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16);
     if (rc) return rc;
   }
   {
@@ -608,7 +608,7 @@ int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, cons
     return launch_attention_pair(N, V, (unsigned)grid, map_q, map_qr, map_kn, map_kr, map_vt, ap, st);
   }
   const unsigned grid = (unsigned)(cap * H);
-  return launch_attention_tc(N, V, grid, map_q, map_kn, map_kr, map_vt, ap, st);
+  return launch_attention_tc(N, V, grid, map_q, map_qr, map_kn, map_kr, map_vt, ap, st);
 }
 
 template <typename T>

@@ -8,9 +8,11 @@
 // scores are scaled, causally masked, normalized with a softmax in fp32 and
 // used to mix the values.
 //
-// Operands of both tensor-core products are fp16 (q is converted in shared
-// memory after its TMA load; k_nope, k_rot and the values come in fp16 from
-// the GEMM; P is packed to fp16), accumulators fp32, output bf16.
+// Operands: the non-rotary score atoms multiply q as given (bf16) with k_nope
+// in bf16; the rotary atom multiplies q's rotary part, rotated once per row
+// by the preparation kernel, with the rotated shared key, both fp16; P and
+// the values are fp16; accumulators fp32, output bf16. Q therefore needs no
+// work on the SM: the first score product starts when its copy lands.
 //
 // One CTA = one (128-query tile, head). Warp 0 issues TMA loads, warp 1 issues
 // the MMAs, warps 2-5 own one query row per thread (TMEM lane = row):
@@ -18,9 +20,8 @@
 //   P_j   = exp2(S_j * scale * log2 e - m)   (online softmax, registers)
 //   O    += P_j V_j           (tcgen05, fp32 accumulator in TMEM)
 // The shared rotary key tile is loaded once per key tile and serves every
-// query row of the head; q's rotary part is rotated in shared memory right
-// after its TMA load. O is rescaled (in TMEM, by the softmax warps) whenever
-// a row's running max grows.
+// query row of the head. O is rescaled (in TMEM, by the softmax warps)
+// whenever a row's running max grows.
 #pragma once
 #include "tc_gemm.cuh"
 
@@ -67,7 +68,7 @@ struct AttParams {
 
 template <int kStages>
 struct AttBarriers {
-  uint64_t q_full, q_ready;
+  uint64_t q_full;
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t s_full[2], s_free[2];
   uint64_t p_full, pv_done, mma_done;
@@ -77,9 +78,9 @@ struct AttBarriers {
 
 template <int kN, int kV, int kStages>
 __global__ void __launch_bounds__(kAttThreads, 1)
-attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_kn,
-                 const __grid_constant__ CUtensorMap map_kr, const __grid_constant__ CUtensorMap map_vt,
-                 AttParams p) {
+attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constant__ CUtensorMap map_qr,
+                 const __grid_constant__ CUtensorMap map_kn, const __grid_constant__ CUtensorMap map_kr,
+                 const __grid_constant__ CUtensorMap map_vt, AttParams p) {
   using C = AttCfg<kN, kV, kStages>;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   __shared__ AttBarriers<kStages> bars;
@@ -107,7 +108,6 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
 
   if (threadIdx.x == 0) {
     mbar_init(&bars.q_full, 1);
-    mbar_init(&bars.q_ready, 128);
     for (int s = 0; s < kStages; ++s) { mbar_init(&bars.kv_full[s], 1); mbar_init(&bars.kv_empty[s], 1); }
     for (int b = 0; b < 2; ++b) { mbar_init(&bars.s_full[b], 1); mbar_init(&bars.s_free[b], 128); }
     mbar_init(&bars.p_full, 128);
@@ -126,12 +126,17 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     // ---------------- TMA producer ----------------
     if (lane == 0) {
       tma_prefetch_desc(&map_q);
+      tma_prefetch_desc(&map_qr);
       tma_prefetch_desc(&map_kn);
       tma_prefetch_desc(&map_kr);
       tma_prefetch_desc(&map_vt);
+      // Q's non-rotary atoms as given (bf16) and its rotary atom rotated by the
+      // preparation kernel (fp16; that kernel finished before the previous one
+      // started)
       mbar_arrive_expect_tx(&bars.q_full, C::kQBytes);
-      for (int a = 0; a < C::kQAtoms; ++a)
+      for (int a = 0; a < kN / 64; ++a)
         tma_load_3d(sQ + a * kTile * 128, &map_q, &bars.q_full, a * 64, h, (int)(seq0 + q0));
+      tma_load_3d(sQ + (kN / 64) * kTile * 128, &map_qr, &bars.q_full, 0, h, (int)(seq0 + q0));
       pdl_wait();   // k_nope, the values and k_rot come from the previous kernel
       bool ok = true;
       int j = 0;
@@ -155,10 +160,11 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer (whole warp; one elected lane issues) ----------------
-    const uint32_t idesc_s = idesc_f16_f32(kTile, kAttBKV);
+    const uint32_t idesc_s_nope = idesc_bf16_f32(kTile, kAttBKV);   // q as given, k_nope in bf16
+    const uint32_t idesc_s_rope = idesc_f16_f32(kTile, kAttBKV);    // rotated q and key in fp16
     const uint32_t idesc_o = idesc_f16_f32(kTile, kV);
     const uint32_t o_tmem = tmem + C::kOCol;
-    bool ok = mbar_wait_warp(&bars.q_ready, 0, abort_flag);
+    bool ok = mbar_wait_warp(&bars.q_full, 0, abort_flag);
     tc_fence_after();
     auto issue_pv = [&](int jj) -> bool {
       if (!mbar_wait_warp(&bars.p_full, (uint32_t)jj & 1u, abort_flag)) return false;
@@ -184,6 +190,7 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       for (int a = 0; a < C::kQAtoms; ++a) {
         const uint64_t qd = desc_kmajor_sw128(smem_u32(sQ + a * kTile * 128));
         const uint64_t kd = desc_kmajor_sw128(smem_u32(sK + a * C::kKAtomBytes));
+        const uint32_t idesc_s = a < kN / 64 ? idesc_s_nope : idesc_s_rope;
 #pragma unroll
         for (int k = 0; k < 4; ++k)
           mma_ss_elect(s_tmem, desc_advance(qd, k * 32), desc_advance(kd, k * 32), idesc_s, (a | k) != 0);
@@ -203,68 +210,7 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     const bool valid = (q0 + row) < L;
     const int qi = min(q0 + row, L - 1);          // in-sequence query index used by the mask
     const int64_t t = seq0 + q0 + row;
-    bool ok = mbar_wait_warp(&bars.q_full, 0, abort_flag);
-    if (ok) {
-      // this row of q: bf16 -> fp16 in place; the rotary part (last atom) is
-      // rotated at the token's position on the way
-      float qmax = 0.f;
-#pragma unroll 1
-      for (int a = 0; a < C::kQAtoms - 1; ++a) {
-        uint8_t* qa = sQ + a * kTile * 128;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint4* ptr = reinterpret_cast<uint4*>(qa + sw128_offset(row, c));
-          const uint4 v = *ptr;
-          const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-          uint32_t o4[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const float2 f = unpack_bf16x2(w4[e]);
-            qmax = fmaxf(qmax, fmaxf(fabsf(f.x), fabsf(f.y)));
-            o4[e] = pack_f16x2(f.x, f.y);
-          }
-          *ptr = make_uint4(o4[0], o4[1], o4[2], o4[3]);
-        }
-      }
-      uint8_t* qr = sQ + (C::kQAtoms - 1) * kTile * 128;
-      float x[64];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint4 v = *reinterpret_cast<const uint4*>(qr + sw128_offset(row, c));
-        const uint32_t w4[4] = {v.x, v.y, v.z, v.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const float2 f = unpack_bf16x2(w4[e]);
-          x[c * 8 + 2 * e] = f.x;
-          x[c * 8 + 2 * e + 1] = f.y;
-        }
-      }
-      const int64_t pos = valid ? checked_pos(p.positions[t], p.max_pos) : 0;
-      const float* ct = p.cos_t + pos * 32;
-      const float* st = p.sin_t + pos * 32;
-      float y[64];
-      if (p.interleaved) {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) rope_turn(x[2 * i], x[2 * i + 1], ct[i], st[i], y[2 * i], y[2 * i + 1]);
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) rope_turn(x[i], x[i + 32], ct[i], st[i], y[i], y[i + 32]);
-      }
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        uint4 v;
-        v.x = pack_f16x2(y[c * 8 + 0], y[c * 8 + 1]);
-        v.y = pack_f16x2(y[c * 8 + 2], y[c * 8 + 3]);
-        v.z = pack_f16x2(y[c * 8 + 4], y[c * 8 + 5]);
-        v.w = pack_f16x2(y[c * 8 + 6], y[c * 8 + 7]);
-        *reinterpret_cast<uint4*>(qr + sw128_offset(row, c)) = v;
-#pragma unroll
-        for (int e = 0; e < 8; ++e) qmax = fmaxf(qmax, fabsf(y[c * 8 + e]));
-      }
-      if (valid && !(qmax <= kF16Max)) raise_device_error(kDevErrRange);
-    }
-    fence_proxy_async_smem();
-    mbar_arrive(&bars.q_ready);
+    bool ok = true;
 
     float m = -INFINITY;      // running max (log2 units) used as the exponent's reference
     float l = 0.f;            // running sum of P at that reference

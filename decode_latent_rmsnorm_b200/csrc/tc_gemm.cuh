@@ -10,16 +10,15 @@
 // Precision: the normalized latent c_hat = w * x / rms(x) is formed in fp32
 // and handed to the tensor cores in fp16 (11 significant bits), against an
 // fp16 copy of the weight (exact for weights in fp16's normal range), with
-// fp32 accumulation; the values are stored in fp16, k_nope in bf16 for the
-// two-tile attention (whose non-rotary score atoms take q as given, in bf16)
-// and in fp16 for the one-tile attention. A value beyond the fp16 range sets
-// the device error word.
+// fp32 accumulation; the values are stored in fp16 and k_nope in bf16 (the
+// attention's non-rotary score atoms take q as given, in bf16). A value
+// beyond the fp16 range sets the device error word.
 //
 // Workspace layout ("padded token space"): every sequence starts on a
 // 128-row boundary, so a 128-token tile never straddles two sequences and
 // every TMA coordinate along tokens is a multiple of 64 elements. Rows past a
 // sequence's end are written as zeros.
-//   k_nope [H, Tpad, N]  bf16 / fp16   (row tp, N contiguous)
+//   k_nope [H, Tpad, N]  bf16   (row tp, N contiguous)
 //   vt     [H, V, Tpad]  fp16   (values transposed: tokens contiguous)
 //   k_rot  [Tpad, P]     fp16   (the shared rotary key, rotated)
 #pragma once
@@ -275,7 +274,7 @@ constexpr int kPrepThreads = 1024;
 constexpr int kPrepUnroll = 8;
 
 // The rotary part of every query head, turned at its token's position once
-// for all key steps: qr [Ttot, H, 64] fp16 (the two-tile attention's last
+// for all key steps: qr [Ttot, H, 64] fp16 (the attention kernels' last
 // score atom). Source: Kimi-K2 "RoPE coefficients" page, "Query heads": each
 // head's rotary query part is rotated at the token's position like the key's.
 struct QRopeParams {
@@ -489,8 +488,8 @@ struct GemmParams {
   // already in the padded layout (tile t = rows 128 t ..) and k_rot has been
   // written with it, so the tile's A rows are padded rows and k_rot is left
   int a_padded;
-  // 1: k_nope is stored as bf16 (the two-tile attention's score operand),
-  // 0: as fp16 (the one-tile attention's); the buffer holds 16-bit codes
+  // 1: k_nope is stored as bf16 (the attention's score operand), 0: as fp16;
+  // the buffer holds 16-bit codes
   int knope_bf16;
 };
 

@@ -25,12 +25,11 @@
  *   - MLA_BF16 runs read and write bfloat16 tensors and accumulate in fp32;
  *     MLA_FP32 runs are fp32 throughout (exact-fp32 SIMT kernels). Inside a
  *     bf16 prefill on the tensor cores the normalized latent and kv_b_proj
- *     enter the up-projection in fp16; the two-tile attention (qk_nope and
- *     v_head 64 or 128) multiplies q as given with k_nope rounded to bf16 for
- *     the non-rotary scores and the rotated q_pe and k_pe rounded to fp16 for
- *     the rotary ones, and the softmax weights with the values in fp16; the
- *     other head shapes use fp16 for all of these. Values beyond the fp16
- *     range in those fp16 buffers set the device error word.
+ *     enter the up-projection in fp16; the attention multiplies q as given
+ *     with k_nope rounded to bf16 for the non-rotary scores and the rotated
+ *     q_pe and k_pe rounded to fp16 for the rotary ones, and the softmax
+ *     weights with the values in fp16. Values beyond the fp16 range in those
+ *     fp16 buffers set the device error word.
  */
 #ifndef MLA_H_
 #define MLA_H_
