@@ -19,6 +19,7 @@
 #include "tc_decode.cuh"
 #include "chunk.cuh"
 #include "tc_chunk.cuh"
+#include "tc_linear.cuh"
 #include "proj.cuh"
 #include "selftest.cuh"
 
@@ -1145,54 +1146,101 @@ ChunkEagerWs chunk_eager_ws_layout(const mla_dims* d, int64_t n, int nseq, int m
 namespace {
 constexpr int64_t kMaxProjRows = (int64_t)1 << 20;   // grid limits of the Linear kernels
 
-// out[t, j] = sum_k x[t, k] w[j, k] for x [n, K], w [Nout, K], out [n, Nout]
-// (row-major). x and w are in the run dtype, or both fp16 when `f16_operands`;
-// out in the run dtype, or fp32 into out_f32 when that is set. bf16 / fp16 with
-// K a multiple of 64 and 16-byte aligned operands: tcgen05 (head_gemm_kernel
-// with one head, M = 128 output features x N = 64 rows per CTA); otherwise the
-// CUDA-core Linear.
+// bf16 / fp16 Linears with K a multiple of 64, Nout a multiple of 32 and
+// 16-byte aligned operands run on tcgen05 (linear_tc_kernel: 128 rows x bn
+// features per CTA, optionally split over K); the others on the CUDA cores.
 bool linear_tc(const mla_dims* d, const void* x, const void* w, int K) {
   return d->dtype == MLA_BF16 && K % 64 == 0 && aligned16(x) && aligned16(w);
 }
 
+// Most K splits of a Linear whose fp32 result is read by a kernel that adds
+// the partials (the workspaces hold this many).
+constexpr int kMaxLinSplits = 4;
+
+// Product width (bn) and K splits of a tensor-core Linear: the pair with the
+// least estimated time, waves of one CTA per SM times a CTA's work (two
+// cycles per feature and K stage at the full tensor rate, plus a fixed cost).
+struct LinPlan {
+  int bn, splits;
+};
+LinPlan plan_linear(int64_t n, int K, int Nout, int max_splits) {
+  const int cands[4] = {128, 192, 224, 256};
+  const int ns = K / 64;
+  LinPlan best{256, 1};
+  double best_cost = 0.0;
+  for (int bn : cands)
+    for (int sp = 1; sp <= max_splits && sp <= ns; ++sp) {
+      const int64_t ctas = (int64_t)((Nout + bn - 1) / bn) * ((n + 127) / 128) * sp;
+      const int64_t waves = (ctas + num_sms() - 1) / num_sms();
+      const double cost = (double)waves * ((double)((ns + sp - 1) / sp) * 2.0 * bn + 6000.0);
+      if (best_cost == 0.0 || cost < best_cost) {
+        best_cost = cost;
+        best = LinPlan{bn, sp};
+      }
+    }
+  return best;
+}
+
+extern "C++" {   // a template: C++ linkage inside the C-ABI block
+template <int kBN, bool kF16>
+int launch_linear_tc_t(const CUtensorMap& mx, const CUtensorMap& mw, const mla::tc::LinParams& lp, int64_t n,
+                       cudaStream_t st) {
+  using C = mla::tc::LinCfg<kBN>;
+  auto kern = mla::tc::linear_tc_kernel<kBN, kF16>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)C::kSmem);
+  if (e != cudaSuccess) return cuda_status(e, "linear smem attribute");
+  kern<<<dim3((unsigned)((lp.Nout + kBN - 1) / kBN), (unsigned)((n + 127) / 128), (unsigned)lp.splits),
+         mla::tc::kLinThreads, C::kSmem, st>>>(mx, mw, lp);
+  return cuda_status(cudaGetLastError(), "linear launch");
+}
+}  // extern "C++"
+
+// out[t, j] = sum_k x[t, k] w[j, k] for x [n, K], w [Nout, K], out [n, Nout]
+// (row-major). x and w are in the run dtype, or both fp16 when `f16_operands`;
+// the result goes to `out` in the run dtype, or to out_f32 in fp32 when that
+// is set. With max_splits > 1 the tensor-core Linear may split K: out_f32
+// then holds *splits partials [splits][n][Nout] that the consumer adds in
+// split order (*splits is 1 otherwise).
 int launch_linear(const mla_dims* d, const void* x, const void* w, void* out, int64_t n, int K, int Nout,
-                  cudaStream_t st, const char* name, float* out_f32 = nullptr, bool f16_operands = false) {
+                  cudaStream_t st, const char* name, float* out_f32 = nullptr, bool f16_operands = false,
+                  int max_splits = 1, int* splits = nullptr) {
   namespace T = mla::tc;
-  if (linear_tc(d, x, w, K)) {
+  if (splits) *splits = 1;
+  if (linear_tc(d, x, w, K) && Nout % 32 == 0 && aligned16(out_f32 ? (const void*)out_f32 : out)) {
     const CUtensorMapDataType dt = f16_operands ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16;
+    const LinPlan pl = plan_linear(n, K, Nout, out_f32 ? max_splits : 1);
     CUtensorMap map_w, map_x;
     {
       const uint64_t dims[2] = {(uint64_t)K, (uint64_t)Nout};
       const uint64_t strides[1] = {(uint64_t)K * 2};
-      const uint32_t box[2] = {64, 128};
+      const uint32_t box[2] = {64, (uint32_t)pl.bn};
       int rc = make_map(&map_w, w, 2, dims, strides, box, dt);
       if (rc) return rc;
     }
     {
-      const uint64_t dims[3] = {(uint64_t)K, 1, (uint64_t)n};
-      const uint64_t strides[2] = {(uint64_t)K * 2, (uint64_t)K * 2};
-      const uint32_t box[3] = {64, 1, 64};
-      int rc = make_map(&map_x, x, 3, dims, strides, box, dt);
+      const uint64_t dims[2] = {(uint64_t)K, (uint64_t)n};
+      const uint64_t strides[1] = {(uint64_t)K * 2};
+      const uint32_t box[2] = {64, 128};
+      int rc = make_map(&map_x, x, 2, dims, strides, box, dt);
       if (rc) return rc;
     }
-    auto kern = f16_operands ? T::head_gemm_kernel<false, true> : T::head_gemm_kernel<false, false>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)T::kHgSmem);
-    if (e != cudaSuccess) return cuda_status(e, "linear smem attribute");
-    T::HgParams hp{};
-    hp.out = static_cast<__nv_bfloat16*>(out);
-    hp.out_f32 = out_f32;
-    hp.out_bs = Nout;
-    hp.out_hs = 0;
-    hp.B = (int)n;
-    hp.Nout = Nout;
-    hp.K = K;
-    hp.a_row0 = 0;
-    hp.a_hstride = 0;
+    T::LinParams lp{};
+    lp.n = n;
+    lp.K = K;
+    lp.Nout = Nout;
+    lp.splits = pl.splits;
+    lp.out = static_cast<__nv_bfloat16*>(out);
+    lp.out_f32 = out_f32;
+    if (splits) *splits = pl.splits;
     prof_begin(st, name);
-    kern<<<dim3(1, (unsigned)((Nout + 127) / 128), (unsigned)((n + 63) / 64)), 192, T::kHgSmem, st>>>(map_w, map_x,
-                                                                                                       hp);
+    int rc = MLA_OK;
+#define MLA_LIN_CASE(c)                                                                     \
+    if (pl.bn == c) rc = f16_operands ? launch_linear_tc_t<c, true>(map_x, map_w, lp, n, st) \
+                                      : launch_linear_tc_t<c, false>(map_x, map_w, lp, n, st);
+    MLA_LIN_CASE(128) MLA_LIN_CASE(192) MLA_LIN_CASE(224) MLA_LIN_CASE(256)
+#undef MLA_LIN_CASE
     prof_end(st);
-    return cuda_status(cudaGetLastError(), name);
+    return rc;
   }
   const dim3 grid((unsigned)((Nout + mla::kLinTile - 1) / mla::kLinTile),
                   (unsigned)((n + mla::kLinTile - 1) / mla::kLinTile));
@@ -1225,21 +1273,24 @@ int launch_linear_f32x(const float* x, const void* w, void* out, int64_t n, int 
   return cuda_status(cudaGetLastError(), name);
 }
 
-// Workspace of mla_kv_down_append: the fp32 result of the Linear (bf16 runs).
+// Workspace of mla_kv_down_append: the fp32 result of the Linear (bf16 runs),
+// room for kMaxLinSplits K-split partials.
 size_t kv_down_ws_bytes(const mla_dims* d, int64_t n) {
-  return d->dtype == MLA_BF16 ? align_up((size_t)n * (d->kv_lora_rank + d->qk_rope) * 4, 256) : 0;
+  return d->dtype == MLA_BF16 ? align_up((size_t)kMaxLinSplits * n * (d->kv_lora_rank + d->qk_rope) * 4, 256) : 0;
 }
 
 // Workspace of mla_q_proj. fp32 runs: q_a [n, q_rank] fp32, normalized in
-// place. bf16 runs: q_a [n, q_rank] fp32, its normalized copy [n, q_rank] (fp16
-// for the tensor-core q_b_proj), and the fp16 copy of w_qb.
+// place. bf16 runs: q_a as up to kMaxLinSplits fp32 partials [n, q_rank], its
+// normalized copy [n, q_rank] (fp16 for the tensor-core q_b_proj), and the
+// fp16 copy of w_qb.
 struct QProjWs {
   size_t q_a, q_an, w16, total;
 };
 QProjWs q_proj_ws_layout(const mla_dims* d, int32_t q_rank, int64_t n) {
   QProjWs L{};
   size_t off = 0;
-  L.q_a = off; off = align_up(off + (size_t)n * q_rank * 4, 256);
+  // bf16: q_a_proj's fp32 partials (up to kMaxLinSplits K splits)
+  L.q_a = off; off = align_up(off + (size_t)(d->dtype == MLA_BF16 ? kMaxLinSplits : 1) * n * q_rank * 4, 256);
   if (d->dtype == MLA_BF16) {
     L.q_an = off; off = align_up(off + (size_t)n * q_rank * 4, 256);   // fp16 (tensor cores) or fp32 (CUDA cores)
     L.w16 = off;  off = align_up(off + (size_t)d->num_heads * (d->qk_nope + d->qk_rope) * q_rank * 2, 256);
@@ -1644,15 +1695,19 @@ int mla_kv_down_append(const mla_dims* dims, int32_t hidden_size, const void* hi
   }
   // bf16: the Linear's fp32 result, then compressed_kv and the cache row from it
   float* x32 = static_cast<float*>(workspace);
-  rc = launch_linear(dims, hidden, w_kva, nullptr, n, hidden_size, W, stream, "kv_a_proj", x32);
+  int splits = 1;
+  rc = launch_linear(dims, hidden, w_kva, nullptr, n, hidden_size, W, stream, "kv_a_proj", x32, false,
+                     kMaxLinSplits, &splits);
   if (rc) return rc;
   prof_begin(stream, "kv_latent_append");
-  mla::kv_latent_append_kernel<<<(unsigned)((n + mla::kKvRowsPerBlock - 1) / mla::kKvRowsPerBlock),
-                                 32 * mla::kKvRowsPerBlock, 0, stream>>>(
-      x32, static_cast<__nv_bfloat16*>(latent), n, dims->kv_lora_rank, dims->qk_rope,
+  cudaError_t e = launch_dependent(
+      mla::kv_latent_append_kernel, dim3((unsigned)((n + mla::kKvRowsPerBlock - 1) / mla::kKvRowsPerBlock)),
+      dim3(32 * mla::kKvRowsPerBlock), 0, stream, (const float*)x32, splits, (int64_t)(n * W),
+      static_cast<__nv_bfloat16*>(latent), n, dims->kv_lora_rank, dims->qk_rope,
       static_cast<const __nv_bfloat16*>(w_norm), positions, cos_table, sin_table, max_pos, dims->rope_interleaved,
-      dims->eps, append ? static_cast<__nv_bfloat16*>(cache) : nullptr, cache_num_rows, cache_rows);
+      dims->eps, append ? static_cast<__nv_bfloat16*>(cache) : (__nv_bfloat16*)nullptr, cache_num_rows, cache_rows);
   prof_end(stream);
+  if (e != cudaSuccess) return cuda_status(e, "kv latent append launch");
   return cuda_status(cudaGetLastError(), "kv latent append launch");
 }
 
@@ -1700,7 +1755,9 @@ int mla_q_proj(const mla_dims* dims, int32_t hidden_size, int32_t q_rank, const 
   // the normalized q_a feeds q_b_proj in fp16 against an fp16 copy of w_qb
   // (tensor cores), or in fp32 (CUDA cores)
   float* qa32 = reinterpret_cast<float*>(ws + L.q_a);
-  rc = launch_linear(dims, hidden, w_qa, nullptr, n, hidden_size, q_rank, stream, "q_a_proj", qa32);
+  int splits = 1;
+  rc = launch_linear(dims, hidden, w_qa, nullptr, n, hidden_size, q_rank, stream, "q_a_proj", qa32, false,
+                     kMaxLinSplits, &splits);
   if (rc) return rc;
   const bool tc_b = linear_tc(dims, ws + L.q_an, w_qb, q_rank) && aligned16(q);
   if (tc_b) {
@@ -1717,7 +1774,7 @@ int mla_q_proj(const mla_dims* dims, int32_t hidden_size, int32_t q_rank, const 
       if (rc) return rc;
       prof_begin(stream, "q_a_layernorm");
       mla::rmsnorm_f32_rows_kernel<__half><<<blocks, 32 * mla::kRowsPerNormBlock, 0, stream>>>(
-          qa32, static_cast<const __nv_bfloat16*>(w_qnorm), qan, n, q_rank, dims->eps);
+          qa32, splits, n * q_rank, static_cast<const __nv_bfloat16*>(w_qnorm), qan, n, q_rank, dims->eps);
       prof_end(stream);
       rc = cuda_status(cudaGetLastError(), "q_a_layernorm launch");
       if (rc) return rc;
@@ -1727,7 +1784,7 @@ int mla_q_proj(const mla_dims* dims, int32_t hidden_size, int32_t q_rank, const 
   float* qan32 = reinterpret_cast<float*>(ws + L.q_an);
   prof_begin(stream, "q_a_layernorm");
   mla::rmsnorm_f32_rows_kernel<float><<<blocks, 32 * mla::kRowsPerNormBlock, 0, stream>>>(
-      qa32, static_cast<const __nv_bfloat16*>(w_qnorm), qan32, n, q_rank, dims->eps);
+      qa32, splits, n * q_rank, static_cast<const __nv_bfloat16*>(w_qnorm), qan32, n, q_rank, dims->eps);
   prof_end(stream);
   rc = cuda_status(cudaGetLastError(), "q_a_layernorm launch");
   if (rc) return rc;

@@ -11,7 +11,7 @@
 // (head_gemm_kernel with one head); these kernels are the rest: the query
 // RMSNorm, and a CUDA-core Linear for fp32 runs and other K.
 #pragma once
-#include "common.cuh"
+#include "tc_ptx.cuh"
 
 namespace mla {
 
@@ -43,20 +43,29 @@ rmsnorm_rows_kernel(const T* x, const T* __restrict__ w, T* y, int64_t rows, int
 // TO (fp16 for the tensor-core q_b_proj, fp32 for the CUDA-core one).
 template <typename TO>
 __global__ void __launch_bounds__(32 * kRowsPerNormBlock)
-rmsnorm_f32_rows_kernel(const float* __restrict__ x, const __nv_bfloat16* __restrict__ w, TO* __restrict__ y,
-                        int64_t rows, int width, float eps) {
+rmsnorm_f32_rows_kernel(const float* __restrict__ x, int splits, int64_t split_stride,
+                        const __nv_bfloat16* __restrict__ w, TO* __restrict__ y, int64_t rows, int width, float eps) {
   const int64_t t = (int64_t)blockIdx.x * kRowsPerNormBlock + (threadIdx.x >> 5);
   const int lane = threadIdx.x & 31;
   if (t >= rows) return;
   const float* xr = x + t * width;
+  // x holds `splits` partial sums of the Linear, split_stride apart: added in split order
+  auto xv = [&](int k) {
+    float v = xr[k];
+    for (int s = 1; s < splits; ++s) v += xr[(int64_t)s * split_stride + k];
+    return v;
+  };
   float ss = 0.f;
-  for (int k = lane; k < width; k += 32) ss = fmaf(xr[k], xr[k], ss);
+  for (int k = lane; k < width; k += 32) {
+    const float v = xv(k);
+    ss = fmaf(v, v, ss);
+  }
   ss = warp_sum(ss);
   const float r = 1.0f / sqrtf(ss / (float)width + eps);
   TO* yr = y + t * width;
   bool over = false;
   for (int k = lane; k < width; k += 32) {
-    const float v = __bfloat162float(w[k]) * (xr[k] * r);
+    const float v = __bfloat162float(w[k]) * (xv(k) * r);
     if constexpr (sizeof(TO) == 2) {
       over |= !(fabsf(v) <= 65504.f);
       yr[k] = __float2half_rn(v);
@@ -72,47 +81,79 @@ rmsnorm_f32_rows_kernel(const float* __restrict__ x, const __nv_bfloat16* __rest
 // input), and when `cache` is set the cache row
 //   RMSNorm(x[t, :R]) || rope(x[t, R:], positions[t])
 // into cache[cache_rows[t]], both computed from the fp32 values (the cache
-// append of the GLM-5 "KV cache" section fused onto the Linear's result). A
-// destination row or position out of range skips the row's append and sets
-// the device error word.
+// append of the GLM-5 "KV cache" section fused onto the Linear's result). x
+// holds `splits` partial sums of the Linear, split_stride apart: the warp adds
+// them in split order (16-byte loads, all of a lane's in flight) into its row
+// in shared memory, and the rest reads the row from there. A destination row
+// or position out of range skips the row's append and sets the device error
+// word. R + P <= 768.
 constexpr int kKvRowsPerBlock = 8;
+constexpr int kKvMaxWidth = 768;
 __global__ void __launch_bounds__(32 * kKvRowsPerBlock)
-kv_latent_append_kernel(const float* __restrict__ x, __nv_bfloat16* __restrict__ latent, int64_t n, int R, int P,
+kv_latent_append_kernel(const float* __restrict__ x, int splits, int64_t split_stride,
+                        __nv_bfloat16* __restrict__ latent, int64_t n, int R, int P,
                         const __nv_bfloat16* __restrict__ w_norm, const int32_t* __restrict__ positions,
                         const float* __restrict__ cos_t, const float* __restrict__ sin_t, int max_pos, int interleaved,
                         float eps, __nv_bfloat16* __restrict__ cache, int64_t cache_num_rows,
                         const int64_t* __restrict__ cache_rows) {
-  const int64_t t = (int64_t)blockIdx.x * kKvRowsPerBlock + (threadIdx.x >> 5);
+  __shared__ __align__(16) float s_row[kKvRowsPerBlock][kKvMaxWidth];
+  const int wi = threadIdx.x >> 5;
+  const int64_t t = (int64_t)blockIdx.x * kKvRowsPerBlock + wi;
   const int lane = threadIdx.x & 31;
+  // the destination row and position are the caller's: read before the wait
+  // for the Linear (launched as its programmatic dependent)
+  const int64_t crow = (cache && t < n) ? cache_rows[t] : 0;
+  const int64_t pos = (cache && t < n) ? positions[t] : 0;
+  tc::pdl_wait();
+  tc::pdl_allow_next();
   if (t >= n) return;
   const int W = R + P;
   const float* xr = x + t * W;
+  float* row = s_row[wi];
+  if (W % 4 == 0) {     // rows start on 16-byte boundaries
+    const float4* x4 = reinterpret_cast<const float4*>(xr);
+    const int64_t st4 = split_stride / 4;
+#pragma unroll 4
+    for (int c = lane; c < W / 4; c += 32) {
+      float4 v = x4[c];
+      for (int sp = 1; sp < splits; ++sp) {
+        const float4 u = x4[sp * st4 + c];
+        v.x += u.x; v.y += u.y; v.z += u.z; v.w += u.w;
+      }
+      reinterpret_cast<float4*>(row)[c] = v;
+    }
+  } else {
+    for (int k = lane; k < W; k += 32) {
+      float v = xr[k];
+      for (int sp = 1; sp < splits; ++sp) v += xr[(int64_t)sp * split_stride + k];
+      row[k] = v;
+    }
+  }
+  __syncwarp();
   __nv_bfloat16* lr = latent + t * W;
   float ss = 0.f;
   for (int k = lane; k < W; k += 32) {
-    const float v = xr[k];
+    const float v = row[k];
     lr[k] = __float2bfloat16_rn(v);
     if (k < R) ss = fmaf(v, v, ss);
   }
   if (!cache) return;
   ss = warp_sum(ss);
-  const int64_t row = cache_rows[t];
-  const int64_t pos = positions[t];
-  if (row < 0 || row >= cache_num_rows || pos < 0 || pos >= max_pos) {
+  if (crow < 0 || crow >= cache_num_rows || pos < 0 || pos >= max_pos) {
     if (lane == 0) raise_device_error(kDevErrBadInput);
     return;
   }
   const float r = 1.0f / sqrtf(ss / (float)R + eps);
-  __nv_bfloat16* dst = cache + row * W;
-  for (int k = lane; k < R; k += 32) dst[k] = __float2bfloat16_rn(__bfloat162float(w_norm[k]) * (xr[k] * r));
+  __nv_bfloat16* dst = cache + crow * W;
+  for (int k = lane; k < R; k += 32) dst[k] = __float2bfloat16_rn(__bfloat162float(w_norm[k]) * (row[k] * r));
   const int half = P / 2;
   for (int i = lane; i < half; i += 32) {
-    int a, b;
-    rope_pair_slots(i, P, interleaved, a, b);
+    int a2, b2;
+    rope_pair_slots(i, P, interleaved, a2, b2);
     float ox, oy;
-    rope_turn(xr[R + a], xr[R + b], cos_t[pos * half + i], sin_t[pos * half + i], ox, oy);
-    dst[R + a] = __float2bfloat16_rn(ox);
-    dst[R + b] = __float2bfloat16_rn(oy);
+    rope_turn(row[R + a2], row[R + b2], cos_t[pos * half + i], sin_t[pos * half + i], ox, oy);
+    dst[R + a2] = __float2bfloat16_rn(ox);
+    dst[R + b2] = __float2bfloat16_rn(oy);
   }
 }
 

@@ -293,12 +293,16 @@ int mla_prefill_cached_form(const mla_dims* dims, const void* latent, const void
  * gives the nn.Linear shapes, mla-queries the query order; "Key heads": mla-kv
  * the joint down-projection). A Linear is out[t, j] = sum_k x[t, k] w[j, k],
  * with w the nn.Linear weight [out, in]; no bias. In bf16 runs with the
- * reduced dimension K a multiple of 64 and 16-byte aligned x and w it runs on
- * the tensor cores (fp32 accumulation, bf16 result); otherwise on the CUDA
- * cores. At most 2^20 rows (tokens) per call (MLA_ERR_UNSUPPORTED_SHAPE). */
+ * reduced dimension K a multiple of 64, the output width a multiple of 32 and
+ * 16-byte aligned tensors it runs on the tensor cores (fp32 accumulation, bf16
+ * result, 128 rows by up to 256 outputs per CTA; the down-projection and
+ * q_a_proj may split K into up to 4 fp32 partials, added in a fixed order by
+ * the step that reads them); otherwise on the CUDA cores. At most 2^20 rows
+ * (tokens) per call (MLA_ERR_UNSUPPORTED_SHAPE). */
 
 /* Workspace bytes of mla_kv_down_append for n rows: the Linear's fp32
- * result [n, R + P] in bf16 runs, 0 in fp32 runs. */
+ * result [n, R + P] (room for 4 K-split partials) in bf16 runs, 0 in fp32
+ * runs. */
 int mla_kv_down_append_workspace_size(const mla_dims* dims, int64_t n, size_t* bytes);
 
 /* kv_a_proj_with_mqa, optionally followed by the cache append:
@@ -318,8 +322,9 @@ int mla_kv_down_append(const mla_dims* dims, int32_t hidden_size, const void* hi
                        const int64_t* cache_rows, void* workspace, size_t workspace_bytes,
                        cudaStream_t stream);
 
-/* Workspace bytes of mla_q_proj: the [n, q_rank] fp32 intermediate; in bf16
- * runs also its normalized copy and an fp16 copy of w_qb. */
+/* Workspace bytes of mla_q_proj: the [n, q_rank] fp32 intermediate (in bf16
+ * runs room for 4 K-split partials, its normalized copy and an fp16 copy of
+ * w_qb). */
 int mla_q_proj_workspace_size(const mla_dims* dims, int32_t q_rank, int64_t n, size_t* bytes);
 
 /* q = q_b_proj(q_a_layernorm(q_a_proj(hidden))):
