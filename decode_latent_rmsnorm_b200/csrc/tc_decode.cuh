@@ -18,26 +18,25 @@
 // sum) goes to its own slot, b + cta, and `combine` merges the slots of a
 // sequence by their log-sum-exp.
 //
-// Tensor-core mapping (M = 128 for both products, the shape tcgen05 runs at
-// full rate; see decode_attn_kernel for the data flow):
-//   S^T[t, h] : M = 128 cache rows, N = 64 heads, K = 576.
-//   O^T[d, h] : M = 128 latent dims (4 blocks), N = 64 heads, K = 128 rows.
+// Tensor-core mapping (see decode_attn_kernel for the data flow):
+//   S^T[t, h] : M = 64 cache rows, N = 64 heads, K = 576.
+//   O^T[d, h] : M = 128 latent dims (4 blocks), N = 64 heads, K = 64 rows.
 #pragma once
 #include "tc_gemm.cuh"
 
 namespace mla {
 namespace tc {
 
-constexpr int kDecRows = 128;                   // cache rows per tile (M of the score MMAs)
+constexpr int kDecRows = 64;                    // cache rows per tile (M of the score MMAs)
 constexpr int kDecHeads = 64;                   // heads per CTA (N of both MMAs)
 constexpr int kDecBoxes = 9;                    // 576 columns = 9 x 64
 constexpr int kDecLatBoxes = 8;                 // the 512 latent columns
-constexpr int kDecBoxBytes = kDecRows * 128;    // [128 rows x 64 cols] bf16 = 16 KB
-constexpr int kDecSlots = kDecBoxes;            // one smem slot per box of a tile
+constexpr int kDecBoxBytes = kDecRows * 128;    // [64 rows x 64 cols] bf16 = 8 KB
+constexpr int kDecBufs = 2;                     // tile buffers: one fills while the other is in use
+constexpr int kDecBufBytes = kDecBoxes * kDecBoxBytes;
 constexpr int kDecQBytes = kDecBoxes * kDecHeads * 128;
-constexpr int kDecPBytes = kDecRows * 128;      // P^T [128 rows x 64 heads] bf16
 constexpr int kDecThreads = 192;
-constexpr size_t kDecSmem = (size_t)kDecQBytes + kDecSlots * (size_t)kDecBoxBytes + 1024;   // P^T reuses the rope slot
+constexpr size_t kDecSmem = (size_t)kDecQBytes + kDecBufs * (size_t)kDecBufBytes + 1024;   // P^T reuses a rope box
 constexpr int kDecOCol = 0;                     // O^T: 4 blocks x 64 columns
 constexpr int kDecSCol = 256;                   // S^T: 64 columns
 
@@ -227,76 +226,56 @@ struct DecTileIter {
 
 struct DecBarriers {
   uint64_t q_full, q_empty;
-  uint64_t full[kDecSlots], empty[kDecSlots];
-  uint64_t s_full, s_free;           // S^T (TMEM)
-  uint64_t p_full, pv_done;          // P^T (smem, in the rope slot)
-  uint64_t o_free, mma_done;
-  uint64_t sm_sync;                  // bounded barrier of the 128 softmax threads
+  uint64_t full[kDecBufs], empty[kDecBufs];   // a tile buffer: its nine boxes landed / free again
+  uint64_t s_full[2], s_free[2];              // S^T buffers (TMEM)
+  uint64_t p_full[2];                         // P^T of the tile in buffer b (smem, its rope box)
+  uint64_t pv_done, o_free, mma_done;
+  uint64_t sm_sync;                           // bounded barrier of the 128 softmax threads
   uint32_t tmem_base;
   int abort_flag;
   int vote[2][4];                    // per tile parity: a vote is read after one sync, rewritten after two
-  float m_ref[kDecHeads];            // per-head reference max (log2 units)
+  alignas(16) float m_ref[kDecHeads];   // per-head reference max (log2 units; read as float4)
   float alpha[kDecHeads];
   float red[4][kDecHeads];           // per-warp column maxima / sums
 };
 
-// Column reduction of a warp: lane l holds v[0..63] (one value per head) and
-// ends with the reduction over the warp's 32 lanes of heads 2l and 2l + 1
-// (a halving exchange: 32 + 16 + 8 + 4 + 2 shuffles).
+// Column reduction over each half of a warp: lane l holds v[0..31], the
+// values of heads 32 (l >> 4) + i of one row, and ends with the reduction
+// over the 16 lanes of its half of heads 32 (l >> 4) + 2 (l & 15) and the
+// one after (a halving exchange: 16 + 8 + 4 + 2 shuffles).
 template <bool kMax>
-__device__ __forceinline__ float2 warp_column_reduce(float (&v)[kDecHeads], int lane) {
+__device__ __forceinline__ float2 half_column_reduce(float (&v)[32], int lane) {
 #pragma unroll
-  for (int c = 0; c < 32; ++c) {
-    const bool up = lane & 16;
-    const float send = up ? v[c] : v[c + 32];
-    const float keep = up ? v[c + 32] : v[c];
-    const float recv = __shfl_xor_sync(0xffffffffu, send, 16);
-    v[c] = kMax ? fmaxf(keep, recv) : keep + recv;
-  }
+  for (int m = 8; m >= 1; m >>= 1) {
+    const bool up = (lane & m) != 0;
 #pragma unroll
-  for (int c = 0; c < 16; ++c) {
-    const bool up = lane & 8;
-    const float send = up ? v[c] : v[c + 16];
-    const float keep = up ? v[c + 16] : v[c];
-    const float recv = __shfl_xor_sync(0xffffffffu, send, 8);
-    v[c] = kMax ? fmaxf(keep, recv) : keep + recv;
-  }
-#pragma unroll
-  for (int c = 0; c < 8; ++c) {
-    const bool up = lane & 4;
-    const float send = up ? v[c] : v[c + 8];
-    const float keep = up ? v[c + 8] : v[c];
-    const float recv = __shfl_xor_sync(0xffffffffu, send, 4);
-    v[c] = kMax ? fmaxf(keep, recv) : keep + recv;
-  }
-#pragma unroll
-  for (int c = 0; c < 4; ++c) {
-    const bool up = lane & 2;
-    const float send = up ? v[c] : v[c + 4];
-    const float keep = up ? v[c + 4] : v[c];
-    const float recv = __shfl_xor_sync(0xffffffffu, send, 2);
-    v[c] = kMax ? fmaxf(keep, recv) : keep + recv;
-  }
-#pragma unroll
-  for (int c = 0; c < 2; ++c) {
-    const bool up = lane & 1;
-    const float send = up ? v[c] : v[c + 2];
-    const float keep = up ? v[c + 2] : v[c];
-    const float recv = __shfl_xor_sync(0xffffffffu, send, 1);
-    v[c] = kMax ? fmaxf(keep, recv) : keep + recv;
+    for (int c = 0; c < 2 * m; ++c) {
+      const float send = up ? v[c] : v[c + 2 * m];
+      const float keep = up ? v[c + 2 * m] : v[c];
+      const float recv = __shfl_xor_sync(0xffffffffu, send, m);
+      v[c] = kMax ? fmaxf(keep, recv) : keep + recv;
+    }
   }
   return make_float2(v[0], v[1]);
 }
 
 // One persistent CTA per SM; warp 0 issues TMA loads, warp 1 the MMAs, warps
-// 2-5 run the softmax (one cache row per thread: S^T lane = row).
-//   S^T[t, h] = C[t, :] . q[h, :]      M = 128 rows, N = 64 heads, K = 576
-//   O^T[d, h] += C[:, d]^T . P^T[:, h]  M = 128 latent dims (4 blocks), N = 64, K = 128
-// Shared memory holds the resident q (72 KB) and one 128 x 576 tile as nine
-// 16 KB boxes, one slot per box. The 8 latent boxes stay from the scores to
-// the latent product; P^T is written into the rope box's slot once the
-// scores have read it. Slots free up block by block as the latent product
-// retires, and the next tile's boxes stream into them right away. The
+// 2-5 run the softmax.
+//   S^T[t, h] = C[t, :] . q[h, :]      M = 64 rows, N = 64 heads, K = 576
+//   O^T[d, h] += C[:, d]^T . P^T[:, h]  M = 128 latent dims (4 blocks), N = 64, K = 64
+// Shared memory holds the resident q (72 KB) and two buffers of one 64 x 576
+// tile each, as nine 8 KB boxes: the next tile streams into one buffer while
+// the products and the softmax work on the other. A tile's boxes stay from
+// its scores to its latent product; P^T is written into its rope box once
+// the scores have read it.
+// The tensor core takes about as long for an M = 64 as for an M = 128
+// product and has a floor per instruction, so the issue order matters: the
+// MMA warp issues the scores of tile j + 1 (into the second S^T buffer) as
+// soon as that tile has landed, ahead of the latent product of tile j, which
+// waits for the softmax; the tensor core then works through the softmax.
+// The M = 64 score accumulator keeps row 16 q + i (i < 16) in TMEM lane
+// 32 q + i: the softmax warp of lane quarter q reads its 16 rows with the
+// two-halves load, a thread taking 32 of the 64 heads of one row. The
 // softmax keeps a per-head reference max that it raises only when a score
 // exceeds it by more than 8 (2^8 bounds P), so the common path needs one
 // CTA-wide vote per tile and no column reduction.
@@ -315,17 +294,18 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_c
   if (r_lo >= r_hi) return;   // uniform over the CTA
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
-  uint8_t* sSlot = smem + kDecQBytes;                       // slot a holds box a of the current tile
-  uint8_t* sP = sSlot + (kDecSlots - 1) * kDecBoxBytes;     // P^T [128 rows x 64 heads] in the rope slot
+  uint8_t* sBuf = smem + kDecQBytes;   // buffer b: box a at b * kDecBufBytes + a * kDecBoxBytes
   volatile int* abort_flag = &bars.abort_flag;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars.q_full, 1);
     mbar_init(&bars.q_empty, 1);
-    for (int a = 0; a < kDecSlots; ++a) { mbar_init(&bars.full[a], 1); mbar_init(&bars.empty[a], 1); }
-    mbar_init(&bars.s_full, 1);
-    mbar_init(&bars.s_free, 128);
-    mbar_init(&bars.p_full, 128);
+    for (int b = 0; b < kDecBufs; ++b) { mbar_init(&bars.full[b], 1); mbar_init(&bars.empty[b], 1); }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&bars.s_full[b], 1);
+      mbar_init(&bars.s_free[b], 128);
+      mbar_init(&bars.p_full[b], 128);
+    }
     mbar_init(&bars.pv_done, 1);
     mbar_init(&bars.o_free, 128);
     mbar_init(&bars.mma_done, 1);
@@ -342,11 +322,12 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_c
 
   if (warp == 0) {
     // ---------------- TMA producer ----------------
+    // tile j goes to buffer j & 1 once the latent product of tile j - 2 is done
     if (lane == 0) {
       tma_prefetch_desc(&map_cache);
       tma_prefetch_desc(&map_q);
       bool ok = true;
-      int j = 0;
+      int j = 0, nq = 0;   // tiles issued, q loads issued
       DecTileIter tiles;
       tiles.init(p, r_lo, r_hi);
       DecTile t;
@@ -356,72 +337,104 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_c
           mbar_arrive_expect_tx(&bars.q_full, kDecQBytes);
           for (int a = 0; a < kDecBoxes; ++a)
             tma_load_2d(sQ + a * kDecHeads * 128, &map_q, &bars.q_full, a * 64, t.b * kDecHeads);
+          ++nq;
         }
-        for (int a = 0; a < kDecBoxes; ++a) {   // latent boxes first: they free up first
-          if (!mbar_wait(&bars.empty[a], ((uint32_t)j & 1u) ^ 1u, abort_flag)) { ok = false; break; }
-          mbar_arrive_expect_tx(&bars.full[a], kDecBoxBytes);
-          tma_load_2d(sSlot + a * kDecBoxBytes, &map_cache, &bars.full[a], a * 64, (int)t.row0);
-        }
+        const int bj = j & 1;
+        if (!mbar_wait(&bars.empty[bj], ((uint32_t)(j >> 1) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
+        uint8_t* buf = sBuf + bj * kDecBufBytes;
+        mbar_arrive_expect_tx(&bars.full[bj], kDecBufBytes);
+        for (int a = 0; a < kDecBoxes; ++a)
+          tma_load_2d(buf + a * kDecBoxBytes, &map_cache, &bars.full[bj], a * 64, (int)t.row0);
         ++j;
       }
       if (!ok) {   // let the copies in flight land before the CTA exits
-        mbar_wait_drain(&bars.q_full, 0);
-        for (int a = 0; a < kDecSlots; ++a) mbar_wait_drain(&bars.full[a], (uint32_t)(j > 0 ? j - 1 : 0) & 1u);
+        if (nq > 0) mbar_wait_drain(&bars.q_full, (uint32_t)(nq - 1) & 1u);
+        for (int b = 0; b < kDecBufs; ++b) {
+          const int n = (j + 1 - b) / 2;   // tiles j' < j with j' & 1 == b
+          if (n > 0) mbar_wait_drain(&bars.full[b], (uint32_t)(n - 1) & 1u);
+        }
       }
     }
   } else if (warp == 1) {
     // ---------------- MMA issuer (whole warp; one elected lane issues) ----------------
+    // Polls, in this order: the latent product of tile jo (its P^T written),
+    // then the scores of tile js (its buffer landed, its S^T buffer read),
+    // with js at most one tile ahead of jo. Decisions are warp-uniform.
     const uint32_t idesc_s = idesc_bf16_f32(kDecRows, kDecHeads);
     const uint32_t idesc_o = idesc_bf16_f32(128, kDecHeads) | kIdescAMajorMN | kIdescBMajorMN;
-    bool ok = true;
-    int j = 0;
-    DecTileIter tiles;
-    tiles.init(p, r_lo, r_hi);
-    DecTile t;
-    while (ok && tiles.next(t)) {
-      const uint32_t ph = (uint32_t)j & 1u;
-      // ---- S^T(j) ----
-      if (t.first && !(ok = mbar_wait_warp(&bars.q_full, (uint32_t)t.seg & 1u, abort_flag))) break;
-      if (!(ok = mbar_wait_warp(&bars.s_free, ph ^ 1u, abort_flag))) break;
-      tc_fence_after();
-      for (int a = 0; a < kDecBoxes && ok; ++a) {
-        if (!(ok = mbar_wait_warp(&bars.full[a], ph, abort_flag))) break;
-        tc_fence_after();
-        const uint64_t cd = desc_kmajor_sw128(smem_u32(sSlot + a * kDecBoxBytes));
-        const uint64_t qd = desc_kmajor_sw128(smem_u32(sQ + a * kDecHeads * 128));
+    DecTileIter its, ito;
+    its.init(p, r_lo, r_hi);
+    ito.init(p, r_lo, r_hi);
+    DecTile ts, to;
+    bool have_s = its.next(ts), have_o = ito.next(to);
+    int js = 0, jo = 0;
+    uint64_t t_idle = global_timer_ns();
+    uint32_t spins = 0;
+    while (have_o) {
+      if (js > jo) {   // ---- O^T(jo) += C^T P^T ----
+        bool ready = mbar_test(&bars.p_full[jo & 1], (uint32_t)(jo >> 1) & 1u);
+        if (to.first && to.seg > 0) ready = ready && mbar_test(&bars.o_free, (uint32_t)(to.seg - 1) & 1u);
+        if (__all_sync(0xffffffffu, ready)) {
+          tc_fence_after();
+          uint8_t* buf = sBuf + (jo & 1) * kDecBufBytes;
+          const uint64_t pd = desc_mnmajor_sw128(smem_u32(buf + kDecLatBoxes * kDecBoxBytes), kDecBoxBytes, 1024);
+          for (int blk = 0; blk < 4; ++blk) {
+            // latent columns [128 blk, 128 blk + 128): boxes 2 blk, 2 blk + 1, read MN-major
+            const uint64_t ad = desc_mnmajor_sw128(smem_u32(buf + 2 * blk * kDecBoxBytes), kDecBoxBytes, 1024);
 #pragma unroll
-        for (int k = 0; k < 4; ++k)
-          mma_ss_elect(tmem + kDecSCol, desc_advance(cd, k * 32), desc_advance(qd, k * 32), idesc_s, (a | k) != 0);
+            for (int k = 0; k < kDecRows / 16; ++k)
+              mma_ss_elect(tmem + kDecOCol + blk * kDecHeads, desc_advance(ad, k * 2048),
+                           desc_advance(pd, k * 2048), idesc_o, (to.first && k == 0) ? 0u : 1u);
+          }
+          mma_commit_elect(&bars.empty[jo & 1]);   // the buffer (and the P^T in it) is free
+          mma_commit_elect(&bars.pv_done);
+          ++jo;
+          have_o = ito.next(to);
+          t_idle = global_timer_ns();
+          continue;
+        }
       }
-      if (!ok) break;
-      mma_commit_elect(&bars.s_full);
-      if (t.last) mma_commit_elect(&bars.q_empty);     // q may be replaced once these are done
-      // ---- O^T(j) += C^T P^T ----
-      if (t.first && t.seg > 0 && !(ok = mbar_wait_warp(&bars.o_free, (uint32_t)(t.seg - 1) & 1u, abort_flag))) break;
-      if (!(ok = mbar_wait_warp(&bars.p_full, ph, abort_flag))) break;
-      tc_fence_after();
-      const uint64_t pd = desc_mnmajor_sw128(smem_u32(sP), kDecBoxBytes, 1024);
-      for (int blk = 0; blk < 4; ++blk) {
-        // latent columns [128 blk, 128 blk + 128): slots 2 blk, 2 blk + 1, read MN-major
-        const uint64_t ad = desc_mnmajor_sw128(smem_u32(sSlot + 2 * blk * kDecBoxBytes), kDecBoxBytes, 1024);
+      if (have_s && js <= jo + 1) {   // ---- S^T(js) ----
+        const uint32_t u = (uint32_t)(js >> 1) & 1u;
+        bool ready = mbar_test(&bars.full[js & 1], u) && mbar_test(&bars.s_free[js & 1], u ^ 1u);
+        if (ts.first) ready = ready && mbar_test(&bars.q_full, (uint32_t)ts.seg & 1u);
+        if (__all_sync(0xffffffffu, ready)) {
+          tc_fence_after();
+          uint8_t* buf = sBuf + (js & 1) * kDecBufBytes;
+          const uint32_t sd = tmem + kDecSCol + (uint32_t)(js & 1) * kDecHeads;
+          for (int a = 0; a < kDecBoxes; ++a) {
+            const uint64_t cd = desc_kmajor_sw128(smem_u32(buf + a * kDecBoxBytes));
+            const uint64_t qd = desc_kmajor_sw128(smem_u32(sQ + a * kDecHeads * 128));
 #pragma unroll
-        for (int k = 0; k < kDecRows / 16; ++k)
-          mma_ss_elect(tmem + kDecOCol + blk * kDecHeads, desc_advance(ad, k * 2048), desc_advance(pd, k * 2048),
-                       idesc_o, (t.first && k == 0) ? 0u : 1u);
-        mma_commit_elect(&bars.empty[2 * blk]);
-        mma_commit_elect(&bars.empty[2 * blk + 1]);
+            for (int k = 0; k < 4; ++k)
+              mma_ss_elect(sd, desc_advance(cd, k * 32), desc_advance(qd, k * 32), idesc_s, (a | k) != 0);
+          }
+          mma_commit_elect(&bars.s_full[js & 1]);
+          if (ts.last) mma_commit_elect(&bars.q_empty);   // q may be replaced once these are done
+          ++js;
+          have_s = its.next(ts);
+          t_idle = global_timer_ns();
+          continue;
+        }
       }
-      mma_commit_elect(&bars.empty[kDecSlots - 1]);    // P^T read: the rope slot is free
-      mma_commit_elect(&bars.pv_done);
-      ++j;
+      if ((++spins & 255u) == 0) {   // bounded: give up after kWaitLimitNs without progress
+        bool stop = *abort_flag != 0;
+        if (!stop && global_timer_ns() - t_idle > kWaitLimitNs) {
+          if (lane == 0) { *abort_flag = 1; raise_device_error(kDevErrTimeout); }
+          stop = true;
+        }
+        if (__any_sync(0xffffffffu, stop)) break;
+      }
     }
     mma_commit_elect(&bars.mma_done);          // every MMA done before TMEM is freed
     if (lane == 0) mbar_wait_drain(&bars.mma_done, 0);
     __syncwarp();
   } else {
     // ---------------- softmax / correction / partial epilogue (warps 2-5) ----------------
-    const int grp = warp & 3;                       // TMEM quadrant
-    const int tix = grp * 32 + lane;                // cache row of the tile == O^T latent row
+    const int grp = warp & 3;                       // TMEM lane quarter
+    const int tix = grp * 32 + lane;                // O^T latent row of this thread
+    const int hh = lane >> 4;                       // scores of heads [32 hh, 32 hh + 32) ...
+    const int row = grp * 16 + (lane & 15);         // ... of this tile row
     const uint32_t lane_base = (uint32_t)(grp * 32) << 16;
     int sync_ph = 0;
     auto cta_sync = [&]() -> bool {                 // bounded barrier of the 128 softmax threads
@@ -430,9 +443,9 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_c
       ++sync_ph;
       return r;
     };
-    float lpart[kDecHeads];
+    float lpart[32];
 #pragma unroll
-    for (int h = 0; h < kDecHeads; ++h) lpart[h] = 0.f;
+    for (int i = 0; i < 32; ++i) lpart[i] = 0.f;
     DecTileIter tiles;
     tiles.init(p, r_lo, r_hi);
     DecTile t;
@@ -440,31 +453,30 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_c
     bool ok = true;
     while (ok && tiles.next(t)) {
       const int b2 = j & 1;
-      if (!mbar_wait_warp(&bars.s_full, (uint32_t)j & 1u, abort_flag)) { ok = false; break; }
+      uint8_t* sP = sBuf + (j & 1) * kDecBufBytes + kDecLatBoxes * kDecBoxBytes;   // P^T [64 rows x 64 heads]
+      const uint32_t u = (uint32_t)(j >> 1) & 1u;
+      if (!mbar_wait_warp(&bars.s_full[j & 1], u, abort_flag)) { ok = false; break; }
       tc_fence_after();
-      float x[kDecHeads];
-      {   // the row's 64 scores: two loads in flight, one wait
-        uint32_t v[kDecHeads];
+      float x[32];
+      {
+        uint32_t v[32];
+        tmem_ld_halves32(tmem + lane_base + (uint32_t)(kDecSCol + (j & 1) * kDecHeads), v);
 #pragma unroll
-        for (int cc = 0; cc < kDecHeads / 32; ++cc)
-          tmem_ld32_nowait(tmem + lane_base + (uint32_t)(kDecSCol + cc * 32), v + cc * 32);
-        tmem_wait_ld64(v);
-#pragma unroll
-        for (int h = 0; h < kDecHeads; ++h) x[h] = __uint_as_float(v[h]);
+        for (int i = 0; i < 32; ++i) x[i] = __uint_as_float(v[i]);
       }
       tc_fence_before();
-      mbar_arrive(&bars.s_free);
-      const bool valid = tix < t.nvalid;
+      mbar_arrive(&bars.s_free[j & 1]);
+      const bool valid = row < t.nvalid;
       bool exceed = false;
 #pragma unroll
-      for (int q4 = 0; q4 < kDecHeads / 4; ++q4) {
-        const float4 mr = *reinterpret_cast<const float4*>(&bars.m_ref[q4 * 4]);
+      for (int q4 = 0; q4 < 8; ++q4) {
+        const float4 mr = *reinterpret_cast<const float4*>(&bars.m_ref[32 * hh + q4 * 4]);
         const float mrv[4] = {mr.x, mr.y, mr.z, mr.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          const int h = q4 * 4 + e;
-          const float xv = valid ? x[h] * p.scale_log2 : -INFINITY;
-          x[h] = xv;
+          const int i = q4 * 4 + e;
+          const float xv = valid ? x[i] * p.scale_log2 : -INFINITY;
+          x[i] = xv;
           exceed |= xv > mrv[e] + 8.f;
         }
       }
@@ -474,12 +486,12 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_c
       const bool any = (bars.vote[b2][0] | bars.vote[b2][1] | bars.vote[b2][2] | bars.vote[b2][3]) != 0;
       if (any) {
         // rare path: raise the reference max of heads whose scores outgrew it
-        float tmp[kDecHeads];
+        float tmp[32];
 #pragma unroll
-        for (int h = 0; h < kDecHeads; ++h) tmp[h] = x[h];
-        const float2 cm = warp_column_reduce<true>(tmp, lane);
-        bars.red[grp][2 * lane] = cm.x;
-        bars.red[grp][2 * lane + 1] = cm.y;
+        for (int i = 0; i < 32; ++i) tmp[i] = x[i];
+        const float2 cm = half_column_reduce<true>(tmp, lane);
+        bars.red[grp][32 * hh + 2 * (lane & 15)] = cm.x;
+        bars.red[grp][32 * hh + 2 * (lane & 15) + 1] = cm.y;
         if (!cta_sync()) { ok = false; break; }
         if (tix < kDecHeads) {
           const float mo = bars.m_ref[tix];
@@ -493,9 +505,13 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_c
         }
         if (!cta_sync()) { ok = false; break; }
 #pragma unroll
-        for (int h = 0; h < kDecHeads; ++h) lpart[h] *= bars.alpha[h];
+        for (int i = 0; i < 32; ++i) lpart[i] *= bars.alpha[32 * hh + i];
         if (!t.first) {
-          // O^T holds the segment's earlier tiles (their P V finished before S^T(j) began)
+          // O^T holds the segment's earlier tiles once the latent product of
+          // tile j - 1 is done (that of tile j - 2 is: tile j's buffer was
+          // loaded after it, so the parity names phase j - 1)
+          if (!mbar_wait_warp(&bars.pv_done, (uint32_t)(j - 1) & 1u, abort_flag)) { ok = false; break; }
+          tc_fence_after();
 #pragma unroll 1
           for (int blk = 0; blk < 4; ++blk)
 #pragma unroll 1
@@ -510,11 +526,11 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_c
           tmem_st_wait();
         }
       }
-      // P^T row of this thread (relative to the reference max), bf16, into the rope slot
-      uint32_t pk[kDecHeads / 2];
+      // this thread's half row of P^T (relative to the reference max), bf16, into the rope box
+      uint32_t pk[16];
 #pragma unroll
-      for (int q4 = 0; q4 < kDecHeads / 4; ++q4) {
-        const float4 mr = *reinterpret_cast<const float4*>(&bars.m_ref[q4 * 4]);
+      for (int q4 = 0; q4 < 8; ++q4) {
+        const float4 mr = *reinterpret_cast<const float4*>(&bars.m_ref[32 * hh + q4 * 4]);
         const uint32_t a0 = pack_bf16x2(ex2_approx(x[q4 * 4] - mr.x), ex2_approx(x[q4 * 4 + 1] - mr.y));
         const uint32_t a1 = pack_bf16x2(ex2_approx(x[q4 * 4 + 2] - mr.z), ex2_approx(x[q4 * 4 + 3] - mr.w));
         pk[q4 * 2] = a0;
@@ -526,15 +542,20 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_c
         lpart[q4 * 4 + 3] += f1.y;
       }
 #pragma unroll
-      for (int cc = 0; cc < 8; ++cc)
-        *reinterpret_cast<uint4*>(sP + sw128_offset(tix, cc)) =
+      for (int cc = 0; cc < 4; ++cc)
+        *reinterpret_cast<uint4*>(sP + sw128_offset(row, 4 * hh + cc)) =
             make_uint4(pk[4 * cc], pk[4 * cc + 1], pk[4 * cc + 2], pk[4 * cc + 3]);
       fence_proxy_async_smem();
       tc_fence_before();
-      mbar_arrive(&bars.p_full);
+      mbar_arrive(&bars.p_full[j & 1]);
       if (t.last) {
         // segment epilogue: unnormalized partial to slot (b + cta)
         const int slot = t.b + c;
+        // pv_done completes once per tile, in order. The latent product of
+        // tile j - 1 may still run (the scores of tile j can be issued ahead
+        // of it), so its phase is awaited first: only then does the parity of
+        // phase j name phase j.
+        if (j > 0 && !mbar_wait_warp(&bars.pv_done, (uint32_t)(j - 1) & 1u, abort_flag)) { ok = false; break; }
         if (!mbar_wait_warp(&bars.pv_done, (uint32_t)j & 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll 1
@@ -547,9 +568,9 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_c
             for (int e = 0; e < 16; ++e)
               p.o_part[((int64_t)slot * p.H + cc * 16 + e) * p.R + blk * 128 + tix] = __uint_as_float(v[e]);
           }
-        const float2 ls = warp_column_reduce<false>(lpart, lane);
-        bars.red[grp][2 * lane] = ls.x;
-        bars.red[grp][2 * lane + 1] = ls.y;
+        const float2 ls = half_column_reduce<false>(lpart, lane);
+        bars.red[grp][32 * hh + 2 * (lane & 15)] = ls.x;
+        bars.red[grp][32 * hh + 2 * (lane & 15) + 1] = ls.y;
         if (!cta_sync()) { ok = false; break; }
         if (tix < kDecHeads) {
           p.m_part[(int64_t)slot * p.H + tix] = bars.m_ref[tix];
@@ -558,7 +579,7 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_c
           bars.m_ref[tix] = -INFINITY;   // the next segment starts afresh
         }
 #pragma unroll
-        for (int h = 0; h < kDecHeads; ++h) lpart[h] = 0.f;
+        for (int i = 0; i < 32; ++i) lpart[i] = 0.f;
         if (!cta_sync()) { ok = false; break; }
         tc_fence_before();
         mbar_arrive(&bars.o_free);
