@@ -668,19 +668,22 @@ int launch_decode_tc(const mla_dims* d, const void* q, const void* cache, int64_
   float* l_part = reinterpret_cast<float*>(ws + L.l_part);
   bf16* o_lat = reinterpret_cast<bf16*>(ws + L.o_lat);
 
+  // The cache rows and the absorbed queries as {64 columns, rows, 9 column
+  // blocks}: one box brings a whole [rows x 576] tile, laid out in shared
+  // memory as nine [rows x 64] blocks (the layout the score product reads).
   CUtensorMap map_cache, map_q;
   {
-    const uint64_t dims[2] = {(uint64_t)(R + P), (uint64_t)cache_rows};
-    const uint64_t strides[1] = {(uint64_t)(R + P) * 2};
-    const uint32_t box[2] = {64, (uint32_t)T::kDecRows};
-    int rc = make_map(&map_cache, cache, 2, dims, strides, box);
+    const uint64_t dims[3] = {64, (uint64_t)cache_rows, (uint64_t)T::kDecBoxes};
+    const uint64_t strides[2] = {(uint64_t)(R + P) * 2, 128};
+    const uint32_t box[3] = {64, (uint32_t)T::kDecRows, (uint32_t)T::kDecBoxes};
+    int rc = make_map(&map_cache, cache, 3, dims, strides, box);
     if (rc) return rc;
   }
   {
-    const uint64_t dims[2] = {(uint64_t)(R + P), (uint64_t)B * Hp};
-    const uint64_t strides[1] = {(uint64_t)(R + P) * 2};
-    const uint32_t box[2] = {64, (uint32_t)Hp};
-    int rc = make_map(&map_q, qf, 2, dims, strides, box);
+    const uint64_t dims[3] = {64, (uint64_t)B * Hp, (uint64_t)T::kDecBoxes};
+    const uint64_t strides[2] = {(uint64_t)(R + P) * 2, 128};
+    const uint32_t box[3] = {64, (uint32_t)Hp, (uint32_t)T::kDecBoxes};
+    int rc = make_map(&map_q, qf, 3, dims, strides, box);
     if (rc) return rc;
   }
   // q_lat[b, h, :] = q_nope[b, h, :] W_UK_h   (W_UK_h = rows j < N of head h: [N, R], R contiguous)

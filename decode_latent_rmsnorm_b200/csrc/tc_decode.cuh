@@ -335,16 +335,14 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_c
         if (t.first) {
           if (!mbar_wait(&bars.q_empty, ((uint32_t)t.seg & 1u) ^ 1u, abort_flag)) { ok = false; break; }
           mbar_arrive_expect_tx(&bars.q_full, kDecQBytes);
-          for (int a = 0; a < kDecBoxes; ++a)
-            tma_load_2d(sQ + a * kDecHeads * 128, &map_q, &bars.q_full, a * 64, t.b * kDecHeads);
+          tma_load_3d(sQ, &map_q, &bars.q_full, 0, t.b * kDecHeads, 0);   // nine [64 heads x 64] blocks
           ++nq;
         }
         const int bj = j & 1;
         if (!mbar_wait(&bars.empty[bj], ((uint32_t)(j >> 1) & 1u) ^ 1u, abort_flag)) { ok = false; break; }
         uint8_t* buf = sBuf + bj * kDecBufBytes;
         mbar_arrive_expect_tx(&bars.full[bj], kDecBufBytes);
-        for (int a = 0; a < kDecBoxes; ++a)
-          tma_load_2d(buf + a * kDecBoxBytes, &map_cache, &bars.full[bj], a * 64, (int)t.row0);
+        tma_load_3d(buf, &map_cache, &bars.full[bj], 0, (int)t.row0, 0);   // nine [64 rows x 64] boxes
         ++j;
       }
       if (!ok) {   // let the copies in flight land before the CTA exits
