@@ -38,7 +38,7 @@ constexpr int kDecQBytes = kDecBoxes * kDecHeads * 128;
 constexpr int kDecThreads = 192;
 constexpr size_t kDecSmem = (size_t)kDecQBytes + kDecBufs * (size_t)kDecBufBytes + 1024;   // P^T reuses a rope box
 constexpr int kDecOCol = 0;                     // O^T: 4 blocks x 64 columns
-constexpr int kDecSCol = 256;                   // S^T: 64 columns
+constexpr int kDecSCol = 256;                   // S^T: two buffers of 64 columns
 
 // ---- split schedule -----------------------------------------------------------
 // prefix[b] = rows of sequences before b (invalid sequences count 0 rows);
@@ -328,10 +328,17 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_c
       tma_prefetch_desc(&map_q);
       bool ok = true;
       int j = 0, nq = 0;   // tiles issued, q loads issued
-      DecTileIter tiles;
+      DecTileIter tiles, ahead;
       tiles.init(p, r_lo, r_hi);
-      DecTile t;
+      ahead.init(p, r_lo, r_hi);
+      DecTile t, ta;
+      // Tile j + 1 is prefetched into L2 when the copy of tile j is issued,
+      // before its own buffer frees up: its copy into shared memory then
+      // reads L2 instead of waiting on DRAM (a third tile in flight without
+      // shared memory; prefetching further ahead measured slower).
+      ahead.next(ta);
       while (ok && tiles.next(t)) {
+        if (ahead.next(ta)) tma_prefetch_l2_3d(&map_cache, 0, (int)ta.row0, 0);
         if (t.first) {
           if (!mbar_wait(&bars.q_empty, ((uint32_t)t.seg & 1u) ^ 1u, abort_flag)) { ok = false; break; }
           mbar_arrive_expect_tx(&bars.q_full, kDecQBytes);
