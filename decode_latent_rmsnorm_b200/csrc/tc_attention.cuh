@@ -17,11 +17,15 @@
 // One CTA = one (128-query tile, head). Warp 0 issues TMA loads, warp 1 issues
 // the MMAs, warps 2-5 own one query row per thread (TMEM lane = row):
 //   S_j   = Q K_j^T           (tcgen05, fp32 in TMEM, double buffered)
-//   P_j   = exp2(S_j * scale * log2 e - m)   (online softmax, registers)
-//   O    += P_j V_j           (tcgen05, fp32 accumulator in TMEM)
-// The shared rotary key tile is loaded once per key tile and serves every
-// query row of the head. O is rescaled (in TMEM, by the softmax warps)
-// whenever a row's running max grows.
+//   P_j   = exp2(S_j * scale * log2 e - m)   (online softmax, registers; fp16
+//           P written back over S_j in TMEM)
+//   O    += P_j V_j           (tcgen05, P read from TMEM, fp32 accumulator)
+// With P in TMEM and S double-buffered, the softmax of step j + 1 does not
+// wait for the P V product of step j. The shared rotary key tile is loaded
+// once per key tile and serves every query row of the head. The reference m
+// of a row is raised only when a score exceeds it by more than kAttLazy
+// (log2 units; P <= 2^kAttLazy stays well inside fp16), and O is rescaled
+// (in TMEM, by the softmax warps) only then.
 #pragma once
 #include "tc_gemm.cuh"
 
@@ -30,6 +34,7 @@ namespace tc {
 
 constexpr int kAttBKV = 64;                       // keys per tile (MMA N of S, K of PV)
 constexpr int kAttThreads = 192;
+constexpr float kAttLazy = 8.f;                   // reference max slack (log2 units)
 
 template <int kN, int kV, int kStages>
 struct AttCfg {
@@ -40,8 +45,7 @@ struct AttCfg {
   static constexpr int kKBytes = kQAtoms * kKAtomBytes;
   static constexpr int kVBytes = kV * 128;         // [kV rows x 64 keys]
   static constexpr int kStageBytes = kKBytes + kVBytes;
-  static constexpr int kPBytes = kTile * 128;      // [128 rows x 64 keys]
-  static constexpr size_t kSmem = (size_t)kQBytes + (size_t)kStages * kStageBytes + kPBytes + 1024;
+  static constexpr size_t kSmem = (size_t)kQBytes + (size_t)kStages * kStageBytes + 1024;
   static constexpr int kSCol = 0;                  // S buffers: columns [0, 128)
   static constexpr int kOCol = 2 * kAttBKV;        // O: columns [128, 128 + kV)
   static constexpr uint32_t kTmemCols = (kOCol + kV) <= 256 ? 256 : 512;
@@ -71,7 +75,8 @@ struct AttBarriers {
   uint64_t q_full;
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t s_full[2], s_free[2];
-  uint64_t p_full, pv_done, mma_done;
+  uint64_t p_full[2];              // P of the step in S buffer b written (TMEM)
+  uint64_t pv_done, mma_done;
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -103,14 +108,13 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sQ = smem;
   uint8_t* sKV = smem + C::kQBytes;
-  uint8_t* sP = sKV + kStages * C::kStageBytes;
   volatile int* abort_flag = &bars.abort_flag;
 
   if (threadIdx.x == 0) {
     mbar_init(&bars.q_full, 1);
     for (int s = 0; s < kStages; ++s) { mbar_init(&bars.kv_full[s], 1); mbar_init(&bars.kv_empty[s], 1); }
     for (int b = 0; b < 2; ++b) { mbar_init(&bars.s_full[b], 1); mbar_init(&bars.s_free[b], 128); }
-    mbar_init(&bars.p_full, 128);
+    for (int b = 0; b < 2; ++b) mbar_init(&bars.p_full[b], 128);
     mbar_init(&bars.pv_done, 1);
     mbar_init(&bars.mma_done, 1);
     bars.abort_flag = 0;
@@ -167,14 +171,14 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     bool ok = mbar_wait_warp(&bars.q_full, 0, abort_flag);
     tc_fence_after();
     auto issue_pv = [&](int jj) -> bool {
-      if (!mbar_wait_warp(&bars.p_full, (uint32_t)jj & 1u, abort_flag)) return false;
+      if (!mbar_wait_warp(&bars.p_full[jj & 1], (uint32_t)(jj >> 1) & 1u, abort_flag)) return false;
       tc_fence_after();
       const int s = jj % kStages;
-      const uint64_t pd = desc_kmajor_sw128(smem_u32(sP));
+      const uint32_t pa = tmem + C::kSCol + (uint32_t)((jj & 1) * kAttBKV);   // P over S_jj, 8 columns per 16 keys
       const uint64_t vd = desc_kmajor_sw128(smem_u32(sKV + s * C::kStageBytes + C::kKBytes));
 #pragma unroll
       for (int k = 0; k < kAttBKV / 16; ++k)
-        mma_ss_elect(o_tmem, desc_advance(pd, k * 32), desc_advance(vd, k * 32), idesc_o, (jj | k) != 0);
+        mma_ts_elect(o_tmem, pa + (uint32_t)(k * 8), desc_advance(vd, k * 32), idesc_o, (jj | k) != 0);
       mma_commit_elect(&bars.kv_empty[s]);
       mma_commit_elect(&bars.pv_done);
       return true;
@@ -236,11 +240,9 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         sc[e] = v;
         mx = fmaxf(mx, v);
       }
-      // the reference is the exact running max, so the dominant key of a row
-      // gets the weight 1.0 exactly (a lazier reference would round it)
       float alpha = 1.f;
       bool rescale = false;
-      if (mx > m) {
+      if (mx > m + kAttLazy) {
         if (m != -INFINITY) { alpha = ex2_approx(m - mx); rescale = true; }
         m = mx;
       }
@@ -256,11 +258,12 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
         rs += pr.x + pr.y;
       }
       l = l * alpha + rs;
-      if (j >= 1) {
-        // P buffer free and O stable once the previous P V product is done
+      if (j >= 1 && __any_sync(0xffffffffu, rescale)) {   // warp-collective TMEM access: whole warp, alpha = 1 elsewhere
+        // O is stable once the P V product of step j - 1 is done (that of
+        // step j - 2 is: S_j was issued after it, so the parity names j - 1)
         if (!mbar_wait_warp(&bars.pv_done, (uint32_t)(j - 1) & 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
-        if (__any_sync(0xffffffffu, rescale)) {   // warp-collective TMEM access: whole warp, alpha = 1 elsewhere
+        {
           for (int c = 0; c < kV / 16; ++c) {
             uint32_t v[16];
             const uint32_t ta = tmem + lane_base + (uint32_t)(C::kOCol + c * 16);
@@ -272,14 +275,22 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
           tmem_st_wait();
         }
       }
+      // P over this step's S columns (this thread's lane; its scores are read)
+      {
+        const uint32_t tp = tmem + lane_base + (uint32_t)(C::kSCol + b * kAttBKV);
+        uint32_t h0[16], h1[16];
 #pragma unroll
-      for (int c = 0; c < 8; ++c)
-        *reinterpret_cast<uint4*>(sP + sw128_offset(row, c)) =
-            make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
-      fence_proxy_async_smem();
+        for (int e = 0; e < 16; ++e) { h0[e] = pk[e]; h1[e] = pk[16 + e]; }
+        tmem_st16(tp, h0);
+        tmem_st16(tp + 16, h1);
+        tmem_st_wait();
+      }
       tc_fence_before();
-      mbar_arrive(&bars.p_full);
+      mbar_arrive(&bars.p_full[b]);
     }
+    // the P V products complete in order; the one of the step before the last
+    // may still run when the last softmax ends, so its phase is awaited first
+    if (ok && n_kv > 1) ok = mbar_wait_warp(&bars.pv_done, (uint32_t)(n_kv - 2) & 1u, abort_flag);
     if (ok && n_kv > 0) ok = mbar_wait_warp(&bars.pv_done, (uint32_t)(n_kv - 1) & 1u, abort_flag);
     if (ok) {
       tc_fence_after();
