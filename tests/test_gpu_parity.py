@@ -163,6 +163,21 @@ def test_decode_glm_heads_interleaved_b70(gpu_lib):
     compare(f64(got), ref, "bf16", "decode glm b70")
 
 
+def test_decode_many_short_sequences(gpu_lib):
+    # 400 short sequences around the 64-row tile edges: each CTA's row range
+    # holds several sequences, so segments of one or two tiles follow each
+    # other (a query block reloaded between back-to-back scores, segment ends
+    # next to the first tile of the next segment, single-row sequences)
+    lens = tuple((1, 2, 63, 64, 65, 127, 128, 129)[(7 * i) % 8] for i in range(400))
+    wl = W.scaled(W.DECODE, batch=400, cache_lens=lens, seed=17)
+    inp = W.decode_inputs(wl)
+    got = run_decode(wl, inp)
+    assert mla.mla_last_dispatch().startswith("tensor-core"), mla.mla_last_dispatch()
+    picks = sorted(set(range(0, 400, 11)) | {1, 2, 3, 4, 5, 6, 7, 398, 399})
+    ref = oracle_decode(wl, inp, batches=picks, absorbed=True)
+    compare(f64(got), ref, "bf16", "decode 400 short")
+
+
 @pytest.mark.parametrize("heads", [8, 16, 32])
 def test_decode_fewer_heads_tensor_core(gpu_lib, heads):
     # one GPU's share of a head-sharded Kimi-K2 decode: the tensor-core
