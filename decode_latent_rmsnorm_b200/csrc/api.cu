@@ -472,7 +472,7 @@ int launch_prefill_tc(const mla_dims* d, const void* latent, const void* q, cons
   qrp.qr = q_rope;
   qrp.rows = T_tot * H;
   qrp.H = H; qrp.D = N + P; qrp.N = N; qrp.max_pos = max_pos; qrp.interleaved = d->rope_interleaved;
-  const int qr_blocks = (int)((4 * qrp.rows + mla::tc::kPrepThreads - 1) / mla::tc::kPrepThreads);
+  const int qr_blocks = (int)mla::tc::q_rope_blocks(qrp.rows, H, mla::tc::kPrepThreads);
   prof_begin(st, "tc_prep");
   mla::tc::prefill_prep_kernel<<<(unsigned)(1 + w_blocks + norm_blocks + qr_blocks), mla::tc::kPrepThreads, 0,
                                  st>>>(
@@ -1447,7 +1447,7 @@ int launch_prefill_cached_eager(const mla_dims* d, const void* latent, const voi
   qrp.H = H; qrp.D = N + P; qrp.N = N; qrp.max_pos = max_pos; qrp.interleaved = d->rope_interleaved;
   if (qrp.rows > 0) {
     prof_begin(st, "tc_q_rope");
-    e = launch_dependent(T::q_rope_kernel, dim3((unsigned)((4 * qrp.rows + T::kPrepThreads - 1) / T::kPrepThreads)),
+    e = launch_dependent(T::q_rope_kernel, dim3((unsigned)T::q_rope_blocks(qrp.rows, H, T::kPrepThreads)),
                          dim3(T::kPrepThreads), 0, st, qrp);
     prof_end(st);
     if (e != cudaSuccess) return cuda_status(e, "q rope launch");

@@ -45,7 +45,7 @@
 //
 // Score operands: the non-rotary atoms multiply q as given (bf16) with k_nope
 // stored in bf16; the rotary atom multiplies the query's rotary part, turned
-// at its position once before this kernel (q_rope_group, run by the
+// at its position once before this kernel (q_rope_warp, run by the
 // up-projection GEMM's epilogue warps or a preparation kernel), with the
 // rotated shared key, both fp16; all products accumulate in one fp32 TMEM
 // tile. So Q needs no work on this SM: its first score product starts when

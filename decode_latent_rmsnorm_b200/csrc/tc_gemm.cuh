@@ -267,8 +267,8 @@ __device__ __forceinline__ void schedule_block(const int32_t* __restrict__ cu, i
 // Block 0 builds the schedule (schedule_block); blocks 1 .. w_blocks convert
 // the weight, kPrepUnroll x 8 values per thread; the next norm_blocks (when
 // launched) write the normalized latent in fp16 for the transposed-value
-// GEMM, and the blocks after those the rotated query rows (q_rope_group,
-// four threads per row). A value beyond the fp16 range sets the device error
+// GEMM, and the blocks after those the rotated query rows (q_rope_warp,
+// four warps per token). A value beyond the fp16 range sets the device error
 // word.
 constexpr int kPrepThreads = 1024;
 constexpr int kPrepUnroll = 8;
@@ -287,65 +287,76 @@ struct QRopeParams {
   int H, D, N, max_pos, interleaved;
 };
 
-// Pairs 8g .. 8g + 7 (g < 4) of row `row` = (t, h) of qr: pair i is
-// (x_i, x_{i+32}) (half-split) or (x_{2i}, x_{2i+1}) (interleaved), turned by
-// the angle of pair i at positions[t], each result rounded once to fp16.
-// Their values are the row's 16-byte chunks g and g + 4 (half-split) or 2g and
-// 2g + 1 (interleaved), so four threads with g = 0 .. 3 write a row's 128
-// bytes. mx takes the largest magnitude written (the caller checks the fp16
-// range).
-__device__ __forceinline__ void q_rope_group(const QRopeParams& p, int64_t row, int g, float& mx) {
-  const int64_t t = row / p.H;
-  const int64_t pos = checked_pos(p.positions[t], p.max_pos);
-  const uint4* src = reinterpret_cast<const uint4*>(p.q + row * p.D + p.N);
-  uint4* dst = reinterpret_cast<uint4*>(p.qr + row * 64);
-  const float4* c4 = reinterpret_cast<const float4*>(p.cos_t + pos * 32);
-  const float4* s4 = reinterpret_cast<const float4*>(p.sin_t + pos * 32);
-  const int ca = p.interleaved ? 2 * g : g, cb = p.interleaved ? 2 * g + 1 : g + 4;
-  const uint4 va = src[ca], vb = src[cb];
-  const float4 c0 = c4[2 * g], c1 = c4[2 * g + 1], s0 = s4[2 * g], s1 = s4[2 * g + 1];
-  const float cs[8] = {c0.x, c0.y, c0.z, c0.w, c1.x, c1.y, c1.z, c1.w};
-  const float sn[8] = {s0.x, s0.y, s0.z, s0.w, s1.x, s1.y, s1.z, s1.w};
-  const uint32_t wa[4] = {va.x, va.y, va.z, va.w}, wb[4] = {vb.x, vb.y, vb.z, vb.w};
-  float x[16];                        // chunk a, then chunk b
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    const float2 fa = unpack_bf16x2(wa[e]), fb = unpack_bf16x2(wb[e]);
-    x[2 * e] = fa.x; x[2 * e + 1] = fa.y;
-    x[8 + 2 * e] = fb.x; x[8 + 2 * e + 1] = fb.y;
-  }
-  float y[16];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    if (p.interleaved) rope_turn(x[2 * i], x[2 * i + 1], cs[i], sn[i], y[2 * i], y[2 * i + 1]);
-    else rope_turn(x[i], x[8 + i], cs[i], sn[i], y[i], y[8 + i]);
-  }
-  uint32_t oa[4], ob[4];
-#pragma unroll
-  for (int e = 0; e < 4; ++e) {
-    mx = fmaxf(mx, fmaxf(fmaxf(fabsf(y[2 * e]), fabsf(y[2 * e + 1])), fmaxf(fabsf(y[8 + 2 * e]), fabsf(y[9 + 2 * e]))));
-    oa[e] = pack_f16x2(y[2 * e], y[2 * e + 1]);
-    ob[e] = pack_f16x2(y[8 + 2 * e], y[9 + 2 * e]);
-  }
-  dst[ca] = make_uint4(oa[0], oa[1], oa[2], oa[3]);
-  dst[cb] = make_uint4(ob[0], ob[1], ob[2], ob[3]);
-}
-
-// Thread i of a grid-stride range: group i % 4 of row i / 4; a value beyond
+// The rotation runs one token per group of kQrWarpsPerToken warps: the
+// token's position and its cosine / sine row are read once by each warp, and
+// lane l of a warp turns the pairs 2 (l & 15) and 2 (l & 15) + 1 of the heads
+// h = 8 k + 2 w + (l >> 4) (w the warp of the token, k = 0, 1, ...): pair i
+// is (x_i, x_{i+32}) (half-split) or (x_{2i}, x_{2i+1}) (interleaved), turned
+// by the angle of pair i at positions[t], each result rounded once to fp16.
+// Four heads of a lane have their loads in flight together. A value beyond
 // the fp16 range sets the device error word.
-__device__ __forceinline__ void q_rope_unit(const QRopeParams& p, int64_t i) {
+constexpr int kQrWarpsPerToken = 4;
+__device__ __forceinline__ void q_rope_warp(const QRopeParams& p, int64_t w, int lane) {
+  const int64_t T = p.rows / p.H;
+  const int64_t t = w / kQrWarpsPerToken;
+  if (t >= T) return;
+  const int wq = (int)(w % kQrWarpsPerToken), hs = lane >> 4, l = lane & 15;
+  const int64_t pos = checked_pos(p.positions[t], p.max_pos);
+  const float2 cs = *reinterpret_cast<const float2*>(p.cos_t + pos * 32 + 2 * l);
+  const float2 sn = *reinterpret_cast<const float2*>(p.sin_t + pos * 32 + 2 * l);
+  const int nk = (p.H + 7) / 8;
   float mx = 0.f;
-  if (i < 4 * p.rows) q_rope_group(p, i >> 2, (int)(i & 3), mx);
+  for (int k0 = 0; k0 < nk; k0 += 4) {
+    uint32_t ra[4], rb[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int h = 8 * (k0 + u) + 2 * wq + hs;
+      if (h < p.H) {
+        const __nv_bfloat16* src = p.q + (t * p.H + h) * p.D + p.N;
+        if (p.interleaved) {
+          const uint2 v = *reinterpret_cast<const uint2*>(src + 4 * l);
+          ra[u] = v.x;
+          rb[u] = v.y;
+        } else {
+          ra[u] = *reinterpret_cast<const uint32_t*>(src + 2 * l);
+          rb[u] = *reinterpret_cast<const uint32_t*>(src + 32 + 2 * l);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int h = 8 * (k0 + u) + 2 * wq + hs;
+      if (h >= p.H) continue;
+      const float2 a = unpack_bf16x2(ra[u]), b = unpack_bf16x2(rb[u]);
+      __half* dst = p.qr + (t * p.H + h) * 64;
+      float y0, y1, y2, y3;
+      if (p.interleaved) {   // pairs (a.x, a.y) and (b.x, b.y)
+        rope_turn(a.x, a.y, cs.x, sn.x, y0, y1);
+        rope_turn(b.x, b.y, cs.y, sn.y, y2, y3);
+        *reinterpret_cast<uint2*>(dst + 4 * l) = make_uint2(pack_f16x2(y0, y1), pack_f16x2(y2, y3));
+      } else {               // pairs (a.x, b.x) and (a.y, b.y)
+        rope_turn(a.x, b.x, cs.x, sn.x, y0, y2);
+        rope_turn(a.y, b.y, cs.y, sn.y, y1, y3);
+        *reinterpret_cast<uint32_t*>(dst + 2 * l) = pack_f16x2(y0, y1);
+        *reinterpret_cast<uint32_t*>(dst + 32 + 2 * l) = pack_f16x2(y2, y3);
+      }
+      mx = fmaxf(mx, fmaxf(fmaxf(fabsf(y0), fabsf(y1)), fmaxf(fabsf(y2), fabsf(y3))));
+    }
+  }
   if (!(mx <= kF16Max)) raise_device_error(kDevErrRange);
+}
+// Blocks of the rotation for `rows` = tokens x heads.
+__host__ __device__ constexpr int64_t q_rope_blocks(int64_t rows, int H, int threads) {
+  return (rows / H * kQrWarpsPerToken * 32 + threads - 1) / threads;
 }
 
 // The rotated query rows on their own (chunks over a cached prefix, whose
-// positions the previous kernel writes), four threads per row.
+// positions the previous kernel writes).
 __global__ void __launch_bounds__(kPrepThreads)
 q_rope_kernel(QRopeParams p) {
   pdl_wait();
   pdl_allow_next();
-  q_rope_unit(p, (int64_t)blockIdx.x * kPrepThreads + threadIdx.x);
+  q_rope_warp(p, ((int64_t)blockIdx.x * kPrepThreads + threadIdx.x) >> 5, (int)(threadIdx.x & 31));
 }
 
 // Block `blk` of the fp16 weight copy: kPrepUnroll x 8 values per thread
@@ -392,7 +403,8 @@ prefill_prep_kernel(const int32_t* __restrict__ cu, int nseq, int64_t Ttot, int 
     return;
   }
   if ((int)blockIdx.x > w_blocks + norm_blocks) {
-    q_rope_unit(qrp, (int64_t)((int)blockIdx.x - 1 - w_blocks - norm_blocks) * kPrepThreads + threadIdx.x);
+    q_rope_warp(qrp, ((int64_t)((int)blockIdx.x - 1 - w_blocks - norm_blocks) * kPrepThreads + threadIdx.x) >> 5,
+                (int)(threadIdx.x & 31));
     return;
   }
   if ((int)blockIdx.x > w_blocks) {
