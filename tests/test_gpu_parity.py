@@ -122,6 +122,21 @@ def test_prefill_varlen_sampled(gpu_lib):
     compare(f64(got), ref, "bf16", "varlen")
 
 
+def test_prefill_many_short_sequences(gpu_lib):
+    """240 sequences whose lengths sit on and around the 128- and 256-row
+    tile edges (1, 2, 127, 128, 129, 255, 256, 257 in turn): single-tile query
+    blocks alternate with two-tile ones, so consecutive work items of the
+    persistent attention change sequence, tile count and key-step count at
+    nearly every claim. Every row of three heads is compared."""
+    base = (1, 2, 127, 128, 129, 255, 256, 257)
+    wl = W.scaled(W.KIMI, seqlens=tuple(base[(5 * i) % 8] for i in range(240)), seed=23)
+    inp = W.prefill_inputs(wl)
+    got = run_prefill(wl, inp)
+    assert mla.mla_last_dispatch().startswith("tensor-core"), mla.mla_last_dispatch()
+    ref = oracle_prefill(wl, inp, heads=[0, 21, 63])
+    compare(f64(got), ref, "bf16", "many short sequences")
+
+
 def test_prefill_output_guard_bytes(gpu_lib):
     # Writes stay inside `out`: guard regions around it keep their bytes.
     wl = W.scaled(W.KIMI, seqlens=(200, 57), seed=13)
