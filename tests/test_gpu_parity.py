@@ -122,6 +122,19 @@ def test_prefill_varlen_sampled(gpu_lib):
     compare(f64(got), ref, "bf16", "varlen")
 
 
+def test_prefill_longest_sampled(gpu_lib):
+    """One sequence of 32 768 tokens (the longest length the configs use):
+    256 key steps for the last query block, 128 blocks x 64 heads = 8192 work
+    items for the persistent attention. Sampled rows (both ends, around tile
+    edges, random) of the first and last head."""
+    wl = W.scaled(W.KIMI, seqlens=(32768,), seed=29)
+    inp = W.prefill_inputs(wl)
+    got = run_prefill(wl, inp)
+    assert mla.mla_last_dispatch().startswith("tensor-core"), mla.mla_last_dispatch()
+    ref = oracle_prefill(wl, inp, heads=[0, 63], rows=_varlen_rows(wl.seqlens, seed=5))
+    compare(f64(got), ref, "bf16", "prefill 32768")
+
+
 def test_prefill_many_short_sequences(gpu_lib):
     """240 sequences whose lengths sit on and around the 128- and 256-row
     tile edges (1, 2, 127, 128, 129, 255, 256, 257 in turn): single-tile query
