@@ -76,7 +76,7 @@ struct AttBarriers {
   uint64_t kv_full[kStages], kv_empty[kStages];
   uint64_t s_full[2], s_free[2];
   uint64_t p_full[2];              // P of the step in S buffer b written (TMEM)
-  uint64_t pv_done, mma_done;
+  uint64_t pv_done[2], mma_done;   // pv_done[j & 1]: the P V product of step j
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -115,7 +115,8 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
     for (int s = 0; s < kStages; ++s) { mbar_init(&bars.kv_full[s], 1); mbar_init(&bars.kv_empty[s], 1); }
     for (int b = 0; b < 2; ++b) { mbar_init(&bars.s_full[b], 1); mbar_init(&bars.s_free[b], 128); }
     for (int b = 0; b < 2; ++b) mbar_init(&bars.p_full[b], 128);
-    mbar_init(&bars.pv_done, 1);
+    mbar_init(&bars.pv_done[0], 1);
+    mbar_init(&bars.pv_done[1], 1);
     mbar_init(&bars.mma_done, 1);
     bars.abort_flag = 0;
     mbar_fence_init();
@@ -180,7 +181,7 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       for (int k = 0; k < kAttBKV / 16; ++k)
         mma_ts_elect(o_tmem, pa + (uint32_t)(k * 8), desc_advance(vd, k * 32), idesc_o, (jj | k) != 0);
       mma_commit_elect(&bars.kv_empty[s]);
-      mma_commit_elect(&bars.pv_done);
+      mma_commit_elect(&bars.pv_done[jj & 1]);
       return true;
     };
     for (int j = 0; j < n_kv && ok; ++j) {
@@ -260,8 +261,11 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       l = l * alpha + rs;
       if (j >= 1 && __any_sync(0xffffffffu, rescale)) {   // warp-collective TMEM access: whole warp, alpha = 1 elsewhere
         // O is stable once the P V product of step j - 1 is done (that of
-        // step j - 2 is: S_j was issued after it, so the parity names j - 1)
-        if (!mbar_wait_warp(&bars.pv_done, (uint32_t)(j - 1) & 1u, abort_flag)) { ok = false; break; }
+        // step j - 2 is: S_j was issued after it; step j + 1's is not issued)
+        if (!mbar_wait_warp(&bars.pv_done[(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
         tc_fence_after();
         {
           for (int c = 0; c < kV / 16; ++c) {
@@ -288,10 +292,13 @@ attention_kernel(const __grid_constant__ CUtensorMap map_q, const __grid_constan
       tc_fence_before();
       mbar_arrive(&bars.p_full[b]);
     }
-    // the P V products complete in order; the one of the step before the last
-    // may still run when the last softmax ends, so its phase is awaited first
-    if (ok && n_kv > 1) ok = mbar_wait_warp(&bars.pv_done, (uint32_t)(n_kv - 2) & 1u, abort_flag);
-    if (ok && n_kv > 0) ok = mbar_wait_warp(&bars.pv_done, (uint32_t)(n_kv - 1) & 1u, abort_flag);
+    // the last two P V products, each on the barrier of its step's parity
+    // (the previous phase of either is complete and no later one is issued,
+    // so each wait is at most one phase behind)
+    if (ok && n_kv > 1)
+      ok = mbar_wait_warp(&bars.pv_done[(n_kv - 2) & 1], (uint32_t)((n_kv - 2) >> 1) & 1u, abort_flag);
+    if (ok && n_kv > 0)
+      ok = mbar_wait_warp(&bars.pv_done[(n_kv - 1) & 1], (uint32_t)((n_kv - 1) >> 1) & 1u, abort_flag);
     if (ok) {
       tc_fence_after();
       const float inv = 1.f / l;

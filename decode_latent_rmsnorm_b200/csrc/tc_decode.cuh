@@ -229,7 +229,7 @@ struct DecBarriers {
   uint64_t full[kDecBufs], empty[kDecBufs];   // a tile buffer: its nine boxes landed / free again
   uint64_t s_full[2], s_free[2];              // S^T buffers (TMEM)
   uint64_t p_full[2];                         // P^T of the tile in buffer b (smem, its rope box)
-  uint64_t pv_done, o_free, mma_done;
+  uint64_t pv_done[2], o_free, mma_done;   // pv_done[j & 1]: the latent product of tile j
   uint64_t sm_sync;                           // bounded barrier of the 128 softmax threads
   uint32_t tmem_base;
   int abort_flag;
@@ -306,7 +306,8 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_c
       mbar_init(&bars.s_free[b], 128);
       mbar_init(&bars.p_full[b], 128);
     }
-    mbar_init(&bars.pv_done, 1);
+    mbar_init(&bars.pv_done[0], 1);
+    mbar_init(&bars.pv_done[1], 1);
     mbar_init(&bars.o_free, 128);
     mbar_init(&bars.mma_done, 1);
     mbar_init(&bars.sm_sync, 128);
@@ -392,7 +393,7 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_c
                            desc_advance(pd, k * 2048), idesc_o, (to.first && k == 0) ? 0u : 1u);
           }
           mma_commit_elect(&bars.empty[jo & 1]);   // the buffer (and the P^T in it) is free
-          mma_commit_elect(&bars.pv_done);
+          mma_commit_elect(&bars.pv_done[jo & 1]);
           ++jo;
           have_o = ito.next(to);
           t_idle = global_timer_ns();
@@ -513,9 +514,13 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_c
         for (int i = 0; i < 32; ++i) lpart[i] *= bars.alpha[32 * hh + i];
         if (!t.first) {
           // O^T holds the segment's earlier tiles once the latent product of
-          // tile j - 1 is done (that of tile j - 2 is: tile j's buffer was
-          // loaded after it, so the parity names phase j - 1)
-          if (!mbar_wait_warp(&bars.pv_done, (uint32_t)(j - 1) & 1u, abort_flag)) { ok = false; break; }
+          // tile j - 1 is done. Its barrier's previous phase (tile j - 3) is
+          // complete, as is that of tile j - 2 (tile j's buffer was loaded
+          // after it), and tile j + 1's is not issued: the parity is exact.
+          if (!mbar_wait_warp(&bars.pv_done[(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1u, abort_flag)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
 #pragma unroll 1
           for (int blk = 0; blk < 4; ++blk)
@@ -556,12 +561,16 @@ decode_attn_kernel(const __grid_constant__ CUtensorMap map_cache, const __grid_c
       if (t.last) {
         // segment epilogue: unnormalized partial to slot (b + cta)
         const int slot = t.b + c;
-        // pv_done completes once per tile, in order. The latent product of
-        // tile j - 1 may still run (the scores of tile j can be issued ahead
-        // of it), so its phase is awaited first: only then does the parity of
-        // phase j name phase j.
-        if (j > 0 && !mbar_wait_warp(&bars.pv_done, (uint32_t)(j - 1) & 1u, abort_flag)) { ok = false; break; }
-        if (!mbar_wait_warp(&bars.pv_done, (uint32_t)j & 1u, abort_flag)) { ok = false; break; }
+        // the latent products of tiles j - 1 (which may still run: the
+        // scores of tile j can be issued ahead of it) and j, each on the
+        // barrier of its tile's parity. On either barrier the previous phase
+        // (tile j - 3 or j - 2) is complete and the next (tile j + 1 or j + 2)
+        // not issued, so each wait is at most one phase behind.
+        if (j > 0 && !mbar_wait_warp(&bars.pv_done[(j - 1) & 1], (uint32_t)((j - 1) >> 1) & 1u, abort_flag)) {
+          ok = false;
+          break;
+        }
+        if (!mbar_wait_warp(&bars.pv_done[j & 1], (uint32_t)(j >> 1) & 1u, abort_flag)) { ok = false; break; }
         tc_fence_after();
 #pragma unroll 1
         for (int blk = 0; blk < 4; ++blk)
